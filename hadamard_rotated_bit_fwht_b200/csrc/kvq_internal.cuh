@@ -1,0 +1,119 @@
+// kvq_internal.cuh -- device helpers and launcher declarations shared by the
+// kernels of the KV-cache library.  Nothing here is part of the C ABI.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kDim = 256;       // Q4_0 path head dimension
+constexpr int kQBlock = 32;     // values per Q4_0 block
+constexpr int kRowCodeBytes = 128;
+constexpr int kRowScales = 8;
+constexpr int kNumSMs = 148;    // B200
+
+// ---------------------------------------------------------------- loads
+__device__ __forceinline__ uint4 ldg_stream_u4(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ---------------------------------------------------------------- packed fp32
+// Packed fp32x2 arithmetic through PTX instructions that carry an explicit
+// rounding modifier: ptxas never contracts those into a fused multiply-add,
+// so a product followed by a sum keeps its two roundings (the compiler
+// intrinsics of the same operations may be contracted).
+__device__ __forceinline__ uint64_t pk(float2 a) {
+  return (uint64_t)__float_as_uint(a.x) | ((uint64_t)__float_as_uint(a.y) << 32);
+}
+__device__ __forceinline__ float2 upk(uint64_t v) {
+  return make_float2(__uint_as_float((uint32_t)v), __uint_as_float((uint32_t)(v >> 32)));
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
+  return upk(r);
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
+  return upk(r);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
+  return upk(r);
+}
+__device__ __forceinline__ float2 add2_rz(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
+  return upk(r);
+}
+
+// ---------------------------------------------------------------- row index
+// Row of (sequence b, kv head h, token t) in the structure-of-arrays Q4_0
+// cache; -1 when the position lies outside the cache.
+__device__ __forceinline__ int64_t q4_row(const kvq_cache &c, int b, int h, int t) {
+  if (t < 0) return -1;
+  if (c.block_table == nullptr) {
+    if (t >= c.max_tokens) return -1;
+    return ((int64_t)b * c.num_kv_heads + h) * c.max_tokens + t;
+  }
+  int pi = t / c.page_size;
+  if (pi >= c.max_pages_per_seq) return -1;
+  int page = __ldg(c.block_table + (int64_t)b * c.max_pages_per_seq + pi);
+  if (page < 0 || page >= c.num_pages) return -1;
+  return ((int64_t)page * c.num_kv_heads + h) * c.page_size + (t - pi * c.page_size);
+}
+
+// ---------------------------------------------------------------- launchers
+cudaError_t launch_rotate(const void *x, int bf16, float *y, int64_t n_vec, cudaStream_t s);
+cudaError_t launch_q4_append(const kvq_cache &c, const void *k, const void *v, int bf16,
+                             int batch, int t_new, const int32_t *start_pos, cudaStream_t s);
+
+struct DecodePlan {
+  int splits;       // splits per (sequence, kv head)
+  int split_tokens; // tokens per split (multiple of 64)
+};
+DecodePlan plan_decode(int batch, int n_kv_heads, int max_seq_len);
+cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, int batch,
+                                 int n_q_heads, const int32_t *seq_lens, int max_seq_len,
+                                 float scale, float *ws, const DecodePlan &p, cudaStream_t s);
+size_t decode_workspace_bytes(int batch, int n_q_heads, const DecodePlan &p);
+cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int batch,
+                             int n_q_heads, const int32_t *seq_lens, int max_seq_len,
+                             float scale, float *out, float *ws, const DecodePlan &p,
+                             cudaStream_t s);
+
+struct OctaveParams {
+  int head_size, rope_dim, v_bits;
+  int off_k_nope, off_v, off_scales, slot_bytes;
+  uint32_t sign_words[16];  // up to 512 dims
+  int8_t lut3[8];
+  int8_t lut4[16];
+  float mult3, mult4;
+};
+cudaError_t launch_octave_quantize(const OctaveParams &p, const void *key, const void *value,
+                                   int bf16, int num_tokens, int n_kv_heads,
+                                   const int64_t *slot_mapping, uint8_t *cache,
+                                   int block_size, int64_t num_blocks, cudaStream_t s);
+DecodePlan plan_octave_decode(int num_q, int n_kv_heads, int max_klen);
+size_t octave_workspace_bytes(int num_q, int n_q_heads, int head_size, const DecodePlan &p);
+cudaError_t launch_octave_decode(const OctaveParams &p, const void *query, int bf16, int num_q,
+                                 int n_q_heads, const uint8_t *cache, int n_kv_heads,
+                                 int block_size, int64_t num_blocks, const int32_t *block_table,
+                                 int num_reqs, int max_blocks, const int32_t *q_to_req,
+                                 const int32_t *q_to_klen, int max_klen, float scale,
+                                 float *out, float *ws, const DecodePlan &plan, cudaStream_t s);
+
+}  // namespace kvq

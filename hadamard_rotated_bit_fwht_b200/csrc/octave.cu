@@ -1,0 +1,509 @@
+// octave.cu -- the Octave KV-cache variant (vLLM API page
+// "vllm.v1.attention.ops.rocm_octave"): quantize into per-(token, head) byte
+// slots, and decode attention over the paged slot cache.
+//
+// Quantize (reference_quantize): one warp per (token, kv head); lane l holds
+// dims l, l+32, l+64, l+96 of the 128-dim head.
+//   K: x * signs, FWHT over each 64-dim block (stages h = 1..16 across lanes
+//      with xor-shuffles, h = 32 in registers, then x 1/8), then per block
+//      _quantize_lut with 4-bit codes for RoPE blocks and 3-bit codes for NoPE
+//      blocks.
+//   V: x * signs, FWHT-128 over the head (h = 32, 64 in registers), x
+//      fp32(1/sqrt(128)), _quantize_lut with v_bits codes.
+//   _quantize_lut: ss = sum x^2 and dot = sum x * LUT[c] in the fixed pairwise
+//      order (v[i] + v[i + n/2], halving n: in-register levels first, then
+//      xor-shuffles 16, 8, 4, 2, 1, which add exactly the same pairs);
+//      rms = max(sqrt(ss / n), 1e-12); y = x / rms * LUT_MULT; code = number
+//      of LUT midpoints below y (ties go to the lower code);
+//      scale = (dot > 0 ? ss / max(dot, 1e-30) : 0) * LUT_ONE, LUT_ONE = 64,
+//      stored as fp16.
+//   The slot is assembled in shared memory (bit packing of the page's module
+//   text / _pack) and written with one 128-byte warp store.
+// Decode (reference_attention, computed in the rotated space): one CTA per
+//   (split, q-head group, query token); the query is rotated like K (signs +
+//   64-dim blocks), each warp streams slots (one 32-bit word per lane,
+//   shuffles to fetch its nibbles), dequantizes LUT[c] * s / 64, keeps an
+//   online softmax, and the combine kernel merges the splits and rotates the
+//   output back (FWHT-128 x fp32(1/sqrt(128)), then signs).
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kHead = 128;
+constexpr int kORec = 132;  // m, l, pad, pad, o[128]
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLutOne = 64.f;
+
+__device__ __forceinline__ float load_in(const void *p, int bf16, int64_t idx) {
+  return bf16 ? __uint_as_float((uint32_t)static_cast<const uint16_t *>(p)[idx] << 16)
+              : static_cast<const float *>(p)[idx];
+}
+
+__device__ __forceinline__ float sign_of(const OctaveParams &P, int d) {
+  return ((P.sign_words[d >> 5] >> (d & 31)) & 1u) ? -1.f : 1.f;
+}
+
+// one cross-lane butterfly stage on lane-index bit h
+__device__ __forceinline__ float xstage(float v, int lane, int h) {
+  const float o = __shfl_xor_sync(kFull, v, h);
+  return (lane & h) ? __fsub_rn(o, v) : __fadd_rn(v, o);
+}
+
+// sum over the 32 lanes of one value per lane, pairs (i, i + 16), (i, i + 8), ...
+__device__ __forceinline__ float xsum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(kFull, v, off));
+  return v;
+}
+
+struct LutSmem {
+  float lut[2][16];  // [0]: 3-bit (8 entries), [1]: 4-bit
+  float mid[2][15];
+};
+
+// _quantize_lut over n = 64 (two values per lane: dims l, l + 32 of the block)
+// or n = 128 (four values per lane); codes out per value, returns the scale.
+template <int NV>
+__device__ __forceinline__ float quantize_lut(const float (&x)[NV], int bits, float mult,
+                                              const LutSmem &L, int (&code)[NV]) {
+  const int tb = bits == 4 ? 1 : 0;
+  const int nmid = (1 << bits) - 1;
+  float sq[NV];
+#pragma unroll
+  for (int k = 0; k < NV; k++) sq[k] = __fmul_rn(x[k], x[k]);
+  // in-register levels: NV = 4 holds (l, l+32, l+64, l+96): first (l, l+64),
+  // (l+32, l+96) [n = 128 -> 64], then their sum [64 -> 32]; NV = 2: (l, l+32).
+  float ss;
+  if (NV == 4) ss = __fadd_rn(__fadd_rn(sq[0], sq[2]), __fadd_rn(sq[1], sq[3]));
+  else ss = __fadd_rn(sq[0], sq[1]);
+  ss = xsum(ss);
+  const float n = (float)(NV * 32);
+  float rms = __fsqrt_rn(__fdiv_rn(ss, n));
+  rms = rms < 1e-12f ? 1e-12f : rms;
+  float pr[NV];
+#pragma unroll
+  for (int k = 0; k < NV; k++) {
+    const float y = __fmul_rn(__fdiv_rn(x[k], rms), mult);
+    int c = 0;
+    for (int i = 0; i < nmid; i++) c += (L.mid[tb][i] < y) ? 1 : 0;
+    code[k] = c;
+    pr[k] = __fmul_rn(x[k], L.lut[tb][c]);
+  }
+  float dot;
+  if (NV == 4) dot = __fadd_rn(__fadd_rn(pr[0], pr[2]), __fadd_rn(pr[1], pr[3]));
+  else dot = __fadd_rn(pr[0], pr[1]);
+  dot = xsum(dot);
+  const float q = __fdiv_rn(ss, dot > 1e-30f ? dot : 1e-30f);
+  return __fmul_rn(dot > 0.f ? q : 0.f, kLutOne);
+}
+
+// Byte p of the packed codes of `n` dims starting at codes[base] (layout of
+// the page's module text).
+__device__ __forceinline__ uint32_t pack_byte(const uint8_t *codes, int n, int bits, int p) {
+  if (bits == 4) {
+    const int w = p >> 2, j = p & 3;
+    return (uint32_t)(codes[8 * w + j] & 15) | ((uint32_t)(codes[8 * w + 4 + j] & 15) << 4);
+  }
+  uint32_t byte = 0;
+  if (p < n / 4) {  // 2-bit plane
+    const int w = p >> 2, j = p & 3;
+#pragma unroll
+    for (int i = 0; i < 4; i++) byte |= (uint32_t)(codes[16 * w + 4 * i + j] & 3) << (2 * i);
+  } else {          // 1-bit plane
+    const int q = p - n / 4, w = q >> 2, j = q & 3;
+#pragma unroll
+    for (int i = 0; i < 8; i++) byte |= (uint32_t)((codes[32 * w + 4 * i + j] >> 2) & 1) << i;
+  }
+  return byte;
+}
+
+__global__ void __launch_bounds__(kThreads)
+    octave_quantize_kernel(OctaveParams P, const void *__restrict__ key,
+                           const void *__restrict__ value, int bf16, int num_tokens,
+                           int n_kv_heads, const int64_t *__restrict__ slot_mapping,
+                           uint8_t *__restrict__ cache, int block_size, int64_t num_blocks) {
+  __shared__ LutSmem L;
+  __shared__ uint8_t kcodes[kWarps][kHead], vcodes[kWarps][kHead];
+  __shared__ __align__(16) uint8_t slot[kWarps][256];
+  for (int i = threadIdx.x; i < 16; i += blockDim.x) {
+    L.lut[0][i] = i < 8 ? (float)P.lut3[i] : 0.f;
+    L.lut[1][i] = (float)P.lut4[i];
+    if (i < 7) L.mid[0][i] = ((float)P.lut3[i + 1] + (float)P.lut3[i]) / 2.0f;
+    if (i < 15) L.mid[1][i] = ((float)P.lut4[i + 1] + (float)P.lut4[i]) / 2.0f;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t items = (int64_t)num_tokens * n_kv_heads;
+  const float vscale = 0.08838834764831845f;  // fp32(1 / sqrt(128))
+  for (int64_t it = (int64_t)blockIdx.x * kWarps + warp; it < items;
+       it += (int64_t)gridDim.x * kWarps) {
+    const int tok = (int)(it / n_kv_heads), h = (int)(it % n_kv_heads);
+    const int64_t base = it * kHead;
+    // ---- K
+    float x[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const int d = lane + 32 * k;
+      x[k] = __fmul_rn(load_in(key, bf16, base + d), sign_of(P, d));
+    }
+#pragma unroll
+    for (int hh = 1; hh < 32; hh <<= 1)
+#pragma unroll
+      for (int k = 0; k < 4; k++) x[k] = xstage(x[k], lane, hh);
+    {  // h = 32 inside each 64-block: (l, l+32), (l+64, l+96)
+      float a = x[0], b = x[1];
+      x[0] = __fadd_rn(a, b);
+      x[1] = __fsub_rn(a, b);
+      a = x[2];
+      b = x[3];
+      x[2] = __fadd_rn(a, b);
+      x[3] = __fsub_rn(a, b);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; k++) x[k] = __fmul_rn(x[k], 0.125f);
+    float ks[2];
+#pragma unroll
+    for (int kb = 0; kb < 2; kb++) {
+      const int bits = (kb * 64 < P.rope_dim) ? 4 : 3;
+      float xb[2] = {x[2 * kb], x[2 * kb + 1]};
+      int cb[2];
+      ks[kb] = quantize_lut<2>(xb, bits, bits == 4 ? P.mult4 : P.mult3, L, cb);
+      kcodes[warp][64 * kb + lane] = (uint8_t)cb[0];
+      kcodes[warp][64 * kb + lane + 32] = (uint8_t)cb[1];
+    }
+    // ---- V
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const int d = lane + 32 * k;
+      x[k] = __fmul_rn(load_in(value, bf16, base + d), sign_of(P, d));
+    }
+#pragma unroll
+    for (int hh = 1; hh < 32; hh <<= 1)
+#pragma unroll
+      for (int k = 0; k < 4; k++) x[k] = xstage(x[k], lane, hh);
+    {
+      float a = x[0], b = x[1];  // h = 32
+      x[0] = __fadd_rn(a, b);
+      x[1] = __fsub_rn(a, b);
+      a = x[2];
+      b = x[3];
+      x[2] = __fadd_rn(a, b);
+      x[3] = __fsub_rn(a, b);
+      a = x[0];                  // h = 64
+      b = x[2];
+      x[0] = __fadd_rn(a, b);
+      x[2] = __fsub_rn(a, b);
+      a = x[1];
+      b = x[3];
+      x[1] = __fadd_rn(a, b);
+      x[3] = __fsub_rn(a, b);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; k++) x[k] = __fmul_rn(x[k], vscale);
+    int cv[4];
+    const float vs = quantize_lut<4>(x, P.v_bits, P.v_bits == 4 ? P.mult4 : P.mult3, L, cv);
+#pragma unroll
+    for (int k = 0; k < 4; k++) vcodes[warp][lane + 32 * k] = (uint8_t)cv[k];
+    __syncwarp();
+    // ---- slot bytes
+    uint8_t *sl = slot[warp];
+    for (int p = lane; p < P.slot_bytes; p += 32) {
+      uint32_t byte = 0;
+      if (p < P.off_k_nope) byte = pack_byte(kcodes[warp], P.rope_dim, 4, p);
+      else if (p < P.off_v) byte = pack_byte(kcodes[warp] + P.rope_dim, kHead - P.rope_dim, 3, p - P.off_k_nope);
+      else if (p < P.off_scales) byte = pack_byte(vcodes[warp], kHead, P.v_bits, p - P.off_v);
+      else if (p < P.off_scales + 6) {
+        const int si = (p - P.off_scales) >> 1;
+        const float sv = si == 0 ? ks[0] : (si == 1 ? ks[1] : vs);
+        const uint32_t hb = __half_as_ushort(__float2half_rn(sv));
+        byte = (p - P.off_scales) & 1 ? (hb >> 8) : (hb & 0xFF);
+      }
+      sl[p] = (uint8_t)byte;
+    }
+    __syncwarp();
+    const int64_t sm = __ldg(slot_mapping + tok);
+    if (sm >= 0) {
+      const int64_t blk = sm / block_size, off = sm % block_size;
+      if (blk < num_blocks) {
+        uint32_t *dst = reinterpret_cast<uint32_t *>(
+            cache + ((blk * n_kv_heads + h) * block_size + off) * P.slot_bytes);
+        for (int w = lane; w < P.slot_bytes / 4; w += 32) dst[w] = reinterpret_cast<const uint32_t *>(sl)[w];
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// ------------------------------------------------------------------ decode
+__device__ __forceinline__ uint32_t slot_byte(uint32_t myword, int p) {
+  const uint32_t w = __shfl_sync(kFull, myword, p >> 2);
+  return (w >> (8 * (p & 3))) & 0xFFu;
+}
+
+template <int GC, bool BF16>
+__global__ void __launch_bounds__(kThreads)
+    octave_decode_split_kernel(OctaveParams P, const void *__restrict__ query, int n_q_heads,
+                               int group, const uint8_t *__restrict__ cache, int n_kv_heads,
+                               int block_size, int64_t num_blocks,
+                               const int32_t *__restrict__ block_table, int num_reqs,
+                               int max_blocks, const int32_t *__restrict__ q_to_req,
+                               const int32_t *__restrict__ q_to_klen, int max_klen,
+                               float scale_log2, int split_tokens, int splits,
+                               float *__restrict__ ws) {
+  __shared__ float qs[GC][kHead];
+  __shared__ float lut[2][16];
+  __shared__ float red_m[kWarps][GC], red_l[kWarps][GC];
+  __shared__ float red_o[kWarps][GC][kHead];
+  const int s = blockIdx.x, hg = blockIdx.y, qi = blockIdx.z;
+  const int h0 = hg * GC, kvh = h0 / group;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < 16; i += blockDim.x) {
+    lut[0][i] = i < 8 ? (float)P.lut3[i] : 0.f;
+    lut[1][i] = (float)P.lut4[i];
+  }
+  const int req = __ldg(q_to_req + qi);
+  int klen = min(max(__ldg(q_to_klen + qi), 0), min(max_klen, max_blocks * block_size));
+  if (req < 0 || req >= num_reqs) klen = 0;
+  const int t0 = s * split_tokens, t1 = min(klen, t0 + split_tokens);
+
+  // query: signs, FWHT over 64-dim blocks, x 1/8, x scale*log2(e)
+  for (int p = threadIdx.x; p < GC * kHead; p += blockDim.x) {
+    const int hh = p / kHead, d = p % kHead;
+    qs[hh][d] = load_in(query, BF16, ((int64_t)qi * n_q_heads + h0 + hh) * kHead + d) * sign_of(P, d);
+  }
+  for (int h = 1; h < 64; h <<= 1) {
+    __syncthreads();
+    for (int p = threadIdx.x; p < GC * 64; p += blockDim.x) {
+      const int vv = p / 64, pi = p % 64;  // 2 blocks x 32 pairs per head
+      const int blk = pi / 32, pj = pi % 32;
+      const int i0 = blk * 64 + (pj / h) * 2 * h + (pj % h);
+      const float a = qs[vv][i0], b = qs[vv][i0 + h];
+      qs[vv][i0] = a + b;
+      qs[vv][i0 + h] = a - b;
+    }
+  }
+  __syncthreads();
+  float qr[GC][4];
+#pragma unroll
+  for (int hh = 0; hh < GC; hh++)
+#pragma unroll
+    for (int k = 0; k < 4; k++) qr[hh][k] = qs[hh][lane + 32 * k] * (0.125f * scale_log2);
+
+  float m[GC], l[GC], o[GC][4];
+#pragma unroll
+  for (int hh = 0; hh < GC; hh++) {
+    m[hh] = -INFINITY;
+    l[hh] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; k++) o[hh][k] = 0.f;
+  }
+  const int rope = P.rope_dim;
+  for (int t = t0 + warp; t < t1; t += kWarps) {
+    const int blk = __ldg(block_table + (int64_t)req * max_blocks + t / block_size);
+    if (blk < 0 || blk >= num_blocks) continue;
+    const uint8_t *sp = cache + (((int64_t)blk * n_kv_heads + kvh) * block_size + (t % block_size)) * P.slot_bytes;
+    const uint32_t myword = lane < P.slot_bytes / 4 ? __ldg(reinterpret_cast<const uint32_t *>(sp) + lane) : 0u;
+    // scales
+    const uint32_t s01 = slot_byte(myword, P.off_scales) | (slot_byte(myword, P.off_scales + 1) << 8);
+    const uint32_t s23 = slot_byte(myword, P.off_scales + 2) | (slot_byte(myword, P.off_scales + 3) << 8);
+    const uint32_t s45 = slot_byte(myword, P.off_scales + 4) | (slot_byte(myword, P.off_scales + 5) << 8);
+    const float sk0 = __half2float(__ushort_as_half((uint16_t)s01)) / kLutOne;
+    const float sk1 = __half2float(__ushort_as_half((uint16_t)s23)) / kLutOne;
+    const float sv = __half2float(__ushort_as_half((uint16_t)s45)) / kLutOne;
+    float kd[4], vd[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const int d = lane + 32 * k;
+      int code;
+      if (d < rope) {  // 4-bit rope dims
+        const uint32_t byte = slot_byte(myword, 4 * (d >> 3) + (d & 3));
+        code = (byte >> (4 * ((d >> 2) & 1))) & 15;
+        kd[k] = lut[1][code] * (d < 64 ? sk0 : sk1);
+      } else {         // 3-bit nope dims
+        const int n = d - rope;
+        const uint32_t lo = slot_byte(myword, P.off_k_nope + 4 * (n >> 4) + (n & 3));
+        const uint32_t hi = slot_byte(myword, P.off_k_nope + (kHead - rope) / 4 + 4 * (n >> 5) + (n & 3));
+        code = ((lo >> (2 * ((n >> 2) & 3))) & 3) + 4 * ((hi >> ((n >> 2) & 7)) & 1);
+        kd[k] = lut[0][code] * (d < 64 ? sk0 : sk1);
+      }
+      if (P.v_bits == 4) {
+        const uint32_t byte = slot_byte(myword, P.off_v + 4 * (d >> 3) + (d & 3));
+        vd[k] = lut[1][(byte >> (4 * ((d >> 2) & 1))) & 15] * sv;
+      } else {
+        const uint32_t lo = slot_byte(myword, P.off_v + 4 * (d >> 4) + (d & 3));
+        const uint32_t hi = slot_byte(myword, P.off_v + kHead / 4 + 4 * (d >> 5) + (d & 3));
+        vd[k] = lut[0][((lo >> (2 * ((d >> 2) & 3))) & 3) + 4 * ((hi >> ((d >> 2) & 7)) & 1)] * sv;
+      }
+    }
+    float sc[GC];
+#pragma unroll
+    for (int hh = 0; hh < GC; hh++) {
+      float a = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; k++) a = fmaf(qr[hh][k], kd[k], a);
+      sc[hh] = a;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+      for (int hh = 0; hh < GC; hh++) sc[hh] += __shfl_xor_sync(kFull, sc[hh], off);
+#pragma unroll
+    for (int hh = 0; hh < GC; hh++) {
+      const float mn = fmaxf(m[hh], sc[hh]);
+      const float alpha = exp2f(m[hh] - mn);
+      const float p = exp2f(sc[hh] - mn);
+      m[hh] = mn;
+      l[hh] = l[hh] * alpha + p;
+#pragma unroll
+      for (int k = 0; k < 4; k++) o[hh][k] = fmaf(p, vd[k], o[hh][k] * alpha);
+    }
+  }
+  if (lane == 0)
+#pragma unroll
+    for (int hh = 0; hh < GC; hh++) {
+      red_m[warp][hh] = m[hh];
+      red_l[warp][hh] = l[hh];
+    }
+#pragma unroll
+  for (int hh = 0; hh < GC; hh++)
+#pragma unroll
+    for (int k = 0; k < 4; k++) red_o[warp][hh][lane + 32 * k] = o[hh][k];
+  __syncthreads();
+  for (int p = threadIdx.x; p < GC * kHead; p += blockDim.x) {
+    const int hh = p / kHead, j = p % kHead;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++) M = fmaxf(M, red_m[w][hh]);
+    float Ls = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; w++) {
+        const float f = exp2f(red_m[w][hh] - M);
+        Ls += red_l[w][hh] * f;
+        O += red_o[w][hh][j] * f;
+      }
+    }
+    float *rec = ws + (((int64_t)qi * n_q_heads + h0 + hh) * splits + s) * kORec;
+    rec[4 + j] = O;
+    if (j == 0) {
+      rec[0] = M;
+      rec[1] = Ls;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kHead)
+    octave_combine_kernel(OctaveParams P, const float *__restrict__ ws,
+                          const int32_t *__restrict__ q_to_req,
+                          const int32_t *__restrict__ q_to_klen, int num_reqs, int n_q_heads,
+                          int splits, int max_klen, int cap, float *__restrict__ out) {
+  __shared__ float ob[kHead];
+  const int qh = blockIdx.x, j = threadIdx.x;
+  const int qi = qh / n_q_heads;
+  const int req = __ldg(q_to_req + qi);
+  int klen = min(max(__ldg(q_to_klen + qi), 0), min(max_klen, cap));
+  if (req < 0 || req >= num_reqs) klen = 0;
+  const float *rec = ws + (int64_t)qh * splits * kORec;
+  float M = -INFINITY;
+  for (int s = 0; s < splits && klen > 0; s++) M = fmaxf(M, rec[s * kORec]);
+  float L = 0.f, O = 0.f;
+  if (klen > 0 && M != -INFINITY) {
+    for (int s = 0; s < splits; s++) {
+      const float ms = rec[s * kORec];
+      if (ms == -INFINITY) continue;
+      const float f = exp2f(ms - M);
+      L += rec[s * kORec + 1] * f;
+      O += rec[s * kORec + 4 + j] * f;
+    }
+  }
+  ob[j] = L > 0.f ? O / L : 0.f;
+  for (int h = 1; h < kHead; h <<= 1) {
+    __syncthreads();
+    if (j < 64) {
+      const int i0 = (j / h) * 2 * h + (j % h);
+      const float a = ob[i0], b = ob[i0 + h];
+      ob[i0] = a + b;
+      ob[i0 + h] = a - b;
+    }
+  }
+  __syncthreads();
+  out[(int64_t)qh * kHead + j] = ob[j] * 0.08838834764831845f * sign_of(P, j);
+}
+
+}  // namespace
+
+cudaError_t launch_octave_quantize(const OctaveParams &p, const void *key, const void *value,
+                                   int bf16, int num_tokens, int n_kv_heads,
+                                   const int64_t *slot_mapping, uint8_t *cache,
+                                   int block_size, int64_t num_blocks, cudaStream_t s) {
+  const int64_t items = (int64_t)num_tokens * n_kv_heads;
+  if (items == 0) return cudaSuccess;
+  int64_t blocks = (items + kWarps - 1) / kWarps;
+  const int grid = (int)(blocks < kNumSMs * 16 ? blocks : kNumSMs * 16);
+  octave_quantize_kernel<<<grid, kThreads, 0, s>>>(p, key, value, bf16, num_tokens, n_kv_heads,
+                                                  slot_mapping, cache, block_size, num_blocks);
+  return cudaGetLastError();
+}
+
+DecodePlan plan_octave_decode(int num_q, int n_kv_heads, int max_klen) {
+  DecodePlan p;
+  const int units = max(num_q * n_kv_heads, 1);
+  const int target = kNumSMs * 4;
+  int splits = max(1, (target + units - 1) / units);
+  int per = (max(max_klen, 1) + splits - 1) / splits;
+  per = ((per + 63) / 64) * 64;
+  if (per < 256) per = 256;
+  p.split_tokens = per;
+  p.splits = max(1, (max(max_klen, 1) + per - 1) / per);
+  return p;
+}
+
+size_t octave_workspace_bytes(int num_q, int n_q_heads, int head_size, const DecodePlan &p) {
+  (void)head_size;
+  return (size_t)num_q * n_q_heads * p.splits * kORec * sizeof(float);
+}
+
+cudaError_t launch_octave_decode(const OctaveParams &P, const void *query, int bf16, int num_q,
+                                 int n_q_heads, const uint8_t *cache, int n_kv_heads,
+                                 int block_size, int64_t num_blocks, const int32_t *block_table,
+                                 int num_reqs, int max_blocks, const int32_t *q_to_req,
+                                 const int32_t *q_to_klen, int max_klen, float scale,
+                                 float *out, float *ws, const DecodePlan &plan, cudaStream_t s) {
+  if (num_q == 0) return cudaSuccess;
+  const int group = n_q_heads / n_kv_heads;
+  const int gc = group < 8 ? group : 8;
+  dim3 grid(plan.splits, n_q_heads / gc, num_q);
+  const float sl2 = scale * kLog2e;
+#define KVQ_LAUNCH(G)                                                                         \
+  do {                                                                                        \
+    if (bf16)                                                                                 \
+      octave_decode_split_kernel<G, true><<<grid, kThreads, 0, s>>>(                         \
+          P, query, n_q_heads, group, cache, n_kv_heads, block_size, num_blocks, block_table, \
+          num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2, plan.split_tokens,        \
+          plan.splits, ws);                                                                   \
+    else                                                                                      \
+      octave_decode_split_kernel<G, false><<<grid, kThreads, 0, s>>>(                        \
+          P, query, n_q_heads, group, cache, n_kv_heads, block_size, num_blocks, block_table, \
+          num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2, plan.split_tokens,        \
+          plan.splits, ws);                                                                   \
+  } while (0)
+  switch (gc) {
+    case 1: KVQ_LAUNCH(1); break;
+    case 2: KVQ_LAUNCH(2); break;
+    case 4: KVQ_LAUNCH(4); break;
+    default: KVQ_LAUNCH(8); break;
+  }
+#undef KVQ_LAUNCH
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  octave_combine_kernel<<<num_q * n_q_heads, kHead, 0, s>>>(P, ws, q_to_req, q_to_klen, num_reqs,
+                                                           n_q_heads, plan.splits, max_klen,
+                                                           max_blocks * block_size, out);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

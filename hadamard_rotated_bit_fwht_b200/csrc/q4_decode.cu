@@ -1,0 +1,97 @@
+// q4_decode.cu -- single-token decode attention over the Q4_0 + FWHT-256 cache.
+//
+// Method: Strata PR #21 "Q4_0 KV cache + FWHT-256": What (score invariance
+// <Hq, Hk> = <q, k>, so the query is rotated like K), How 2 (nibbles are
+// dequantized in registers during the flash-attention score accumulation) and
+// the merge note (the per-token path rotates Q and the output).
+//
+// Split-K flash decoding: the split kernel (tensor cores, q4_decode_mma.cu)
+// writes one partial record (m, l, o[256]) per (sequence, q head, split); the
+// combine kernel here merges the splits with a log-sum-exp and applies the
+// back-rotation H o (FWHT-256) -- once per query head, after the combine.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kRec = 260;  // floats per partial record: m, l, pad, pad, o[256]
+
+// In-place FWHT-256 of n_vec vectors in shared memory (all threads of the CTA
+// take part; fp32, stage order h = 1, 2, ..., 128; no scaling).
+__device__ void smem_fwht256(float *x, int n_vec) {
+  for (int h = 1; h < kDim; h <<= 1) {
+    __syncthreads();
+    for (int p = threadIdx.x; p < n_vec * 128; p += blockDim.x) {
+      const int vv = p >> 7, pi = p & 127;
+      const int i0 = ((pi / h) * 2 * h) + (pi % h);
+      float *y = x + vv * kDim;
+      const float a = y[i0], b = y[i0 + h];
+      y[i0] = a + b;
+      y[i0 + h] = a - b;
+    }
+  }
+  __syncthreads();
+}
+
+// Log-sum-exp combine of the splits and back-rotation; one CTA of 256 threads
+// per (sequence, q head).
+__global__ void __launch_bounds__(256)
+    q4_decode_combine_kernel(const float *__restrict__ ws, const int32_t *__restrict__ seq_lens,
+                             int n_q_heads, int splits, int max_seq_len, int cap,
+                             float *__restrict__ out) {
+  __shared__ float ob[kDim];
+  const int bh = blockIdx.x, j = threadIdx.x;
+  const int b = bh / n_q_heads;
+  const int len = min(max(__ldg(seq_lens + b), 0), min(max_seq_len, cap));
+  const float *rec = ws + (int64_t)bh * splits * kRec;
+  float M = -INFINITY;
+  for (int s = 0; s < splits && len > 0; s++) M = fmaxf(M, rec[s * kRec]);
+  float L = 0.f, O = 0.f;
+  if (len > 0 && M != -INFINITY) {
+    for (int s = 0; s < splits; s++) {
+      const float ms = rec[s * kRec];
+      if (ms == -INFINITY) continue;
+      const float f = exp2f(ms - M);
+      L += rec[s * kRec + 1] * f;
+      O += rec[s * kRec + 4 + j] * f;
+    }
+  }
+  ob[j] = L > 0.f ? O / L : 0.f;
+  smem_fwht256(ob, 1);
+  out[(int64_t)bh * kDim + j] = ob[j] * 0.0625f;
+}
+
+}  // namespace
+
+DecodePlan plan_decode(int batch, int n_kv_heads, int max_seq_len) {
+  DecodePlan p;
+  const int units = max(batch * n_kv_heads, 1);
+  const int target = kNumSMs * 2;  // resident CTAs of the tensor-core split kernel
+  int splits = max(1, (target + units - 1) / units);
+  int per = (max(max_seq_len, 1) + splits - 1) / splits;
+  per = ((per + 63) / 64) * 64;
+  if (per < 256) per = 256;
+  p.split_tokens = per;
+  p.splits = max(1, (max(max_seq_len, 1) + per - 1) / per);
+  return p;
+}
+
+size_t decode_workspace_bytes(int batch, int n_q_heads, const DecodePlan &p) {
+  return (size_t)batch * n_q_heads * p.splits * kRec * sizeof(float);
+}
+
+cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int batch,
+                             int n_q_heads, const int32_t *seq_lens, int max_seq_len,
+                             float scale, float *out, float *ws, const DecodePlan &p,
+                             cudaStream_t s) {
+  if (batch == 0) return cudaSuccess;
+  cudaError_t e = launch_q4_decode_mma(c, q, bf16, batch, n_q_heads, seq_lens, max_seq_len,
+                                       scale, ws, p, s);
+  if (e != cudaSuccess) return e;
+  const int cap = c.block_table ? c.max_pages_per_seq * c.page_size : c.max_tokens;
+  q4_decode_combine_kernel<<<batch * n_q_heads, 256, 0, s>>>(ws, seq_lens, n_q_heads, p.splits,
+                                                             max_seq_len, cap, out);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

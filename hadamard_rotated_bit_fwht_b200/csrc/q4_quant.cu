@@ -1,0 +1,324 @@
+// q4_quant.cu -- FWHT-256 rotation and Q4_0 quantize-on-append for B200.
+//
+// Method: Strata PR #21 "Q4_0 KV cache + FWHT-256", How 1 (orthonormal
+// Walsh-Hadamard transform of each D = 256 head vector, scale 1/16) and How 2
+// (Q4_0 blocks: 32 values, one fp16 scale, 16 bytes of nibbles), with the
+// maintainer's deterministic tie-break a > amax || (a == amax && v > mval).
+// Stage order and end scaling: vLLM rocm_octave page, fwht_blocks.
+//
+// Work decomposition (one warp = 4 vectors, 8 lanes per vector, 32 values
+// per lane; no shared-memory barrier, only __syncwarp):
+//   L0 (after the load): lane i holds x[u + 8i + 64j] in r[u + 8j] -- each
+//       lane reads four 16-byte chunks, so a warp instruction reads 512
+//       contiguous bytes of bf16 input.  Stages h = 1, 2, 4 run in registers.
+//   One register transpose through 1 KB of shared memory per vector
+//   (128-bit stores and loads, XOR swizzle, no bank conflicts) gives
+//   L1: lane i holds x[i + 8u + 64j] in r[u + 8j]; stages h = 8 ... 128 run in
+//       registers.  The two halves of each packed fp32x2 operation are
+//       r[k] and r[k + 16], so every stage but h = 128 uses add/sub.f32x2.
+//   Quantization in L1: a 32-value block is (8 lanes) x (4 registers); its
+//   max-abs key is reduced with three xor-shuffles; lane i computes the scale
+//   of block i and broadcasts 1/d; codes are formed with the fp32 magic
+//   number 2^23 (round-toward-zero add) instead of a float-to-int conversion;
+//   the 16 nibble bytes of block i are regrouped through shared memory so
+//   each lane stores one 16-byte chunk.
+// Every fp32 operation is the IEEE round-to-nearest operation of the stated
+// sequence (explicit _rn intrinsics, no contraction), so codes and scales are
+// bit-identical to that sequence.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kVecPerWarp = 4;
+constexpr int kVecPerCta = kWarps * kVecPerWarp;
+constexpr unsigned kFull = 0xffffffffu;
+
+// ------------------------------------------------------------------ load (L0)
+template <bool BF16>
+__device__ __forceinline__ void load_l0(const void *vec, int i, bool valid, float r[32]) {
+  if (!valid) {
+#pragma unroll
+    for (int k = 0; k < 32; k++) r[k] = 0.f;
+    return;
+  }
+  if (BF16) {
+    const uint16_t *p = static_cast<const uint16_t *>(vec);
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      uint4 w = ldg_stream_u4(p + 8 * (i + 8 * j));
+      r[8 * j + 0] = bf16lo(w.x);
+      r[8 * j + 1] = bf16hi(w.x);
+      r[8 * j + 2] = bf16lo(w.y);
+      r[8 * j + 3] = bf16hi(w.y);
+      r[8 * j + 4] = bf16lo(w.z);
+      r[8 * j + 5] = bf16hi(w.z);
+      r[8 * j + 6] = bf16lo(w.w);
+      r[8 * j + 7] = bf16hi(w.w);
+    }
+  } else {
+    const float *p = static_cast<const float *>(vec);
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      uint4 a = ldg_stream_u4(p + 8 * (i + 8 * j));
+      uint4 b = ldg_stream_u4(p + 8 * (i + 8 * j) + 4);
+      r[8 * j + 0] = __uint_as_float(a.x);
+      r[8 * j + 1] = __uint_as_float(a.y);
+      r[8 * j + 2] = __uint_as_float(a.z);
+      r[8 * j + 3] = __uint_as_float(a.w);
+      r[8 * j + 4] = __uint_as_float(b.x);
+      r[8 * j + 5] = __uint_as_float(b.y);
+      r[8 * j + 6] = __uint_as_float(b.z);
+      r[8 * j + 7] = __uint_as_float(b.w);
+    }
+  }
+}
+
+// Butterfly on register-index bit M (M in {1,2,4,8}): pairs (k, k+M) become
+// (a+b, a-b); r[k] and r[k+16] travel together in one fp32x2 operation.
+template <int M>
+__device__ __forceinline__ void bfly_packed(float r[32]) {
+#pragma unroll
+  for (int k = 0; k < 16; k++) {
+    if (k & M) continue;
+    float2 a = make_float2(r[k], r[k + 16]);
+    float2 b = make_float2(r[k + M], r[k + M + 16]);
+    float2 s = add2(a, b), d = sub2(a, b);
+    r[k] = s.x;
+    r[k + 16] = s.y;
+    r[k + M] = d.x;
+    r[k + M + 16] = d.y;
+  }
+}
+
+// Butterfly on register-index bit 16 (the packed pair itself): scalar.
+__device__ __forceinline__ void bfly16(float r[32]) {
+#pragma unroll
+  for (int k = 0; k < 16; k++) {
+    float a = r[k], b = r[k + 16];
+    r[k] = __fadd_rn(a, b);
+    r[k + 16] = __fsub_rn(a, b);
+  }
+}
+
+// L0 -> L1 through shared memory.  Slot of element e (low 6 bits): float4 at
+// index ((e & 7) ^ ((e >> 3) & 7)) + 8 * ((e >> 3) & 7), holding e + 64j for
+// j = 0..3.  Both the stores (L0) and the loads (L1) of 8 lanes of a vector
+// touch 8 distinct bank quads.
+__device__ __forceinline__ void transpose_l0_l1(float r[32], float4 *buf, int i) {
+#pragma unroll
+  for (int u = 0; u < 8; u++)
+    buf[(u ^ i) + 8 * i] = make_float4(r[u], r[u + 8], r[u + 16], r[u + 24]);
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < 8; u++) {
+    float4 w = buf[(i ^ u) + 8 * u];
+    r[u] = w.x;
+    r[u + 8] = w.y;
+    r[u + 16] = w.z;
+    r[u + 24] = w.w;
+  }
+  __syncwarp();
+}
+
+// Full FWHT-256 of the 4 vectors of this warp: load, stages, transpose,
+// stages, end scaling.  Leaves layout L1.
+template <bool BF16>
+__device__ __forceinline__ void fwht256_warp(const void *vec, bool valid, int i, float4 *buf,
+                                             float r[32]) {
+  load_l0<BF16>(vec, i, valid, r);
+  bfly_packed<1>(r);  // h = 1
+  bfly_packed<2>(r);  // h = 2
+  bfly_packed<4>(r);  // h = 4
+  transpose_l0_l1(r, buf, i);
+  bfly_packed<1>(r);  // h = 8
+  bfly_packed<2>(r);  // h = 16
+  bfly_packed<4>(r);  // h = 32
+  bfly_packed<8>(r);  // h = 64
+  bfly16(r);          // h = 128
+  const float2 s = make_float2(0.0625f, 0.0625f);
+#pragma unroll
+  for (int k = 0; k < 16; k++) {
+    float2 v = mul2(make_float2(r[k], r[k + 16]), s);
+    r[k] = v.x;
+    r[k + 16] = v.y;
+  }
+}
+
+// ------------------------------------------------------------------ rotate
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads) rotate_kernel(const void *__restrict__ x,
+                                                          float *__restrict__ y, int64_t n_vec) {
+  __shared__ float4 smem[kWarps][kVecPerWarp][64];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int vg = lane >> 3, i = lane & 7;
+  float4 *buf = smem[warp][vg];
+  const int64_t ngroups = (n_vec + kVecPerCta - 1) / kVecPerCta;
+  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
+    const int64_t v = g * kVecPerCta + warp * kVecPerWarp + vg;
+    const bool valid = v < n_vec;
+    const size_t esz = BF16 ? 2 : 4;
+    const void *src = static_cast<const char *>(x) + (valid ? v : 0) * kDim * esz;
+    float r[32];
+    fwht256_warp<BF16>(src, valid, i, buf, r);
+    if (valid) {
+      float *dst = y + v * kDim;
+#pragma unroll
+      for (int j = 0; j < 4; j++)
+#pragma unroll
+        for (int u = 0; u < 8; u++) dst[i + 8 * u + 64 * j] = r[u + 8 * j];
+    }
+  }
+}
+
+// ------------------------------------------------------------------ quantize
+// Max-abs key of a value: rotl(bits, 1) ^ 1 orders values by |z| first and puts
+// the positive one above the negative one of equal magnitude, so the maximum
+// key over a block is the element the sequential tie-break scan keeps.  The
+// start value (amax = 0, mval = +0) has key 1.
+__device__ __forceinline__ uint32_t amax_key(float z) {
+  uint32_t b = __float_as_uint(z);
+  return __funnelshift_l(b, b, 1) ^ 1u;
+}
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key >> 1) | ((~key & 1u) << 31));
+}
+
+struct QuantOut {
+  uint32_t items[8];  // block B: byte i | byte (i + 8) << 8 of the block's 16 code bytes
+  uint16_t scale;     // fp16 bits of this lane's block (block index = lane i)
+};
+
+// Quantize the 8 blocks of one vector held in layout L1 (this lane: i).
+__device__ __forceinline__ void q4_quantize_l1(const float r[32], int lane, int i, QuantOut &o) {
+  // register of block B, in-block row m: 4 * (B & 1) + m + 8 * (B >> 1)
+  uint32_t key[8];
+#pragma unroll
+  for (int B = 0; B < 8; B++) {
+    uint32_t k = 1u;
+#pragma unroll
+    for (int m = 0; m < 4; m++) k = max(k, amax_key(r[4 * (B & 1) + m + 8 * (B >> 1)]));
+    key[B] = k;
+  }
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1)
+#pragma unroll
+    for (int B = 0; B < 8; B++) key[B] = max(key[B], __shfl_xor_sync(kFull, key[B], off));
+  uint32_t kmine = key[0];
+#pragma unroll
+  for (int B = 1; B < 8; B++) kmine = (i == B) ? key[B] : kmine;
+  const float mval = key_value(kmine);
+  const float d = __fmul_rn(mval, -0.125f);  // == mval / -8 (exact power-of-two scaling)
+  const float id = (d != 0.f) ? __frcp_rn(d) : 0.f;
+  o.scale = __half_as_ushort(__float2half_rn(d));
+  float idb[8];
+#pragma unroll
+  for (int B = 0; B < 8; B++) idb[B] = __shfl_sync(kFull, id, (lane & ~7) | B);
+
+  uint32_t mq[32];
+  const float2 half8 = make_float2(8.5f, 8.5f), magic = make_float2(8388608.f, 8388608.f);
+#pragma unroll
+  for (int k = 0; k < 16; k++) {
+    // register k belongs to block B = ((k >> 2) & 1) + 2 * (k >> 3); k + 16 to B + 4
+    const int B = ((k >> 2) & 1) + 2 * (k >> 3);
+    float2 t = mul2(make_float2(r[k], r[k + 16]), make_float2(idb[B], idb[B + 4]));
+    t = add2(t, half8);
+    float2 f = add2_rz(t, magic);  // 2^23 + floor(t), t >= 0
+    mq[k] = min(__float_as_uint(f.x), 0x4B00000Fu);
+    mq[k + 16] = min(__float_as_uint(f.y), 0x4B00000Fu);
+  }
+#pragma unroll
+  for (int B = 0; B < 8; B++) {
+    const int r0 = 4 * (B & 1) + 8 * (B >> 1);
+    // element-in-block i + 8m: byte i = m0 | m2 << 4, byte i + 8 = m1 | m3 << 4
+    uint32_t lo = (mq[r0 + 0] & 15u) | ((mq[r0 + 2] & 15u) << 4);
+    uint32_t hi = (mq[r0 + 1] & 15u) | ((mq[r0 + 3] & 15u) << 4);
+    o.items[B] = lo | (hi << 8);
+  }
+}
+
+// Regroup the per-lane items so lane i holds the 16 code bytes of block i.
+__device__ __forceinline__ uint4 gather_block_bytes(const QuantOut &o, uint8_t *stage, int i) {
+  uint16_t *s16 = reinterpret_cast<uint16_t *>(stage);
+#pragma unroll
+  for (int B = 0; B < 8; B++) s16[B * 8 + i] = (uint16_t)o.items[B];
+  __syncwarp();
+  uint4 w = *reinterpret_cast<const uint4 *>(stage + 16 * i);  // (b0,b8,b1,b9 | b2,b10,b3,b11 | ...)
+  __syncwarp();
+  uint4 out;
+  out.x = __byte_perm(w.x, w.y, 0x6420);
+  out.y = __byte_perm(w.z, w.w, 0x6420);
+  out.z = __byte_perm(w.x, w.y, 0x7531);
+  out.w = __byte_perm(w.z, w.w, 0x7531);
+  return out;
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads)
+    q4_append_kernel(kvq_cache c, const void *__restrict__ k, const void *__restrict__ v,
+                     int batch, int t_new, const int32_t *__restrict__ start_pos) {
+  __shared__ float4 smem[kWarps][kVecPerWarp][64];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int vg = lane >> 3, i = lane & 7;
+  float4 *buf = smem[warp][vg];
+  // code regrouping reuses 128 bytes of this vector's buffer, offset by 16
+  // bytes per vector so the four vectors of a warp use different banks
+  uint8_t *stage = reinterpret_cast<uint8_t *>(buf) + 16 * vg;
+  const int64_t per_tensor = (int64_t)batch * t_new * c.num_kv_heads;
+  const int64_t n_vec = 2 * per_tensor;
+  const int64_t ngroups = (n_vec + kVecPerCta - 1) / kVecPerCta;
+  const size_t esz = BF16 ? 2 : 4;
+  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
+    const int64_t vid = g * kVecPerCta + warp * kVecPerWarp + vg;
+    bool valid = vid < n_vec;
+    const bool is_v = valid && vid >= per_tensor;
+    const int64_t e = valid ? (is_v ? vid - per_tensor : vid) : 0;
+    const void *src = static_cast<const char *>(is_v ? v : k) + e * kDim * esz;
+    float r[32];
+    fwht256_warp<BF16>(src, valid, i, buf, r);
+    QuantOut o;
+    q4_quantize_l1(r, lane, i, o);
+    uint4 bytes = gather_block_bytes(o, stage, i);
+    if (valid) {
+      const int h = (int)(e % c.num_kv_heads);
+      const int64_t bt = e / c.num_kv_heads;
+      const int tok = (int)(bt % t_new), b = (int)(bt / t_new);
+      const int64_t row = q4_row(c, b, h, __ldg(start_pos + b) + tok);
+      if (row >= 0) {
+        uint8_t *codes = (is_v ? c.v_codes : c.k_codes) + row * kRowCodeBytes;
+        uint16_t *scales = (is_v ? c.v_scales : c.k_scales) + row * kRowScales;
+        *reinterpret_cast<uint4 *>(codes + 16 * i) = bytes;
+        scales[i] = o.scale;
+      }
+    }
+  }
+}
+
+int grid_for(int64_t groups) {
+  int64_t cap = (int64_t)kNumSMs * 8;
+  return (int)(groups < cap ? (groups > 0 ? groups : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_rotate(const void *x, int bf16, float *y, int64_t n_vec, cudaStream_t s) {
+  if (n_vec == 0) return cudaSuccess;
+  const int grid = grid_for((n_vec + kVecPerCta - 1) / kVecPerCta);
+  if (bf16) rotate_kernel<true><<<grid, kThreads, 0, s>>>(x, y, n_vec);
+  else rotate_kernel<false><<<grid, kThreads, 0, s>>>(x, y, n_vec);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_q4_append(const kvq_cache &c, const void *k, const void *v, int bf16,
+                             int batch, int t_new, const int32_t *start_pos, cudaStream_t s) {
+  const int64_t n_vec = 2LL * batch * t_new * c.num_kv_heads;
+  if (n_vec == 0) return cudaSuccess;
+  const int grid = grid_for((n_vec + kVecPerCta - 1) / kVecPerCta);
+  if (bf16) q4_append_kernel<true><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos);
+  else q4_append_kernel<false><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

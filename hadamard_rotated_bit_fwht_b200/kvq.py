@@ -1,0 +1,339 @@
+"""Python binding of libkvq (include/kvq.h): argument marshalling only.
+
+Every step of the hot path runs in the CUDA kernels behind the C ABI.  This
+module loads ``libkvq.so`` with ctypes, turns torch CUDA tensors into raw
+pointers and torch's current stream into a ``cudaStream_t``, and raises
+``KVQError`` on any non-OK status.  There is no CPU fallback: if the library
+is missing the import of the first call fails with a message saying so.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkvq.so")
+
+KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA = range(5)
+KVQ_F32, KVQ_BF16 = 0, 1
+
+EXPORTED = (
+    "kvq_status_string", "kvq_version", "kvq_rotate", "kvq_quantize_append",
+    "kvq_decode_attn_workspace", "kvq_decode_attn", "kvq_octave_layout_of",
+    "kvq_octave_codebook", "kvq_octave_quantize", "kvq_octave_decode_attn_workspace",
+    "kvq_octave_decode_attn",
+)
+
+
+class KVQError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn} failed: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class CacheDesc(C.Structure):
+    _fields_ = [
+        ("k_codes", C.c_void_p), ("k_scales", C.c_void_p),
+        ("v_codes", C.c_void_p), ("v_scales", C.c_void_p),
+        ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32),
+        ("max_tokens", C.c_int32), ("batch_capacity", C.c_int32),
+        ("block_table", C.c_void_p), ("page_size", C.c_int32),
+        ("max_pages_per_seq", C.c_int32), ("num_pages", C.c_int32),
+    ]
+
+
+class OctaveFmtDesc(C.Structure):
+    _fields_ = [("head_size", C.c_int32), ("rope_dim", C.c_int32),
+                ("v_bits", C.c_int32), ("compact", C.c_int32)]
+
+
+class OctaveLayoutDesc(C.Structure):
+    _fields_ = [(n, C.c_int32) for n in ("off_k_nope", "off_v", "off_scales", "num_k_scales",
+                                        "num_scales", "slot_bytes", "kernel_code")]
+
+
+_lib = None
+
+
+def lib():
+    """Load libkvq.so (built by hadamard_rotated_bit_fwht_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m hadamard_rotated_bit_fwht_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        L.kvq_status_string.restype = C.c_char_p
+        L.kvq_status_string.argtypes = [C.c_int]
+        L.kvq_version.restype = C.c_int
+        L.kvq_rotate.argtypes = [C.c_void_p, C.c_int, C.c_void_p, C.c_int64, C.c_int32, C.c_void_p]
+        L.kvq_quantize_append.argtypes = [C.POINTER(CacheDesc), C.c_void_p, C.c_void_p, C.c_int,
+                                          C.c_int32, C.c_int32, C.c_void_p, C.c_void_p]
+        L.kvq_decode_attn_workspace.restype = C.c_size_t
+        L.kvq_decode_attn_workspace.argtypes = [C.POINTER(CacheDesc), C.c_int32, C.c_int32,
+                                                C.c_int32]
+        L.kvq_decode_attn.argtypes = [C.POINTER(CacheDesc), C.c_void_p, C.c_int, C.c_int32,
+                                      C.c_int32, C.c_void_p, C.c_int32, C.c_float, C.c_void_p,
+                                      C.c_void_p, C.c_size_t, C.c_void_p]
+        L.kvq_octave_layout_of.argtypes = [C.POINTER(OctaveFmtDesc), C.POINTER(OctaveLayoutDesc)]
+        L.kvq_octave_codebook.argtypes = [C.c_int32, C.c_void_p, C.POINTER(C.c_float)]
+        L.kvq_octave_quantize.argtypes = [C.POINTER(OctaveFmtDesc), C.c_void_p, C.c_void_p,
+                                          C.c_int, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
+                                          C.c_int32, C.c_int64, C.c_void_p, C.c_void_p]
+        L.kvq_octave_decode_attn_workspace.restype = C.c_size_t
+        L.kvq_octave_decode_attn_workspace.argtypes = [C.POINTER(OctaveFmtDesc), C.c_int32,
+                                                       C.c_int32, C.c_int32]
+        L.kvq_octave_decode_attn.argtypes = [
+            C.POINTER(OctaveFmtDesc), C.c_void_p, C.c_int, C.c_int32, C.c_int32, C.c_void_p,
+            C.c_int32, C.c_int32, C.c_int64, C.c_void_p, C.c_int32, C.c_int32, C.c_void_p,
+            C.c_void_p, C.c_int32, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t,
+            C.c_void_p]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().kvq_status_string(status).decode()
+
+
+def _check(fn, status):
+    if status != KVQ_OK:
+        raise KVQError(fn, status)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KVQ_F32
+    if t.dtype == torch.bfloat16:
+        return KVQ_BF16
+    raise TypeError(f"expected float32 or bfloat16, got {t.dtype}")
+
+
+def _cuda_contig(name, t):
+    if not (t.is_cuda and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+# --------------------------------------------------------------------------
+# Q4_0 + FWHT-256
+# --------------------------------------------------------------------------
+class Q4Cache:
+    """Caller-owned structure-of-arrays Q4_0 cache (layout in include/kvq.h)."""
+
+    def __init__(self, n_rows, num_kv_heads, device, *, max_tokens=0, batch_capacity=0,
+                 block_table=None, page_size=0, num_pages=0):
+        dev = torch.device(device)
+        self.num_kv_heads = num_kv_heads
+        self.max_tokens = max_tokens
+        self.batch_capacity = batch_capacity
+        self.block_table = block_table
+        self.page_size = page_size
+        self.num_pages = num_pages
+        self.k_codes = torch.zeros((n_rows, 128), dtype=torch.uint8, device=dev)
+        self.v_codes = torch.zeros((n_rows, 128), dtype=torch.uint8, device=dev)
+        self.k_scales = torch.zeros((n_rows, 8), dtype=torch.int16, device=dev)
+        self.v_scales = torch.zeros((n_rows, 8), dtype=torch.int16, device=dev)
+
+    @classmethod
+    def contiguous(cls, batch, num_kv_heads, max_tokens, device="cuda"):
+        return cls(batch * num_kv_heads * max_tokens, num_kv_heads, device,
+                   max_tokens=max_tokens, batch_capacity=batch)
+
+    @classmethod
+    def paged(cls, num_pages, num_kv_heads, page_size, block_table, device="cuda"):
+        bt = block_table.to(device=device, dtype=torch.int32).contiguous()
+        return cls(num_pages * num_kv_heads * page_size, num_kv_heads, device,
+                   block_table=bt, page_size=page_size, num_pages=num_pages)
+
+    def with_block_table(self, block_table: torch.Tensor) -> "Q4Cache":
+        """The same planes seen through another block table (e.g. one row, to
+        append a single sequence of a paged batch)."""
+        view = Q4Cache.__new__(Q4Cache)
+        view.__dict__.update(self.__dict__)
+        view.block_table = block_table.to(device=self.k_codes.device,
+                                          dtype=torch.int32).contiguous()
+        return view
+
+    @property
+    def capacity(self):
+        if self.block_table is None:
+            return self.max_tokens
+        return self.block_table.shape[1] * self.page_size
+
+    def desc(self) -> CacheDesc:
+        bt = self.block_table
+        return CacheDesc(self.k_codes.data_ptr(), self.k_scales.data_ptr(),
+                         self.v_codes.data_ptr(), self.v_scales.data_ptr(),
+                         self.num_kv_heads, 256, self.max_tokens, self.batch_capacity,
+                         None if bt is None else bt.data_ptr(), self.page_size,
+                         0 if bt is None else bt.shape[1], self.num_pages)
+
+    def nbytes_per_row(self):
+        return 2 * (128 + 16)
+
+
+def rotate(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = H x over the last dim (256), fp32 output."""
+    _cuda_contig("x", x)
+    if x.shape[-1] != 256:
+        raise ValueError("kvq_rotate: last dim must be 256")
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.float32, device=x.device)
+    n = x.numel() // 256
+    _check("kvq_rotate", lib().kvq_rotate(_ptr(x), _dtype_code(x), _ptr(out), n, 256,
+                                          _stream(stream)))
+    return out
+
+
+def quantize_append(cache: Q4Cache, k: torch.Tensor, v: torch.Tensor,
+                    start_pos: torch.Tensor, stream=None) -> None:
+    """Rotate + Q4_0-quantize k, v ([batch, t_new, Hkv, 256]) into the cache."""
+    _cuda_contig("k", k)
+    _cuda_contig("v", v)
+    _cuda_contig("start_pos", start_pos)
+    if k.shape != v.shape or k.dtype != v.dtype or k.dim() != 4:
+        raise ValueError("k and v must have the same [batch, t_new, Hkv, 256] shape and dtype")
+    if start_pos.dtype != torch.int32:
+        raise TypeError("start_pos must be int32")
+    batch, t_new, hkv, _ = k.shape
+    if hkv != cache.num_kv_heads:
+        raise ValueError("kv head count does not match the cache")
+    d = cache.desc()
+    _check("kvq_quantize_append",
+           lib().kvq_quantize_append(C.byref(d), _ptr(k), _ptr(v), _dtype_code(k), batch, t_new,
+                                     _ptr(start_pos), _stream(stream)))
+
+
+def decode_attn_workspace(cache: Q4Cache, batch: int, num_q_heads: int, max_seq_len: int) -> int:
+    d = cache.desc()
+    return int(lib().kvq_decode_attn_workspace(C.byref(d), batch, num_q_heads, max_seq_len))
+
+
+def decode_attn(cache: Q4Cache, q: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int,
+                scale: float, out: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One query token per sequence: q [batch, Hq, 256] -> out [batch, Hq, 256] fp32."""
+    _cuda_contig("q", q)
+    _cuda_contig("seq_lens", seq_lens)
+    if seq_lens.dtype != torch.int32:
+        raise TypeError("seq_lens must be int32")
+    batch, hq, dim = q.shape
+    if out is None:
+        out = torch.empty((batch, hq, dim), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = decode_attn_workspace(cache, batch, hq, max_seq_len)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    d = cache.desc()
+    _check("kvq_decode_attn",
+           lib().kvq_decode_attn(C.byref(d), _ptr(q), _dtype_code(q), batch, hq, _ptr(seq_lens),
+                                 int(max_seq_len), float(scale), _ptr(out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+# --------------------------------------------------------------------------
+# Octave
+# --------------------------------------------------------------------------
+@dataclass(frozen=True)
+class OctaveFormat:
+    head_size: int
+    rope_dim: int
+    v_bits: int
+    compact: bool = False
+
+    CACHE_DTYPES = {"octave_k3v4": (4, False), "octave_k3v3": (3, False),
+                    "octave_k3v3_compact": (3, True)}
+
+    @classmethod
+    def from_cache_dtype(cls, cache_dtype: str, head_size: int, rope_dim: int):
+        v_bits, compact = cls.CACHE_DTYPES[cache_dtype]
+        return cls(head_size, rope_dim, v_bits, compact)
+
+    def desc(self) -> OctaveFmtDesc:
+        return OctaveFmtDesc(self.head_size, self.rope_dim, self.v_bits, int(self.compact))
+
+    def layout(self) -> dict:
+        out = OctaveLayoutDesc()
+        f = self.desc()
+        _check("kvq_octave_layout_of", lib().kvq_octave_layout_of(C.byref(f), C.byref(out)))
+        return {n: getattr(out, n) for n, _ in OctaveLayoutDesc._fields_}
+
+
+def octave_codebook(bits: int):
+    lut = np.zeros(1 << bits, np.int8)
+    mult = C.c_float(0)
+    _check("kvq_octave_codebook",
+           lib().kvq_octave_codebook(bits, lut.ctypes.data_as(C.c_void_p), C.byref(mult)))
+    return lut, float(np.float32(mult.value))
+
+
+def sign_words(signs) -> np.ndarray:
+    """+-1 pattern -> int32 words with bit i set where the sign is -1."""
+    neg = (np.asarray(signs) < 0).astype(np.uint64).reshape(-1, 32)
+    words = (neg << np.arange(32, dtype=np.uint64)).sum(axis=1).astype(np.uint32)
+    return words.view(np.int32).copy()
+
+
+def octave_quantize(fmt: OctaveFormat, key: torch.Tensor, value: torch.Tensor,
+                    slot_mapping: torch.Tensor, cache: torch.Tensor, sign_bits: np.ndarray,
+                    stream=None) -> None:
+    """key/value [T, Hkv, D] -> slots of cache [num_blocks, Hkv, block_size, slot]."""
+    for n, t in (("key", key), ("value", value), ("slot_mapping", slot_mapping),
+                 ("cache", cache)):
+        _cuda_contig(n, t)
+    if slot_mapping.dtype != torch.int64 or cache.dtype != torch.uint8:
+        raise TypeError("slot_mapping must be int64 and cache uint8")
+    T, hkv, _ = key.shape
+    num_blocks, _, block_size, _ = cache.shape
+    f = fmt.desc()
+    sb = np.ascontiguousarray(sign_bits, dtype=np.int32)
+    _check("kvq_octave_quantize",
+           lib().kvq_octave_quantize(C.byref(f), _ptr(key), _ptr(value), _dtype_code(key), T, hkv,
+                                     _ptr(slot_mapping), _ptr(cache), block_size, num_blocks,
+                                     sb.ctypes.data_as(C.c_void_p), _stream(stream)))
+
+
+def octave_decode_attn_workspace(fmt: OctaveFormat, num_q: int, num_q_heads: int,
+                                 max_klen: int) -> int:
+    f = fmt.desc()
+    return int(lib().kvq_octave_decode_attn_workspace(C.byref(f), num_q, num_q_heads, max_klen))
+
+
+def octave_decode_attn(fmt: OctaveFormat, query: torch.Tensor, cache: torch.Tensor,
+                       block_table: torch.Tensor, q_to_req: torch.Tensor,
+                       q_to_klen: torch.Tensor, max_klen: int, scale: float,
+                       sign_bits: np.ndarray, out: torch.Tensor | None = None,
+                       workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    for n, t in (("query", query), ("cache", cache), ("block_table", block_table),
+                 ("q_to_req", q_to_req), ("q_to_klen", q_to_klen)):
+        _cuda_contig(n, t)
+    nq, hq, d = query.shape
+    num_blocks, hkv, block_size, _ = cache.shape
+    if out is None:
+        out = torch.empty((nq, hq, d), dtype=torch.float32, device=query.device)
+    if workspace is None:
+        nbytes = octave_decode_attn_workspace(fmt, nq, hq, max_klen)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=query.device)
+    f = fmt.desc()
+    sb = np.ascontiguousarray(sign_bits, dtype=np.int32)
+    _check("kvq_octave_decode_attn",
+           lib().kvq_octave_decode_attn(
+               C.byref(f), _ptr(query), _dtype_code(query), nq, hq, _ptr(cache), hkv, block_size,
+               num_blocks, _ptr(block_table), block_table.shape[0], block_table.shape[1],
+               _ptr(q_to_req), _ptr(q_to_klen), int(max_klen), float(scale),
+               sb.ctypes.data_as(C.c_void_p), _ptr(out), _ptr(workspace),
+               workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out

@@ -151,6 +151,13 @@ class Q4Cache:
         self.k_scales = np.zeros((n_rows, 8), np.uint16)
         self.v_scales = np.zeros((n_rows, 8), np.uint16)
 
+    def with_block_table(self, block_table):
+        view = Q4Cache.__new__(Q4Cache)
+        view.__dict__.update(self.__dict__)
+        view.block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+        view.max_pages = view.block_table.shape[1]
+        return view
+
     def _args(self):
         return (_p(self.k_codes), _p(self.k_scales), _p(self.v_codes), _p(self.v_scales),
                 self.n_kv_heads, self.max_tokens, _p(self.block_table), self.page_size,

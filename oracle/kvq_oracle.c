@@ -223,6 +223,7 @@ static int64_t q4_row(int b, int h, int t, int n_kv_heads, int max_tokens,
                       const int32_t *block_table, int page_size, int max_pages) {
   if (!block_table) return ((int64_t)b * n_kv_heads + h) * max_tokens + t;
   int32_t page = block_table[(int64_t)b * max_pages + t / page_size];
+  if (page < 0) return -1;
   return ((int64_t)page * n_kv_heads + h) * page_size + (t % page_size);
 }
 
@@ -245,6 +246,7 @@ int orc_q4_append(uint8_t *k_codes, uint16_t *k_scales, uint8_t *v_codes,
         int64_t src = (((int64_t)b * t_new + i) * n_kv_heads + h) * Q4_DIM;
         int64_t row = q4_row(b, h, t, n_kv_heads, max_tokens, block_table,
                              page_size, max_pages);
+        if (row < 0) return -1;
         int r = q4_quantize_one(k, dtype, src, k_codes + row * 128, k_scales + row * 8);
         if (r) return r;
         r = q4_quantize_one(v, dtype, src, v_codes + row * 128, v_scales + row * 8);
@@ -304,6 +306,7 @@ int orc_q4_decode_attn(const uint8_t *k_codes, const uint16_t *k_scales,
       for (int t = 0; t < len; t++) {
         int64_t row = q4_row(b, g, t, n_kv_heads, max_tokens, block_table, page_size,
                              max_pages);
+        if (row < 0) { free(sc); free(qv); return -1; }
         q4_row_unrotated(k_codes, k_scales, row, kd);
         for (int hh = 0; hh < group; hh++) {
           double s = 0.0;
@@ -326,6 +329,7 @@ int orc_q4_decode_attn(const uint8_t *k_codes, const uint16_t *k_scales,
       for (int t = 0; t < len; t++) {
         int64_t row = q4_row(b, g, t, n_kv_heads, max_tokens, block_table, page_size,
                              max_pages);
+        if (row < 0) { free(sc); free(qv); return -1; }
         q4_row_unrotated(v_codes, v_scales, row, kd);
         for (int hh = 0; hh < group; hh++) {
           double p = sc[(int64_t)t * group + hh];

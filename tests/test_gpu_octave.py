@@ -1,0 +1,137 @@
+"""GPU parity of the Octave variant (vLLM rocm_octave page) against the CPU
+oracle through the C ABI: slots bit-identical, attention within 2e-3."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hadamard_rotated_bit_fwht_b200 import build, kvq, synth
+
+pytestmark = pytest.mark.gpu
+ATOL = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    kvq.lib()
+
+
+def to_dev(a):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if a.dtype == np.uint16:
+        t = t.view(torch.bfloat16)
+    return t.cuda()
+
+
+def make_cache(fmt, T, Hkv, bs, seed, dt="bf16", outliers=16.0, shuffle=True):
+    """T tokens into ceil(T / bs) + 2 blocks through a shuffled slot mapping."""
+    nblk = (T + bs - 1) // bs + 2
+    k = synth.apply_outliers(synth.gaussian(seed, (T, Hkv, 128)),
+                             synth.outlier_channels(seed, Hkv, 128), outliers)
+    v = synth.apply_outliers(synth.gaussian(seed + 1, (T, Hkv, 128)),
+                             synth.outlier_channels(seed, Hkv, 128), outliers)
+    if dt == "bf16":
+        k, v = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+    g = np.random.default_rng(seed)
+    blocks = g.permutation(nblk) if shuffle else np.arange(nblk)
+    slot = (blocks[np.arange(T) // bs] * bs + np.arange(T) % bs).astype(np.int64)
+    return k, v, slot, nblk
+
+
+@pytest.mark.parametrize("v_bits", [4, 3])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_quantize_bitexact(v_bits, dt):
+    fmt = (128, 64, v_bits, 0)
+    F = kvq.OctaveFormat(*fmt[:3])
+    slot_bytes = F.layout()["slot_bytes"]
+    T, Hkv, bs = 333, 3, 16
+    k, v, slot, nblk = make_cache(fmt, T, Hkv, bs, 7 + v_bits, dt)
+    signs = synth.sign_pattern(128)
+    cache = torch.zeros((nblk, Hkv, bs, slot_bytes), dtype=torch.uint8, device="cuda")
+    kvq.octave_quantize(F, to_dev(k), to_dev(v), to_dev(slot), cache, kvq.sign_words(signs))
+    want = oracle.octave_quantize(k, v, fmt, signs)  # (T, H, slot)
+    got = cache.cpu().numpy().transpose(0, 2, 1, 3).reshape(-1, Hkv, slot_bytes)[slot]
+    bad = np.nonzero(np.any(got != want, axis=-1))
+    assert bad[0].size == 0, f"{bad[0].size} slots differ, first token {bad[0][:3]}"
+
+
+def test_quantize_skips_negative_and_out_of_range_slots():
+    F = kvq.OctaveFormat(128, 64, 4)
+    T, Hkv, bs = 8, 2, 16
+    k, v, slot, nblk = make_cache((128, 64, 4, 0), T, Hkv, bs, 3, shuffle=False)
+    slot[2] = -1
+    slot[5] = nblk * bs + 3  # block out of range
+    cache = torch.zeros((nblk, Hkv, bs, 128), dtype=torch.uint8, device="cuda")
+    kvq.octave_quantize(F, to_dev(k), to_dev(v), to_dev(slot), cache,
+                        kvq.sign_words(synth.sign_pattern(128)))
+    c = cache.cpu().numpy()
+    assert np.all(c[0, :, 2] == 0) and np.all(c[0, :, 5] == 0)
+    assert np.any(c[0, :, 3] != 0)
+
+
+@pytest.mark.parametrize("G", [1, 4, 8])
+def test_decode_vs_oracle(G):
+    fmt = (128, 64, 4, 0)
+    F = kvq.OctaveFormat(128, 64, 4)
+    Hkv, bs = 2, 16
+    Hq = Hkv * G
+    lens = np.array([300, 45, 0, 129], np.int32)
+    nreq = 3
+    T = 600
+    k, v, slot, nblk = make_cache(fmt, T, Hkv, bs, 21)
+    signs = synth.sign_pattern(128)
+    cache = torch.zeros((nblk, Hkv, bs, 128), dtype=torch.uint8, device="cuda")
+    kvq.octave_quantize(F, to_dev(k), to_dev(v), to_dev(slot), cache, kvq.sign_words(signs))
+    # requests: req r owns tokens [200 r, 200 r + 200) through their blocks
+    maxb = 200 // bs + 1
+    bt = np.zeros((nreq, maxb), np.int32)
+    for r in range(nreq):
+        for j in range(maxb):
+            tok = min(200 * r + j * bs, T - 1)
+            bt[r, j] = slot[tok] // bs
+    # only use request prefixes that are block aligned with the mapping above
+    q_to_req = np.array([0, 1, 2, 0], np.int32)
+    q_to_klen = np.minimum(lens, 192)
+    q = synth.to_bf16_bits(synth.queries(31, len(lens), Hq, 128))
+    got = kvq.octave_decode_attn(F, to_dev(q), cache, to_dev(bt), to_dev(q_to_req),
+                                 to_dev(q_to_klen), 192, 128 ** -0.5,
+                                 kvq.sign_words(signs)).cpu().numpy()
+    want = oracle.octave_attention(q, cache.cpu().numpy(), bt, q_to_req, q_to_klen, fmt,
+                                   128 ** -0.5, signs)
+    assert np.all(got[2] == 0)
+    assert np.abs(got - want).max() <= ATOL
+
+
+def test_octave_workload_sampled():
+    """Octave workload shape (k3v4, head 128, rope 64, 32 q / 8 kv heads,
+    bf16, 256-token blocks, shuffled table) with 4 requests of 4096 tokens:
+    sampled slots bit-exact and attention within 2e-3."""
+    W = synth.WORKLOADS["octave"]
+    fmt = (W["head_size"], W["rope_dim"], W["v_bits"], 0)
+    F = kvq.OctaveFormat(*fmt[:3])
+    nreq, ctx, Hkv, Hq, bs = 4, 4096, W["n_kv_heads"], W["n_q_heads"], W["block_size"]
+    T = nreq * ctx
+    nblk = T // bs
+    k, v = synth.kv_tokens(W["seed"], 1, T, Hkv, 128, W["outlier_frac"], W["outlier_factor"])
+    k, v = synth.to_bf16_bits(k[0]), synth.to_bf16_bits(v[0])
+    bt, _ = synth.page_table(W["seed"], nreq, np.full(nreq, ctx // bs), ctx // bs)
+    slot = np.concatenate([bt[r, np.arange(ctx) // bs] * bs + np.arange(ctx) % bs
+                           for r in range(nreq)]).astype(np.int64)
+    signs = synth.sign_pattern(128)
+    cache = torch.zeros((nblk, Hkv, bs, 128), dtype=torch.uint8, device="cuda")
+    kvq.octave_quantize(F, to_dev(k), to_dev(v), to_dev(slot), cache, kvq.sign_words(signs))
+    rng = np.random.default_rng(1)
+    pick = rng.choice(T, 512, replace=False)
+    want_slots = oracle.octave_quantize(k[pick], v[pick], fmt, signs)
+    c = cache.cpu().numpy()
+    got_slots = c.transpose(0, 2, 1, 3).reshape(-1, Hkv, 128)[slot[pick]]
+    assert np.array_equal(got_slots, want_slots)
+    q = synth.to_bf16_bits(synth.queries(W["seed"], nreq, Hq, 128))
+    q_to_req = np.arange(nreq, dtype=np.int32)
+    q_to_klen = np.full(nreq, ctx, np.int32)
+    got = kvq.octave_decode_attn(F, to_dev(q), cache, to_dev(bt), to_dev(q_to_req),
+                                 to_dev(q_to_klen), ctx, 128 ** -0.5,
+                                 kvq.sign_words(signs)).cpu().numpy()
+    want = oracle.octave_attention(q, c, bt, q_to_req, q_to_klen, fmt, 128 ** -0.5, signs)
+    assert np.abs(got - want).max() <= ATOL
