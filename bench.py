@@ -1,19 +1,22 @@
 """Benchmark of the Hadamard-rotated Q4_0 KV cache on B200.
 
-One step = one pass of the whole hot path on the long-context decode workload
-(1 sequence, 131072 tokens, 32 query / 4 kv heads, D = 256, bf16 inputs):
-kvq_quantize_append of the new token's K and V (rotate + Q4_0 + store), then
-kvq_decode_attn over the whole cache (rotate q, stream and dequantize the
-nibbles, online softmax, split-K combine, back-rotation).
+One step = one pass of the whole hot path over one batch.  The default
+workload is the long-context decode (1 sequence, 131072 tokens, 32 query /
+4 kv heads, D = 256, bf16 inputs): kvq_quantize_append of the new token's K
+and V (rotate + Q4_0 + store), then kvq_decode_attn over the whole cache
+(rotate q, stream and dequantize the nibbles, online softmax, split-K
+combine, back-rotation).
 
-`value` is decode-step HBM throughput in GB/s: algorithmic bytes per step
-(every cache byte read once, inputs read and outputs written once) / device
-time per step, summed over ranks.  Three copies of the cache (453 MB, over 3x
-the 126 MB L2) are rotated so no step reads bytes the previous step left in L2.
-The other workloads (quantize prefill, paged decode, Octave) are timed the same
-way and reported under "workloads".
+`value` is HBM throughput in GB/s: algorithmic bytes per step (every cache
+byte read once, inputs read and outputs written once) / device time per
+step, summed over ranks.  Every workload's data is larger than the 126 MB L2;
+the long-decode cache (151 MB) is additionally kept in three copies (453 MB)
+that steps rotate through.  The other workloads are timed per call (with a
+512 MB L2 flush before each call, outside the timed events) and reported
+under "workloads"; `--workload NAME` makes one of them the main line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+                    [--workload long_decode|quantize|paged_decode|octave]
 """
 from __future__ import annotations
 
@@ -53,17 +56,34 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from a committed ncu capture, only if the kernel
+def recorded_traffic(key: str):
+    """DRAM bytes per call from a committed ncu capture, only if the kernel
     sources are unchanged since it was taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    e = d.get(kernel)
+    e = json.load(open(p)).get(key)
     if not e or e.get("source_hash") != kernel_source_hash():
         return None
-    return e.get("bytes_per_launch")
+    return e.get("bytes_per_call")
+
+
+# ----------------------------------------------------------------- ranks
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of per-rank timings (no-op without a process
+    group); every rank gets the same result."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput_gbs(bytes_per_step_per_rank, world, ms_per_step):
+    """Whole-job GB/s: every rank processes its own replica of the step; the
+    job's step time is the slowest rank's."""
+    return bytes_per_step_per_rank * world / ms_per_step / 1e6
 
 
 # ----------------------------------------------------------------- clocks
@@ -122,23 +142,47 @@ class ClockSampler:
 # ----------------------------------------------------------------- workloads
 def bf16_tensor(a, dev):
     import torch
-    return torch.from_numpy(a).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)
 
 
-class LongDecode:
-    """Long-context decode workload and its per-step byte count."""
+class Workload:
+    """One step of the hot path on a synthetic batch: pre(i) (the append of
+    the step's new tokens, if any) then kernel_call(i) (the dominant call).
+    Subclasses set step_bytes / kernel_bytes (algorithmic), launches_per_step,
+    kernel_name, traffic_key, config, and h2d / d2h tensors for e2e."""
+    launches_per_step = 0
+    kernel_name = ""
+    traffic_key = ""
+
+    def pre(self, i):
+        pass
+
+    def kernel_call(self, i):
+        raise NotImplementedError
+
+    def step(self, i):
+        self.pre(i)
+        self.kernel_call(i)
+
+    def extra(self, call_ms):
+        return {}
+
+
+class LongDecode(Workload):
+    """Long-context decode: append the new token, decode over 131072 tokens."""
+    launches_per_step = 3  # append + decode split + combine
+    kernel_name = "kvq_decode_attn (q4_decode_mma_kernel + q4_decode_combine_kernel)"
+    traffic_key = "q4_decode_long"
 
     def __init__(self, dev, copies=3):
         import torch
         from hadamard_rotated_bit_fwht_b200 import kvq
         W = synth.WORKLOADS["long_decode"]
-        self.W = W
         B, H, T, Hq = W["batch"], W["n_kv_heads"], W["ctx"], W["n_q_heads"]
         self.B, self.H, self.T, self.Hq = B, H, T, Hq
         k, v = synth.kv_tokens(W["seed"], B, T, H, 256, W["outlier_frac"], W["outlier_factor"])
         kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
         del k, v
-        self.host_k, self.host_v = kb, vb
         kd, vd = bf16_tensor(kb, dev), bf16_tensor(vb, dev)
         self.caches = []
         zero = torch.zeros(B, dtype=torch.int32, device=dev)
@@ -147,48 +191,249 @@ class LongDecode:
             kvq.quantize_append(c, kd, vd, zero)
             self.caches.append(c)
         del kd, vd
-        self.q_host = synth.to_bf16_bits(synth.queries(W["seed"], B, Hq, 256))
-        self.q = bf16_tensor(self.q_host, dev)
-        # the step's new token: the last position of each sequence
-        self.new_k_host = np.ascontiguousarray(kb[:, T - 1:T])
-        self.new_v_host = np.ascontiguousarray(vb[:, T - 1:T])
-        self.new_k = bf16_tensor(self.new_k_host, dev)
-        self.new_v = bf16_tensor(self.new_v_host, dev)
+        self.q = bf16_tensor(synth.to_bf16_bits(synth.queries(W["seed"], B, Hq, 256)), dev)
+        self.new_k = bf16_tensor(kb[:, T - 1:T], dev)
+        self.new_v = bf16_tensor(vb[:, T - 1:T], dev)
         self.pos = torch.full((B,), T - 1, dtype=torch.int32, device=dev)
         self.lens = torch.full((B,), T, dtype=torch.int32, device=dev)
         self.out = torch.empty((B, Hq, 256), dtype=torch.float32, device=dev)
-        ws = kvq.decode_attn_workspace(self.caches[0], B, Hq, T)
-        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self.ws = torch.empty(kvq.decode_attn_workspace(self.caches[0], B, Hq, T),
+                              dtype=torch.uint8, device=dev)
         self.kvq = kvq
-        torch.cuda.synchronize()
+        self.kernel_bytes = B * H * T * 288 + B * Hq * 256 * (2 + 4)
+        self.step_bytes = self.kernel_bytes + 2 * B * H * (512 + 144)
+        self.h2d = [self.new_k, self.new_v, self.q]
+        self.d2h = [self.out]
+        self.config = {"workload": "long_decode", "batch": B, "n_q_heads": Hq,
+                       "n_kv_heads": H, "head_dim": 256, "ctx": T,
+                       "step": "kvq_quantize_append(1 token) + kvq_decode_attn",
+                       "l2": "3 cache copies (453 MB) rotated per step, inputs > L2"}
 
-    def decode_bytes(self):
-        return (self.B * self.H * self.T * 288 + self.B * self.Hq * 256 * 2
-                + self.B * self.Hq * 256 * 4)
+    def pre(self, i):
+        self.kvq.quantize_append(self.caches[i % len(self.caches)], self.new_k, self.new_v,
+                                 self.pos)
 
-    def append_bytes(self):
-        return 2 * self.B * self.H * (512 + 144)
-
-    def step_bytes(self):
-        return self.decode_bytes() + self.append_bytes()
-
-    def append(self, i):
-        self.kvq.quantize_append(self.caches[i % len(self.caches)], self.new_k, self.new_v, self.pos)
-
-    def decode(self, i):
+    def kernel_call(self, i):
         self.kvq.decode_attn(self.caches[i % len(self.caches)], self.q, self.lens, self.T,
                              1.0 / 16.0, out=self.out, workspace=self.ws)
 
-    def step(self, i):
-        self.append(i)
-        self.decode(i)
-
-    launches_per_step = 3  # append + decode split + combine
+    def extra(self, call_ms):
+        th = self.B * self.H * self.T / call_ms * 1e3
+        return {"tok_head_per_s": th, "tok_qhead_per_s": th * self.Hq / self.H}
 
 
+class QuantizePrefill(Workload):
+    """Quantize-on-append: 4096-token prefill of 8 sequences x 8 kv heads."""
+    launches_per_step = 1
+    kernel_name = "kvq_quantize_append (q4_append_kernel)"
+    traffic_key = "q4_append_prefill"
+
+    def __init__(self, dev):
+        import torch
+        from hadamard_rotated_bit_fwht_b200 import kvq
+        W = synth.WORKLOADS["quantize"]
+        B, H, P, A, cap = W["batch"], W["n_kv_heads"], W["prefill"], W["appends"], W["capacity"]
+        self.B, self.H, self.P, self.A = B, H, P, A
+        k, v = synth.kv_tokens(W["seed"], B, P + A, H, 256, W["outlier_frac"],
+                               W["outlier_factor"])
+        kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+        del k, v
+        self.k = bf16_tensor(kb[:, :P], dev)
+        self.v = bf16_tensor(vb[:, :P], dev)
+        self.singles = [(bf16_tensor(kb[:, P + i:P + i + 1], dev),
+                         bf16_tensor(vb[:, P + i:P + i + 1], dev),
+                         torch.full((B,), P + i, dtype=torch.int32, device=dev))
+                        for i in range(A)]
+        self.cache = kvq.Q4Cache.contiguous(B, H, cap, device=dev)
+        self.zero = torch.zeros(B, dtype=torch.int32, device=dev)
+        self.kvq = kvq
+        self.kernel_bytes = self.step_bytes = 2 * B * P * H * (512 + 144)
+        self.h2d = [self.k, self.v]
+        self.d2h = [self.cache.k_scales[:1]]
+        self.config = {"workload": "quantize", "batch": B, "n_kv_heads": H, "head_dim": 256,
+                       "prefill": P, "dtype_in": "bf16",
+                       "step": "kvq_quantize_append(4096-token prefill)",
+                       "l2": "inputs 268 MB > L2"}
+
+    def kernel_call(self, i):
+        self.kvq.quantize_append(self.cache, self.k, self.v, self.zero)
+
+    def extra(self, call_ms):
+        return {"Mtok_s": self.B * self.P / call_ms / 1e3,
+                "tok_head_s": self.B * self.P * self.H / call_ms * 1e3}
+
+    def single_token_appends(self):
+        """The 256 single-token appends, eager and captured in one CUDA graph."""
+        import torch
+        s = torch.cuda.current_stream()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for kk, vv, pp in self.singles[:8]:
+            self.kvq.quantize_append(self.cache, kk, vv, pp)
+        torch.cuda.synchronize()
+        a.record(s)
+        for kk, vv, pp in self.singles:
+            self.kvq.quantize_append(self.cache, kk, vv, pp)
+        b.record(s)
+        torch.cuda.synchronize()
+        eager = a.elapsed_time(b) * 1e3 / self.A
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for kk, vv, pp in self.singles:
+                self.kvq.quantize_append(self.cache, kk, vv, pp)
+        g.replay()
+        torch.cuda.synchronize()
+        a.record(s)
+        g.replay()
+        b.record(s)
+        torch.cuda.synchronize()
+        graph = a.elapsed_time(b) * 1e3 / self.A
+        del g
+        return {"us_per_append_eager": eager, "us_per_append_cuda_graph": graph,
+                "appends": self.A, "shape": f"batch {self.B}, {self.H} kv heads, 1 token each"}
+
+
+class PagedDecode(Workload):
+    """Batched paged decode: 32 sequences, lengths U[8192, 32768], 256-token
+    shuffled pages; a step appends one token per sequence and decodes."""
+    launches_per_step = 3
+    kernel_name = "kvq_decode_attn, paged (q4_decode_mma_kernel + combine)"
+    traffic_key = "q4_decode_paged"
+
+    def __init__(self, dev):
+        import torch
+        from hadamard_rotated_bit_fwht_b200 import kvq
+        W = synth.WORKLOADS["paged_decode"]
+        B, H, Hq, ps = W["batch"], W["n_kv_heads"], W["n_q_heads"], W["page_size"]
+        self.B, self.H, self.Hq = B, H, Hq
+        lens = synth.seq_lens(W["seed"], B, W["ctx_lo"], W["ctx_hi"])
+        npp = (lens + ps - 1) // ps
+        bt, n_pages = synth.page_table(W["seed"], B, npp, int(npp.max()))
+        self.cache = kvq.Q4Cache.paged(n_pages, H, ps, torch.from_numpy(bt), device=dev)
+        new_k, new_v = [], []
+        for b0 in range(0, B, 8):  # generate 8 sequences at a time, append each alone
+            Lc = int(lens[b0:b0 + 8].max())
+            k, v = synth.kv_tokens(W["seed"] * 100 + b0, 8, Lc, H, 256, W["outlier_frac"],
+                                   W["outlier_factor"])
+            kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+            del k, v
+            for j in range(8):
+                L = int(lens[b0 + j])
+                one = self.cache.with_block_table(torch.from_numpy(bt[b0 + j:b0 + j + 1]))
+                kvq.quantize_append(one, bf16_tensor(kb[j:j + 1, :L], dev),
+                                    bf16_tensor(vb[j:j + 1, :L], dev),
+                                    torch.zeros(1, dtype=torch.int32, device=dev))
+                new_k.append(kb[j, L - 1:L])
+                new_v.append(vb[j, L - 1:L])
+            del kb, vb
+        self.new_k = bf16_tensor(np.stack(new_k), dev)  # (B, 1, H, 256)
+        self.new_v = bf16_tensor(np.stack(new_v), dev)
+        self.pos = torch.from_numpy(lens - 1).to(dev)
+        self.lens = torch.from_numpy(lens).to(dev)
+        self.Tm = int(lens.max())
+        self.q = bf16_tensor(synth.to_bf16_bits(synth.queries(W["seed"], B, Hq, 256)), dev)
+        self.out = torch.empty((B, Hq, 256), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(kvq.decode_attn_workspace(self.cache, B, Hq, self.Tm),
+                              dtype=torch.uint8, device=dev)
+        self.kvq = kvq
+        self.total = int(lens.sum())
+        self.kernel_bytes = self.total * H * 288 + B * Hq * 256 * 6
+        self.step_bytes = self.kernel_bytes + 2 * B * H * (512 + 144)
+        self.h2d = [self.new_k, self.new_v, self.q]
+        self.d2h = [self.out]
+        self.config = {"workload": "paged_decode", "batch": B, "n_q_heads": Hq,
+                       "n_kv_heads": H, "head_dim": 256, "tokens": self.total,
+                       "page_size": ps, "step": "kvq_quantize_append(1 token/seq) + "
+                       "kvq_decode_attn", "l2": "cache 369 MB > L2"}
+
+    def pre(self, i):
+        self.kvq.quantize_append(self.cache, self.new_k, self.new_v, self.pos)
+
+    def kernel_call(self, i):
+        self.kvq.decode_attn(self.cache, self.q, self.lens, self.Tm, 1 / 16, out=self.out,
+                             workspace=self.ws)
+
+    def extra(self, call_ms):
+        return {"tok_head_per_s": self.total * self.H / call_ms * 1e3}
+
+
+class OctaveDecode(Workload):
+    """Octave k3v4 (head 128, rope 64), 16 requests x 16384 tokens, 32 q / 8 kv
+    heads, 256-token shuffled blocks; a step quantizes one new token per
+    request into its slot and decodes."""
+    launches_per_step = 3  # quantize + split + combine
+    kernel_name = "kvq_octave_decode_attn (octave split + combine)"
+    traffic_key = "octave_decode"
+
+    def __init__(self, dev):
+        import torch
+        from hadamard_rotated_bit_fwht_b200 import kvq
+        W = synth.WORKLOADS["octave"]
+        B, H, Hq, ctx, bs = W["batch"], W["n_kv_heads"], W["n_q_heads"], W["ctx"], W["block_size"]
+        self.B, self.H, self.Hq, self.ctx = B, H, Hq, ctx
+        self.F = kvq.OctaveFormat(W["head_size"], W["rope_dim"], W["v_bits"])
+        self.signs = kvq.sign_words(synth.sign_pattern(128))
+        bt, _ = synth.page_table(W["seed"], B, np.full(B, ctx // bs), ctx // bs)
+        self.cache = torch.zeros((B * ctx // bs, H, bs, 128), dtype=torch.uint8, device=dev)
+        new_k, new_v = [], []
+        for r in range(B):
+            k, v = synth.kv_tokens(W["seed"] * 100 + r, 1, ctx, H, 128, W["outlier_frac"],
+                                   W["outlier_factor"])
+            kb, vb = synth.to_bf16_bits(k[0]), synth.to_bf16_bits(v[0])
+            slot = torch.from_numpy((bt[r, np.arange(ctx) // bs] * bs + np.arange(ctx) % bs)
+                                    .astype(np.int64)).to(dev)
+            kd, vd = bf16_tensor(kb, dev), bf16_tensor(vb, dev)
+            kvq.octave_quantize(self.F, kd, vd, slot, self.cache, self.signs)
+            if r == 0:  # kept for the quantize-throughput figure
+                self.qk, self.qv, self.qslot = kd, vd, slot
+            new_k.append(kb[ctx - 1])
+            new_v.append(vb[ctx - 1])
+        self.new_k = bf16_tensor(np.stack(new_k), dev)  # (B, H, 128): token r -> request r
+        self.new_v = bf16_tensor(np.stack(new_v), dev)
+        self.new_slot = torch.from_numpy((bt[:, (ctx - 1) // bs] * bs + (ctx - 1) % bs)
+                                         .astype(np.int64)).to(dev)
+        self.q = bf16_tensor(synth.to_bf16_bits(synth.queries(W["seed"], B, Hq, 128)), dev)
+        self.bt = torch.from_numpy(bt).to(dev)
+        self.q2r = torch.arange(B, dtype=torch.int32, device=dev)
+        self.q2l = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+        self.out = torch.empty((B, Hq, 128), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(kvq.octave_decode_attn_workspace(self.F, B, Hq, ctx),
+                              dtype=torch.uint8, device=dev)
+        self.kvq = kvq
+        self.kernel_bytes = B * ctx * H * 128 + B * Hq * 128 * 6
+        self.step_bytes = self.kernel_bytes + B * H * (2 * 256 + 128)
+        self.quant_bytes = ctx * H * (2 * 256 + 128)
+        self.h2d = [self.new_k, self.new_v, self.q]
+        self.d2h = [self.out]
+        self.config = {"workload": "octave", "format": "k3v4", "head_size": 128, "rope_dim": 64,
+                       "batch": B, "n_q_heads": Hq, "n_kv_heads": H, "ctx": ctx,
+                       "block_size": bs, "step": "kvq_octave_quantize(1 token/request) + "
+                       "kvq_octave_decode_attn", "l2": "cache 268 MB > L2"}
+
+    def pre(self, i):
+        self.kvq.octave_quantize(self.F, self.new_k, self.new_v, self.new_slot, self.cache,
+                                 self.signs)
+
+    def kernel_call(self, i):
+        self.kvq.octave_decode_attn(self.F, self.q, self.cache, self.bt, self.q2r, self.q2l,
+                                    self.ctx, 128 ** -0.5, self.signs, out=self.out,
+                                    workspace=self.ws)
+
+    def quantize_call(self):
+        self.kvq.octave_quantize(self.F, self.qk, self.qv, self.qslot, self.cache, self.signs)
+
+    def extra(self, call_ms):
+        return {"tok_head_per_s": self.B * self.ctx * self.H / call_ms * 1e3}
+
+
+WORKLOAD_CLASSES = {"long_decode": LongDecode, "quantize": QuantizePrefill,
+                    "paged_decode": PagedDecode, "octave": OctaveDecode}
+
+
+# ----------------------------------------------------------------- timing
 def time_steps(wl, steps, warmup, dist=None):
-    """Device time of `steps` steps (CUDA events around the region, barrier and
-    synchronize on both sides); also per-launch time of the decode call."""
+    """Device time of `steps` steps (CUDA events on the launching stream around
+    the region, barrier + synchronize on both sides) and the mean device time
+    of the dominant call inside those steps (events around each call)."""
     import torch
     for i in range(warmup):
         wl.step(i)
@@ -203,35 +448,32 @@ def time_steps(wl, steps, warmup, dist=None):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(s)
     for i in range(steps):
-        wl.append(i)
+        wl.pre(i)
         ev[i][0].record(s)
-        wl.decode(i)
+        wl.kernel_call(i)
         ev[i][1].record(s)
     t1.record(s)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     total_ms = t0.elapsed_time(t1)
-    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
-    return total_ms, dec_ms
+    call_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    return total_ms, call_ms
 
 
 def time_e2e(wl, steps, warmup):
-    """Same step through the C ABI with host buffers: H2D of the new token's
-    K, V and the query from pinned memory, the step, D2H of the output."""
+    """The same step with its inputs copied host -> device from pinned memory
+    and its output copied back, inside the timed region."""
     import torch
-    dev = wl.q.device
-    hk = torch.from_numpy(wl.new_k_host).view(torch.bfloat16).pin_memory()
-    hv = torch.from_numpy(wl.new_v_host).view(torch.bfloat16).pin_memory()
-    hq = torch.from_numpy(wl.q_host).view(torch.bfloat16).pin_memory()
-    ho = torch.empty(wl.out.shape, dtype=torch.float32).pin_memory()
+    hin = [t.cpu().pin_memory() for t in wl.h2d]
+    hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in wl.d2h]
 
     def one(i):
-        wl.new_k.copy_(hk, non_blocking=True)
-        wl.new_v.copy_(hv, non_blocking=True)
-        wl.q.copy_(hq, non_blocking=True)
+        for d, h in zip(wl.h2d, hin):
+            d.copy_(h, non_blocking=True)
         wl.step(i)
-        ho.copy_(wl.out, non_blocking=True)
+        for d, h in zip(wl.d2h, hout):
+            h.copy_(d, non_blocking=True)
 
     for i in range(warmup):
         one(i)
@@ -243,9 +485,8 @@ def time_e2e(wl, steps, warmup):
         one(i)
     b.record(s)
     torch.cuda.synchronize()
-    h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 2
-    d2h = ho.numel() * 4
-    _ = dev
+    h2d = sum(t.numel() * t.element_size() for t in hin)
+    d2h = sum(t.numel() * t.element_size() for t in hout)
     return a.elapsed_time(b) / steps, h2d, d2h
 
 
@@ -267,151 +508,38 @@ def time_call(fn, reps, flush=None):
     return float(np.mean([a.elapsed_time(b) for a, b in ts]))
 
 
-def other_workloads(dev, reps, peak):
-    """Quantize prefill / single-token appends, paged decode and Octave."""
+def other_workloads(dev, main_name, reps, peak):
+    """Per-call timing of every workload other than the main one."""
     import torch
-    from hadamard_rotated_bit_fwht_b200 import kvq
     flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
     def flush():
         flush_buf.fill_(1)
 
     res = {}
-    # ---- quantize-on-append (B=8, Hkv=8, 4096-token prefill, 256 appends)
-    W = synth.WORKLOADS["quantize"]
-    B, H, P, A, cap = W["batch"], W["n_kv_heads"], W["prefill"], W["appends"], W["capacity"]
-    k, v = synth.kv_tokens(W["seed"], B, P + A, H, 256, W["outlier_frac"], W["outlier_factor"])
-    kd, vd = bf16_tensor(synth.to_bf16_bits(k), dev), bf16_tensor(synth.to_bf16_bits(v), dev)
-    del k, v
-    cache = kvq.Q4Cache.contiguous(B, H, cap, device=dev)
-    kp, vp = kd[:, :P].contiguous(), vd[:, :P].contiguous()
-    zero = torch.zeros(B, dtype=torch.int32, device=dev)
-    for _ in range(3):
-        kvq.quantize_append(cache, kp, vp, zero)
-    ms = time_call(lambda: kvq.quantize_append(cache, kp, vp, zero), reps, flush)
-    nbytes = 2 * B * P * H * (512 + 144)
-    res["quantize_prefill"] = {
-        "ms": ms, "GB_s": nbytes / ms / 1e6, "frac_of_peak": nbytes / ms / 1e6 / peak,
-        "Mtok_s": B * P / ms / 1e3, "tok_head_s": B * P * H / ms * 1e3, "bytes": nbytes,
-        "shape": f"batch {B}, {H} kv heads, {P}-token prefill, bf16 -> Q4_0"}
-    singles = [(kd[:, P + i:P + i + 1].contiguous(), vd[:, P + i:P + i + 1].contiguous(),
-                torch.full((B,), P + i, dtype=torch.int32, device=dev)) for i in range(A)]
-    torch.cuda.synchronize()
-    s = torch.cuda.current_stream()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(s)
-    for kk, vv, pp in singles:
-        kvq.quantize_append(cache, kk, vv, pp)
-    b.record(s)
-    torch.cuda.synchronize()
-    us_eager = a.elapsed_time(b) * 1e3 / A
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for kk, vv, pp in singles:
-            kvq.quantize_append(cache, kk, vv, pp)
-    g.replay()
-    torch.cuda.synchronize()
-    a.record(s)
-    g.replay()
-    b.record(s)
-    torch.cuda.synchronize()
-    res["quantize_single_token_append"] = {
-        "us_per_append_eager": us_eager, "us_per_append_cuda_graph": a.elapsed_time(b) * 1e3 / A,
-        "appends": A, "shape": f"batch {B}, {H} kv heads, 1 token each"}
-    del g, singles, kd, vd, kp, vp, cache
-
-    # ---- paged decode (B=32, 16 q / 2 kv heads, lens U[8192, 32768], 256-token pages)
-    W = synth.WORKLOADS["paged_decode"]
-    B, H, Hq, ps = W["batch"], W["n_kv_heads"], W["n_q_heads"], W["page_size"]
-    lens = synth.seq_lens(W["seed"], B, W["ctx_lo"], W["ctx_hi"])
-    npp = (lens + ps - 1) // ps
-    maxp = int(npp.max())
-    bt, n_pages = synth.page_table(W["seed"], B, npp, maxp)
-    pc = kvq.Q4Cache.paged(n_pages, H, ps, torch.from_numpy(bt), device=dev)
-    Tm = int(lens.max())
-    for b0 in range(0, B, 8):  # generate 8 sequences at a time, append each alone
-        Lc = int(lens[b0:b0 + 8].max())
-        k, v = synth.kv_tokens(W["seed"] * 100 + b0, 8, Lc, H, 256, W["outlier_frac"],
-                               W["outlier_factor"])
-        kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
-        del k, v
-        for j in range(8):
-            L = int(lens[b0 + j])
-            one = pc.with_block_table(torch.from_numpy(bt[b0 + j:b0 + j + 1]))
-            kvq.quantize_append(one, bf16_tensor(np.ascontiguousarray(kb[j:j + 1, :L]), dev),
-                                bf16_tensor(np.ascontiguousarray(vb[j:j + 1, :L]), dev),
-                                torch.zeros(1, dtype=torch.int32, device=dev))
-        del kb, vb
-    q = bf16_tensor(synth.to_bf16_bits(synth.queries(W["seed"], B, Hq, 256)), dev)
-    lens_d = torch.from_numpy(lens).to(dev)
-    out = torch.empty((B, Hq, 256), dtype=torch.float32, device=dev)
-    wsz = kvq.decode_attn_workspace(pc, B, Hq, Tm)
-    ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
-
-    def dec():
-        kvq.decode_attn(pc, q, lens_d, Tm, 1 / 16, out=out, workspace=ws)
-
-    for _ in range(3):
-        dec()
-    ms = time_call(dec, reps, flush)
-    tot = int(lens.sum())
-    nbytes = tot * H * 288 + B * Hq * 256 * 6
-    res["paged_decode"] = {
-        "ms": ms, "GB_s": nbytes / ms / 1e6, "frac_of_peak": nbytes / ms / 1e6 / peak,
-        "tok_head_s": tot * H / ms * 1e3, "bytes": nbytes,
-        "shape": f"batch {B}, {Hq} q / {H} kv heads, {tot} tokens, 256-token shuffled pages"}
-    del pc, ws
-
-    # ---- Octave k3v4 (B=16, 32 q / 8 kv heads, head 128, ctx 16384, 256-token blocks)
-    W = synth.WORKLOADS["octave"]
-    B, H, Hq, ctx, bs = W["batch"], W["n_kv_heads"], W["n_q_heads"], W["ctx"], W["block_size"]
-    F = kvq.OctaveFormat(W["head_size"], W["rope_dim"], W["v_bits"])
-    signs = kvq.sign_words(synth.sign_pattern(128))
-    nb = B * ctx // bs
-    bt, _ = synth.page_table(W["seed"], B, np.full(B, ctx // bs), ctx // bs)
-    ocache = torch.zeros((nb, H, bs, 128), dtype=torch.uint8, device=dev)
-    qtime = []
-    for r in range(B):
-        k, v = synth.kv_tokens(W["seed"] * 100 + r, 1, ctx, H, 128, W["outlier_frac"],
-                               W["outlier_factor"])
-        kd = bf16_tensor(synth.to_bf16_bits(k[0]), dev)
-        vd = bf16_tensor(synth.to_bf16_bits(v[0]), dev)
-        slot = torch.from_numpy((bt[r, np.arange(ctx) // bs] * bs + np.arange(ctx) % bs)
-                                .astype(np.int64)).to(dev)
-        kvq.octave_quantize(F, kd, vd, slot, ocache, signs)
-        if r == 0:
+    for name, cls in WORKLOAD_CLASSES.items():
+        if name == main_name:
+            continue
+        wl = cls(dev)
+        for i in range(3):
+            wl.kernel_call(i)
+        ms = time_call(lambda: wl.kernel_call(0), reps, flush)
+        gbs = wl.kernel_bytes / ms / 1e6
+        res[name] = {"call": wl.kernel_name, "ms": ms, "GB_s": gbs, "frac_of_peak": gbs / peak,
+                     "bytes": wl.kernel_bytes, "config": wl.config, **wl.extra(ms)}
+        if isinstance(wl, QuantizePrefill):
+            res["quantize_single_token_append"] = wl.single_token_appends()
+        if isinstance(wl, OctaveDecode):
             for _ in range(2):
-                kvq.octave_quantize(F, kd, vd, slot, ocache, signs)
-            qtime.append(time_call(lambda: kvq.octave_quantize(F, kd, vd, slot, ocache, signs),
-                                   reps, flush))
-    qo = bf16_tensor(synth.to_bf16_bits(synth.queries(W["seed"], B, Hq, 128)), dev)
-    btd = torch.from_numpy(bt).to(dev)
-    q2r = torch.arange(B, dtype=torch.int32, device=dev)
-    q2l = torch.full((B,), ctx, dtype=torch.int32, device=dev)
-    oout = torch.empty((B, Hq, 128), dtype=torch.float32, device=dev)
-    wsz = kvq.octave_decode_attn_workspace(F, B, Hq, ctx)
-    ows = torch.empty(wsz, dtype=torch.uint8, device=dev)
-
-    def odec():
-        kvq.octave_decode_attn(F, qo, ocache, btd, q2r, q2l, ctx, 128 ** -0.5, signs, out=oout,
-                               workspace=ows)
-
-    for _ in range(3):
-        odec()
-    ms = time_call(odec, reps, flush)
-    nbytes = B * ctx * H * 128 + B * Hq * 128 * 6
-    qbytes = ctx * H * (2 * 128 * 2 + 128)
-    res["octave_decode"] = {
-        "ms": ms, "GB_s": nbytes / ms / 1e6, "frac_of_peak": nbytes / ms / 1e6 / peak,
-        "tok_head_s": B * ctx * H / ms * 1e3, "bytes": nbytes,
-        "shape": f"k3v4 head 128 rope 64, batch {B}, {Hq} q / {H} kv heads, ctx {ctx}, "
-                 "256-token shuffled blocks"}
-    res["octave_quantize"] = {
-        "ms": qtime[0], "GB_s": qbytes / qtime[0] / 1e6,
-        "frac_of_peak": qbytes / qtime[0] / 1e6 / peak, "Mtok_s": ctx / qtime[0] / 1e3,
-        "shape": f"{ctx} tokens x {H} kv heads, bf16 -> 128-byte slots"}
-    del ocache, flush_buf
-    torch.cuda.synchronize()
+                wl.quantize_call()
+            qms = time_call(wl.quantize_call, reps, flush)
+            res["octave_quantize"] = {
+                "ms": qms, "GB_s": wl.quant_bytes / qms / 1e6,
+                "frac_of_peak": wl.quant_bytes / qms / 1e6 / peak, "Mtok_s": wl.ctx / qms / 1e3,
+                "shape": f"{wl.ctx} tokens x {wl.H} kv heads, bf16 -> 128-byte slots"}
+        del wl
+        torch.cuda.synchronize()
+    del flush_buf
     return res
 
 
@@ -463,13 +591,29 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------- main
+def busy(wl, seconds, start):
+    """Keep the GPU on the step for a while (for the clock sampler)."""
+    import torch
+    t_end = time.time() + seconds
+    i = start
+    while time.time() < t_end:
+        wl.step(i)
+        i += 1
+        if i % 64 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    return i
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
-    ap.add_argument("--no-workloads", action="store_true", help="skip the other workloads")
+    ap.add_argument("--workload", default="long_decode", choices=list(WORKLOAD_CLASSES))
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="report the main workload only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -492,82 +636,61 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     from hadamard_rotated_bit_fwht_b200 import build as kbuild
-    if rank == 0 or world == 1:
+    if rank == 0:
         kbuild.build()
     if dist is not None:
         dist.barrier()
     peak, peak_kind = load_peaks()
 
-    wl = LongDecode(dev)
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                          else local)
+    wl = WORKLOAD_CLASSES[args.workload](dev)
+    clocks = ClockSampler(local)
     clocks.start()
-    # keep the GPU busy ~0.5 s before and after the timed region for the sampler
-    t_end = time.time() + 0.5
-    i = 0
-    while time.time() < t_end:
-        wl.step(i)
-        i += 1
-        if i % 200 == 0:
-            torch.cuda.synchronize()
-    total_ms, dec_ms = time_steps(wl, args.steps, args.warmup, dist)
-    t_end = time.time() + 0.5
-    while time.time() < t_end:
-        wl.step(i)
-        i += 1
-        if i % 200 == 0:
-            torch.cuda.synchronize()
-    torch.cuda.synchronize()
+    i = busy(wl, 0.5, 0)
+    total_ms, call_ms = time_steps(wl, args.steps, args.warmup, dist)
+    busy(wl, 0.5, i)
     clk = clocks.stop()
 
-    ms_step = total_ms / args.steps
-    if dist is not None:
-        t = torch.tensor([ms_step, dec_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, dec_ms = float(t[0]), float(t[1])
-    value = wl.step_bytes() * world / ms_step / 1e6  # GB/s, whole job
-    achieved = wl.decode_bytes() / dec_ms / 1e6
-    e2e_ms, h2d, d2h = time_e2e(wl, max(50, args.steps // 10), 10)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e_value = wl.step_bytes() * world / e2e_ms / 1e6
+    ms_step, call_ms = max_over_ranks([total_ms / args.steps, call_ms], dist, dev)
+    value = job_throughput_gbs(wl.step_bytes, world, ms_step)
+    achieved = wl.kernel_bytes / call_ms / 1e6
+    e2e_ms, h2d, d2h = time_e2e(wl, max(20, args.steps // 10), 5)
+    (e2e_ms,) = max_over_ranks([e2e_ms], dist, dev)
+    e2e_value = job_throughput_gbs(wl.step_bytes, world, e2e_ms)
+    info = {"config": wl.config, "extra": wl.extra(call_ms), "kernel": wl.kernel_name,
+            "kernel_bytes": wl.kernel_bytes, "traffic_key": wl.traffic_key,
+            "launches": wl.launches_per_step}
+    del wl
+    torch.cuda.synchronize()
 
     workloads = None
     if not args.no_workloads and rank == 0:
-        workloads = other_workloads(dev, reps=20, peak=peak)
+        workloads = other_workloads(dev, args.workload, reps=20, peak=peak)
     if dist is not None:
         dist.barrier()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "long_decode":
         gbs, dt, sample = cpu_oracle_long_decode(steps=5)
         cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
                "seconds": dt}
 
     if rank == 0:
-        tok_head = wl.B * wl.H * wl.T / dec_ms * 1e3
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": "long_decode", "batch": wl.B, "n_q_heads": wl.Hq,
-                       "n_kv_heads": wl.H, "head_dim": 256, "ctx": wl.T,
-                       "step": "kvq_quantize_append(1 token) + kvq_decode_attn",
-                       "l2": "3 cache copies (453 MB) rotated per step, inputs > L2",
-                       "parallelism": f"replicas x{world}"},
+            "config": {**info["config"], "parallelism": f"replicas x{world}"},
             "frac_of_peak": value / world / peak,
-            "tok_head_per_s": tok_head, "tok_qhead_per_s": tok_head * wl.Hq / wl.H,
-            "roofline": {"bound": "hbm", "kernel": "kvq_decode_attn (split + combine launches)",
-                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
-                         "unit": "GB/s", "frac": achieved / peak,
-                         "algorithmic_bytes_per_launch": wl.decode_bytes(),
-                         "traffic": recorded_traffic("q4_decode_long")},
+            **info["extra"],
+            "roofline": {"bound": "hbm", "kernel": info["kernel"], "achieved": achieved,
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak,
+                         "algorithmic_bytes_per_launch": info["kernel_bytes"],
+                         "traffic": recorded_traffic(info["traffic_key"])},
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": wl.launches_per_step * args.steps,
+            "gpu_launches": info["launches"] * args.steps,
             "clocks": clk,
             "cpu_baseline": cpu,
             "workloads": workloads,

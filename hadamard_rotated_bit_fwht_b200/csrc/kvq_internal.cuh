@@ -29,10 +29,10 @@ __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w <
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // ---------------------------------------------------------------- packed fp32
-// Packed fp32x2 arithmetic through PTX instructions that carry an explicit
-// rounding modifier: ptxas never contracts those into a fused multiply-add,
-// so a product followed by a sum keeps its two roundings (the compiler
-// intrinsics of the same operations may be contracted).
+// Packed fp32x2 arithmetic through PTX instructions with an explicit rounding
+// modifier.  Used only where no multiply feeds an add (butterflies, scaling):
+// a packed multiply followed by a packed add has been observed to be fused
+// even with .rn, so that pattern uses the scalar __fmul_rn / __fadd_rn.
 __device__ __forceinline__ uint64_t pk(float2 a) {
   return (uint64_t)__float_as_uint(a.x) | ((uint64_t)__float_as_uint(a.y) << 32);
 }

@@ -34,28 +34,59 @@ __device__ void smem_fwht256(float *x, int n_vec) {
 }
 
 // Log-sum-exp combine of the splits and back-rotation; one CTA of 256 threads
-// per (sequence, q head).
+// per (sequence, q head).  The split maxima are reduced cooperatively, the
+// split weights exp2(m_s - M) are computed once into shared memory, and each
+// thread sums its dimension over the splits with independent loads.
+constexpr int kMaxSplitsSmem = 1024;
+
 __global__ void __launch_bounds__(256)
     q4_decode_combine_kernel(const float *__restrict__ ws, const int32_t *__restrict__ seq_lens,
                              int n_q_heads, int splits, int max_seq_len, int cap,
                              float *__restrict__ out) {
   __shared__ float ob[kDim];
-  const int bh = blockIdx.x, j = threadIdx.x;
+  __shared__ float wgt[kMaxSplitsSmem];
+  __shared__ float red[8];
+  const int bh = blockIdx.x, j = threadIdx.x, lane = j & 31, warp = j >> 5;
   const int b = bh / n_q_heads;
   const int len = min(max(__ldg(seq_lens + b), 0), min(max_seq_len, cap));
   const float *rec = ws + (int64_t)bh * splits * kRec;
+  const int ns = len > 0 ? min(splits, kMaxSplitsSmem) : 0;
+  // max over splits
   float M = -INFINITY;
-  for (int s = 0; s < splits && len > 0; s++) M = fmaxf(M, rec[s * kRec]);
-  float L = 0.f, O = 0.f;
-  if (len > 0 && M != -INFINITY) {
-    for (int s = 0; s < splits; s++) {
-      const float ms = rec[s * kRec];
-      if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - M);
-      L += rec[s * kRec + 1] * f;
-      O += rec[s * kRec + 4 + j] * f;
-    }
+  for (int s = j; s < ns; s += 256) M = fmaxf(M, __ldg(rec + (int64_t)s * kRec));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; w++) M = fmaxf(M, red[w]);
+  __syncthreads();
+  // split weights and the total
+  float L = 0.f;
+  for (int s = j; s < ns; s += 256) {
+    const float ms = __ldg(rec + (int64_t)s * kRec);
+    const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M);
+    wgt[s] = f;
+    L += f * __ldg(rec + (int64_t)s * kRec + 1);
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  if (lane == 0) red[warp] = L;
+  __syncthreads();
+  L = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; w++) L += red[w];
+  float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
+  int s = 0;
+  for (; s + 4 <= ns; s += 4) {
+    O0 += wgt[s] * __ldg(rec + (int64_t)s * kRec + 4 + j);
+    O1 += wgt[s + 1] * __ldg(rec + (int64_t)(s + 1) * kRec + 4 + j);
+    O2 += wgt[s + 2] * __ldg(rec + (int64_t)(s + 2) * kRec + 4 + j);
+    O3 += wgt[s + 3] * __ldg(rec + (int64_t)(s + 3) * kRec + 4 + j);
+  }
+  for (; s < ns; s++) O0 += wgt[s] * __ldg(rec + (int64_t)s * kRec + 4 + j);
+  const float O = (O0 + O1) + (O2 + O3);
   ob[j] = L > 0.f ? O / L : 0.f;
   smem_fwht256(ob, 1);
   out[(int64_t)bh * kDim + j] = ob[j] * 0.0625f;
@@ -73,6 +104,10 @@ DecodePlan plan_decode(int batch, int n_kv_heads, int max_seq_len) {
   if (per < 256) per = 256;
   p.split_tokens = per;
   p.splits = max(1, (max(max_seq_len, 1) + per - 1) / per);
+  while (p.splits > kMaxSplitsSmem) {  // very long contexts: larger splits
+    p.split_tokens *= 2;
+    p.splits = (max(max_seq_len, 1) + p.split_tokens - 1) / p.split_tokens;
+  }
   return p;
 }
 

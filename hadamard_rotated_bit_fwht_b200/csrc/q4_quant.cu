@@ -23,7 +23,8 @@
 //   the 16 nibble bytes of block i are regrouped through shared memory so
 //   each lane stores one 16-byte chunk.
 // Every fp32 operation is the IEEE round-to-nearest operation of the stated
-// sequence (explicit _rn intrinsics, no contraction), so codes and scales are
+// sequence (explicit-rounding PTX for the packed butterflies, scalar _rn
+// intrinsics where a product is followed by a sum), so codes and scales are
 // bit-identical to that sequence.
 #include "kvq_internal.cuh"
 
@@ -218,13 +219,17 @@ __device__ __forceinline__ void q4_quantize_l1(const float r[32], int lane, int 
   for (int B = 0; B < 8; B++) idb[B] = __shfl_sync(kFull, id, (lane & ~7) | B);
 
   uint32_t mq[32];
-  const float2 half8 = make_float2(8.5f, 8.5f), magic = make_float2(8388608.f, 8388608.f);
+  const float2 magic = make_float2(8388608.f, 8388608.f);
 #pragma unroll
   for (int k = 0; k < 16; k++) {
-    // register k belongs to block B = ((k >> 2) & 1) + 2 * (k >> 3); k + 16 to B + 4
+    // register k belongs to block B = ((k >> 2) & 1) + 2 * (k >> 3); k + 16 to B + 4.
+    // z * id and + 8.5 must round separately: scalar __fmul_rn / __fadd_rn are
+    // never merged into a multiply-add (the packed fp32x2 forms were observed
+    // to be, which moves a value sitting on a rounding tie).
     const int B = ((k >> 2) & 1) + 2 * (k >> 3);
-    float2 t = mul2(make_float2(r[k], r[k + 16]), make_float2(idb[B], idb[B + 4]));
-    t = add2(t, half8);
+    float2 t;
+    t.x = __fadd_rn(__fmul_rn(r[k], idb[B]), 8.5f);
+    t.y = __fadd_rn(__fmul_rn(r[k + 16], idb[B + 4]), 8.5f);
     float2 f = add2_rz(t, magic);  // 2^23 + floor(t), t >= 0
     mq[k] = min(__float_as_uint(f.x), 0x4B00000Fu);
     mq[k + 16] = min(__float_as_uint(f.y), 0x4B00000Fu);
