@@ -25,7 +25,7 @@ EXPORTED = (
     "kvq_status_string", "kvq_version", "kvq_rotate", "kvq_quantize_append",
     "kvq_decode_attn_workspace", "kvq_decode_attn", "kvq_octave_layout_of",
     "kvq_octave_codebook", "kvq_octave_quantize", "kvq_octave_decode_attn_workspace",
-    "kvq_octave_decode_attn",
+    "kvq_octave_decode_attn", "kvq_decode_attn_noalloc",
 )
 
 
@@ -92,6 +92,9 @@ def lib():
             C.c_int32, C.c_int32, C.c_int64, C.c_void_p, C.c_int32, C.c_int32, C.c_void_p,
             C.c_void_p, C.c_int32, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t,
             C.c_void_p]
+        L.kvq_decode_attn_noalloc.argtypes = [C.POINTER(CacheDesc), C.c_void_p, C.c_int, C.c_int32,
+                                              C.c_int32, C.c_void_p, C.c_int32, C.c_float,
+                                              C.c_void_p, C.c_void_p]
         _lib = L
     return _lib
 
@@ -241,6 +244,26 @@ def decode_attn(cache: Q4Cache, q: torch.Tensor, seq_lens: torch.Tensor, max_seq
            lib().kvq_decode_attn(C.byref(d), _ptr(q), _dtype_code(q), batch, hq, _ptr(seq_lens),
                                  int(max_seq_len), float(scale), _ptr(out), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def decode_attn_noalloc(cache: Q4Cache, q: torch.Tensor, seq_lens: torch.Tensor,
+                        max_seq_len: int, scale: float, out: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """decode_attn with the split-K scratch taken from the library's fixed
+    device array instead of a caller workspace (kvq_decode_attn_noalloc)."""
+    _cuda_contig("q", q)
+    _cuda_contig("seq_lens", seq_lens)
+    if seq_lens.dtype != torch.int32:
+        raise TypeError("seq_lens must be int32")
+    batch, hq, dim = q.shape
+    if out is None:
+        out = torch.empty((batch, hq, dim), dtype=torch.float32, device=q.device)
+    d = cache.desc()
+    _check("kvq_decode_attn_noalloc",
+           lib().kvq_decode_attn_noalloc(C.byref(d), _ptr(q), _dtype_code(q), batch, hq,
+                                         _ptr(seq_lens), int(max_seq_len), float(scale),
+                                         _ptr(out), _stream(stream)))
     return out
 
 

@@ -157,6 +157,33 @@ KVQ_API kvq_status kvq_decode_attn(const kvq_cache *cache, const void *q, kvq_dt
                            float *out, void *workspace, size_t workspace_bytes,
                            void *stream);
 
+/* kvq_decode_attn_noalloc -- kvq_decode_attn without a caller-provided
+ * workspace.  (The pages have no counterpart: this is an interface
+ * convenience, not part of the method.)
+ * Some callers cannot hand the library device scratch memory: a plugin
+ * interface that passes only the input and output tensors, a C host program
+ * without a device allocator, or a latency-critical decode loop that must
+ * never call cudaMalloc (slow, and it can synchronize the device).  This call
+ * allocates nothing: its split-K partials live in a fixed device array inside
+ * the library, KVQ_DECODE_NOALLOC_SCRATCH_BYTES large, which every GPU that
+ * loads the library holds until the process exits.
+ *   Arguments, layouts and results are those of kvq_decode_attn.
+ *   A shape whose workspace (kvq_decode_attn_workspace) exceeds
+ *   KVQ_DECODE_NOALLOC_SCRATCH_BYTES returns KVQ_ERR_WORKSPACE before any
+ *   launch; use kvq_decode_attn with a workspace for such shapes.
+ *   The first call on a device looks up the array's device address with that
+ *   device current (KVQ_ERR_CUDA if the lookup fails); make that first call
+ *   before any stream capture.
+ *   All calls on a device share the one array: every call overwrites the
+ *   records it reads, so nothing carries over from the previous call, but two
+ *   calls whose kernels overlap on the GPU (different streams, no ordering
+ *   between them) race on it and give undefined results. */
+#define KVQ_DECODE_NOALLOC_SCRATCH_BYTES (8u << 20)
+KVQ_API kvq_status kvq_decode_attn_noalloc(const kvq_cache *cache, const void *q,
+                                           kvq_dtype dtype, int32_t batch, int32_t num_q_heads,
+                                           const int32_t *d_seq_lens, int32_t max_seq_len,
+                                           float scale, float *out, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Octave variant (vLLM API page "vllm.v1.attention.ops.rocm_octave")        */
 /* ------------------------------------------------------------------------ */
