@@ -159,6 +159,8 @@ kvq_status kvq_quantize_append(const kvq_cache *cache, const void *k, const void
   if (!cache->block_table && batch > cache->batch_capacity) return KVQ_ERR_INVALID_ARG;
   if (batch == 0 || t_new == 0) return KVQ_OK;
   if (!k || !v || !d_start_pos || !aligned(k, 16) || !aligned(v, 16)) return KVQ_ERR_INVALID_ARG;
+  // the kernel indexes the 2 * batch * t_new * heads vectors with 31-bit counts
+  if (2LL * batch * t_new * cache->num_kv_heads >= (1LL << 31)) return KVQ_ERR_UNSUPPORTED;
   return from_cuda(launch_q4_append(*cache, k, v, dtype == KVQ_BF16, batch, t_new, d_start_pos,
                                     as_stream(stream)));
 }

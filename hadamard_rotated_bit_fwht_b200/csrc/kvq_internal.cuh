@@ -29,31 +29,21 @@ __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w <
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // ---------------------------------------------------------------- packed fp32
-// Packed fp32x2 arithmetic through PTX instructions with an explicit rounding
-// modifier.  Used only where no multiply feeds an add (butterflies, scaling):
-// a packed multiply followed by a packed add has been observed to be fused
-// even with .rn, so that pattern uses the scalar __fmul_rn / __fadd_rn.
+// Packed fp32x2 arithmetic.  Used only where no multiply feeds an add
+// (butterflies, end scaling, the round-toward-zero add): a packed multiply
+// followed by a packed add has been observed to be fused into one rounding
+// even with an explicit .rn, so that pattern uses scalar __fmul_rn / __fadd_rn.
 __device__ __forceinline__ uint64_t pk(float2 a) {
   return (uint64_t)__float_as_uint(a.x) | ((uint64_t)__float_as_uint(a.y) << 32);
 }
 __device__ __forceinline__ float2 upk(uint64_t v) {
   return make_float2(__uint_as_float((uint32_t)v), __uint_as_float((uint32_t)(v >> 32)));
 }
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
-  return upk(r);
-}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-  uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
-  return upk(r);
+  return __fadd2_rn(a, make_float2(-b.x, -b.y));
 }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
-  return upk(r);
-}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 add2_rz(float2 a, float2 b) {
   uint64_t r;
   asm("add.rz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
@@ -86,6 +76,7 @@ struct DecodePlan {
   int split_tokens; // tokens per split (multiple of 64)
 };
 DecodePlan plan_decode(int batch, int n_kv_heads, int max_seq_len);
+int q4_decode_ctas_per_sm();
 cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, int batch,
                                  int n_q_heads, const int32_t *seq_lens, int max_seq_len,
                                  float scale, float *ws, const DecodePlan &p, cudaStream_t s);
@@ -108,6 +99,14 @@ cudaError_t launch_octave_quantize(const OctaveParams &p, const void *key, const
                                    const int64_t *slot_mapping, uint8_t *cache,
                                    int block_size, int64_t num_blocks, cudaStream_t s);
 DecodePlan plan_octave_decode(int num_q, int n_kv_heads, int max_klen);
+bool octave_mma_supported(const OctaveParams &p);
+cudaError_t launch_octave_decode_mma(const OctaveParams &P, const void *query, int bf16, int num_q,
+                                     int n_q_heads, const uint8_t *cache, int n_kv_heads,
+                                     int block_size, int64_t num_blocks,
+                                     const int32_t *block_table, int num_reqs, int max_blocks,
+                                     const int32_t *q_to_req, const int32_t *q_to_klen,
+                                     int max_klen, float scale, float *ws,
+                                     const DecodePlan &plan, cudaStream_t s);
 size_t octave_workspace_bytes(int num_q, int n_q_heads, int head_size, const DecodePlan &p);
 cudaError_t launch_octave_decode(const OctaveParams &p, const void *query, int bf16, int num_q,
                                  int n_q_heads, const uint8_t *cache, int n_kv_heads,

@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(256)
 DecodePlan plan_decode(int batch, int n_kv_heads, int max_seq_len) {
   DecodePlan p;
   const int units = max(batch * n_kv_heads, 1);
-  const int target = kNumSMs * 2;  // resident CTAs of the tensor-core split kernel
+  const int target = kNumSMs * q4_decode_ctas_per_sm();  // one wave of split CTAs
   int splits = max(1, (target + units - 1) / units);
   int per = (max(max_seq_len, 1) + splits - 1) / splits;
   per = ((per + 63) / 64) * 64;

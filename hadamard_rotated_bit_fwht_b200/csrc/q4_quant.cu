@@ -38,18 +38,40 @@ constexpr int kVecPerCta = kWarps * kVecPerWarp;
 constexpr unsigned kFull = 0xffffffffu;
 
 // ------------------------------------------------------------------ load (L0)
+// 16-byte chunks per lane: bf16 -> 4 chunks (8 values each), fp32 -> 8 chunks.
 template <bool BF16>
-__device__ __forceinline__ void load_l0(const void *vec, int i, bool valid, float r[32]) {
+struct Raw {
+  uint4 w[BF16 ? 4 : 8];
+};
+
+template <bool BF16>
+__device__ __forceinline__ void fetch_raw(const void *vec, int i, bool valid, Raw<BF16> &raw) {
   if (!valid) {
 #pragma unroll
-    for (int k = 0; k < 32; k++) r[k] = 0.f;
+    for (int j = 0; j < (BF16 ? 4 : 8); j++) raw.w[j] = make_uint4(0u, 0u, 0u, 0u);
     return;
   }
   if (BF16) {
     const uint16_t *p = static_cast<const uint16_t *>(vec);
 #pragma unroll
+    for (int j = 0; j < 4; j++) raw.w[j] = ldg_stream_u4(p + 8 * (i + 8 * j));
+  } else {
+    const float *p = static_cast<const float *>(vec);
+#pragma unroll
     for (int j = 0; j < 4; j++) {
-      uint4 w = ldg_stream_u4(p + 8 * (i + 8 * j));
+      raw.w[2 * j] = ldg_stream_u4(p + 8 * (i + 8 * j));
+      raw.w[2 * j + 1] = ldg_stream_u4(p + 8 * (i + 8 * j) + 4);
+    }
+  }
+}
+
+// L0: lane i holds x[u + 8i + 64j] in r[u + 8j]
+template <bool BF16>
+__device__ __forceinline__ void unpack_l0(const Raw<BF16> &raw, float r[32]) {
+#pragma unroll
+  for (int j = 0; j < 4; j++) {
+    if (BF16) {
+      const uint4 w = raw.w[j];
       r[8 * j + 0] = bf16lo(w.x);
       r[8 * j + 1] = bf16hi(w.x);
       r[8 * j + 2] = bf16lo(w.y);
@@ -58,13 +80,8 @@ __device__ __forceinline__ void load_l0(const void *vec, int i, bool valid, floa
       r[8 * j + 5] = bf16hi(w.z);
       r[8 * j + 6] = bf16lo(w.w);
       r[8 * j + 7] = bf16hi(w.w);
-    }
-  } else {
-    const float *p = static_cast<const float *>(vec);
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-      uint4 a = ldg_stream_u4(p + 8 * (i + 8 * j));
-      uint4 b = ldg_stream_u4(p + 8 * (i + 8 * j) + 4);
+    } else {
+      const uint4 a = raw.w[2 * j], b = raw.w[2 * j + 1];
       r[8 * j + 0] = __uint_as_float(a.x);
       r[8 * j + 1] = __uint_as_float(a.y);
       r[8 * j + 2] = __uint_as_float(a.z);
@@ -124,12 +141,9 @@ __device__ __forceinline__ void transpose_l0_l1(float r[32], float4 *buf, int i)
   __syncwarp();
 }
 
-// Full FWHT-256 of the 4 vectors of this warp: load, stages, transpose,
-// stages, end scaling.  Leaves layout L1.
-template <bool BF16>
-__device__ __forceinline__ void fwht256_warp(const void *vec, bool valid, int i, float4 *buf,
-                                             float r[32]) {
-  load_l0<BF16>(vec, i, valid, r);
+// Full FWHT-256 of the 4 vectors of this warp from layout L0: stages,
+// transpose, stages, end scaling.  Leaves layout L1.
+__device__ __forceinline__ void fwht256_warp(int i, float4 *buf, float r[32]) {
   bfly_packed<1>(r);  // h = 1
   bfly_packed<2>(r);  // h = 2
   bfly_packed<4>(r);  // h = 4
@@ -162,8 +176,11 @@ __global__ void __launch_bounds__(kThreads) rotate_kernel(const void *__restrict
     const bool valid = v < n_vec;
     const size_t esz = BF16 ? 2 : 4;
     const void *src = static_cast<const char *>(x) + (valid ? v : 0) * kDim * esz;
+    Raw<BF16> raw;
+    fetch_raw<BF16>(src, i, valid, raw);
     float r[32];
-    fwht256_warp<BF16>(src, valid, i, buf, r);
+    unpack_l0<BF16>(raw, r);
+    fwht256_warp(i, buf, r);
     if (valid) {
       float *dst = y + v * kDim;
 #pragma unroll
@@ -175,16 +192,20 @@ __global__ void __launch_bounds__(kThreads) rotate_kernel(const void *__restrict
 }
 
 // ------------------------------------------------------------------ quantize
-// Max-abs key of a value: rotl(bits, 1) ^ 1 orders values by |z| first and puts
-// the positive one above the negative one of equal magnitude, so the maximum
-// key over a block is the element the sequential tie-break scan keeps.  The
-// start value (amax = 0, mval = +0) has key 1.
-__device__ __forceinline__ uint32_t amax_key(float z) {
-  uint32_t b = __float_as_uint(z);
-  return __funnelshift_l(b, b, 1) ^ 1u;
-}
+// The tie-break scan (start (amax, mval) = (0, +0); take z when |z| > amax, or
+// |z| == amax and z > mval) ends on the lexicographic maximum of (|z|, z).
+// Each lane reduces its 4 values of a block to amax_t = max |z| and a flag
+// "+amax_t occurs"; the key (bits(amax_t) << 1) | flag orders exactly like
+// (|z|, z), so the maximum key over the 8 lanes identifies mval.  An all-zero
+// block gives key 1, i.e. mval = +0, like the scan.
 __device__ __forceinline__ float key_value(uint32_t key) {
   return __uint_as_float((key >> 1) | ((~key & 1u) << 31));
+}
+
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
 struct QuantOut {
@@ -198,10 +219,11 @@ __device__ __forceinline__ void q4_quantize_l1(const float r[32], int lane, int 
   uint32_t key[8];
 #pragma unroll
   for (int B = 0; B < 8; B++) {
-    uint32_t k = 1u;
-#pragma unroll
-    for (int m = 0; m < 4; m++) k = max(k, amax_key(r[4 * (B & 1) + m + 8 * (B >> 1)]));
-    key[B] = k;
+    const int r0 = 4 * (B & 1) + 8 * (B >> 1);
+    const float z0 = r[r0], z1 = r[r0 + 1], z2 = r[r0 + 2], z3 = r[r0 + 3];
+    const float am = fmaxf(fmaxf(fabsf(z0), fabsf(z1)), fmaxf(fabsf(z2), fabsf(z3)));
+    const float mz = fmaxf(fmaxf(z0, z1), fmaxf(z2, z3));
+    key[B] = (__float_as_uint(am) << 1) | (mz == am ? 1u : 0u);
   }
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1)
@@ -218,29 +240,25 @@ __device__ __forceinline__ void q4_quantize_l1(const float r[32], int lane, int 
 #pragma unroll
   for (int B = 0; B < 8; B++) idb[B] = __shfl_sync(kFull, id, (lane & ~7) | B);
 
-  uint32_t mq[32];
   const float2 magic = make_float2(8388608.f, 8388608.f);
-#pragma unroll
-  for (int k = 0; k < 16; k++) {
-    // register k belongs to block B = ((k >> 2) & 1) + 2 * (k >> 3); k + 16 to B + 4.
-    // z * id and + 8.5 must round separately: scalar __fmul_rn / __fadd_rn are
-    // never merged into a multiply-add (the packed fp32x2 forms were observed
-    // to be, which moves a value sitting on a rounding tie).
-    const int B = ((k >> 2) & 1) + 2 * (k >> 3);
-    float2 t;
-    t.x = __fadd_rn(__fmul_rn(r[k], idb[B]), 8.5f);
-    t.y = __fadd_rn(__fmul_rn(r[k + 16], idb[B + 4]), 8.5f);
-    float2 f = add2_rz(t, magic);  // 2^23 + floor(t), t >= 0
-    mq[k] = min(__float_as_uint(f.x), 0x4B00000Fu);
-    mq[k + 16] = min(__float_as_uint(f.y), 0x4B00000Fu);
-  }
+  const uint32_t fifteen = 0x000F000Fu;
 #pragma unroll
   for (int B = 0; B < 8; B++) {
     const int r0 = 4 * (B & 1) + 8 * (B >> 1);
-    // element-in-block i + 8m: byte i = m0 | m2 << 4, byte i + 8 = m1 | m3 << 4
-    uint32_t lo = (mq[r0 + 0] & 15u) | ((mq[r0 + 2] & 15u) << 4);
-    uint32_t hi = (mq[r0 + 1] & 15u) | ((mq[r0 + 3] & 15u) << 4);
-    o.items[B] = lo | (hi << 8);
+    // z * id and + 8.5 round separately: scalar __fmul_rn / __fadd_rn are
+    // never merged into a multiply-add (the packed fp32x2 forms were observed
+    // to be, which moves a value sitting on a rounding tie).
+    float t[4];
+#pragma unroll
+    for (int m = 0; m < 4; m++) t[m] = __fadd_rn(__fmul_rn(r[r0 + m], idb[B]), 8.5f);
+    // 2^23 + floor(t) for t >= 0; the low 16 bits are floor(t) in 0..16
+    const float2 f02 = add2_rz(make_float2(t[0], t[2]), magic);
+    const float2 f13 = add2_rz(make_float2(t[1], t[3]), magic);
+    // element-in-block i + 8m: byte i = c0 | c2 << 4, byte i + 8 = c1 | c3 << 4
+    const uint32_t x02 = min_u16x2(__byte_perm(__float_as_uint(f02.x), __float_as_uint(f02.y), 0x5410), fifteen);
+    const uint32_t x13 = min_u16x2(__byte_perm(__float_as_uint(f13.x), __float_as_uint(f13.y), 0x5410), fifteen);
+    const uint32_t y02 = x02 | (x02 >> 12), y13 = x13 | (x13 >> 12);
+    o.items[B] = __byte_perm(y02, y13, 0x0040);  // (byte i, byte i + 8) in the low 16 bits
   }
 }
 
@@ -260,10 +278,23 @@ __device__ __forceinline__ uint4 gather_block_bytes(const QuantOut &o, uint8_t *
   return out;
 }
 
+// n / d for n < 2^31 by one 64-bit multiply: m = ceil(2^(31+p) / d) with
+// 2^(p-1) < d <= 2^p gives floor(n * m / 2^(31+p)) = floor(n / d).
+struct FastDiv {
+  uint64_t m;
+  uint32_t shift;
+  uint32_t d;
+};
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
+  return (uint32_t)(((uint64_t)n * f.m) >> f.shift);
+}
+
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads)
     q4_append_kernel(kvq_cache c, const void *__restrict__ k, const void *__restrict__ v,
-                     int batch, int t_new, const int32_t *__restrict__ start_pos) {
+                     int batch, int t_new, const int32_t *__restrict__ start_pos,
+                     FastDiv div_heads, FastDiv div_tnew) {
   __shared__ float4 smem[kWarps][kVecPerWarp][64];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int vg = lane >> 3, i = lane & 7;
@@ -271,26 +302,47 @@ __global__ void __launch_bounds__(kThreads)
   // code regrouping reuses 128 bytes of this vector's buffer, offset by 16
   // bytes per vector so the four vectors of a warp use different banks
   uint8_t *stage = reinterpret_cast<uint8_t *>(buf) + 16 * vg;
-  const int64_t per_tensor = (int64_t)batch * t_new * c.num_kv_heads;
-  const int64_t n_vec = 2 * per_tensor;
-  const int64_t ngroups = (n_vec + kVecPerCta - 1) / kVecPerCta;
-  const size_t esz = BF16 ? 2 : 4;
-  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
-    const int64_t vid = g * kVecPerCta + warp * kVecPerWarp + vg;
-    bool valid = vid < n_vec;
-    const bool is_v = valid && vid >= per_tensor;
-    const int64_t e = valid ? (is_v ? vid - per_tensor : vid) : 0;
-    const void *src = static_cast<const char *>(is_v ? v : k) + e * kDim * esz;
+  // counts fit in 31 bits (checked on the host)
+  const uint32_t per_tensor = (uint32_t)batch * (uint32_t)t_new * (uint32_t)c.num_kv_heads;
+  const uint32_t n_vec = 2u * per_tensor;
+  const uint32_t ngroups = (n_vec + kVecPerCta - 1) / kVecPerCta;
+  constexpr size_t esz = BF16 ? 2 : 4;
+  auto source = [&](uint32_t vid) -> const void * {
+    const bool is_v = vid >= per_tensor;
+    const uint32_t e = is_v ? vid - per_tensor : vid;
+    return static_cast<const char *>(is_v ? v : k) + (size_t)e * kDim * esz;
+  };
+  // the next group's input is fetched before the current one is processed
+  Raw<BF16> raw;
+  uint32_t g = blockIdx.x;
+  {
+    const uint32_t vid = g * kVecPerCta + warp * kVecPerWarp + vg;
+    const bool valid = g < ngroups && vid < n_vec;
+    fetch_raw<BF16>(valid ? source(vid) : k, i, valid, raw);
+  }
+  for (; g < ngroups; g += gridDim.x) {
+    const uint32_t vid = g * kVecPerCta + warp * kVecPerWarp + vg;
+    const bool valid = vid < n_vec;
     float r[32];
-    fwht256_warp<BF16>(src, valid, i, buf, r);
+    unpack_l0<BF16>(raw, r);
+    {
+      const uint32_t gn = g + gridDim.x;
+      const uint32_t vn = gn * kVecPerCta + warp * kVecPerWarp + vg;
+      const bool vnext = gn < ngroups && vn < n_vec;
+      fetch_raw<BF16>(vnext ? source(vn) : k, i, vnext, raw);
+    }
+    fwht256_warp(i, buf, r);
     QuantOut o;
     q4_quantize_l1(r, lane, i, o);
     uint4 bytes = gather_block_bytes(o, stage, i);
     if (valid) {
-      const int h = (int)(e % c.num_kv_heads);
-      const int64_t bt = e / c.num_kv_heads;
-      const int tok = (int)(bt % t_new), b = (int)(bt / t_new);
-      const int64_t row = q4_row(c, b, h, __ldg(start_pos + b) + tok);
+      const bool is_v = vid >= per_tensor;
+      const uint32_t e = is_v ? vid - per_tensor : vid;
+      const uint32_t bt = fdiv(e, div_heads);
+      const int h = (int)(e - bt * div_heads.d);
+      const uint32_t b = fdiv(bt, div_tnew);
+      const int tok = (int)(bt - b * div_tnew.d);
+      const int64_t row = q4_row(c, (int)b, h, __ldg(start_pos + b) + tok);
       if (row >= 0) {
         uint8_t *codes = (is_v ? c.v_codes : c.k_codes) + row * kRowCodeBytes;
         uint16_t *scales = (is_v ? c.v_scales : c.k_scales) + row * kRowScales;
@@ -299,6 +351,16 @@ __global__ void __launch_bounds__(kThreads)
       }
     }
   }
+}
+
+FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  uint32_t p = 0;
+  while ((1u << p) < d) p++;
+  f.shift = 31 + p;
+  f.m = (((uint64_t)1 << f.shift) + d - 1) / d;
+  f.d = d;
+  return f;
 }
 
 int grid_for(int64_t groups) {
@@ -321,8 +383,11 @@ cudaError_t launch_q4_append(const kvq_cache &c, const void *k, const void *v, i
   const int64_t n_vec = 2LL * batch * t_new * c.num_kv_heads;
   if (n_vec == 0) return cudaSuccess;
   const int grid = grid_for((n_vec + kVecPerCta - 1) / kVecPerCta);
-  if (bf16) q4_append_kernel<true><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos);
-  else q4_append_kernel<false><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos);
+  const FastDiv dh = make_fastdiv((uint32_t)c.num_kv_heads), dt = make_fastdiv((uint32_t)t_new);
+  if (bf16)
+    q4_append_kernel<true><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
+  else
+    q4_append_kernel<false><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
   return cudaGetLastError();
 }
 

@@ -123,7 +123,9 @@ KVQ_API kvq_status kvq_rotate(const void *x, kvq_dtype dtype, float *y, int64_t 
  * per 32-value block d = mval / -8, id = d ? 1/d : 0,
  * code = min(15, trunc(z * id + 8.5)) (product and sum rounded separately),
  * scale = fp16(d) (round to nearest even).
- * batch must be <= batch_capacity for a contiguous cache. */
+ * batch must be <= batch_capacity for a contiguous cache; one call handles
+ * fewer than 2^30 vectors per tensor (batch * t_new * num_kv_heads),
+ * KVQ_ERR_UNSUPPORTED otherwise. */
 KVQ_API kvq_status kvq_quantize_append(const kvq_cache *cache, const void *k, const void *v,
                                kvq_dtype dtype, int32_t batch, int32_t t_new,
                                const int32_t *d_start_pos, void *stream);
