@@ -165,10 +165,16 @@ kvq_status kvq_quantize_append(const kvq_cache *cache, const void *k, const void
                                     as_stream(stream)));
 }
 
+// CTAs per (sequence, split): q heads in groups of at most 8 per kv head
+static int head_groups(int num_q_heads, int num_kv_heads) {
+  const int group = num_q_heads / num_kv_heads;
+  return num_q_heads / (group < 8 ? (group > 0 ? group : 1) : 8);
+}
+
 size_t kvq_decode_attn_workspace(const kvq_cache *cache, int32_t batch, int32_t num_q_heads,
                                  int32_t max_seq_len) {
   if (!cache || batch <= 0 || num_q_heads <= 0 || cache->num_kv_heads <= 0) return 0;
-  DecodePlan p = plan_decode(batch, cache->num_kv_heads, max_seq_len);
+  DecodePlan p = plan_decode(batch, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len);
   return decode_workspace_bytes(batch, num_q_heads, p);
 }
 
@@ -187,7 +193,7 @@ kvq_status kvq_decode_attn(const kvq_cache *cache, const void *q, kvq_dtype dtyp
   if (!isfinite(scale)) return KVQ_ERR_INVALID_ARG;
   if (batch == 0) return KVQ_OK;
   if (!q || !d_seq_lens || !out) return KVQ_ERR_INVALID_ARG;
-  DecodePlan p = plan_decode(batch, cache->num_kv_heads, max_seq_len);
+  DecodePlan p = plan_decode(batch, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len);
   const size_t need = decode_workspace_bytes(batch, num_q_heads, p);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return KVQ_ERR_WORKSPACE;
   return from_cuda(launch_q4_decode(*cache, q, dtype == KVQ_BF16, batch, num_q_heads, d_seq_lens,
@@ -227,9 +233,11 @@ kvq_status kvq_octave_quantize(const kvq_octave_fmt *fmt, const void *key, const
 size_t kvq_octave_decode_attn_workspace(const kvq_octave_fmt *fmt, int32_t num_q,
                                         int32_t num_q_heads, int32_t max_klen) {
   if (!fmt || num_q <= 0 || num_q_heads <= 0) return 0;
-  // the split plan depends on num_q * num_kv_heads; size for the worst case
-  // (one kv head) so any valid head count fits
-  DecodePlan p = plan_octave_decode(num_q, 1, max_klen);
+  // the split plan depends on the kv head count, unknown here: size for the
+  // most splits any plan makes (256-token splits)
+  DecodePlan p;
+  p.splits = (max(max_klen, 1) + 255) / 256;
+  p.split_tokens = 256;
   return octave_workspace_bytes(num_q, num_q_heads, fmt->head_size, p);
 }
 
@@ -255,7 +263,7 @@ kvq_status kvq_octave_decode_attn(const kvq_octave_fmt *fmt, const void *query, 
   if (!query || !cache || !d_block_table || !d_q_to_req || !d_q_to_klen || !out ||
       !aligned(cache, 4))
     return KVQ_ERR_INVALID_ARG;
-  DecodePlan plan = plan_octave_decode(num_q, num_kv_heads, max_klen);
+  DecodePlan plan = plan_octave_decode(num_q, head_groups(num_q_heads, num_kv_heads), max_klen);
   const size_t need = octave_workspace_bytes(num_q, num_q_heads, fmt->head_size, plan);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return KVQ_ERR_WORKSPACE;
   return from_cuda(launch_octave_decode(p, query, dtype == KVQ_BF16, num_q, num_q_heads, cache,

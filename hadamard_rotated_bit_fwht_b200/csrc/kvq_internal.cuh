@@ -75,7 +75,10 @@ struct DecodePlan {
   int splits;       // splits per (sequence, kv head)
   int split_tokens; // tokens per split (multiple of 64)
 };
-DecodePlan plan_decode(int batch, int n_kv_heads, int max_seq_len);
+// split-K plan over `units` independent problems with `slots` resident CTAs
+DecodePlan plan_split_k(int units, int max_len, int slots, int max_splits);
+// n_head_groups: q heads / min(group, 8), the CTAs per sequence and split
+DecodePlan plan_decode(int batch, int n_head_groups, int max_seq_len);
 int q4_decode_ctas_per_sm();
 cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, int batch,
                                  int n_q_heads, const int32_t *seq_lens, int max_seq_len,
@@ -98,7 +101,7 @@ cudaError_t launch_octave_quantize(const OctaveParams &p, const void *key, const
                                    int bf16, int num_tokens, int n_kv_heads,
                                    const int64_t *slot_mapping, uint8_t *cache,
                                    int block_size, int64_t num_blocks, cudaStream_t s);
-DecodePlan plan_octave_decode(int num_q, int n_kv_heads, int max_klen);
+DecodePlan plan_octave_decode(int num_q, int n_head_groups, int max_klen);
 bool octave_mma_supported(const OctaveParams &p);
 cudaError_t launch_octave_decode_mma(const OctaveParams &P, const void *query, int bf16, int num_q,
                                      int n_q_heads, const uint8_t *cache, int n_kv_heads,

@@ -449,17 +449,8 @@ cudaError_t launch_octave_quantize(const OctaveParams &p, const void *key, const
   return cudaGetLastError();
 }
 
-DecodePlan plan_octave_decode(int num_q, int n_kv_heads, int max_klen) {
-  DecodePlan p;
-  const int units = max(num_q * n_kv_heads, 1);
-  const int target = kNumSMs * 4;
-  int splits = max(1, (target + units - 1) / units);
-  int per = (max(max_klen, 1) + splits - 1) / splits;
-  per = ((per + 63) / 64) * 64;
-  if (per < 256) per = 256;
-  p.split_tokens = per;
-  p.splits = max(1, (max(max_klen, 1) + per - 1) / per);
-  return p;
+DecodePlan plan_octave_decode(int num_q, int n_head_groups, int max_klen) {
+  return plan_split_k(num_q * n_head_groups, max_klen, kNumSMs * 4, 1 << 20);
 }
 
 size_t octave_workspace_bytes(int num_q, int n_q_heads, int head_size, const DecodePlan &p) {
@@ -478,6 +469,18 @@ cudaError_t launch_octave_decode(const OctaveParams &P, const void *query, int b
   const int gc = group < 8 ? group : 8;
   dim3 grid(plan.splits, n_q_heads / gc, num_q);
   const float sl2 = scale * kLog2e;
+  if (octave_mma_supported(P)) {  // k3v4, head 128, rope 64: tensor-core split kernel
+    cudaError_t e = launch_octave_decode_mma(P, query, bf16, num_q, n_q_heads, cache, n_kv_heads,
+                                             block_size, num_blocks, block_table, num_reqs,
+                                             max_blocks, q_to_req, q_to_klen, max_klen, scale, ws,
+                                             plan, s);
+    if (e != cudaSuccess) return e;
+    octave_combine_kernel<<<num_q * n_q_heads, kHead, 0, s>>>(P, ws, q_to_req, q_to_klen,
+                                                             num_reqs, n_q_heads, plan.splits,
+                                                             max_klen, max_blocks * block_size,
+                                                             out);
+    return cudaGetLastError();
+  }
 #define KVQ_LAUNCH(G)                                                                         \
   do {                                                                                        \
     if (bf16)                                                                                 \

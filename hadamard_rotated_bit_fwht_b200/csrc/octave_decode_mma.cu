@@ -1,0 +1,529 @@
+// octave_decode_mma.cu -- tensor-core split-K decode over the Octave cache
+// (vLLM API page "vllm.v1.attention.ops.rocm_octave": module text -- scores in
+// the rotated space, output rotated back once per query head -- and
+// reference_attention), for the k3v4 format with head 128 and rope 64:
+//   slot bytes  0..31  K RoPE block, 4-bit codes (word w: byte j = dims 8w+j | 8w+j+4 << 4)
+//              32..55  K NoPE block, 3-bit codes (2-bit plane 32..47, 1-bit plane 48..55)
+//              56..119 V, 4-bit codes over 128 dims
+//             120..125 fp16 scales: K RoPE, K NoPE, V.
+// A code c of a block with scale s stands for LUT[c] * s / 64.
+//   * QK on the integer tensor path (mma.sync m16n8k32, s8 x s8 -> s32).  The
+//     signed int8 codebook sits in registers; prmt selects four table bytes at
+//     a time from nibble-packed codes (two 8-entry halves plus a
+//     sign-replicated mask for 4-bit codes, one prmt for 3-bit codes), and
+//     those bytes are B-fragment registers as they stand.  The rotated query
+//     of each head is scaled by S = 127 * 128 / max|q| and split exactly into
+//     int8 H and L (S q = 128 H + L, |L| <= 64), rows 0-7 H and rows 8-15 L;
+//     its columns are stored in the order the codes arrive in.  Per (block,
+//     8 tokens) 128 d_H + d_L is the exact integer dot product, converted to
+//     fp32 once and multiplied by the block scale; 1 / S joins the softmax
+//     scale.  The query is thereby carried to 3e-5 of its largest element.
+//   * PV on the fp16 path (m16n8k16, fp32 accumulation): A = V^T codes through
+//     the biased table (each byte u becomes the exact fp16 1024 + u by pairing
+//     it with 0x64; one half2 subtract of 1152 leaves LUT[c]), read by
+//     ldmatrix.trans from the swizzled tile; B = p * s_v / 64 split hi + lo.
+//     The V region starts 8 bytes into a 16-byte chunk: the used halves of
+//     chunks 3 and 7 are joined by one lane shuffle, so the 64 V bytes make
+//     exactly 8 M-tiles.
+// Tiles of 64 slots (one 128-byte row per token) are staged by cp.async with
+// the 128-byte XOR swizzle through a 3-stage ring; each row is addressed
+// through the block table by one lookup, so any block size works, and a
+// token whose block entry names no block contributes nothing.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kTile = 64;
+constexpr int kStages = 3;
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kHead = 128;
+constexpr int kORec = 132;  // m, l, pad, pad, o[128]
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kQRange = 16256.f;  // 127 * 128
+constexpr int kStageBytes = kTile * 128;
+constexpr int kOffF = kStages * kStageBytes;  // fp32 scales [3][64] of the current tile
+constexpr int kOffV = kOffF + 3 * kTile * 4;  // per stage, per token: 1 if its block is mapped
+constexpr int kQStride = 144;                 // int8 query row: 128 B + 16 B pad
+constexpr int kOffQ = kOffV + kStages * kTile;  // int8 query rows (0-7 H, 8-15 L)
+constexpr int kSmemBytes = kOffQ + 16 * kQStride;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t (&r)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// d += A(s8, 16 x 32) * B(s8, 32 x 8)
+__device__ __forceinline__ void imma16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(s));
+  return r;
+}
+__device__ __forceinline__ uint32_t lop3_sel(uint32_t lo, uint32_t hi, uint32_t m) {
+  uint32_t r;  // m ? hi : lo, bitwise
+  asm("lop3.b32 %0, %1, %2, %3, 0xD8;" : "=r"(r) : "r"(lo), "r"(hi), "r"(m));
+  return r;
+}
+
+// Table bytes T[c] for four nibble-packed 4-bit codes (sel bits 0-15): two
+// 8-entry lookups on the low three bits, then a per-byte choice by the fourth
+// bit (sign-replicated into a mask by prmt).
+struct Lut4 {
+  uint32_t lo0, lo1, hi0, hi1;
+};
+__device__ __forceinline__ uint32_t lut4_bytes(uint32_t sel, const Lut4 &T) {
+  const uint32_t s = sel & 0x7777u;
+  const uint32_t plo = prmt(T.lo0, T.lo1, s);
+  const uint32_t phi = prmt(T.hi0, T.hi1, s);
+  const uint32_t m = prmt(sel << 4, sel, 0xD9C8u);
+  return lop3_sel(plo, phi, m);
+}
+// biased bytes (a, b) of R -> half2 (LUT, LUT) exactly: (1024 + U) - 1152
+__device__ __forceinline__ uint32_t lut_half2(uint32_t R, uint32_t selector) {
+  const uint32_t h = prmt(R, 0x64646464u, selector);
+  const __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&h),
+                            __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+__device__ __forceinline__ void split_hilo(float2 w, uint32_t &hi, uint32_t &lo) {
+  __half2 h = __float22half2_rn(w);
+  float2 hf = __half22float2(h);
+  __half2 l = __float22half2_rn(make_float2(w.x - hf.x, w.y - hf.y));
+  hi = *reinterpret_cast<uint32_t *>(&h);
+  lo = *reinterpret_cast<uint32_t *>(&l);
+}
+
+// Head dim of column k (0..31) of the query's virtual chunk vc: chunks 0, 1
+// follow the RoPE codes as lut4_bytes returns them (word of lane tg = dims
+// 32 vc + 8 tg + 0..7, bytes in the order 0 4 1 5 | 2 6 3 7); chunks 2, 3 the
+// NoPE codes (lane tg: dims 64 + 16 tg + 8 (vc - 2) + 0..7 in order).
+__device__ __forceinline__ int qcol_dim(int vc, int k) {
+  const int tg = (k & 15) >> 2, j = k & 3, hi = k >> 4;
+  return vc < 2 ? 32 * vc + 8 * tg + 2 * hi + (j >> 1) + 4 * (j & 1)
+                : 64 + 16 * tg + 8 * (vc - 2) + 4 * hi + j;
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads, 4)
+    octave_decode_mma_kernel(OctaveParams P, const void *__restrict__ query, int n_q_heads,
+                             int group, int gc, const uint8_t *__restrict__ cache, int n_kv_heads,
+                             int block_size, int64_t num_blocks,
+                             const int32_t *__restrict__ block_table, int num_reqs,
+                             int max_blocks, const int32_t *__restrict__ q_to_req,
+                             const int32_t *__restrict__ q_to_klen, int max_klen,
+                             float scale_log2, int split_tokens, int splits,
+                             float *__restrict__ ws) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int s = blockIdx.x, hg = blockIdx.y, qi = blockIdx.z;
+  const int h0 = hg * gc, kvh = h0 / group;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tg = lane & 3;
+  const int req = __ldg(q_to_req + qi);
+  int klen = min(max(__ldg(q_to_klen + qi), 0), min(max_klen, max_blocks * block_size));
+  if (req < 0 || req >= num_reqs) klen = 0;
+  const int t0 = s * split_tokens, t1 = min(klen, t0 + split_tokens);
+  const int ntiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
+
+  // codebook tables: signed bytes for QK, biased (+128) bytes for PV
+  Lut4 T4, U4;
+  uint32_t T3lo, T3hi;
+  {
+    uint32_t b[16], u[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+      b[i] = (uint32_t)P.lut4[i] & 0xFFu;
+      u[i] = (uint32_t)(P.lut4[i] + 128) & 0xFFu;
+    }
+    T4.lo0 = b[0] | b[1] << 8 | b[2] << 16 | b[3] << 24;
+    T4.lo1 = b[4] | b[5] << 8 | b[6] << 16 | b[7] << 24;
+    T4.hi0 = b[8] | b[9] << 8 | b[10] << 16 | b[11] << 24;
+    T4.hi1 = b[12] | b[13] << 8 | b[14] << 16 | b[15] << 24;
+    U4.lo0 = u[0] | u[1] << 8 | u[2] << 16 | u[3] << 24;
+    U4.lo1 = u[4] | u[5] << 8 | u[6] << 16 | u[7] << 24;
+    U4.hi0 = u[8] | u[9] << 8 | u[10] << 16 | u[11] << 24;
+    U4.hi1 = u[12] | u[13] << 8 | u[14] << 16 | u[15] << 24;
+    uint32_t c[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) c[i] = (uint32_t)P.lut3[i] & 0xFFu;
+    T3lo = c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24;
+    T3hi = c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24;
+  }
+
+  // ---- query: signs, FWHT over the two 64-dim blocks; int8 H / L rows
+  float *qs = reinterpret_cast<float *>(smem);  // [8][128]
+  {
+    // thread tid always holds dim tid: sign bit (tid & 31) of word tid / 32
+    // (constant indices only, so the parameter block stays in constant memory)
+    const uint32_t sw = warp == 0 ? P.sign_words[0]
+                        : warp == 1 ? P.sign_words[1]
+                        : warp == 2 ? P.sign_words[2]
+                                    : P.sign_words[3];
+    const float sgn = ((sw >> lane) & 1u) ? -1.f : 1.f;
+    for (int hh = 0; hh < 8; hh++) {
+      float v = 0.f;
+      if (hh < gc) {
+        const int64_t off = ((int64_t)qi * n_q_heads + h0 + hh) * kHead + tid;
+        v = (BF16 ? __uint_as_float((uint32_t)static_cast<const uint16_t *>(query)[off] << 16)
+                  : static_cast<const float *>(query)[off]) *
+            sgn;
+      }
+      qs[hh * kHead + tid] = v;
+    }
+  }
+  for (int h = 1; h < 64; h <<= 1) {
+    __syncthreads();
+    for (int p = tid; p < 8 * 64; p += kThreads) {
+      const int vv = p >> 6, pi = p & 63, blk = pi >> 5, pj = pi & 31;
+      const int i0 = blk * 64 + (pj / h) * 2 * h + (pj % h);
+      float *y = qs + vv * kHead;
+      const float a = y[i0], bb = y[i0 + h];
+      y[i0] = a + bb;
+      y[i0 + h] = a - bb;
+    }
+  }
+  __syncthreads();
+  float *qmax = reinterpret_cast<float *>(smem + kOffF);  // [8]
+#pragma unroll
+  for (int i = 0; i < 2; i++) {  // warp w: heads 2w, 2w + 1
+    const int hh = 2 * warp + i;
+    float m = fmaxf(fmaxf(fabsf(qs[hh * kHead + lane]), fabsf(qs[hh * kHead + lane + 32])),
+                    fmaxf(fabsf(qs[hh * kHead + lane + 64]), fabsf(qs[hh * kHead + lane + 96])));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+    if (lane == 0) qmax[hh] = m;
+  }
+  __syncthreads();
+  uint8_t *qrow = smem + kOffQ;
+  for (int p = tid; p < 8 * kHead; p += kThreads) {
+    const int hh = p >> 7, col = p & 127;
+    const float m = qmax[hh];
+    const int dim = qcol_dim(col >> 5, col & 31);
+    const float x = m > 0.f ? qs[hh * kHead + dim] * (kQRange / m) : 0.f;
+    const float hi = rintf(x * 0.0078125f);
+    const float lo = rintf(x - 128.f * hi);  // exact difference, |lo| <= 64
+    qrow[hh * kQStride + col] = (uint8_t)(int8_t)(int)hi;
+    qrow[(8 + hh) * kQStride + col] = (uint8_t)(int8_t)(int)lo;
+  }
+  __syncthreads();
+  uint32_t qa[4][4];  // A fragments of the virtual chunks
+  {
+    const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+    const uint32_t qaddr = smem_u32(qrow) + row * kQStride + 16 * (lane >> 4);
+#pragma unroll
+    for (int vc = 0; vc < 4; vc++) ldsm_x4(qaddr + 32 * vc, qa[vc]);
+  }
+  // FWHT-64 blocks carry 1 / 8; the query ints carry S
+  const float sl = scale_log2 * (qmax[g] * (0.125f / kQRange));
+  __syncthreads();
+
+  // ---- loader: thread tid copies chunks 4 (tid & 1) .. + 3 of row tid / 2
+  const int lr = tid >> 1, lc0 = 4 * (tid & 1);
+  auto issue = [&](int it) {
+    uint8_t *st = smem + (it % kStages) * kStageBytes;
+    const int t = t0 + it * kTile + lr;
+    bool ok = t < t1;
+    const uint8_t *src = cache;
+    if (ok) {
+      const int blk = __ldg(block_table + (int64_t)req * max_blocks + t / block_size);
+      ok = blk >= 0 && blk < num_blocks;
+      if (ok)
+        src = cache + (((int64_t)blk * n_kv_heads + kvh) * block_size + (t % block_size)) *
+                          P.slot_bytes;
+    }
+    if (lc0 == 0) smem[kOffV + (it % kStages) * kTile + lr] = ok ? 1 : 0;
+    const uint32_t rowa = smem_u32(st) + lr * 128;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const int ch = lc0 + i;
+      cp_async16(rowa + ((ch ^ (lr & 7)) << 4), ok ? src + ch * 16 : cache, ok);
+    }
+  };
+
+  float o[8][4];
+#pragma unroll
+  for (int mt = 0; mt < 8; mt++) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  float *fsc = reinterpret_cast<float *>(smem + kOffF);
+
+#pragma unroll
+  for (int i = 0; i < kStages - 1; i++) {
+    if (i < ntiles) issue(i);
+    cp_async_commit();
+  }
+  for (int it = 0; it < ntiles; it++) {
+    cp_async_wait<kStages - 2>();
+    __syncthreads();
+    uint8_t *st = smem + (it % kStages) * kStageBytes;
+    if (tid < kTile) {  // scales at bytes 120..125 (chunk 7, offset 8): fp16 -> fp32 / 64
+      const int r = tid;
+      const uint8_t *row = st + r * 128 + ((7 ^ (r & 7)) << 4) + 8;
+      const uint32_t w01 = *reinterpret_cast<const uint32_t *>(row);
+      const uint32_t w2 = *reinterpret_cast<const uint16_t *>(row + 4);
+      const float2 f01 = __half22float2(*reinterpret_cast<const __half2 *>(&w01));
+      fsc[r] = f01.x * 0.015625f;
+      fsc[kTile + r] = f01.y * 0.015625f;
+      fsc[2 * kTile + r] = __half2float(__ushort_as_half((uint16_t)w2)) * 0.015625f;
+    }
+    if (it + kStages - 1 < ntiles) issue(it + kStages - 1);
+    cp_async_commit();
+    __syncthreads();
+
+    // bit k: token k of this warp's 16 is in range and on a mapped block
+    const unsigned okmask =
+        __ballot_sync(kFull, (lane < 16) &&
+                                 smem[kOffV + (it % kStages) * kTile + 16 * warp + (lane & 15)] != 0) &
+        0xFFFFu;
+    if (okmask != 0) {
+      const bool partial = okmask != 0xFFFFu;
+      const uint32_t base = smem_u32(st);
+      // ldmatrix lane address: matrix m = lane / 8 (x4: T = m & 1, chunk +m >> 1)
+      const int mr = 16 * warp + 8 * ((lane >> 3) & 1) + (lane & 7);
+      const int mc = lane >> 4;
+      auto chunk_addr = [&](int ch) -> uint32_t {
+        return base + mr * 128 + ((ch ^ (mr & 7)) << 4);
+      };
+      // ---- QK: integer MMAs, one accumulator per (block, 8 tokens)
+      int accr[2][4] = {}, accn[2][4] = {};
+      {  // RoPE: chunks 0, 1 (4-bit)
+        uint32_t kr[4];
+        ldsm_x4(chunk_addr(mc), kr);  // (T0, c0), (T1, c0), (T0, c1), (T1, c1)
+#pragma unroll
+        for (int m = 0; m < 4; m++) {
+          const int T = m & 1, c = m >> 1;
+          const uint32_t w = kr[m];
+          imma16832(accr[T], qa[c], lut4_bytes(w & 0xFFFFu, T4), lut4_bytes(w >> 16, T4));
+        }
+      }
+      {  // NoPE: 2-bit plane chunk 2, 1-bit plane in chunk 3 (words 0, 1)
+        uint32_t lo[2], hi[2];
+        {
+          uint32_t r4[4];
+          ldsm_x4(chunk_addr(2 + mc), r4);  // (T0, c2), (T1, c2), (T0, c3), (T1, c3)
+          lo[0] = r4[0];
+          lo[1] = r4[1];
+          // the 1-bit plane word this lane needs (tg >> 1) sits in lane 4g + (tg >> 1)
+          hi[0] = __shfl_sync(kFull, r4[2], (lane & ~3) | (tg >> 1));
+          hi[1] = __shfl_sync(kFull, r4[3], (lane & ~3) | (tg >> 1));
+        }
+#pragma unroll
+        for (int T = 0; T < 2; T++) {
+          uint32_t R[4];
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            // code byte j: (lo >> 2i) & 3 | ((hi >> (4(tg & 1) + i)) & 1) << 2
+            const uint32_t lb = (lo[T] >> (2 * i)) & 0x03030303u;
+            const uint32_t hb = (hi[T] >> (4 * (tg & 1) + i)) & 0x01010101u;
+            uint32_t x = hb * 4u + lb;
+            x = x | (x >> 4);
+            R[i] = prmt(T3lo, T3hi, prmt(x, 0u, 0x0020u));  // dims 16tg + 4i + 0..3
+          }
+          imma16832(accn[T], qa[2], R[0], R[1]);
+          imma16832(accn[T], qa[3], R[2], R[3]);
+        }
+      }
+      float2 sacc[2];
+#pragma unroll
+      for (int T = 0; T < 2; T++) {
+        const float2 dr = *reinterpret_cast<const float2 *>(fsc + 16 * warp + 8 * T + 2 * tg);
+        const float2 dn =
+            *reinterpret_cast<const float2 *>(fsc + kTile + 16 * warp + 8 * T + 2 * tg);
+        sacc[T].x = fmaf(dr.x, (float)(accr[T][0] * 128 + accr[T][2]),
+                         dn.x * (float)(accn[T][0] * 128 + accn[T][2]));
+        sacc[T].y = fmaf(dr.y, (float)(accr[T][1] * 128 + accr[T][3]),
+                         dn.y * (float)(accn[T][1] * 128 + accn[T][3]));
+      }
+      // ---- online softmax (base 2), head g, this warp's 16 tokens
+      float sc[4] = {sacc[0].x * sl, sacc[0].y * sl, sacc[1].x * sl, sacc[1].y * sl};
+      if (partial) {
+#pragma unroll
+        for (int e = 0; e < 4; e++)
+          if (!((okmask >> (8 * (e >> 1) + 2 * tg + (e & 1))) & 1u)) sc[e] = -INFINITY;
+      }
+      float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+      if (__any_sync(kFull, mx > m_run + 8.f)) {
+        const float mn = fmaxf(m_run, mx);
+        const float alpha = exp2f(m_run - mn);
+        m_run = mn;
+        l_run *= alpha;
+        const float a0 = __shfl_sync(kFull, alpha, 8 * tg);
+        const float a1 = __shfl_sync(kFull, alpha, 8 * tg + 4);
+#pragma unroll
+        for (int mt = 0; mt < 8; mt++) {
+          o[mt][0] *= a0;
+          o[mt][1] *= a1;
+          o[mt][2] *= a0;
+          o[mt][3] *= a1;
+        }
+      }
+      float p[4];
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        p[e] = exp2f(sc[e] - m_run);
+        l_run += p[e];
+      }
+      // ---- PV: B = p * s_v / 64 (hi / lo), A = V^T codes through the LUT
+      const float2 dv0 = *reinterpret_cast<const float2 *>(fsc + 2 * kTile + 16 * warp + 2 * tg);
+      const float2 dv1 =
+          *reinterpret_cast<const float2 *>(fsc + 2 * kTile + 16 * warp + 8 + 2 * tg);
+      float2 w0 = make_float2(p[0] * dv0.x, p[1] * dv0.y);
+      float2 w1 = make_float2(p[2] * dv1.x, p[3] * dv1.y);
+      if (partial) {  // a zero-filled or unmapped row: keep its weight out exactly
+        if (!((okmask >> (2 * tg)) & 1u)) w0.x = 0.f;
+        if (!((okmask >> (2 * tg + 1)) & 1u)) w0.y = 0.f;
+        if (!((okmask >> (8 + 2 * tg)) & 1u)) w1.x = 0.f;
+        if (!((okmask >> (9 + 2 * tg)) & 1u)) w1.y = 0.f;
+      }
+      uint32_t bh0, bl0, bh1, bl1;
+      split_hilo(w0, bh0, bl0);
+      split_hilo(w1, bh1, bl1);
+      // x2.trans: matrices (T0, chunk), (T1, chunk); lanes 0..15 give the rows
+      const int vrow = 16 * warp + (lane & 15);
+      const uint32_t vaddr = base + vrow * 128;
+#pragma unroll
+      for (int vc = 0; vc < 4; vc++) {
+        uint32_t vr[2];
+        if (vc == 0) {
+          // joined chunk: row g < 4 <- chunk 3 element g + 4 (V bytes 2g, 2g + 1),
+          // row g >= 4 <- chunk 7 element g - 4 (V bytes 48 + 2g, 49 + 2g)
+          uint32_t c3[2], c7[2];
+          ldsm_x2_t(vaddr + ((3 ^ (vrow & 7)) << 4), c3);
+          ldsm_x2_t(vaddr + ((7 ^ (vrow & 7)) << 4), c7);
+          vr[0] = __shfl_xor_sync(kFull, lane < 16 ? c7[0] : c3[0], 16);
+          vr[1] = __shfl_xor_sync(kFull, lane < 16 ? c7[1] : c3[1], 16);
+        } else {  // chunks 4, 5, 6: V bytes 16 vc - 8 + element
+          ldsm_x2_t(vaddr + (((3 + vc) ^ (vrow & 7)) << 4), vr);
+        }
+#pragma unroll
+        for (int par = 0; par < 2; par++) {
+          // byte 2g + par of tokens (2tg, 2tg+1) [vr[0]] and (2tg+8, 2tg+9) [vr[1]]
+          const uint32_t s0 = prmt(vr[0], 0u, par ? 0x0031u : 0x0020u);
+          const uint32_t s1 = prmt(vr[1], 0u, par ? 0x0031u : 0x0020u);
+          const uint32_t R0 = lut4_bytes(s0, U4);  // (tok a lo, tok a hi, tok b lo, tok b hi)
+          const uint32_t R1 = lut4_bytes(s1, U4);
+          const uint32_t a[4] = {lut_half2(R0, 0x4240u), lut_half2(R0, 0x4341u),
+                                 lut_half2(R1, 0x4240u), lut_half2(R1, 0x4341u)};
+          float(&acc)[4] = o[2 * vc + par];
+          mma16816(acc, a, bh0, bh1);
+          mma16816(acc, a, bl0, bl1);
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // ---- merge the warps and write the partial records
+  float *red_o = reinterpret_cast<float *>(smem);  // [warp][8][128]
+  float *red_m = red_o + kWarps * 8 * kHead;
+  float *red_l = red_m + kWarps * 8;
+  l_run += __shfl_xor_sync(kFull, l_run, 1);
+  l_run += __shfl_xor_sync(kFull, l_run, 2);
+  if (tg == 0) {
+    red_m[warp * 8 + g] = m_run;
+    red_l[warp * 8 + g] = l_run;
+  }
+#pragma unroll
+  for (int vc = 0; vc < 4; vc++)
+#pragma unroll
+    for (int par = 0; par < 2; par++) {
+      // V byte of row g: joined chunk -> 2g (+48 for g >= 4); chunk 3 + vc -> 16 vc - 8 + 2g
+      const int vb = (vc == 0 ? (g < 4 ? 2 * g : 48 + 2 * g) : 16 * vc - 8 + 2 * g) + par;
+      const int d = 8 * (vb >> 2) + (vb & 3);  // low nibble; high nibble is d + 4
+      const float(&acc)[4] = o[2 * vc + par];
+      float *w = red_o + warp * 8 * kHead;
+      w[(2 * tg) * kHead + d] = acc[0];
+      w[(2 * tg + 1) * kHead + d] = acc[1];
+      w[(2 * tg) * kHead + d + 4] = acc[2];
+      w[(2 * tg + 1) * kHead + d + 4] = acc[3];
+    }
+  __syncthreads();
+  for (int p = tid; p < gc * kHead; p += kThreads) {
+    const int hh = p >> 7, j = p & 127;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++) M = fmaxf(M, red_m[w * 8 + hh]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; w++) {
+        const float f = exp2f(red_m[w * 8 + hh] - M);
+        L += red_l[w * 8 + hh] * f;
+        O += red_o[(w * 8 + hh) * kHead + j] * f;
+      }
+    }
+    float *rec = ws + (((int64_t)qi * n_q_heads + h0 + hh) * splits + s) * kORec;
+    rec[4 + j] = O;
+    if (j == 0) {
+      rec[0] = M;
+      rec[1] = L;
+    }
+  }
+}
+
+}  // namespace
+
+bool octave_mma_supported(const OctaveParams &P) {
+  return P.head_size == kHead && P.rope_dim == 64 && P.v_bits == 4 && P.slot_bytes == 128;
+}
+
+cudaError_t launch_octave_decode_mma(const OctaveParams &P, const void *query, int bf16, int num_q,
+                                     int n_q_heads, const uint8_t *cache, int n_kv_heads,
+                                     int block_size, int64_t num_blocks,
+                                     const int32_t *block_table, int num_reqs, int max_blocks,
+                                     const int32_t *q_to_req, const int32_t *q_to_klen,
+                                     int max_klen, float scale, float *ws,
+                                     const DecodePlan &plan, cudaStream_t s) {
+  const int group = n_q_heads / n_kv_heads;
+  const int gc = group < 8 ? group : 8;
+  dim3 grid(plan.splits, n_q_heads / gc, num_q);
+  const float sl2 = scale * kLog2e;
+  if (bf16)
+    octave_decode_mma_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(
+        P, query, n_q_heads, group, gc, cache, n_kv_heads, block_size, num_blocks, block_table,
+        num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2, plan.split_tokens,
+        plan.splits, ws);
+  else
+    octave_decode_mma_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(
+        P, query, n_q_heads, group, gc, cache, n_kv_heads, block_size, num_blocks, block_table,
+        num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2, plan.split_tokens,
+        plan.splits, ws);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

@@ -94,21 +94,42 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-DecodePlan plan_decode(int batch, int n_kv_heads, int max_seq_len) {
-  DecodePlan p;
-  const int units = max(batch * n_kv_heads, 1);
-  const int target = kNumSMs * q4_decode_ctas_per_sm();  // one wave of split CTAs
-  int splits = max(1, (target + units - 1) / units);
-  int per = (max(max_seq_len, 1) + splits - 1) / splits;
-  per = ((per + 63) / 64) * 64;
-  if (per < 256) per = 256;
-  p.split_tokens = per;
-  p.splits = max(1, (max(max_seq_len, 1) + per - 1) / per);
-  while (p.splits > kMaxSplitsSmem) {  // very long contexts: larger splits
-    p.split_tokens *= 2;
-    p.splits = (max(max_seq_len, 1) + p.split_tokens - 1) / p.split_tokens;
+DecodePlan plan_split_k(int units, int max_len, int slots, int max_splits) {
+  // Each of `units` independent problems (sequence, q-head group) is cut into
+  // splits of whole 64-token tiles, at least 256 tokens each.  With `slots`
+  // CTAs resident at once, the kernel takes about waves x tokens-per-split; the
+  // split count minimising that (fewest splits on ties) wins, so a second wave
+  // is only chosen when it shortens every split by more than half.
+  const int len = max(max_len, 1);
+  const int tiles = (len + 63) / 64;
+  units = max(units, 1);
+  DecodePlan best;
+  best.split_tokens = max(tiles * 64, 256);
+  best.splits = 1;
+  int64_t best_cost = -1;
+  const int sp_max = min(tiles, 2 * ((slots + units - 1) / units) + 1);
+  for (int sp = 1; sp <= sp_max; sp++) {
+    const int per = max(((tiles + sp - 1) / sp) * 64, 256);
+    const int splits = (len + per - 1) / per;
+    if (splits > max_splits) continue;
+    const int64_t waves = ((int64_t)units * splits + slots - 1) / slots;
+    const int64_t cost = waves * per;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best.split_tokens = per;
+      best.splits = splits;
+    }
   }
-  return p;
+  while (best.splits > max_splits) {  // very long contexts: larger splits
+    best.split_tokens *= 2;
+    best.splits = (len + best.split_tokens - 1) / best.split_tokens;
+  }
+  return best;
+}
+
+DecodePlan plan_decode(int batch, int n_head_groups, int max_seq_len) {
+  return plan_split_k(batch * n_head_groups, max_seq_len, kNumSMs * q4_decode_ctas_per_sm(),
+                      kMaxSplitsSmem);
 }
 
 size_t decode_workspace_bytes(int batch, int n_q_heads, const DecodePlan &p) {

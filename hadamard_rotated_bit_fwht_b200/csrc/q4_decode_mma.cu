@@ -3,37 +3,44 @@
 // merge note's per-token path that rotates Q and the output).
 //
 // With GQA the decode step is a small dense contraction per kv head:
-// S = Q_rot K^T (G x T) and O = P V (G x 256).  At G = 8 fp32 FMAs alone would
-// cap the kernel near a third of HBM bandwidth, so both products run on the
-// tensor cores (warp-level mma.sync m16n8k16, fp16 inputs, fp32 accumulation)
-// while keeping fp32-level accuracy:
-//   * The nibble codes enter the MMA as exact fp16 values 64 + c: a nibble
-//     sitting in bits 4..7 of a 16-bit lane, OR-ed with the bits of 64.0
-//     (0x5400), is that value -- one LOP3 per pair, no conversion
-//     instruction.  The bias 64 + 8 = 72 is removed in fp32: for scores,
-//     72 * sum(q) per (head, block); for outputs, 72 * sum_t(p d_v) per
-//     (head, block), accumulated alongside and subtracted once at the end.
-//   * The query is split into fp16 hi + lo parts that fill the 16 M-rows of
-//     the QK MMA (rows 0-7 hi, rows 8-15 lo of the 8 heads), so a head's score
-//     is c0 + c2 of the accumulator and carries ~22 mantissa bits.  The query
-//     fragments live in shared memory in ldmatrix order.
-//   * The per-block Q4_0 scale depends on (token, block), so each 32-dim
-//     block has its own fresh QK accumulator, scaled by the block's scale in
-//     fp32 and added to the score.
-//   * PV: A = V^T codes (dims x tokens, exact), B = p * d_v (token x head)
-//     split hi + lo; the 16 dims of one M-tile lie in one block, so the V
-//     scale rides in B.
+// S = Q_rot K^T (G x T) and O = P V (G x 256), G <= 8 heads per CTA.  Both
+// products run on the tensor cores (warp-level mma.sync) at fp32-level
+// accuracy; a CTA of four warps walks its split in 64-token tiles:
+//   * Tiles arrive by TMA (cp.async.bulk.tensor, 2-D maps over the cache's
+//     128-byte code rows and 16-byte scale rows, hardware 128-byte swizzle)
+//     into a ring of shared-memory stages guarded by mbarriers; one thread
+//     issues, every wait is bounded.
+//   * QK: warp w scores tokens 16w..16w+15 of the tile for all 8 heads on the
+//     integer tensor path (m16n8k32, s8 x u8 -> s32).  A Q4_0 block is 32
+//     dims, one MMA K-step; its codes enter as bytes with three logic ops per
+//     8 codes (low nibbles = dims 0..15, high nibbles = dims 16..31 of the
+//     block, the B-fragment rows).  The rotated query of each head is scaled
+//     by S = 127 * 2^14 / max|q| and split exactly into int8 levels H, M, L
+//     with S q = 2^14 H + 2^7 M + L (|M|, |L| <= 64); one MMA takes H and M
+//     (rows 0-7, 8-15), a second takes L.  Their accumulators start at the
+//     bits of 1.5 * 2^23 minus the zero-point term 8 * sum(level), so each
+//     exact integer sum over the block becomes an fp32 by one subtraction;
+//     2^7 F_HM + F_L times the block's scale is added to the score.  The
+//     query is carried to about 2^-22 of its largest element.
+//   * Softmax: the tile maximum per head is shared through shared memory, so
+//     every warp keeps the same running maximum (rescaling lazily, only when
+//     a score passes it by 8); p goes to shared memory.
+//   * PV: warp w owns output dims 64w..64w+63 (Q4_0 blocks 2w, 2w+1) for all
+//     64 tokens of the tile: A = V^T codes as the exact fp16 values 64 + c (a
+//     nibble in bits 4..7 of a 16-bit lane OR-ed with the bits of 64.0, one
+//     LOP3 per pair, read by ldmatrix.trans), B = p * d_v split into fp16
+//     hi + lo (the 16 dims of an M-tile lie in one block, so the V scale rides
+//     in B).  The bias 64 + 8 = 72 is removed at the end with
+//     72 * sum_t(p d_v) per (head, block).
 //   * The QK accumulator layout (head g = lane / 4, tokens 2(lane % 4) + {0,1})
-//     is exactly the PV B-fragment layout for tokens {0..7} and {8..15}, so no
-//     data moves between the two products.
-// Memory path: 64-token tiles of codes (rows of 128 bytes) and scales are
-// staged by cp.async into a 3-stage shared-memory ring; code rows are stored
-// with the 128-byte XOR swizzle (16-byte chunk c of row r at c ^ (r & 7)) so
-// ldmatrix (K) and ldmatrix.trans (V) are conflict-free; the scales of the
-// current tile are widened to fp32 once.  Three CTAs of four warps per SM.
-// Online softmax in base 2 with a lazily updated reference maximum (rescale
-// only when a score exceeds it by 8), split-K partials (m, l, o[256]) per
-// (sequence, q head, split), and the combine + back-rotation kernel.
+//     is the PV B-fragment layout for tokens {0..7} and {8..15}.
+// Split-K partials (m, l, o[256]) per (sequence, q head, split) go to the
+// combine + back-rotation kernel.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -41,36 +48,78 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kTile = 64;          // tokens per pipeline stage (16 per warp)
-constexpr int kStages = 3;
-constexpr int kCtasPerSm = 3;
+constexpr int kTile = 64;          // tokens per stage (16 per warp for QK)
+constexpr int kStages = 2;
+constexpr int kCtasPerSm = 4;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kRec = 260;          // partial record: m, l, pad, pad, o[256]
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kBias = 72.f;      // 64 (magic) + 8 (Q4_0 zero point)
+constexpr float kQRange = 2080768.f;         // 127 * 2^14
+constexpr uint32_t kTileBytes = 2 * kTile * 128 + 2 * kTile * 16;  // one TMA transaction
 
-// shared memory layout (bytes)
-constexpr int kOffKC = 0;                       // K codes: 64 rows x 128 B, swizzled
+// shared memory layout (bytes from a 1024-aligned base: 128-byte swizzle atoms)
+constexpr int kOffKC = 0;                       // K codes: 64 rows x 128 B (TMA-swizzled)
 constexpr int kOffVC = kOffKC + kTile * 128;    // V codes
 constexpr int kOffKS = kOffVC + kTile * 128;    // K scales: 64 rows x 8 fp16
 constexpr int kOffVS = kOffKS + kTile * 16;     // V scales
-constexpr int kStageBytes = kOffVS + kTile * 16;
-constexpr int kOffF = kStages * kStageBytes;    // fp32 scales of the current tile [kv][block][token]
-constexpr int kOffQ = kOffF + 2 * 8 * kTile * 4;  // query fragments: 16 tiles of 16x16 fp16
-constexpr int kSmemBytes = kOffQ + 16 * 512;
+constexpr int kStageBytes = kOffVS + kTile * 16;  // 18432 = 18 KiB
+constexpr int kOffF = kStages * kStageBytes;    // fp32 scales, 2 buffers x [kv][block][token]
+constexpr int kFBuf = 2 * 8 * kTile;            // floats per buffer
+constexpr int kPStride = 72;                    // p rows: 64 tokens + pad (conflict-free)
+constexpr int kOffP = kOffF + 2 * kFBuf * 4;    // p [8 heads][kPStride] fp32
+constexpr int kOffRed = kOffP + 8 * kPStride * 4;  // tile maxima [warp][8], then l [warp][8]
+constexpr int kQStride = 272;                   // int8 query row: 256 B + 16 B pad
+constexpr int kOffQ = kOffRed + 2 * kWarps * 8 * 4;  // rows 0-7 H, 8-15 M, 16-23 L
+constexpr int kOffZ = kOffQ + 24 * kQStride;    // 16 zero bytes (ldmatrix rows of zeros)
+constexpr int kOffBar = kOffZ + 16;             // mbarriers, 8 B each
+constexpr int kSmemUsed = kOffBar + kStages * 8;
+constexpr int kSmemBytes = kSmemUsed + 1024;    // slack for the 1024-byte alignment
+static_assert(kStageBytes % 1024 == 0, "stages must keep the swizzle atoms aligned");
+static_assert(kOffBar % 8 == 0, "mbarrier alignment");
+
+// bounded waits: ~2^20 polls of up to ~1 us each
+constexpr int kWaitPolls = 1 << 20;
+
+struct TmaMaps {
+  CUtensorMap kc, vc, ks, vs;
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(valid ? 16 : 0));
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N));
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// true once the phase with this parity has completed; false after the poll limit
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (int i = 0; i < kWaitPolls; i++) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity), "r"(1000u)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -86,11 +135,18 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                          uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// d = A(s8, 16 x 32) * B(u8, 32 x 8), accumulating from zero
+__device__ __forceinline__ void imma16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%10,%10};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "n"(0));
 }
 
 // nibbles at bits 4..7 and 20..23 of x -> half2 (64 + c) exactly
@@ -109,24 +165,14 @@ __device__ __forceinline__ void split_hilo(float2 w, uint32_t &hi, uint32_t &lo)
   lo = *reinterpret_cast<uint32_t *>(&l);
 }
 
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  return __ffma2_rn(a, b, c);
-}
-
-// byte offset of element (row, col) of one 16x16 fp16 query-fragment tile;
-// the 16-byte halves are XOR-swizzled with bit 2 of the row so the eight rows
-// read by one ldmatrix phase fall in distinct banks
-__device__ __forceinline__ int qfrag_off(int row, int col) {
-  return row * 32 + (((col >> 3) ^ ((row >> 2) & 1)) << 4) + (col & 7) * 2;
-}
-
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    q4_decode_mma_kernel(kvq_cache c, const void *__restrict__ q,
-                         const int32_t *__restrict__ seq_lens, int max_seq_len, int n_q_heads,
-                         int group, int gc, float scale_log2, int split_tokens, int splits,
-                         float *__restrict__ ws) {
-  extern __shared__ __align__(128) uint8_t smem[];
+    q4_decode_mma_kernel(const __grid_constant__ TmaMaps maps, kvq_cache c,
+                         const void *__restrict__ q, const int32_t *__restrict__ seq_lens,
+                         int max_seq_len, int n_q_heads, int group, int gc, float scale_log2,
+                         int split_tokens, int splits, float *__restrict__ ws) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int s = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
   const int h0 = hg * gc, kvh = h0 / group;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -136,9 +182,42 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const int t0 = s * split_tokens;
   const int t1 = min(len, t0 + split_tokens);
   const int ntiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
+  const uint32_t bar0 = smem_u32(smem + kOffBar);
 
-  // ---- query: rotate (FWHT-256 in shared memory), split hi/lo into fragments
-  float *qs = reinterpret_cast<float *>(smem);  // [8][256] in the ring, before it is used
+  // first cache row of a tile, -1 if its page is unmapped
+  auto tile_row0 = [&](int tstart) -> int64_t {
+    if (c.block_table == nullptr) return ((int64_t)b * c.num_kv_heads + kvh) * c.max_tokens + tstart;
+    const int pi = tstart / c.page_size;
+    const int page = __ldg(c.block_table + (int64_t)b * c.max_pages_per_seq + pi);
+    if (page < 0 || page >= c.num_pages) return -1;
+    return ((int64_t)page * c.num_kv_heads + kvh) * c.page_size + (tstart - pi * c.page_size);
+  };
+  // one thread: a whole tile (codes + scales of K and V) onto the stage's barrier
+  auto issue = [&](int it) {
+    const int st = it % kStages;
+    const uint32_t bar = bar0 + 8 * st;
+    const int64_t row0 = tile_row0(t0 + it * kTile);
+    if (row0 < 0) {  // nothing to load: complete the phase without bytes
+      mbar_arrive(bar);
+      return;
+    }
+    const uint32_t dst = smem_u32(smem + st * kStageBytes);
+    mbar_arrive_tx(bar, kTileBytes);
+    tma_load_2d(dst + kOffKC, &maps.kc, 0, (int)row0, bar);
+    tma_load_2d(dst + kOffVC, &maps.vc, 0, (int)row0, bar);
+    tma_load_2d(dst + kOffKS, &maps.ks, 0, (int)row0, bar);
+    tma_load_2d(dst + kOffVS, &maps.vs, 0, (int)row0, bar);
+  };
+
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < kStages; i++) mbar_init(bar0 + 8 * i, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+
+  // ---- query: rotate (FWHT-256 in shared memory), then int8 H / M / L rows
+  float *qs = reinterpret_cast<float *>(smem);  // [8][256] in the stages, before any load
   for (int p = tid; p < 8 * kDim; p += kThreads) {
     const int hh = p >> 8, j = p & 255;
     float v = 0.f;
@@ -161,281 +240,323 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
   }
   __syncthreads();
-  // Fragment tile (bb, kk) row r: hi (r < 8) or lo (r >= 8) of head r & 7;
-  // column k <-> dim 32bb + 16kk + 4((k & 7) >> 1) + (k >> 3) + 2(k & 1).
-  // q_rot = FWHT / 16 is of order one, so its split stays in the normal fp16
-  // range; scale * log2(e) is applied to the scores.
-  uint8_t *qf = smem + kOffQ;
-  for (int p = tid; p < 16 * 8 * 16; p += kThreads) {  // (tile, head, col) for hi and lo
-    const int tile = p >> 7, hh = (p >> 4) & 7, k = p & 15;
-    const int bb = tile >> 1, kk = tile & 1;
-    const int dim = 32 * bb + 16 * kk + 4 * ((k & 7) >> 1) + (k >> 3) + 2 * (k & 1);
-    const float x = qs[hh * kDim + dim] * 0.0625f;
-    const __half hi = __float2half_rn(x);
-    const __half lo = __float2half_rn(x - __half2float(hi));
-    *reinterpret_cast<__half *>(qf + tile * 512 + qfrag_off(hh, k)) = hi;
-    *reinterpret_cast<__half *>(qf + tile * 512 + qfrag_off(hh + 8, k)) = lo;
-  }
-  // bias correction of the scores: 72 * sum over each block of (hi + lo), one
-  // thread per (head, block), into shared memory
-  float *sqs = reinterpret_cast<float *>(smem + kOffF);  // reused by the scale widening later
-  if (tid < 64) {
-    const int hh = tid >> 3, bb = tid & 7;
-    const float *qr = qs + hh * kDim + 32 * bb;
-    float a = 0.f;
-    for (int j = 0; j < 32; j++) {
-      const float x = qr[(j + tid) & 31] * 0.0625f;  // rotated start: spreads the banks
-      const __half hi = __float2half_rn(x);
-      const __half lo = __float2half_rn(x - __half2float(hi));
-      a += __half2float(hi) + __half2float(lo);
-    }
-    sqs[tid] = kBias * a;
+  float *red = reinterpret_cast<float *>(smem + kOffRed);
+#pragma unroll
+  for (int i = 0; i < 2; i++) {  // warp w: max |FWHT(q)| of heads 2w, 2w + 1
+    const int hh = 2 * warp + i;
+    float m = 0.f;
+    for (int j = lane; j < kDim; j += 32) m = fmaxf(m, fabsf(qs[hh * kDim + j]));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+    if (lane == 0) red[hh] = m;
   }
   __syncthreads();
-  float sqb[8];
-#pragma unroll
-  for (int bb = 0; bb < 8; bb++) sqb[bb] = sqs[g * 8 + bb];
-  __syncthreads();  // qs (ring area) is overwritten by the loads below
-
-  // ---- tile loader
-  auto tile_row0 = [&](int tstart) -> int64_t {  // first cache row of the tile, -1 if unmapped
-    if (c.block_table == nullptr) return ((int64_t)b * c.num_kv_heads + kvh) * c.max_tokens + tstart;
-    const int pi = tstart / c.page_size;
-    const int page = __ldg(c.block_table + (int64_t)b * c.max_pages_per_seq + pi);
-    if (page < 0 || page >= c.num_pages) return -1;
-    return ((int64_t)page * c.num_kv_heads + kvh) * c.page_size + (tstart - pi * c.page_size);
-  };
-  auto issue = [&](int it) {
-    uint8_t *st = smem + (it % kStages) * kStageBytes;
-    const int tstart = t0 + it * kTile;
-    const int64_t row0 = tile_row0(tstart);
-    const int nvalid = row0 < 0 ? 0 : min(kTile, t1 - tstart);
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-      const int idx = tid + kThreads * i;  // 0..511
-      const int r = idx >> 3, ch = idx & 7;
-      const bool ok = r < nvalid;
-      const int64_t row = ok ? row0 + r : 0;
-      const uint32_t so = r * 128 + ((ch ^ (r & 7)) << 4);
-      cp_async16(smem_u32(st + kOffKC + so), c.k_codes + row * 128 + ch * 16, ok);
-      cp_async16(smem_u32(st + kOffVC + so), c.v_codes + row * 128 + ch * 16, ok);
-    }
-    {
-      const int r = tid & 63;
-      const bool ok = r < nvalid;
-      const int64_t row = ok ? row0 + r : 0;
-      if (tid < 64) cp_async16(smem_u32(st + kOffKS + r * 16), c.k_scales + row * 8, ok);
-      else cp_async16(smem_u32(st + kOffVS + r * 16), c.v_scales + row * 8, ok);
-    }
-  };
-
-  float o[16][4];
-#pragma unroll
-  for (int mt = 0; mt < 16; mt++) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-  float swb[8];  // sum over tokens of p * d_v, per block, for head g
-#pragma unroll
-  for (int bb = 0; bb < 8; bb++) swb[bb] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
-
-  const uint32_t qbase = smem_u32(qf);
-  // ldmatrix.x4 lane address inside a query tile: matrix m = lane / 8 gives
-  // (rows 8 * (m & 1) + lane % 8, 16-byte half m >> 1)
-  const int qrow = (lane & 7) + 8 * ((lane >> 3) & 1);
-  const uint32_t qlane = qrow * 32 + ((((lane >> 4) & 1) ^ ((qrow >> 2) & 1)) << 4);
-  float *fsc = reinterpret_cast<float *>(smem + kOffF);
-
-#pragma unroll
-  for (int i = 0; i < kStages - 1; i++) {
-    if (i < ntiles) issue(i);
-    cp_async_commit();
+  uint8_t *qi = smem + kOffQ;
+  for (int p = tid; p < 8 * kDim; p += kThreads) {
+    const int hh = p >> 8, j = p & 255;
+    const float m = red[hh];
+    const float x = m > 0.f ? qs[p] * (kQRange / m) : 0.f;  // |x| <= 127 * 2^14 (+ rounding)
+    const float hi = rintf(x * (1.f / 16384.f));
+    const float r = x - 16384.f * hi;          // exact, |r| <= 2^13
+    const float mid = rintf(r * (1.f / 128.f));
+    const float lo = rintf(r - 128.f * mid);   // exact difference, |lo| <= 64
+    qi[hh * kQStride + j] = (uint8_t)(int8_t)(int)hi;
+    qi[(8 + hh) * kQStride + j] = (uint8_t)(int8_t)(int)mid;
+    qi[(16 + hh) * kQStride + j] = (uint8_t)(int8_t)(int)lo;
   }
+  if (tid < 4) reinterpret_cast<uint32_t *>(smem + kOffZ)[tid] = 0u;
+  __syncthreads();
+  // zero-point term of head g, block bb: 8 * sum over the block of 2^14 H + 2^7 M + L
+  int bq[8];
+#pragma unroll
+  for (int bb = 0; bb < 8; bb++) {
+    // lane (g, tg) sums dims 32 bb + 8 tg .. + 7, then the 4 lanes of head g combine
+    int acc = 0;
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+      const int d = 32 * bb + 8 * tg + j;
+      acc += 16384 * (int)(int8_t)qi[g * kQStride + d] + 128 * (int)(int8_t)qi[(8 + g) * kQStride + d] +
+             (int)(int8_t)qi[(16 + g) * kQStride + d];
+    }
+    acc += __shfl_xor_sync(kFull, acc, 1);
+    acc += __shfl_xor_sync(kFull, acc, 2);
+    bq[bb] = 8 * acc;
+  }
+  // A fragments of block bb: rows 0-15 (H, M) by ldmatrix.x4; L rows with a
+  // zero row in place of rows 8-15, also by ldmatrix.x4 (bytes 32 bb + 0..15,
+  // + 16..31)
+  uint32_t qhm[8][4];
+  const uint32_t zrow = smem_u32(smem + kOffZ);
+  const uint32_t qla = ((lane >> 3) & 1) ? zrow : smem_u32(qi) + (16 + (lane & 7)) * kQStride + 16 * (lane >> 4);
+  const uint32_t qlstep = ((lane >> 3) & 1) ? 0u : 32u;
+  {
+    const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+    const uint32_t a4 = smem_u32(qi) + row * kQStride + 16 * (lane >> 4);
+#pragma unroll
+    for (int bb = 0; bb < 8; bb++) ldsm_x4(a4 + 32 * bb, qhm[bb]);
+  }
+  // score scale for head g: max / (16 * 127 * 2^14) undoes S and the FWHT's 1 / 16
+  const float sl2 = scale_log2 * (red[g] * (0.0625f / kQRange));
+  __syncthreads();  // qs, red are reused below; the barriers are initialised
+
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < kStages - 1; i++)
+      if (i < ntiles) issue(i);
+  }
+
+  float o[4][4];  // M-tiles: block 2w + (mt >> 1), parity mt & 1
+#pragma unroll
+  for (int mt = 0; mt < 4; mt++) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  float swb[2] = {0.f, 0.f};  // sum over this lane's tokens of p * d_v, head g, blocks 2w, 2w+1
+  float m_run = -INFINITY, l_run = 0.f;  // head g; m_run is the same in every warp
+  float *pbuf = reinterpret_cast<float *>(smem + kOffP);
+  bool failed = false;
+
   for (int it = 0; it < ntiles; it++) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    uint8_t *st = smem + (it % kStages) * kStageBytes;
-    {  // widen the scales of this tile to fp32: [kv][block][token]
+    const int st = it % kStages;
+    uint8_t *stage = smem + st * kStageBytes;
+    const int tstart = t0 + it * kTile;
+    const bool tile_ok = tile_row0(tstart) >= 0;
+    const int nvalid = min(kTile, t1 - tstart);
+    if (!mbar_wait(bar0 + 8 * st, (it / kStages) & 1)) failed = true;
+    float *fsc = reinterpret_cast<float *>(smem + kOffF) + (it & 1) * kFBuf;
+    {  // widen this tile's scales to fp32 [kv][block][token]; rows past the end are 0
       const int r = tid & 63, kv = tid >> 6;
-      const uint4 w = *reinterpret_cast<const uint4 *>(st + (kv ? kOffVS : kOffKS) + r * 16);
+      const uint4 w = *reinterpret_cast<const uint4 *>(stage + (kv ? kOffVS : kOffKS) + r * 16);
+      const bool ok = r < nvalid;
       float *f = fsc + kv * 8 * kTile;
       const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int k2 = 0; k2 < 4; k2++) {
         const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&ww[k2]));
-        f[(2 * k2) * kTile + r] = p.x;
-        f[(2 * k2 + 1) * kTile + r] = p.y;
+        f[(2 * k2) * kTile + r] = ok ? p.x : 0.f;
+        f[(2 * k2 + 1) * kTile + r] = ok ? p.y : 0.f;
       }
     }
-    if (it + kStages - 1 < ntiles) issue(it + kStages - 1);
-    cp_async_commit();
-    __syncthreads();
+    // (1) scales widened; every warp is done with tile it - 1; a failed wait
+    // anywhere stops the whole CTA
+    if (__syncthreads_or(failed)) {
+      failed = true;
+      break;
+    }
+    if (tid == 0 && it + kStages - 1 < ntiles) issue(it + kStages - 1);
+    if (!tile_ok) continue;  // uniform across the CTA
 
-    const int tstart = t0 + it * kTile;
-    // tokens of this warp's 16; a tile on an unmapped page contributes nothing
-    const int live = tile_row0(tstart) < 0 ? 0 : min(kTile, t1 - tstart) - 16 * warp;
-    if (live > 0) {
-      const uint32_t kbase = smem_u32(st + kOffKC), vbase = smem_u32(st + kOffVC);
+    // ---- QK: warp w, tokens 16w .. 16w + 15
+    const uint32_t kbase = smem_u32(stage + kOffKC), vbase = smem_u32(stage + kOffVC);
+    const int live = nvalid - 16 * warp;  // tokens of this warp's 16 inside the split
+    float2 sacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    {
       const float *fk = fsc + 16 * warp + 2 * tg;
-      const float *fv = fk + 8 * kTile;
-      // ldmatrix row address of this lane in a code tile: matrix m = lane / 8
-      // -> (token group T = m & 1, block offset m >> 1), row = lane % 8
+      // ldmatrix: matrix m = lane / 8 -> (token group T = m & 1, block offset m >> 1)
       const int mr = 16 * warp + 8 * ((lane >> 3) & 1) + (lane & 7);
       const int mb = lane >> 4;
-      // ---- QK
-      float2 sacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int bp = 0; bp < 4; bp++) {
         uint32_t kr[4];
-        const int blk = 2 * bp + mb;
-        ldsm_x4(kbase + mr * 128 + ((blk ^ (mr & 7)) << 4), kr);
+        ldsm_x4(kbase + mr * 128 + (((2 * bp + mb) ^ (mr & 7)) << 4), kr);
 #pragma unroll
         for (int half = 0; half < 2; half++) {
           const int bb = 2 * bp + half;
-          uint32_t qa0[4], qa1[4];
-          ldsm_x4(qbase + (2 * bb) * 512 + qlane, qa0);
-          ldsm_x4(qbase + (2 * bb + 1) * 512 + qlane, qa1);
+          uint32_t ql[4];
+          ldsm_x4(qla + qlstep * bb, ql);
 #pragma unroll
           for (int T = 0; T < 2; T++) {
             const uint32_t w = kr[2 * half + T];
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            // chunk 0: low nibbles of bytes (0, 2) and (1, 3); chunk 1: high nibbles
-            mma16816(acc, qa0, nib64(w << 4), nib64(w >> 4));
-            mma16816(acc, qa1, nib64(w), nib64(w >> 8));
+            const uint32_t b0 = w & 0x0F0F0F0Fu, b1 = (w >> 4) & 0x0F0F0F0Fu;
+            int dhm[4], dl[4];
+            imma16832(dhm, qhm[bb], b0, b1);
+            imma16832(dl, ql, b0, b1);
+            // sum over the block of (2^14 H + 2^7 M + L)(c - 8), exact in int32
+            const int t0 = (dhm[0] << 14) + ((dhm[2] << 7) + dl[0]) - bq[bb];
+            const int t1 = (dhm[1] << 14) + ((dhm[3] << 7) + dl[1]) - bq[bb];
             const float2 d = *reinterpret_cast<const float2 *>(fk + bb * kTile + 8 * T);
-            const float2 hl = make_float2(acc[0] + acc[2] - sqb[bb], acc[1] + acc[3] - sqb[bb]);
-            sacc[T] = ffma2(d, hl, sacc[T]);
+            sacc[T] = __ffma2_rn(d, make_float2((float)t0, (float)t1), sacc[T]);
           }
         }
       }
-      // ---- online softmax (base 2) for head g over this warp's 16 tokens
-      const float2 sl2 = make_float2(scale_log2, scale_log2);
-      const float2 s0 = __fmul2_rn(sacc[0], sl2), s1 = __fmul2_rn(sacc[1], sl2);
-      float sc[4] = {s0.x, s0.y, s1.x, s1.y};
-      if (live < 16) {
+    }
+    // ---- softmax: tile maximum per head across the four warps
+    float sc[4] = {sacc[0].x * sl2, sacc[0].y * sl2, sacc[1].x * sl2, sacc[1].y * sl2};
+    if (live < 16) {
 #pragma unroll
-        for (int e = 0; e < 4; e++)
-          if (8 * (e >> 1) + 2 * tg + (e & 1) >= live) sc[e] = -INFINITY;
+      for (int e = 0; e < 4; e++)
+        if (8 * (e >> 1) + 2 * tg + (e & 1) >= live) sc[e] = -INFINITY;
+    }
+    float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    if (tg == 0) red[warp * 8 + g] = mx;
+    __syncthreads();  // (2)
+    const float mt_ = fmaxf(fmaxf(red[g], red[8 + g]), fmaxf(red[16 + g], red[24 + g]));
+    if (__any_sync(kFull, mt_ > m_run + 8.f)) {
+      const float mn = fmaxf(m_run, mt_);
+      const float alpha = exp2f(m_run - mn);  // 0 while m_run is -inf
+      m_run = mn;
+      l_run *= alpha;
+      swb[0] *= alpha;
+      swb[1] *= alpha;
+      const float a0 = __shfl_sync(kFull, alpha, 8 * tg);      // head 2tg
+      const float a1 = __shfl_sync(kFull, alpha, 8 * tg + 4);  // head 2tg + 1
+#pragma unroll
+      for (int mt = 0; mt < 4; mt++) {
+        o[mt][0] *= a0;
+        o[mt][1] *= a1;
+        o[mt][2] *= a0;
+        o[mt][3] *= a1;
       }
-      float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-      if (__any_sync(kFull, mx > m_run + 8.f)) {
-        const float mn = fmaxf(m_run, mx);
-        const float alpha = exp2f(m_run - mn);  // 0 while m_run is -inf
-        m_run = mn;
-        l_run *= alpha;
-#pragma unroll
-        for (int bb = 0; bb < 8; bb++) swb[bb] *= alpha;
-        const float a0 = __shfl_sync(kFull, alpha, 8 * tg);      // head 2tg
-        const float a1 = __shfl_sync(kFull, alpha, 8 * tg + 4);  // head 2tg + 1
-#pragma unroll
-        for (int mt = 0; mt < 16; mt++) {
-          o[mt][0] *= a0;
-          o[mt][1] *= a1;
-          o[mt][2] *= a0;
-          o[mt][3] *= a1;
-        }
-      }
+    }
+    {
       float p[4];
 #pragma unroll
       for (int e = 0; e < 4; e++) {
         p[e] = exp2f(sc[e] - m_run);
         l_run += p[e];
       }
-      const float2 p01 = make_float2(p[0], p[1]), p23 = make_float2(p[2], p[3]);
-      // ---- PV: per block, B = p * d_v (hi / lo), A = V^T codes
+      float *pr = pbuf + g * kPStride + 16 * warp + 2 * tg;
+      *reinterpret_cast<float2 *>(pr) = make_float2(p[0], p[1]);
+      *reinterpret_cast<float2 *>(pr + 8) = make_float2(p[2], p[3]);
+    }
+    __syncthreads();  // (3) p of all 64 tokens
+    // ---- PV: warp w, blocks 2w, 2w + 1, all 64 tokens in 4 steps of 16
+    {
+      const float *fv = fsc + 8 * kTile + (2 * warp) * kTile + 2 * tg;
+      const float *pp = pbuf + g * kPStride + 2 * tg;
+      const int blk = 2 * warp + (lane >> 4);  // ldmatrix block of this lane's matrices
 #pragma unroll
-      for (int bp = 0; bp < 4; bp++) {
-        uint32_t vr[4];
-        const int blk = 2 * bp + mb;
+      for (int ks = 0; ks < 4; ks++) {
+        const int mr = 16 * ks + 8 * ((lane >> 3) & 1) + (lane & 7);
+        uint32_t vr[4];  // (T0, blk 2w), (T1, blk 2w), (T0, blk 2w+1), (T1, blk 2w+1)
         ldsm_x4_t(vbase + mr * 128 + ((blk ^ (mr & 7)) << 4), vr);
+        const float2 p01 = *reinterpret_cast<const float2 *>(pp + 16 * ks);
+        const float2 p23 = *reinterpret_cast<const float2 *>(pp + 16 * ks + 8);
 #pragma unroll
         for (int half = 0; half < 2; half++) {
-          const int bb = 2 * bp + half;
-          float2 w0 = __fmul2_rn(p01, *reinterpret_cast<const float2 *>(fv + bb * kTile));
-          float2 w1 = __fmul2_rn(p23, *reinterpret_cast<const float2 *>(fv + bb * kTile + 8));
-          if (live < 16) {  // tokens past the end: p is 0, keep a stale scale out too
-            if (2 * tg >= live) w0.x = 0.f;
-            if (2 * tg + 1 >= live) w0.y = 0.f;
-            if (8 + 2 * tg >= live) w1.x = 0.f;
-            if (9 + 2 * tg >= live) w1.y = 0.f;
-          }
-          swb[bb] += (w0.x + w0.y) + (w1.x + w1.y);
+          const float2 w0 =
+              __fmul2_rn(p01, *reinterpret_cast<const float2 *>(fv + half * kTile + 16 * ks));
+          const float2 w1 =
+              __fmul2_rn(p23, *reinterpret_cast<const float2 *>(fv + half * kTile + 16 * ks + 8));
+          swb[half] += (w0.x + w0.y) + (w1.x + w1.y);
           uint32_t bh0, bl0, bh1, bl1;
           split_hilo(w0, bh0, bl0);
           split_hilo(w1, bh1, bl1);
           const uint32_t r0 = vr[2 * half], r1 = vr[2 * half + 1];  // tokens 0-7, 8-15
           {  // even M-tile: rows g <-> low nibble of byte 2g, rows g + 8 <-> its high nibble
             const uint32_t a[4] = {nib64(r0 << 4), nib64(r0), nib64(r1 << 4), nib64(r1)};
-            float(&acc)[4] = o[2 * bb];
-            mma16816(acc, a, bh0, bh1);
-            mma16816(acc, a, bl0, bl1);
+            mma16816(o[2 * half], a, bh0, bh1);
+            mma16816(o[2 * half], a, bl0, bl1);
           }
           {  // odd M-tile: byte 2g + 1
             const uint32_t a[4] = {nib64(r0 >> 4), nib64(r0 >> 8), nib64(r1 >> 4),
                                    nib64(r1 >> 8)};
-            float(&acc)[4] = o[2 * bb + 1];
-            mma16816(acc, a, bh0, bh1);
-            mma16816(acc, a, bl0, bl1);
+            mma16816(o[2 * half + 1], a, bh0, bh1);
+            mma16816(o[2 * half + 1], a, bl0, bl1);
           }
         }
       }
     }
   }
-  cp_async_wait<0>();
-  __syncthreads();
 
-  // ---- remove the 72 * sum(p d_v) bias, merge the four warps, write partials
-#pragma unroll
-  for (int bb = 0; bb < 8; bb++) {
-    swb[bb] += __shfl_xor_sync(kFull, swb[bb], 1);
-    swb[bb] += __shfl_xor_sync(kFull, swb[bb], 2);
+  // ---- partial records: m (same in every warp), l summed over warps, o per warp
+  if (failed) {
+    // a load never arrived: let what was issued land (bounded), then mark the
+    // records of this split invalid with NaN so the output shows it
+    __syncthreads();
+    if (tid == 0)
+      for (int i = 0; i < kStages; i++) (void)mbar_wait(bar0 + 8 * i, 0), (void)mbar_wait(bar0 + 8 * i, 1);
+    __syncthreads();
+    for (int p = tid; p < gc * kRec; p += kThreads) {
+      const int hh = p / kRec, j = p % kRec;
+      ws[(((int64_t)b * n_q_heads + h0 + hh) * splits + s) * kRec + j] = __int_as_float(0x7fc00000);
+    }
+    return;
   }
-  float *red_o = reinterpret_cast<float *>(smem);            // [warp][8 heads][256]
-  float *red_m = red_o + kWarps * 8 * kDim;                 // [warp][8]
-  float *red_l = red_m + kWarps * 8;
   l_run += __shfl_xor_sync(kFull, l_run, 1);
   l_run += __shfl_xor_sync(kFull, l_run, 2);
-  if (tg == 0) {
-    red_m[warp * 8 + g] = m_run;
-    red_l[warp * 8 + g] = l_run;
-  }
+  __syncthreads();  // red is reused
+  if (tg == 0) red[kWarps * 8 + warp * 8 + g] = l_run;
 #pragma unroll
-  for (int bb = 0; bb < 8; bb++) {
-    const float c0 = kBias * __shfl_sync(kFull, swb[bb], 8 * tg);      // head 2tg
-    const float c1 = kBias * __shfl_sync(kFull, swb[bb], 8 * tg + 4);  // head 2tg + 1
-#pragma unroll
-    for (int par = 0; par < 2; par++) {
-      const float(&acc)[4] = o[2 * bb + par];
-      const int d0 = 32 * bb + 2 * g + par;  // dim of row g; row g + 8 is d0 + 16
-      float *w = red_o + warp * 8 * kDim;
-      w[(2 * tg) * kDim + d0] = acc[0] - c0;
-      w[(2 * tg + 1) * kDim + d0] = acc[1] - c1;
-      w[(2 * tg) * kDim + d0 + 16] = acc[2] - c0;
-      w[(2 * tg + 1) * kDim + d0 + 16] = acc[3] - c1;
-    }
+  for (int half = 0; half < 2; half++) {
+    swb[half] += __shfl_xor_sync(kFull, swb[half], 1);
+    swb[half] += __shfl_xor_sync(kFull, swb[half], 2);
   }
   __syncthreads();
-  for (int p = tid; p < gc * kDim; p += kThreads) {
-    const int hh = p >> 8, j = p & 255;
-    float M = -INFINITY;
+  const int hA = 2 * tg, hB = 2 * tg + 1;  // heads of this lane's O columns
 #pragma unroll
-    for (int w = 0; w < kWarps; w++) M = fmaxf(M, red_m[w * 8 + hh]);
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
+  for (int half = 0; half < 2; half++) {
+    const float cA = kBias * __shfl_sync(kFull, swb[half], 4 * hA);
+    const float cB = kBias * __shfl_sync(kFull, swb[half], 4 * hB);
 #pragma unroll
-      for (int w = 0; w < kWarps; w++) {
-        const float f = exp2f(red_m[w * 8 + hh] - M);
-        L += red_l[w * 8 + hh] * f;
-        O += red_o[(w * 8 + hh) * kDim + j] * f;
+    for (int par = 0; par < 2; par++) {
+      const float(&acc)[4] = o[2 * half + par];
+      const int d0 = 64 * warp + 32 * half + 2 * g + par;  // row g; row g + 8 is d0 + 16
+      if (hA < gc) {
+        float *rec = ws + (((int64_t)b * n_q_heads + h0 + hA) * splits + s) * kRec + 4;
+        rec[d0] = acc[0] - cA;
+        rec[d0 + 16] = acc[2] - cA;
+      }
+      if (hB < gc) {
+        float *rec = ws + (((int64_t)b * n_q_heads + h0 + hB) * splits + s) * kRec + 4;
+        rec[d0] = acc[1] - cB;
+        rec[d0 + 16] = acc[3] - cB;
       }
     }
-    float *rec = ws + (((int64_t)b * n_q_heads + h0 + hh) * splits + s) * kRec;
-    rec[4 + j] = O;
-    if (j == 0) {
-      rec[0] = M;
-      rec[1] = L;
-    }
   }
+  if (warp == 0 && tg == 0 && g < gc) {
+    float *rec = ws + (((int64_t)b * n_q_heads + h0 + g) * splits + s) * kRec;
+    rec[0] = m_run;
+    rec[1] = red[kWarps * 8 + g] + red[kWarps * 8 + 8 + g] + red[kWarps * 8 + 16 + g] +
+             red[kWarps * 8 + 24 + g];
+  }
+}
+
+// ---- host: 2-D tensor maps over the cache planes (cached per plane)
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// rows x row_bytes uint8 plane, boxes of 64 rows x row_bytes
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t row_bytes, bool swizzle) {
+  struct Entry {
+    const void *base;
+    uint64_t rows;
+    uint32_t row_bytes;
+    CUtensorMap map;
+  };
+  static Entry cache[16];
+  static int next = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry &e : cache)
+    if (e.base == base && e.rows == rows && e.row_bytes == row_bytes) {
+      *m = e.map;
+      return true;
+    }
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {row_bytes, (cuuint32_t)kTile};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  cache[next] = Entry{base, rows, row_bytes, *m};
+  next = (next + 1) % 16;
+  return true;
 }
 
 }  // namespace
@@ -449,26 +570,42 @@ cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, in
   const int gc = group < 8 ? group : 8;
   dim3 grid(p.splits, n_q_heads / gc, batch);
   const float sl2 = scale * kLog2e;
+  const uint64_t rows = c.block_table
+                            ? (uint64_t)c.num_pages * c.num_kv_heads * c.page_size
+                            : (uint64_t)c.batch_capacity * c.num_kv_heads * c.max_tokens;
+  if (rows >= (1ull << 31)) return cudaErrorInvalidValue;  // TMA row coordinates are 32-bit
+  TmaMaps maps;
+  if (!make_map(&maps.kc, c.k_codes, rows, 128, true) ||
+      !make_map(&maps.vc, c.v_codes, rows, 128, true) ||
+      !make_map(&maps.ks, c.k_scales, rows, 16, false) ||
+      !make_map(&maps.vs, c.v_scales, rows, 16, false))
+    return cudaErrorInvalidValue;
   // opt in to the large dynamic shared-memory carve-out once per device
+  static std::mutex mu;
   static unsigned configured[2] = {0u, 0u};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const unsigned bit = 1u << (dev & 31);
-  if (!(configured[bf16] & bit)) {
-    e = bf16 ? cudaFuncSetAttribute(q4_decode_mma_kernel<true>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)
-             : cudaFuncSetAttribute(q4_decode_mma_kernel<false>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured[bf16] |= bit;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const unsigned bit = 1u << (dev & 31);
+    if (!(configured[bf16] & bit)) {
+      e = bf16 ? cudaFuncSetAttribute(q4_decode_mma_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)
+               : cudaFuncSetAttribute(q4_decode_mma_kernel<false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      if (e != cudaSuccess) return e;
+      configured[bf16] |= bit;
+    }
   }
   if (bf16)
     q4_decode_mma_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(
-        c, q, seq_lens, max_seq_len, n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws);
+        maps, c, q, seq_lens, max_seq_len, n_q_heads, group, gc, sl2, p.split_tokens, p.splits,
+        ws);
   else
     q4_decode_mma_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(
-        c, q, seq_lens, max_seq_len, n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws);
+        maps, c, q, seq_lens, max_seq_len, n_q_heads, group, gc, sl2, p.split_tokens, p.splits,
+        ws);
   return cudaGetLastError();
 }
 

@@ -277,6 +277,6 @@ def octave_attention(query, cache, block_table, q_to_req, q_to_klen, fmt, scale,
     s = np.ascontiguousarray(signs, dtype=np.float32)
     out = np.zeros((nq, hq, d), np.float64)
     _check(lib().orc_octave_attention(*fmt, _p(query), _dtype_code(query), nq, hq, _p(cache),
-                                      hkv, bs, _p(bt), bt.shape[1], _p(qr), _p(ql),
+                                      C.c_int64(cache.shape[0]), hkv, bs, _p(bt), bt.shape[1], _p(qr), _p(ql),
                                       C.c_double(scale), _p(s), _p(out)), "octave_attention")
     return out

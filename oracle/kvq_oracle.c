@@ -676,7 +676,8 @@ int orc_octave_dequantize(int head_size, int rope_dim, int v_bits, int compact,
  * here; klen <= 0 gives a zero row. */
 int orc_octave_attention(int head_size, int rope_dim, int v_bits, int compact,
                          const void *query, int dtype, int n_q, int n_q_heads,
-                         const uint8_t *cache, int n_kv_heads, int block_size,
+                         const uint8_t *cache, int64_t num_blocks, int n_kv_heads,
+                         int block_size,
                          const int32_t *block_table, int max_blocks,
                          const int32_t *q_to_req, const int32_t *q_to_klen, double scale,
                          const float *signs, double *out) {
@@ -693,6 +694,10 @@ int orc_octave_attention(int head_size, int rope_dim, int v_bits, int compact,
     if (klen <= 0) continue;
     if ((klen - 1) / block_size >= max_blocks) return -1;
     int req = q_to_req[i];
+    for (int t = 0; t < klen; t += block_size) {
+      int32_t blk = block_table[(int64_t)req * max_blocks + t / block_size];
+      if (blk < 0 || blk >= num_blocks) return -1;
+    }
     double *k = (double *)malloc(sizeof(double) * (size_t)klen * n_kv_heads * d);
     double *v = (double *)malloc(sizeof(double) * (size_t)klen * n_kv_heads * d);
     uint8_t *slots = (uint8_t *)malloc((size_t)klen * n_kv_heads * f.slot_bytes);

@@ -127,10 +127,11 @@ int orc_octave_dequantize(int head_size, int rope_dim, int v_bits, int compact,
                           const float *signs, int rotated, double *k,
                           double *v);
 /* query: [Q][Hq][d]; cache: [num_blocks][Hkv][block_size][slot];
- * block_table: [num_reqs][max_blocks]; out: [Q][Hq][d] fp64. */
+ * block_table: [num_reqs][max_blocks]; an entry a query reads must name one of
+ * the num_blocks blocks, else -1 is returned.  out: [Q][Hq][d] fp64. */
 int orc_octave_attention(int head_size, int rope_dim, int v_bits, int compact,
                          const void *query, int dtype, int n_q, int n_q_heads,
-                         const uint8_t *cache, int n_kv_heads, int block_size,
+                         const uint8_t *cache, int64_t num_blocks, int n_kv_heads, int block_size,
                          const int32_t *block_table, int max_blocks,
                          const int32_t *q_to_req, const int32_t *q_to_klen,
                          double scale, const float *signs, double *out);

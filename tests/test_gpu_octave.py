@@ -70,30 +70,38 @@ def test_quantize_skips_negative_and_out_of_range_slots():
     assert np.any(c[0, :, 3] != 0)
 
 
-@pytest.mark.parametrize("G", [1, 4, 8])
-def test_decode_vs_oracle(G):
-    fmt = (128, 64, 4, 0)
-    F = kvq.OctaveFormat(128, 64, 4)
-    Hkv, bs = 2, 16
+def decode_case(v_bits, G, bs, qdt, seed=21):
+    """Requests over a shuffled block mapping; returns what both sides need."""
+    fmt = (128, 64, v_bits, 0)
+    F = kvq.OctaveFormat(128, 64, v_bits)
+    slot_bytes = F.layout()["slot_bytes"]
+    Hkv = 2
     Hq = Hkv * G
-    lens = np.array([300, 45, 0, 129], np.int32)
-    nreq = 3
     T = 600
-    k, v, slot, nblk = make_cache(fmt, T, Hkv, bs, 21)
+    k, v, slot, nblk = make_cache(fmt, T, Hkv, bs, seed)
     signs = synth.sign_pattern(128)
-    cache = torch.zeros((nblk, Hkv, bs, 128), dtype=torch.uint8, device="cuda")
+    cache = torch.zeros((nblk, Hkv, bs, slot_bytes), dtype=torch.uint8, device="cuda")
     kvq.octave_quantize(F, to_dev(k), to_dev(v), to_dev(slot), cache, kvq.sign_words(signs))
-    # requests: req r owns tokens [200 r, 200 r + 200) through their blocks
-    maxb = 200 // bs + 1
+    # request r owns the blocks holding tokens [192 r, 192 r + 192)
+    nreq, span = 3, 192
+    maxb = -(-span // bs)
     bt = np.zeros((nreq, maxb), np.int32)
     for r in range(nreq):
         for j in range(maxb):
-            tok = min(200 * r + j * bs, T - 1)
-            bt[r, j] = slot[tok] // bs
-    # only use request prefixes that are block aligned with the mapping above
+            bt[r, j] = slot[min(span * r + j * bs, T - 1)] // bs
+    q = synth.queries(seed + 10, 4, Hq, 128)
+    if qdt == "bf16":
+        q = synth.to_bf16_bits(q)
+    return F, fmt, cache, bt, q, signs
+
+
+@pytest.mark.parametrize("v_bits", [4, 3])  # 4: tensor-core kernel, 3: SIMT kernel
+@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("qdt", ["bf16", "f32"])
+def test_decode_vs_oracle(v_bits, G, qdt):
+    F, fmt, cache, bt, q, signs = decode_case(v_bits, G, 16, qdt)
     q_to_req = np.array([0, 1, 2, 0], np.int32)
-    q_to_klen = np.minimum(lens, 192)
-    q = synth.to_bf16_bits(synth.queries(31, len(lens), Hq, 128))
+    q_to_klen = np.array([192, 45, 0, 129], np.int32)
     got = kvq.octave_decode_attn(F, to_dev(q), cache, to_dev(bt), to_dev(q_to_req),
                                  to_dev(q_to_klen), 192, 128 ** -0.5,
                                  kvq.sign_words(signs)).cpu().numpy()
@@ -101,6 +109,49 @@ def test_decode_vs_oracle(G):
                                    128 ** -0.5, signs)
     assert np.all(got[2] == 0)
     assert np.abs(got - want).max() <= ATOL
+
+
+@pytest.mark.parametrize("v_bits", [4, 3])
+@pytest.mark.parametrize("bs", [1, 24, 64, 256])
+def test_decode_block_sizes(v_bits, bs):
+    """Block sizes below, across and above the 64-token tile."""
+    F, fmt, cache, bt, q, signs = decode_case(v_bits, 4, bs, "bf16", seed=40 + bs)
+    q_to_req = np.array([2, 0, 1, 1], np.int32)
+    q_to_klen = np.array([192, 191, 65, 1], np.int32)
+    got = kvq.octave_decode_attn(F, to_dev(q), cache, to_dev(bt), to_dev(q_to_req),
+                                 to_dev(q_to_klen), 192, 128 ** -0.5,
+                                 kvq.sign_words(signs)).cpu().numpy()
+    want = oracle.octave_attention(q, cache.cpu().numpy(), bt, q_to_req, q_to_klen, fmt,
+                                   128 ** -0.5, signs)
+    assert np.abs(got - want).max() <= ATOL
+
+
+@pytest.mark.parametrize("v_bits", [4, 3])
+def test_decode_unmapped_blocks_contribute_nothing(v_bits):
+    """A block-table entry that names no block (-1 or past the cache) drops its
+    tokens: decode attention has no positional term, so the result equals the
+    oracle over the table with those entries removed."""
+    bs = 16
+    F, fmt, cache, bt, q, signs = decode_case(v_bits, 8, bs, "bf16", seed=60)
+    nblk = cache.shape[0]
+    holes = bt.copy()
+    holes[0, 3] = -1
+    holes[0, 7] = nblk + 5
+    holes[1, 0] = -1
+    keep0 = [j for j in range(bt.shape[1]) if j not in (3, 7)]
+    keep1 = [j for j in range(bt.shape[1]) if j != 0]
+    q_to_req = np.array([0, 1], np.int32)
+    q_to_klen = np.array([192, 192], np.int32)
+    got = kvq.octave_decode_attn(F, to_dev(q[:2]), cache, to_dev(holes), to_dev(q_to_req),
+                                 to_dev(q_to_klen), 192, 128 ** -0.5,
+                                 kvq.sign_words(signs)).cpu().numpy()
+    c = cache.cpu().numpy()
+    for i, keep in enumerate((keep0, keep1)):
+        compact = bt[i, keep][None, :]
+        want = oracle.octave_attention(q[i:i + 1], c, compact, np.zeros(1, np.int32),
+                                       np.array([bs * len(keep)], np.int32), fmt,
+                                       128 ** -0.5, signs)
+        assert np.abs(got[i:i + 1] - want).max() <= ATOL
 
 
 def test_octave_workload_sampled():

@@ -258,6 +258,36 @@ def test_decode_paged_equals_contiguous_and_oracle():
     np.testing.assert_array_equal(gp, gcn)  # same tokens, same splits -> same bits
 
 
+def test_decode_unmapped_pages_contribute_nothing():
+    """Page-table entries that name no page (-1, or past the pool) drop their
+    tokens; with no positional term in decode attention the result equals the
+    oracle over the table with those pages removed."""
+    B, H, G, ps = 2, 2, 4, 64
+    lens = np.array([640, 300], np.int32)
+    T = int(lens.max())
+    bt, n_pages = paged_setup(13, B, H, lens, ps)
+    k = synth.to_bf16_bits(synth.gaussian(95, (B, T, H, 256)))
+    v = synth.to_bf16_bits(synth.gaussian(96, (B, T, H, 256)))
+    q = synth.to_bf16_bits(synth.queries(97, B, H * G, 256))
+    pc = kvq.Q4Cache.paged(n_pages, H, ps, torch.from_numpy(bt))
+    oc = oracle.Q4Cache(n_pages * H * ps, H, block_table=bt, page_size=ps)
+    append_paged(pc, oc, k, v, lens, bt)
+    holes = bt.copy()
+    holes[0, 3] = -1
+    holes[0, 6] = n_pages + 2
+    holes[1, 1] = -1
+    got = kvq.decode_attn(pc.with_block_table(torch.from_numpy(holes)), to_dev(q),
+                          to_dev(lens), T, 0.0625).cpu().numpy()
+    compact = np.full_like(bt, -1)
+    keep0 = [j for j in range(10) if j not in (3, 6)]
+    keep1 = [j for j in range(5) if j != 1]
+    compact[0, :len(keep0)] = bt[0, keep0]
+    compact[1, :len(keep1)] = bt[1, keep1]
+    clens = np.array([640 - 2 * ps, 300 - ps], np.int32)
+    want = oc.with_block_table(compact).decode_attn(q, clens, 0.0625)
+    assert np.abs(got - want).max() <= ATOL
+
+
 # ------------------------------------------------------------------ full size
 def test_long_decode_full_size_sampled():
     """Long-context workload at full size (1 x 131072 tokens, 32 q / 4 kv
