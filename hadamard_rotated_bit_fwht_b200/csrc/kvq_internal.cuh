@@ -76,10 +76,12 @@ struct DecodePlan {
   int split_tokens; // tokens per split (multiple of 64)
 };
 // split-K plan over `units` independent problems with `slots` resident CTAs
-DecodePlan plan_split_k(int units, int max_len, int slots, int max_splits);
+DecodePlan plan_split_k(int units, int max_len, int slots, int max_splits, int granule = 64,
+                        int overhead_tokens = 0);
 // n_head_groups: q heads / min(group, 8), the CTAs per sequence and split
 DecodePlan plan_decode(int batch, int n_head_groups, int max_seq_len);
 int q4_decode_ctas_per_sm();
+int q4_decode_tile_tokens();
 cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, int batch,
                                  int n_q_heads, const int32_t *seq_lens, int max_seq_len,
                                  float scale, float *ws, const DecodePlan &p, cudaStream_t s);

@@ -46,6 +46,8 @@ __global__ void __launch_bounds__(256)
   __shared__ float ob[kDim];
   __shared__ float wgt[kMaxSplitsSmem];
   __shared__ float red[8];
+  // the partial records come from the split kernel launched just before
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x, j = threadIdx.x, lane = j & 31, warp = j >> 5;
   const int b = bh / n_q_heads;
   const int len = min(max(__ldg(seq_lens + b), 0), min(max_seq_len, cap));
@@ -94,26 +96,28 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-DecodePlan plan_split_k(int units, int max_len, int slots, int max_splits) {
+DecodePlan plan_split_k(int units, int max_len, int slots, int max_splits, int granule,
+                        int overhead_tokens) {
   // Each of `units` independent problems (sequence, q-head group) is cut into
-  // splits of whole 64-token tiles, at least 256 tokens each.  With `slots`
-  // CTAs resident at once, the kernel takes about waves x tokens-per-split; the
-  // split count minimising that (fewest splits on ties) wins, so a second wave
-  // is only chosen when it shortens every split by more than half.
+  // splits of whole `granule`-token tiles, at least 256 tokens each.  With
+  // `slots` CTAs resident at once, the kernel takes about
+  // waves x (tokens per split + a fixed per-CTA cost); the split count
+  // minimising that (fewest splits on ties) wins.
   const int len = max(max_len, 1);
-  const int tiles = (len + 63) / 64;
+  const int tiles = (len + granule - 1) / granule;
   units = max(units, 1);
   DecodePlan best;
-  best.split_tokens = max(tiles * 64, 256);
+  const int min_tiles = max(256 / granule, 1);
+  best.split_tokens = max(tiles, min_tiles) * granule;
   best.splits = 1;
   int64_t best_cost = -1;
   const int sp_max = min(tiles, 2 * ((slots + units - 1) / units) + 1);
   for (int sp = 1; sp <= sp_max; sp++) {
-    const int per = max(((tiles + sp - 1) / sp) * 64, 256);
+    const int per = max((tiles + sp - 1) / sp, min_tiles) * granule;
     const int splits = (len + per - 1) / per;
     if (splits > max_splits) continue;
     const int64_t waves = ((int64_t)units * splits + slots - 1) / slots;
-    const int64_t cost = waves * per;
+    const int64_t cost = waves * (per + overhead_tokens);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best.split_tokens = per;
@@ -128,8 +132,10 @@ DecodePlan plan_split_k(int units, int max_len, int slots, int max_splits) {
 }
 
 DecodePlan plan_decode(int batch, int n_head_groups, int max_seq_len) {
+  // ~3 tiles' worth of per-CTA work (query rotation, ring fill, final merge)
+  const int tile = q4_decode_tile_tokens();
   return plan_split_k(batch * n_head_groups, max_seq_len, kNumSMs * q4_decode_ctas_per_sm(),
-                      kMaxSplitsSmem);
+                      kMaxSplitsSmem, tile, 3 * tile);
 }
 
 size_t decode_workspace_bytes(int batch, int n_q_heads, const DecodePlan &p) {
@@ -145,8 +151,20 @@ cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int ba
                                        scale, ws, p, s);
   if (e != cudaSuccess) return e;
   const int cap = c.block_table ? c.max_pages_per_seq * c.page_size : c.max_tokens;
-  q4_decode_combine_kernel<<<batch * n_q_heads, 256, 0, s>>>(ws, seq_lens, n_q_heads, p.splits,
-                                                             max_seq_len, cap, out);
+  // programmatic dependent launch: scheduled while the split kernel drains,
+  // waits for its records with griddepcontrol.wait
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(batch * n_q_heads);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, q4_decode_combine_kernel, (const float *)ws, seq_lens, n_q_heads,
+                         p.splits, max_seq_len, cap, out);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -1,41 +1,39 @@
-// q4_decode_mma.cu -- tensor-core split-K decode attention over the Q4_0 +
-// FWHT-256 cache (Strata PR #21 "Q4_0 KV cache + FWHT-256": What, How 2 and the
+// q4_decode_mma.cu -- split-K decode attention over the Q4_0 + FWHT-256 cache on
+// the tensor cores (Strata PR #21 "Q4_0 KV cache + FWHT-256": What, How 2 and the
 // merge note's per-token path that rotates Q and the output).
 //
 // With GQA the decode step is a small dense contraction per kv head:
-// S = Q_rot K^T (G x T) and O = P V (G x 256), G <= 8 heads per CTA.  Both
-// products run on the tensor cores (warp-level mma.sync) at fp32-level
-// accuracy; a CTA of four warps walks its split in 64-token tiles:
-//   * Tiles arrive by TMA (cp.async.bulk.tensor, 2-D maps over the cache's
-//     128-byte code rows and 16-byte scale rows, hardware 128-byte swizzle)
-//     into a ring of shared-memory stages guarded by mbarriers; one thread
-//     issues, every wait is bounded.
-//   * QK: warp w scores tokens 16w..16w+15 of the tile for all 8 heads on the
-//     integer tensor path (m16n8k32, s8 x u8 -> s32).  A Q4_0 block is 32
-//     dims, one MMA K-step; its codes enter as bytes with three logic ops per
-//     8 codes (low nibbles = dims 0..15, high nibbles = dims 16..31 of the
-//     block, the B-fragment rows).  The rotated query of each head is scaled
-//     by S = 127 * 2^14 / max|q| and split exactly into int8 levels H, M, L
-//     with S q = 2^14 H + 2^7 M + L (|M|, |L| <= 64); one MMA takes H and M
-//     (rows 0-7, 8-15), a second takes L.  Their accumulators start at the
-//     bits of 1.5 * 2^23 minus the zero-point term 8 * sum(level), so each
-//     exact integer sum over the block becomes an fp32 by one subtraction;
-//     2^7 F_HM + F_L times the block's scale is added to the score.  The
-//     query is carried to about 2^-22 of its largest element.
-//   * Softmax: the tile maximum per head is shared through shared memory, so
-//     every warp keeps the same running maximum (rescaling lazily, only when
-//     a score passes it by 8); p goes to shared memory.
-//   * PV: warp w owns output dims 64w..64w+63 (Q4_0 blocks 2w, 2w+1) for all
-//     64 tokens of the tile: A = V^T codes as the exact fp16 values 64 + c (a
-//     nibble in bits 4..7 of a 16-bit lane OR-ed with the bits of 64.0, one
-//     LOP3 per pair, read by ldmatrix.trans), B = p * d_v split into fp16
-//     hi + lo (the 16 dims of an M-tile lie in one block, so the V scale rides
-//     in B).  The bias 64 + 8 = 72 is removed at the end with
-//     72 * sum_t(p d_v) per (head, block).
-//   * The QK accumulator layout (head g = lane / 4, tokens 2(lane % 4) + {0,1})
-//     is the PV B-fragment layout for tokens {0..7} and {8..15}.
+// S = Q_rot K^T (G x T) and O = P V (G x 256), G <= 8 heads per CTA.  One CTA
+// per SM (8 warps, ~200 KB of shared memory):
+//   * 128-token tiles of the split (codes and fp16 scales of K and V, 36 KB)
+//     stream by TMA (2-D maps over the 128-byte code rows and 16-byte scale
+//     rows, hardware 128-byte swizzle) into a ring of 5 stages, each guarded by
+//     a full mbarrier.  The first 5 tiles are issued at kernel start, before
+//     the query is prepared; afterwards the last warp to release a stage (a
+//     shared-memory counter per stage) issues its refill, so no warp is spent
+//     on producing and every warp keeps the full register budget.  Every wait
+//     is bounded.
+//   * warp w owns tokens 16w .. 16w+15 of every tile and runs its own online
+//     softmax over them (no CTA-wide barrier per tile).  The 8 running states
+//     are merged once at the end of the split.
+//   * QK on mma.sync m16n8k16 (f16 x f16 -> f32): A = the rotated query of the
+//     8 heads split exactly into fp16 hi (rows 0-7) and lo (rows 8-15), held in
+//     registers for the whole split; B = K codes of 8 tokens as the exact fp16
+//     values 64 + c (a nibble in bits 4..7 of a 16-bit lane OR-ed with the bits
+//     of 64.0, one LOP3 per pair).  One Q4_0 block (32 dims) is two k-steps; the
+//     dims of a k-step are permuted (the same way in A and B) so that each
+//     thread's code word feeds both k-steps without a byte shuffle.  The
+//     accumulator starts at -72 * sum(q over the block) (zero point 8 plus the
+//     magic 64), and hi + lo times the block's scale is added to the score.
+//   * PV on mma.sync: A = V^T codes (64 + c, via ldmatrix.trans), B = p * d_v
+//     split into fp16 hi + lo (the 32 dims of a block share the token's scale,
+//     so the scale rides in B); O = 16 dims x 8 heads per M-tile, 64 fp32
+//     registers per thread.  The bias 72 * sum_t(p d_v) per (head, block) is
+//     removed at the end.
+//   * The QK accumulator layout (head g = lane / 4, tokens 2(lane % 4) + {0,1},
+//     + 8) is the PV B-fragment layout, so p never leaves registers.
 // Split-K partials (m, l, o[256]) per (sequence, q head, split) go to the
-// combine + back-rotation kernel.
+// combine + back-rotation kernel (q4_decode.cu).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -46,39 +44,47 @@
 namespace kvq {
 namespace {
 
-constexpr int kWarps = 4;
+constexpr int kWarps = 8;           // 2 groups of 4; group gq takes the tiles it with it % 2 == gq
 constexpr int kThreads = 32 * kWarps;
-constexpr int kTile = 64;          // tokens per stage (16 per warp for QK)
-constexpr int kStages = 2;
-constexpr int kCtasPerSm = 4;
+constexpr int kTile = 128;          // tokens per stage, 32 per warp of the group
+constexpr int kSub = 64;            // rows per TMA box (the page-size granule)
+constexpr int kStages = 4;          // even: stage it % 4 always serves group it % 2
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kRec = 260;          // partial record: m, l, pad, pad, o[256]
+constexpr int kRec = 260;           // partial record: m, l, pad, pad, o[256]
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kBias = 72.f;      // 64 (magic) + 8 (Q4_0 zero point)
-constexpr float kQRange = 2080768.f;         // 127 * 2^14
-constexpr uint32_t kTileBytes = 2 * kTile * 128 + 2 * kTile * 16;  // one TMA transaction
+constexpr float kBias = 72.f;       // 64 (magic) + 8 (Q4_0 zero point)
+constexpr uint32_t kSubBytes = 2 * kSub * 128 + 2 * kSub * 16;  // one sub-tile, K + V
 
-// shared memory layout (bytes from a 1024-aligned base: 128-byte swizzle atoms)
-constexpr int kOffKC = 0;                       // K codes: 64 rows x 128 B (TMA-swizzled)
-constexpr int kOffVC = kOffKC + kTile * 128;    // V codes
-constexpr int kOffKS = kOffVC + kTile * 128;    // K scales: 64 rows x 8 fp16
-constexpr int kOffVS = kOffKS + kTile * 16;     // V scales
-constexpr int kStageBytes = kOffVS + kTile * 16;  // 18432 = 18 KiB
-constexpr int kOffF = kStages * kStageBytes;    // fp32 scales, 2 buffers x [kv][block][token]
-constexpr int kFBuf = 2 * 8 * kTile;            // floats per buffer
-constexpr int kPStride = 72;                    // p rows: 64 tokens + pad (conflict-free)
-constexpr int kOffP = kOffF + 2 * kFBuf * 4;    // p [8 heads][kPStride] fp32
-constexpr int kOffRed = kOffP + 8 * kPStride * 4;  // tile maxima [warp][8], then l [warp][8]
-constexpr int kQStride = 272;                   // int8 query row: 256 B + 16 B pad
-constexpr int kOffQ = kOffRed + 2 * kWarps * 8 * 4;  // rows 0-7 H, 8-15 M, 16-23 L
-constexpr int kOffZ = kOffQ + 24 * kQStride;    // 16 zero bytes (ldmatrix rows of zeros)
-constexpr int kOffBar = kOffZ + 16;             // mbarriers, 8 B each
-constexpr int kSmemUsed = kOffBar + kStages * 8;
-constexpr int kSmemBytes = kSmemUsed + 1024;    // slack for the 1024-byte alignment
+// stage layout (bytes from a 1024-aligned stage base)
+constexpr int kOffKC = 0;                      // K codes: 128 rows x 128 B (TMA 128B swizzle)
+constexpr int kOffVC = kOffKC + kTile * 128;   // V codes
+constexpr int kOffKS = kOffVC + kTile * 128;   // K scales: 128 rows x 8 fp16
+constexpr int kOffVS = kOffKS + kTile * 16;    // V scales
+constexpr int kStageBytes = kOffVS + kTile * 16;  // 36 KB
+// after the ring
+constexpr int kFsK = 8 * 32 * 4;               // per-warp K scales fp32 [block][32 pos]
+constexpr int kFsV = 8 * 32 * 2;               // per-warp V scales fp16 [block][32 pos]
+constexpr int kOffFs = kStages * kStageBytes;
+constexpr int kOffQF = kOffFs + kWarps * (kFsK + kFsV);  // query fragments [h][b][ks][tg] x 16 B
+constexpr int kOffQB = kOffQF + 8 * 8 * 2 * 4 * 16;      // accumulator starts [h][b]
+constexpr int kOffBar = kOffQB + 8 * 8 * 4;              // full[kStages]
+constexpr int kOffRel = kOffBar + kStages * 8;           // release counters [kStages]
+constexpr int kOffAbort = kOffRel + kStages * 4;         // abort flag, tiles issued
+constexpr int kSmemUsed = kOffAbort + 8;
+constexpr int kSmemBytes = kSmemUsed + 1024;   // slack for the 1024-byte alignment
+// end-of-split merge, reusing the ring: per warp m[8], l[8], o[8][264]
+// (head stride 264 floats spreads the 4 heads a warp writes at once over banks)
+constexpr int kMergeHead = 264;
+constexpr int kMergeWarpFloats = 16 + 8 * kMergeHead;
+constexpr int kOffMergeF = kWarps * kMergeWarpFloats * 4;  // exp2 factors [warp][8], then M, L
+static_assert(kStages % 2 == 0, "each stage must serve one warp group");
 static_assert(kStageBytes % 1024 == 0, "stages must keep the swizzle atoms aligned");
+static_assert(kOffMergeF + (kWarps + 2) * 8 * 4 <= kStages * kStageBytes, "merge fits the ring");
 static_assert(kOffBar % 8 == 0, "mbarrier alignment");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
-// bounded waits: ~2^20 polls of up to ~1 us each
+// bounded waits: ~2^20 polls of up to ~1 us each, abandoned early once any
+// thread of the CTA has given up
 constexpr int kWaitPolls = 1 << 20;
 
 struct TmaMaps {
@@ -99,17 +105,24 @@ __device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-// true once the phase with this parity has completed; false after the poll limit
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(1000u)
+      : "memory");
+  return done != 0;
+}
+// true once the phase with this parity has completed; false after the poll
+// limit or once *abort is set (by any thread of the CTA)
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          const volatile int *abort) {
+  if (mbar_try(bar, parity)) return true;
   for (int i = 0; i < kWaitPolls; i++) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-        " selp.u32 %0, 1, 0, p;\n}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity), "r"(1000u)
-        : "memory");
-    if (done) return true;
+    if (mbar_try(bar, parity)) return true;
+    if (*abort) return false;
   }
   return false;
 }
@@ -120,6 +133,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+__device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -133,6 +155,13 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
                : "r"(addr));
 }
 
+// d += A(16 x 16, f16, row) * B(16 x 8, f16, col) in fp32
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint4 &a, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                          uint32_t b1) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
@@ -140,13 +169,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-// d = A(s8, 16 x 32) * B(u8, 32 x 8), accumulating from zero
-__device__ __forceinline__ void imma16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                          uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%10,%10,%10,%10};"
-      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "n"(0));
+// d = A * B + c with the accumulator input c kept intact
+__device__ __forceinline__ void mma16816c(float (&d)[4], const uint4 &a, uint32_t b0, uint32_t b1,
+                                          float c0, float c1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%11,%11};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
 }
 
 // nibbles at bits 4..7 and 20..23 of x -> half2 (64 + c) exactly
@@ -156,20 +185,53 @@ __device__ __forceinline__ uint32_t nib64(uint32_t x) {
   return h;
 }
 
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 // fp32 pair -> fp16 hi + lo pairs (w ~= hi + lo to ~22 bits)
 __device__ __forceinline__ void split_hilo(float2 w, uint32_t &hi, uint32_t &lo) {
-  __half2 h = __float22half2_rn(w);
-  float2 hf = __half22float2(h);
-  __half2 l = __float22half2_rn(make_float2(w.x - hf.x, w.y - hf.y));
-  hi = *reinterpret_cast<uint32_t *>(&h);
-  lo = *reinterpret_cast<uint32_t *>(&l);
+  hi = pack_f16x2(w.x, w.y);
+  const float2 hf = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+  lo = pack_f16x2(w.x - hf.x, w.y - hf.y);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// in-register FWHT-256 of one vector held as 8 consecutive values per lane
+// (lane L: dims 8L .. 8L+7); stages h = 1, 2, ..., 128 in order, no scaling
+__device__ __forceinline__ void warp_fwht256(float (&x)[8], int lane) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+      if ((i & h) == 0) {
+        const float a = x[i], c = x[i + h];
+        x[i] = a + c;
+        x[i + h] = a - c;
+      }
+  }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = lane & m;  // this lane holds the i + h half of each pair
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const float o = __shfl_xor_sync(kFull, x[i], m);
+      x[i] = upper ? o - x[i] : x[i] + o;
+    }
+  }
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, 1)
     q4_decode_mma_kernel(const __grid_constant__ TmaMaps maps, kvq_cache c,
                          const void *__restrict__ q, const int32_t *__restrict__ seq_lens,
-                         int max_seq_len, int n_q_heads, int group, int gc, float scale_log2,
+                         int max_seq_len, int n_q_heads, int group, int gc, float sl2,
                          int split_tokens, int splits, float *__restrict__ ws) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -177,340 +239,394 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const int h0 = hg * gc, kvh = h0 / group;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tg = lane & 3;
+  const uint32_t full0 = smem_u32(smem + kOffBar);
+  int *rel = reinterpret_cast<int *>(smem + kOffRel);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffAbort);
+  volatile int *issued = abort_flag + 1;  // tiles issued so far (in order)
+
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < kStages; i++) {
+      mbar_init(full0 + 8 * i, 1);
+      rel[i] = 0;
+    }
+    *abort_flag = 0;
+    *issued = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    prefetch_map(&maps.kc);
+    prefetch_map(&maps.vc);
+    prefetch_map(&maps.ks);
+    prefetch_map(&maps.vs);
+  }
+  // inputs may come from the kernel launched just before this one
+  grid_dependency_wait();
+  launch_dependents();
+  __syncthreads();
+
   const int cap = c.block_table ? c.max_pages_per_seq * c.page_size : c.max_tokens;
   const int len = min(max(__ldg(seq_lens + b), 0), min(max_seq_len, cap));
   const int t0 = s * split_tokens;
   const int t1 = min(len, t0 + split_tokens);
   const int ntiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
-  const uint32_t bar0 = smem_u32(smem + kOffBar);
 
-  // first cache row of a tile, -1 if its page is unmapped
-  auto tile_row0 = [&](int tstart) -> int64_t {
-    if (c.block_table == nullptr) return ((int64_t)b * c.num_kv_heads + kvh) * c.max_tokens + tstart;
-    const int pi = tstart / c.page_size;
+  // first cache row of the 64-token sub-tile starting at token t, -1 if unmapped
+  auto sub_row = [&](int t) -> int {
+    if (c.block_table == nullptr) return (int)(((int64_t)b * c.num_kv_heads + kvh) * c.max_tokens + t);
+    const int pi = t / c.page_size;
     const int page = __ldg(c.block_table + (int64_t)b * c.max_pages_per_seq + pi);
     if (page < 0 || page >= c.num_pages) return -1;
-    return ((int64_t)page * c.num_kv_heads + kvh) * c.page_size + (tstart - pi * c.page_size);
+    return (int)(((int64_t)page * c.num_kv_heads + kvh) * c.page_size + (t - pi * c.page_size));
   };
-  // one thread: a whole tile (codes + scales of K and V) onto the stage's barrier
+  // one thread: tile `it` (both 64-token halves that hold tokens of the split)
+  // onto its stage's full barrier
   auto issue = [&](int it) {
     const int st = it % kStages;
-    const uint32_t bar = bar0 + 8 * st;
-    const int64_t row0 = tile_row0(t0 + it * kTile);
-    if (row0 < 0) {  // nothing to load: complete the phase without bytes
-      mbar_arrive(bar);
-      return;
-    }
-    const uint32_t dst = smem_u32(smem + st * kStageBytes);
-    mbar_arrive_tx(bar, kTileBytes);
-    tma_load_2d(dst + kOffKC, &maps.kc, 0, (int)row0, bar);
-    tma_load_2d(dst + kOffVC, &maps.vc, 0, (int)row0, bar);
-    tma_load_2d(dst + kOffKS, &maps.ks, 0, (int)row0, bar);
-    tma_load_2d(dst + kOffVS, &maps.vs, 0, (int)row0, bar);
-  };
-
-  if (tid == 0) {
-#pragma unroll
-    for (int i = 0; i < kStages; i++) mbar_init(bar0 + 8 * i, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  }
-
-  // ---- query: rotate (FWHT-256 in shared memory), then int8 H / M / L rows
-  float *qs = reinterpret_cast<float *>(smem);  // [8][256] in the stages, before any load
-  for (int p = tid; p < 8 * kDim; p += kThreads) {
-    const int hh = p >> 8, j = p & 255;
-    float v = 0.f;
-    if (hh < gc) {
-      const int64_t off = ((int64_t)b * n_q_heads + h0 + hh) * kDim + j;
-      v = BF16 ? __uint_as_float((uint32_t)static_cast<const uint16_t *>(q)[off] << 16)
-               : static_cast<const float *>(q)[off];
-    }
-    qs[p] = v;
-  }
-  for (int h = 1; h < kDim; h <<= 1) {
-    __syncthreads();
-    for (int p = tid; p < 8 * 128; p += kThreads) {
-      const int vv = p >> 7, pi = p & 127;
-      const int i0 = ((pi / h) * 2 * h) + (pi % h);
-      float *y = qs + vv * kDim;
-      const float a = y[i0], bb = y[i0 + h];
-      y[i0] = a + bb;
-      y[i0 + h] = a - bb;
-    }
-  }
-  __syncthreads();
-  float *red = reinterpret_cast<float *>(smem + kOffRed);
-#pragma unroll
-  for (int i = 0; i < 2; i++) {  // warp w: max |FWHT(q)| of heads 2w, 2w + 1
-    const int hh = 2 * warp + i;
-    float m = 0.f;
-    for (int j = lane; j < kDim; j += 32) m = fmaxf(m, fabsf(qs[hh * kDim + j]));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
-    if (lane == 0) red[hh] = m;
-  }
-  __syncthreads();
-  uint8_t *qi = smem + kOffQ;
-  for (int p = tid; p < 8 * kDim; p += kThreads) {
-    const int hh = p >> 8, j = p & 255;
-    const float m = red[hh];
-    const float x = m > 0.f ? qs[p] * (kQRange / m) : 0.f;  // |x| <= 127 * 2^14 (+ rounding)
-    const float hi = rintf(x * (1.f / 16384.f));
-    const float r = x - 16384.f * hi;          // exact, |r| <= 2^13
-    const float mid = rintf(r * (1.f / 128.f));
-    const float lo = rintf(r - 128.f * mid);   // exact difference, |lo| <= 64
-    qi[hh * kQStride + j] = (uint8_t)(int8_t)(int)hi;
-    qi[(8 + hh) * kQStride + j] = (uint8_t)(int8_t)(int)mid;
-    qi[(16 + hh) * kQStride + j] = (uint8_t)(int8_t)(int)lo;
-  }
-  if (tid < 4) reinterpret_cast<uint32_t *>(smem + kOffZ)[tid] = 0u;
-  __syncthreads();
-  // zero-point term of head g, block bb: 8 * sum over the block of 2^14 H + 2^7 M + L
-  int bq[8];
-#pragma unroll
-  for (int bb = 0; bb < 8; bb++) {
-    // lane (g, tg) sums dims 32 bb + 8 tg .. + 7, then the 4 lanes of head g combine
-    int acc = 0;
-#pragma unroll
-    for (int j = 0; j < 8; j++) {
-      const int d = 32 * bb + 8 * tg + j;
-      acc += 16384 * (int)(int8_t)qi[g * kQStride + d] + 128 * (int)(int8_t)qi[(8 + g) * kQStride + d] +
-             (int)(int8_t)qi[(16 + g) * kQStride + d];
-    }
-    acc += __shfl_xor_sync(kFull, acc, 1);
-    acc += __shfl_xor_sync(kFull, acc, 2);
-    bq[bb] = 8 * acc;
-  }
-  // A fragments of block bb: rows 0-15 (H, M) by ldmatrix.x4; L rows with a
-  // zero row in place of rows 8-15, also by ldmatrix.x4 (bytes 32 bb + 0..15,
-  // + 16..31)
-  uint32_t qhm[8][4];
-  const uint32_t zrow = smem_u32(smem + kOffZ);
-  const uint32_t qla = ((lane >> 3) & 1) ? zrow : smem_u32(qi) + (16 + (lane & 7)) * kQStride + 16 * (lane >> 4);
-  const uint32_t qlstep = ((lane >> 3) & 1) ? 0u : 32u;
-  {
-    const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
-    const uint32_t a4 = smem_u32(qi) + row * kQStride + 16 * (lane >> 4);
-#pragma unroll
-    for (int bb = 0; bb < 8; bb++) ldsm_x4(a4 + 32 * bb, qhm[bb]);
-  }
-  // score scale for head g: max / (16 * 127 * 2^14) undoes S and the FWHT's 1 / 16
-  const float sl2 = scale_log2 * (red[g] * (0.0625f / kQRange));
-  __syncthreads();  // qs, red are reused below; the barriers are initialised
-
-  if (tid == 0) {
-#pragma unroll
-    for (int i = 0; i < kStages - 1; i++)
-      if (i < ntiles) issue(i);
-  }
-
-  float o[4][4];  // M-tiles: block 2w + (mt >> 1), parity mt & 1
-#pragma unroll
-  for (int mt = 0; mt < 4; mt++) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-  float swb[2] = {0.f, 0.f};  // sum over this lane's tokens of p * d_v, head g, blocks 2w, 2w+1
-  float m_run = -INFINITY, l_run = 0.f;  // head g; m_run is the same in every warp
-  float *pbuf = reinterpret_cast<float *>(smem + kOffP);
-  bool failed = false;
-
-  for (int it = 0; it < ntiles; it++) {
-    const int st = it % kStages;
-    uint8_t *stage = smem + st * kStageBytes;
     const int tstart = t0 + it * kTile;
-    const bool tile_ok = tile_row0(tstart) >= 0;
-    const int nvalid = min(kTile, t1 - tstart);
-    if (!mbar_wait(bar0 + 8 * st, (it / kStages) & 1)) failed = true;
-    float *fsc = reinterpret_cast<float *>(smem + kOffF) + (it & 1) * kFBuf;
-    {  // widen this tile's scales to fp32 [kv][block][token]; rows past the end are 0
-      const int r = tid & 63, kv = tid >> 6;
-      const uint4 w = *reinterpret_cast<const uint4 *>(stage + (kv ? kOffVS : kOffKS) + r * 16);
-      const bool ok = r < nvalid;
-      float *f = fsc + kv * 8 * kTile;
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    const int r0 = sub_row(tstart);
+    const int r1 = tstart + kSub < t1 ? sub_row(tstart + kSub) : -1;
+    const uint32_t bar = full0 + 8 * st;
+    const int n = (r0 >= 0) + (r1 >= 0);
+    if (n == 0) {
+      mbar_arrive(bar);
+    } else {
+      mbar_arrive_tx(bar, n * kSubBytes);
+      const uint32_t dst = smem_u32(smem + st * kStageBytes);
 #pragma unroll
-      for (int k2 = 0; k2 < 4; k2++) {
-        const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&ww[k2]));
-        f[(2 * k2) * kTile + r] = ok ? p.x : 0.f;
-        f[(2 * k2 + 1) * kTile + r] = ok ? p.y : 0.f;
+      for (int j = 0; j < 2; j++) {
+        const int r = j ? r1 : r0;
+        if (r < 0) continue;
+        tma_load_2d(dst + kOffKC + j * kSub * 128, &maps.kc, 0, r, bar);
+        tma_load_2d(dst + kOffVC + j * kSub * 128, &maps.vc, 0, r, bar);
+        tma_load_2d(dst + kOffKS + j * kSub * 16, &maps.ks, 0, r, bar);
+        tma_load_2d(dst + kOffVS + j * kSub * 16, &maps.vs, 0, r, bar);
       }
     }
-    // (1) scales widened; every warp is done with tile it - 1; a failed wait
-    // anywhere stops the whole CTA
-    if (__syncthreads_or(failed)) {
-      failed = true;
+    atomicMax(const_cast<int *>(issued), it + 1);
+  };
+  if (lane == 0 && warp < kStages && warp < ntiles) issue(warp);
+
+  // (1) query: warp w rotates head h0 + w, splits it into fp16 hi + lo and
+  // writes the MMA fragments of its 8 blocks x 2 k-steps
+  {
+    float x[8];
+    if (warp < gc) {
+      const int64_t off = ((int64_t)b * n_q_heads + h0 + warp) * kDim + 8 * lane;
+      if (BF16) {
+        const uint4 r = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(q) + off));
+        const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+          x[2 * i] = bf16lo(rr[i]);
+          x[2 * i + 1] = bf16hi(rr[i]);
+        }
+      } else {
+        const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(q) + off);
+        const float4 u = __ldg(p), v = __ldg(p + 1);
+        x[0] = u.x, x[1] = u.y, x[2] = u.z, x[3] = u.w;
+        x[4] = v.x, x[5] = v.y, x[6] = v.z, x[7] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; i++) x[i] = 0.f;
+    }
+    warp_fwht256(x, lane);
+    float hi[8], lo[8], sq = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const float v = x[i] * 0.0625f;  // the FWHT's 1/16 (exact)
+      hi[i] = __half2float(__float2half_rn(v));
+      lo[i] = __half2float(__float2half_rn(v - hi[i]));
+      sq += hi[i] + lo[i];
+    }
+    // lane L holds dims 8L..8L+7 = block L/4, k-step (L/2)&1, tg 2(L&1) and 2(L&1)+1
+    uint4 *qf = reinterpret_cast<uint4 *>(smem + kOffQF) + (warp * 8 + (lane >> 2)) * 8 +
+                ((lane >> 1) & 1) * 4 + 2 * (lane & 1);
+#pragma unroll
+    for (int e = 0; e < 2; e++) {
+      const int i = 4 * e;
+      qf[e] = make_uint4(pack_f16x2(hi[i], hi[i + 2]), pack_f16x2(lo[i], lo[i + 2]),
+                         pack_f16x2(hi[i + 1], hi[i + 3]), pack_f16x2(lo[i + 1], lo[i + 3]));
+    }
+    sq += __shfl_xor_sync(kFull, sq, 1);
+    sq += __shfl_xor_sync(kFull, sq, 2);
+    if ((lane & 3) == 0)
+      reinterpret_cast<float *>(smem + kOffQB)[warp * 8 + (lane >> 2)] = -kBias * sq;
+  }
+  __syncthreads();
+  uint4 qa[8][2];
+  float cb[8];  // accumulator start of the hi rows: -72 * sum over the block of (hi + lo)
+  {
+    const uint4 *qf = reinterpret_cast<const uint4 *>(smem + kOffQF) + g * 64 + tg;
+#pragma unroll
+    for (int bb = 0; bb < 8; bb++) {
+      qa[bb][0] = qf[bb * 8];
+      qa[bb][1] = qf[bb * 8 + 4];
+      cb[bb] = reinterpret_cast<const float *>(smem + kOffQB)[g * 8 + bb];
+    }
+  }
+
+  // (2) the split: warp group gq = warp / 4 takes the tiles it with it % 2 == gq,
+  // warp wi = warp % 4 tokens 32wi .. 32wi + 31 of each of them
+  const int gq = warp >> 2, wi = warp & 3;
+  float o[8][2][4];  // [block][M-tile X (dims 2g, 2g+1) / Y (16 + 2g, 17 + 2g)][reg]
+#pragma unroll
+  for (int bb = 0; bb < 8; bb++)
+#pragma unroll
+    for (int m = 0; m < 2; m++) o[bb][m][0] = o[bb][m][1] = o[bb][m][2] = o[bb][m][3] = 0.f;
+  float wacc[4] = {0.f, 0.f, 0.f, 0.f};  // sum_t p d_v: head g (hi, lo rows) x blocks 2tg, 2tg+1
+  float m_run = -INFINITY, l_run = 0.f;  // head g
+  float *fsk = reinterpret_cast<float *>(smem + kOffFs + warp * (kFsK + kFsV));
+  __half *fsv = reinterpret_cast<__half *>(smem + kOffFs + warp * (kFsK + kFsV) + kFsK);
+  const int row_l = 32 * wi + 8 * ((lane >> 3) & 1) + (lane & 7);  // ldmatrix row (T = 0/1)
+  const int blk_l = lane >> 4;
+
+  for (int it = gq; it < ntiles; it += 2) {
+    const int st = it % kStages;
+    if (!mbar_wait(full0 + 8 * st, (it / kStages) & 1, abort_flag)) {
+      *abort_flag = 1;
       break;
     }
-    if (tid == 0 && it + kStages - 1 < ntiles) issue(it + kStages - 1);
-    if (!tile_ok) continue;  // uniform across the CTA
+    const uint8_t *stage = smem + st * kStageBytes;
+    const int tw = t0 + it * kTile + 32 * wi;  // first token of this warp
+    const int nvalid = min(32, t1 - tw);
+    bool live = nvalid > 0;
+    if (live && c.block_table != nullptr) live = sub_row(tw & ~(kSub - 1)) >= 0;
+    if (live) {
+      {  // widen: lane = token; K scales -> fp32, V scales fp16, [block][pos]; invalid -> 0
+        const int t = lane;
+        const uint4 wk = *reinterpret_cast<const uint4 *>(stage + kOffKS + (32 * wi + t) * 16);
+        const uint4 wv = *reinterpret_cast<const uint4 *>(stage + kOffVS + (32 * wi + t) * 16);
+        // pos: 16 * (T >> 1) + 4 * tg + 2 * (T & 1) + e for t = 8T + 2tg + e
+        const int T = t >> 3, tg2 = (t >> 1) & 3, e = t & 1;
+        const int pos = 16 * (T >> 1) + 4 * tg2 + 2 * (T & 1) + e;
+        const bool ok = t < nvalid;
+        const uint32_t kk[4] = {wk.x, wk.y, wk.z, wk.w}, vv[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int k2 = 0; k2 < 4; k2++) {
+          const float2 pk2 = __half22float2(*reinterpret_cast<const __half2 *>(&kk[k2]));
+          fsk[(2 * k2) * 32 + pos] = ok ? pk2.x : 0.f;
+          fsk[(2 * k2 + 1) * 32 + pos] = ok ? pk2.y : 0.f;
+          const uint32_t v2 = ok ? vv[k2] : 0u;
+          reinterpret_cast<uint16_t *>(fsv)[(2 * k2) * 32 + pos] = (uint16_t)(v2 & 0xffffu);
+          reinterpret_cast<uint16_t *>(fsv)[(2 * k2 + 1) * 32 + pos] = (uint16_t)(v2 >> 16);
+        }
+      }
+      __syncwarp();
+      const uint32_t kbase = smem_u32(stage + kOffKC), vbase = smem_u32(stage + kOffVC);
 
-    // ---- QK: warp w, tokens 16w .. 16w + 15
-    const uint32_t kbase = smem_u32(stage + kOffKC), vbase = smem_u32(stage + kOffVC);
-    const int live = nvalid - 16 * warp;  // tokens of this warp's 16 inside the split
-    float2 sacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-    {
-      const float *fk = fsc + 16 * warp + 2 * tg;
-      // ldmatrix: matrix m = lane / 8 -> (token group T = m & 1, block offset m >> 1)
-      const int mr = 16 * warp + 8 * ((lane >> 3) & 1) + (lane & 7);
-      const int mb = lane >> 4;
+      // ---- QK: head g, tokens 8T + 2tg + {0, 1}, T = 0..3
+      float2 sacc[4];
+#pragma unroll
+      for (int T = 0; T < 4; T++) sacc[T] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int bp = 0; bp < 4; bp++) {
-        uint32_t kr[4];
-        ldsm_x4(kbase + mr * 128 + (((2 * bp + mb) ^ (mr & 7)) << 4), kr);
 #pragma unroll
-        for (int half = 0; half < 2; half++) {
-          const int bb = 2 * bp + half;
-          uint32_t ql[4];
-          ldsm_x4(qla + qlstep * bb, ql);
+        for (int tp = 0; tp < 2; tp++) {  // token groups 2tp, 2tp + 1
+          uint32_t kr[4];  // (T0, block 2bp), (T1, 2bp), (T0, 2bp + 1), (T1, 2bp + 1)
+          ldsm_x4(kbase + (row_l + 16 * tp) * 128 + (((2 * bp + blk_l) ^ (lane & 7)) << 4), kr);
 #pragma unroll
-          for (int T = 0; T < 2; T++) {
-            const uint32_t w = kr[2 * half + T];
-            const uint32_t b0 = w & 0x0F0F0F0Fu, b1 = (w >> 4) & 0x0F0F0F0Fu;
-            int dhm[4], dl[4];
-            imma16832(dhm, qhm[bb], b0, b1);
-            imma16832(dl, ql, b0, b1);
-            // sum over the block of (2^14 H + 2^7 M + L)(c - 8), exact in int32
-            const int t0 = (dhm[0] << 14) + ((dhm[2] << 7) + dl[0]) - bq[bb];
-            const int t1 = (dhm[1] << 14) + ((dhm[3] << 7) + dl[1]) - bq[bb];
-            const float2 d = *reinterpret_cast<const float2 *>(fk + bb * kTile + 8 * T);
-            sacc[T] = __ffma2_rn(d, make_float2((float)t0, (float)t1), sacc[T]);
+          for (int half = 0; half < 2; half++) {
+            const int bb = 2 * bp + half;
+            const float4 dk = *reinterpret_cast<const float4 *>(fsk + bb * 32 + 16 * tp + 4 * tg);
+#pragma unroll
+            for (int T = 0; T < 2; T++) {
+              const uint32_t w = kr[2 * half + T];
+              float acc[4];
+              mma16816c(acc, qa[bb][0], nib64(w << 4), nib64(w >> 4), cb[bb], 0.f);
+              mma16816(acc, qa[bb][1], nib64(w), nib64(w >> 8));
+              const float2 d = T ? make_float2(dk.z, dk.w) : make_float2(dk.x, dk.y);
+              sacc[2 * tp + T] = __ffma2_rn(
+                  d, __fadd2_rn(make_float2(acc[0], acc[1]), make_float2(acc[2], acc[3])), sacc[2 * tp + T]);
+            }
+          }
+        }
+      }
+      // ---- online softmax of head g over this warp's 32 tokens
+      float x[8];
+#pragma unroll
+      for (int T = 0; T < 4; T++) {
+        x[2 * T] = sacc[T].x * sl2;
+        x[2 * T + 1] = sacc[T].y * sl2;
+      }
+      if (nvalid < 32) {
+#pragma unroll
+        for (int e2 = 0; e2 < 8; e2++)
+          if (8 * (e2 >> 1) + 2 * tg + (e2 & 1) >= nvalid) x[e2] = -INFINITY;
+      }
+      float mx = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+      if (__any_sync(kFull, mx > m_run)) {
+        const float mn = fmaxf(m_run, mx);
+        const float alpha = mn == m_run ? 1.f : ex2(m_run - mn);
+        m_run = mn;
+        l_run *= alpha;
+#pragma unroll
+        for (int k = 0; k < 4; k++) wacc[k] *= alpha;  // rows of head g
+        const float a0 = __shfl_sync(kFull, alpha, 8 * tg);
+        const float a1 = __shfl_sync(kFull, alpha, 8 * tg + 4);
+#pragma unroll
+        for (int bb = 0; bb < 8; bb++)
+#pragma unroll
+          for (int m = 0; m < 2; m++) {
+            o[bb][m][0] *= a0;
+            o[bb][m][1] *= a1;
+            o[bb][m][2] *= a0;
+            o[bb][m][3] *= a1;
+          }
+      }
+      uint32_t ph[4], pl[4];  // p of head g as fp16 hi + lo pairs, token groups T
+#pragma unroll
+      for (int T = 0; T < 4; T++) {
+        const float p0 = ex2(x[2 * T] - m_run), p1 = ex2(x[2 * T + 1] - m_run);
+        l_run += p0 + p1;
+        split_hilo(make_float2(p0, p1), ph[T], pl[T]);
+      }
+      // ---- PV: k-steps of 16 tokens (token groups 2ks, 2ks + 1)
+#pragma unroll
+      for (int ks = 0; ks < 2; ks++) {
+        {  // sum_t p d_v for blocks 2tg, 2tg+1 on the tensor cores (d_v exact in fp16)
+          const uint2 dvb = *reinterpret_cast<const uint2 *>(fsv + g * 32 + 16 * ks + 4 * tg);
+          const uint32_t a[4] = {ph[2 * ks], pl[2 * ks], ph[2 * ks + 1], pl[2 * ks + 1]};
+          mma16816(wacc, a, dvb.x, dvb.y);
+        }
+#pragma unroll
+        for (int bp = 0; bp < 4; bp++) {
+          uint32_t vr[4];  // (tokens 0-7, block 2bp), (8-15, 2bp), (0-7, 2bp + 1), (8-15, 2bp + 1)
+          ldsm_x4_t(vbase + (row_l + 16 * ks) * 128 + (((2 * bp + blk_l) ^ (lane & 7)) << 4), vr);
+#pragma unroll
+          for (int half = 0; half < 2; half++) {
+            const int bb = 2 * bp + half;
+            const uint2 dvp = *reinterpret_cast<const uint2 *>(fsv + bb * 32 + 16 * ks + 4 * tg);
+            const __half2 d01 = *reinterpret_cast<const __half2 *>(&dvp.x);
+            const __half2 d89 = *reinterpret_cast<const __half2 *>(&dvp.y);
+            // w = p d_v exactly as hi + lo (TwoProduct with fp16 FMA)
+            const __half2 ph0 = *reinterpret_cast<const __half2 *>(&ph[2 * ks]);
+            const __half2 ph1 = *reinterpret_cast<const __half2 *>(&ph[2 * ks + 1]);
+            const __half2 pl0 = *reinterpret_cast<const __half2 *>(&pl[2 * ks]);
+            const __half2 pl1 = *reinterpret_cast<const __half2 *>(&pl[2 * ks + 1]);
+            const __half2 wh0 = __hmul2_rn(ph0, d01), wh1 = __hmul2_rn(ph1, d89);
+            const __half2 wl0 = __hfma2(pl0, d01, __hfma2(ph0, d01, __hneg2(wh0)));
+            const __half2 wl1 = __hfma2(pl1, d89, __hfma2(ph1, d89, __hneg2(wh1)));
+            const uint32_t bh0 = *reinterpret_cast<const uint32_t *>(&wh0);
+            const uint32_t bh1 = *reinterpret_cast<const uint32_t *>(&wh1);
+            const uint32_t bl0 = *reinterpret_cast<const uint32_t *>(&wl0);
+            const uint32_t bl1 = *reinterpret_cast<const uint32_t *>(&wl1);
+            const uint32_t r0 = vr[2 * half], r1 = vr[2 * half + 1];
+            {
+              const uint32_t a[4] = {nib64(r0 << 4), nib64(r0 >> 4), nib64(r1 << 4), nib64(r1 >> 4)};
+              mma16816(o[bb][0], a, bh0, bh1);
+              mma16816(o[bb][0], a, bl0, bl1);
+            }
+            {
+              const uint32_t a[4] = {nib64(r0), nib64(r0 >> 8), nib64(r1), nib64(r1 >> 8)};
+              mma16816(o[bb][1], a, bh0, bh1);
+              mma16816(o[bb][1], a, bl0, bl1);
+            }
           }
         }
       }
     }
-    // ---- softmax: tile maximum per head across the four warps
-    float sc[4] = {sacc[0].x * sl2, sacc[0].y * sl2, sacc[1].x * sl2, sacc[1].y * sl2};
-    if (live < 16) {
-#pragma unroll
-      for (int e = 0; e < 4; e++)
-        if (8 * (e >> 1) + 2 * tg + (e & 1) >= live) sc[e] = -INFINITY;
-    }
-    float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-    if (tg == 0) red[warp * 8 + g] = mx;
-    __syncthreads();  // (2)
-    const float mt_ = fmaxf(fmaxf(red[g], red[8 + g]), fmaxf(red[16 + g], red[24 + g]));
-    if (__any_sync(kFull, mt_ > m_run + 8.f)) {
-      const float mn = fmaxf(m_run, mt_);
-      const float alpha = exp2f(m_run - mn);  // 0 while m_run is -inf
-      m_run = mn;
-      l_run *= alpha;
-      swb[0] *= alpha;
-      swb[1] *= alpha;
-      const float a0 = __shfl_sync(kFull, alpha, 8 * tg);      // head 2tg
-      const float a1 = __shfl_sync(kFull, alpha, 8 * tg + 4);  // head 2tg + 1
-#pragma unroll
-      for (int mt = 0; mt < 4; mt++) {
-        o[mt][0] *= a0;
-        o[mt][1] *= a1;
-        o[mt][2] *= a0;
-        o[mt][3] *= a1;
-      }
-    }
-    {
-      float p[4];
-#pragma unroll
-      for (int e = 0; e < 4; e++) {
-        p[e] = exp2f(sc[e] - m_run);
-        l_run += p[e];
-      }
-      float *pr = pbuf + g * kPStride + 16 * warp + 2 * tg;
-      *reinterpret_cast<float2 *>(pr) = make_float2(p[0], p[1]);
-      *reinterpret_cast<float2 *>(pr + 8) = make_float2(p[2], p[3]);
-    }
-    __syncthreads();  // (3) p of all 64 tokens
-    // ---- PV: warp w, blocks 2w, 2w + 1, all 64 tokens in 4 steps of 16
-    {
-      const float *fv = fsc + 8 * kTile + (2 * warp) * kTile + 2 * tg;
-      const float *pp = pbuf + g * kPStride + 2 * tg;
-      const int blk = 2 * warp + (lane >> 4);  // ldmatrix block of this lane's matrices
-#pragma unroll
-      for (int ks = 0; ks < 4; ks++) {
-        const int mr = 16 * ks + 8 * ((lane >> 3) & 1) + (lane & 7);
-        uint32_t vr[4];  // (T0, blk 2w), (T1, blk 2w), (T0, blk 2w+1), (T1, blk 2w+1)
-        ldsm_x4_t(vbase + mr * 128 + ((blk ^ (mr & 7)) << 4), vr);
-        const float2 p01 = *reinterpret_cast<const float2 *>(pp + 16 * ks);
-        const float2 p23 = *reinterpret_cast<const float2 *>(pp + 16 * ks + 8);
-#pragma unroll
-        for (int half = 0; half < 2; half++) {
-          const float2 w0 =
-              __fmul2_rn(p01, *reinterpret_cast<const float2 *>(fv + half * kTile + 16 * ks));
-          const float2 w1 =
-              __fmul2_rn(p23, *reinterpret_cast<const float2 *>(fv + half * kTile + 16 * ks + 8));
-          swb[half] += (w0.x + w0.y) + (w1.x + w1.y);
-          uint32_t bh0, bl0, bh1, bl1;
-          split_hilo(w0, bh0, bl0);
-          split_hilo(w1, bh1, bl1);
-          const uint32_t r0 = vr[2 * half], r1 = vr[2 * half + 1];  // tokens 0-7, 8-15
-          {  // even M-tile: rows g <-> low nibble of byte 2g, rows g + 8 <-> its high nibble
-            const uint32_t a[4] = {nib64(r0 << 4), nib64(r0), nib64(r1 << 4), nib64(r1)};
-            mma16816(o[2 * half], a, bh0, bh1);
-            mma16816(o[2 * half], a, bl0, bl1);
-          }
-          {  // odd M-tile: byte 2g + 1
-            const uint32_t a[4] = {nib64(r0 >> 4), nib64(r0 >> 8), nib64(r1 >> 4),
-                                   nib64(r1 >> 8)};
-            mma16816(o[2 * half + 1], a, bh0, bh1);
-            mma16816(o[2 * half + 1], a, bl0, bl1);
-          }
+    // release the stage; the last of its 4 warps refills it with tile it + kStages
+    // (same warp group: kStages is even)
+    __syncwarp();
+    if (lane == 0) {
+      int old;
+      asm volatile("atom.release.cta.shared::cta.add.s32 %0, [%1], 1;"
+                   : "=r"(old)
+                   : "r"(smem_u32(rel + st))
+                   : "memory");
+      if (old == 3) {
+        asm volatile("fence.acq_rel.cta;" ::: "memory");
+        rel[st] = 0;
+        if (it + kStages < ntiles && !*abort_flag) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          issue(it + kStages);
         }
       }
     }
   }
 
-  // ---- partial records: m (same in every warp), l summed over warps, o per warp
-  if (failed) {
-    // a load never arrived: let what was issued land (bounded), then mark the
-    // records of this split invalid with NaN so the output shows it
-    __syncthreads();
-    if (tid == 0)
-      for (int i = 0; i < kStages; i++) (void)mbar_wait(bar0 + 8 * i, 0), (void)mbar_wait(bar0 + 8 * i, 1);
-    __syncthreads();
-    for (int p = tid; p < gc * kRec; p += kThreads) {
-      const int hh = p / kRec, j = p % kRec;
-      ws[(((int64_t)b * n_q_heads + h0 + hh) * splits + s) * kRec + j] = __int_as_float(0x7fc00000);
-    }
-    return;
-  }
+  // (3) merge the 8 warps' states into this split's records
   l_run += __shfl_xor_sync(kFull, l_run, 1);
   l_run += __shfl_xor_sync(kFull, l_run, 2);
-  __syncthreads();  // red is reused
-  if (tg == 0) red[kWarps * 8 + warp * 8 + g] = l_run;
-#pragma unroll
-  for (int half = 0; half < 2; half++) {
-    swb[half] += __shfl_xor_sync(kFull, swb[half], 1);
-    swb[half] += __shfl_xor_sync(kFull, swb[half], 2);
+  // wacc: head g, blocks 2tg (hi + lo rows: [0] + [2]) and 2tg + 1 ([1] + [3])
+  const float wA = wacc[0] + wacc[2], wB = wacc[1] + wacc[3];
+  __syncthreads();  // every warp is done with the ring
+  const bool abort_all = *abort_flag != 0;
+  if (abort_all) {
+    // a load never arrived: let every load still in flight land (bounded,
+    // ignoring the flag) before the CTA's shared memory goes away
+    if (tid == 0) {
+      const int n = *issued;
+      for (int it = n > kStages ? n - kStages : 0; it < n; it++)
+        for (int i = 0; i < kWaitPolls && !mbar_try(full0 + 8 * (it % kStages), (it / kStages) & 1); i++) {
+        }
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  const int hA = 2 * tg, hB = 2 * tg + 1;  // heads of this lane's O columns
+  float *mw = reinterpret_cast<float *>(smem) + warp * kMergeWarpFloats;
+  if (!abort_all) {
+    if (tg == 0) {
+      mw[g] = m_run;
+      mw[8 + g] = l_run;
+    }
 #pragma unroll
-  for (int half = 0; half < 2; half++) {
-    const float cA = kBias * __shfl_sync(kFull, swb[half], 4 * hA);
-    const float cB = kBias * __shfl_sync(kFull, swb[half], 4 * hB);
+    for (int bb = 0; bb < 8; bb++) {
+      // wsum of (head h, block bb) lives in lane 4h + bb/2, as wA (bb even) or wB (odd)
+      const float sA = __shfl_sync(kFull, (bb & 1) ? wB : wA, 8 * tg + (bb >> 1));
+      const float sB = __shfl_sync(kFull, (bb & 1) ? wB : wA, 8 * tg + 4 + (bb >> 1));
+      const float cA = kBias * sA, cB = kBias * sB;
 #pragma unroll
-    for (int par = 0; par < 2; par++) {
-      const float(&acc)[4] = o[2 * half + par];
-      const int d0 = 64 * warp + 32 * half + 2 * g + par;  // row g; row g + 8 is d0 + 16
-      if (hA < gc) {
-        float *rec = ws + (((int64_t)b * n_q_heads + h0 + hA) * splits + s) * kRec + 4;
-        rec[d0] = acc[0] - cA;
-        rec[d0 + 16] = acc[2] - cA;
-      }
-      if (hB < gc) {
-        float *rec = ws + (((int64_t)b * n_q_heads + h0 + hB) * splits + s) * kRec + 4;
-        rec[d0] = acc[1] - cB;
-        rec[d0 + 16] = acc[3] - cB;
+      for (int m = 0; m < 2; m++) {
+        const int d0 = 32 * bb + 16 * m + 2 * g;  // row g; row g + 8 is d0 + 1
+        float *oa = mw + 16 + (2 * tg) * kMergeHead + d0;
+        float *ob = oa + kMergeHead;
+        oa[0] = o[bb][m][0] - cA;
+        ob[0] = o[bb][m][1] - cB;
+        oa[1] = o[bb][m][2] - cA;
+        ob[1] = o[bb][m][3] - cB;
       }
     }
   }
-  if (warp == 0 && tg == 0 && g < gc) {
-    float *rec = ws + (((int64_t)b * n_q_heads + h0 + g) * splits + s) * kRec;
-    rec[0] = m_run;
-    rec[1] = red[kWarps * 8 + g] + red[kWarps * 8 + 8 + g] + red[kWarps * 8 + 16 + g] +
-             red[kWarps * 8 + 24 + g];
+  __syncthreads();
+  float *fac = reinterpret_cast<float *>(smem + kOffMergeF);  // [warp][head] exp2 factors
+  float *mh = fac + kWarps * 8;                                // M, L per head
+  if (!abort_all && tid < 8) {
+    const float *m0 = reinterpret_cast<const float *>(smem);
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++) M = fmaxf(M, m0[w * kMergeWarpFloats + tid]);
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++) {
+      const float mwv = m0[w * kMergeWarpFloats + tid];
+      const float f = mwv == -INFINITY ? 0.f : ex2(mwv - M);
+      fac[w * 8 + tid] = f;
+      L += f * m0[w * kMergeWarpFloats + 8 + tid];
+    }
+    mh[tid] = M;
+    mh[8 + tid] = L;
+  }
+  __syncthreads();
+  const float nan = __int_as_float(0x7fc00000);
+  for (int hh = 0; hh < gc; hh++) {
+    float *rec = ws + (((int64_t)b * n_q_heads + h0 + hh) * splits + s) * kRec;
+    float acc = 0.f;
+    if (!abort_all) {
+#pragma unroll
+      for (int w = 0; w < kWarps; w++)
+        acc += fac[w * 8 + hh] *
+               reinterpret_cast<const float *>(smem)[w * kMergeWarpFloats + 16 + hh * kMergeHead + tid];
+    }
+    rec[4 + tid] = abort_all ? nan : acc;
+    if (tid == 0) {
+      rec[0] = abort_all ? nan : mh[hh];
+      rec[1] = abort_all ? nan : mh[8 + hh];
+    }
   }
 }
-
 // ---- host: 2-D tensor maps over the cache planes (cached per plane)
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -526,7 +642,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// rows x row_bytes uint8 plane, boxes of 64 rows x row_bytes
+// rows x row_bytes uint8 plane, boxes of kSub rows x row_bytes
 bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t row_bytes, bool swizzle) {
   struct Entry {
     const void *base;
@@ -547,7 +663,7 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t row_byte
   if (!fn) return false;
   const cuuint64_t dims[2] = {row_bytes, rows};
   const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {row_bytes, (cuuint32_t)kTile};
+  const cuuint32_t box[2] = {row_bytes, (cuuint32_t)kSub};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -561,14 +677,15 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t row_byte
 
 }  // namespace
 
-int q4_decode_ctas_per_sm() { return kCtasPerSm; }
+int q4_decode_ctas_per_sm() { return 1; }
+int q4_decode_tile_tokens() { return kTile; }
 
 cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, int batch,
                                  int n_q_heads, const int32_t *seq_lens, int max_seq_len,
                                  float scale, float *ws, const DecodePlan &p, cudaStream_t s) {
   const int group = n_q_heads / c.num_kv_heads;
   const int gc = group < 8 ? group : 8;
-  dim3 grid(p.splits, n_q_heads / gc, batch);
+  if (p.split_tokens % kTile) return cudaErrorInvalidValue;
   const float sl2 = scale * kLog2e;
   const uint64_t rows = c.block_table
                             ? (uint64_t)c.num_pages * c.num_kv_heads * c.page_size
@@ -598,14 +715,26 @@ cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, in
       configured[bf16] |= bit;
     }
   }
+  // programmatic dependent launch: this grid may be scheduled while the
+  // previous kernel on the stream finishes; it waits for it (griddepcontrol)
+  // before touching global memory
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.splits, n_q_heads / gc, batch);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (bf16)
-    q4_decode_mma_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(
-        maps, c, q, seq_lens, max_seq_len, n_q_heads, group, gc, sl2, p.split_tokens, p.splits,
-        ws);
+    e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<true>, maps, c, q, seq_lens, max_seq_len,
+                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws);
   else
-    q4_decode_mma_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(
-        maps, c, q, seq_lens, max_seq_len, n_q_heads, group, gc, sl2, p.split_tokens, p.splits,
-        ws);
+    e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<false>, maps, c, q, seq_lens, max_seq_len,
+                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

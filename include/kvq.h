@@ -141,7 +141,10 @@ KVQ_API size_t kvq_decode_attn_workspace(const kvq_cache *cache, int32_t batch,
  *   t < seq_len[b], with k_t, v_t the dequantized cached rows.
  * Split-K flash decoding: partial (max, sum, accumulator) per split in the
  * workspace, then a log-sum-exp combine that also applies the back-rotation.
- *   q: device, [batch][num_q_heads][256] of `dtype`.
+ * Both kernels are launched with programmatic stream serialization: they may
+ * be scheduled while the previous kernel on the stream drains and wait for it
+ * on the device before reading any input.
+ *   q: device, [batch][num_q_heads][256] of `dtype`, 16-byte aligned.
  *   d_seq_lens: device int32[batch]; values are clamped to
  *   [0, min(max_seq_len, capacity)]; a sequence of length 0 gives a zero row.
  *   max_seq_len: host upper bound of the lengths (sizes the grid).
