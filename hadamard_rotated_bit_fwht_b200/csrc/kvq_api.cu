@@ -192,7 +192,7 @@ kvq_status kvq_decode_attn(const kvq_cache *cache, const void *q, kvq_dtype dtyp
   if (!cache->block_table && batch > cache->batch_capacity) return KVQ_ERR_INVALID_ARG;
   if (!isfinite(scale)) return KVQ_ERR_INVALID_ARG;
   if (batch == 0) return KVQ_OK;
-  if (!q || !d_seq_lens || !out || !aligned(q, 16)) return KVQ_ERR_INVALID_ARG;
+  if (!q || !d_seq_lens || !out || !aligned(q, 16) || !aligned(out, 16)) return KVQ_ERR_INVALID_ARG;
   DecodePlan p = plan_decode(batch, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len);
   const size_t need = decode_workspace_bytes(batch, num_q_heads, p);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return KVQ_ERR_WORKSPACE;

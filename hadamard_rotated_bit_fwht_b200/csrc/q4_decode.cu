@@ -16,44 +16,31 @@ namespace {
 
 constexpr int kRec = 260;  // floats per partial record: m, l, pad, pad, o[256]
 
-// In-place FWHT-256 of n_vec vectors in shared memory (all threads of the CTA
-// take part; fp32, stage order h = 1, 2, ..., 128; no scaling).
-__device__ void smem_fwht256(float *x, int n_vec) {
-  for (int h = 1; h < kDim; h <<= 1) {
-    __syncthreads();
-    for (int p = threadIdx.x; p < n_vec * 128; p += blockDim.x) {
-      const int vv = p >> 7, pi = p & 127;
-      const int i0 = ((pi / h) * 2 * h) + (pi % h);
-      float *y = x + vv * kDim;
-      const float a = y[i0], b = y[i0 + h];
-      y[i0] = a + b;
-      y[i0 + h] = a - b;
-    }
-  }
-  __syncthreads();
-}
-
 // Log-sum-exp combine of the splits and back-rotation; one CTA of 256 threads
-// per (sequence, q head).  The split maxima are reduced cooperatively, the
-// split weights exp2(m_s - M) are computed once into shared memory, and each
-// thread sums its dimension over the splits with independent loads.
+// per (sequence, q head).  Thread j owns dimension j: the split maxima and sums
+// are reduced cooperatively, then each thread issues all its loads of o_s[j]
+// (up to kBatch at a time, so a split count of up to kBatch costs one L2 round
+// trip) before accumulating.  Warp 0 applies the FWHT-256 (8 values per lane:
+// strides 1, 2, 4 in registers, 8 .. 128 across lanes) and the 1/16.
 constexpr int kMaxSplitsSmem = 1024;
+constexpr int kBatch = 48;
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 1)
     q4_decode_combine_kernel(const float *__restrict__ ws, const int32_t *__restrict__ seq_lens,
-                             int n_q_heads, int splits, int max_seq_len, int cap,
-                             float *__restrict__ out) {
+                             int n_q_heads, int splits, int split_tokens, int max_seq_len,
+                             int cap, float *__restrict__ out) {
   __shared__ float ob[kDim];
   __shared__ float wgt[kMaxSplitsSmem];
-  __shared__ float red[8];
+  __shared__ float red[16];
   // the partial records come from the split kernel launched just before
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x, j = threadIdx.x, lane = j & 31, warp = j >> 5;
   const int b = bh / n_q_heads;
   const int len = min(max(__ldg(seq_lens + b), 0), min(max_seq_len, cap));
   const float *rec = ws + (int64_t)bh * splits * kRec;
-  const int ns = len > 0 ? min(splits, kMaxSplitsSmem) : 0;
-  // max over splits
+  // splits past the length wrote no record
+  const int ns = min(min(splits, (len + split_tokens - 1) / split_tokens), kMaxSplitsSmem);
+  // split maxima and sums (one pass: thread s < ns holds split s, more if ns > 256)
   float M = -INFINITY;
   for (int s = j; s < ns; s += 256) M = fmaxf(M, __ldg(rec + (int64_t)s * kRec));
 #pragma unroll
@@ -63,8 +50,6 @@ __global__ void __launch_bounds__(256)
   M = red[0];
 #pragma unroll
   for (int w = 1; w < 8; w++) M = fmaxf(M, red[w]);
-  __syncthreads();
-  // split weights and the total
   float L = 0.f;
   for (int s = j; s < ns; s += 256) {
     const float ms = __ldg(rec + (int64_t)s * kRec);
@@ -74,24 +59,54 @@ __global__ void __launch_bounds__(256)
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-  if (lane == 0) red[warp] = L;
+  if (lane == 0) red[8 + warp] = L;
   __syncthreads();
   L = 0.f;
 #pragma unroll
-  for (int w = 0; w < 8; w++) L += red[w];
-  float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
-  int s = 0;
-  for (; s + 4 <= ns; s += 4) {
-    O0 += wgt[s] * __ldg(rec + (int64_t)s * kRec + 4 + j);
-    O1 += wgt[s + 1] * __ldg(rec + (int64_t)(s + 1) * kRec + 4 + j);
-    O2 += wgt[s + 2] * __ldg(rec + (int64_t)(s + 2) * kRec + 4 + j);
-    O3 += wgt[s + 3] * __ldg(rec + (int64_t)(s + 3) * kRec + 4 + j);
+  for (int w = 0; w < 8; w++) L += red[8 + w];
+  float O = 0.f;
+  for (int s0 = 0; s0 < ns; s0 += kBatch) {
+    float v[kBatch];
+    // volatile asm keeps all kBatch loads ahead of the first use
+#pragma unroll
+    for (int k = 0; k < kBatch; k++) {
+      const float *src = rec + (int64_t)min(s0 + k, ns - 1) * kRec + 4 + j;
+      asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v[k]) : "l"(src));
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; k++) {
+      const float w = s0 + k < ns ? wgt[s0 + k] : 0.f;
+      asm volatile("fma.rn.f32 %0, %1, %2, %0;" : "+f"(O) : "f"(w), "f"(v[k]));
+    }
   }
-  for (; s < ns; s++) O0 += wgt[s] * __ldg(rec + (int64_t)s * kRec + 4 + j);
-  const float O = (O0 + O1) + (O2 + O3);
   ob[j] = L > 0.f ? O / L : 0.f;
-  smem_fwht256(ob, 1);
-  out[(int64_t)bh * kDim + j] = ob[j] * 0.0625f;
+  __syncthreads();
+  if (warp == 0) {
+    float x[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) x[i] = ob[8 * lane + i];
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1)
+#pragma unroll
+      for (int i = 0; i < 8; i++)
+        if ((i & h) == 0) {
+          const float a = x[i], c = x[i + h];
+          x[i] = a + c;
+          x[i + h] = a - c;
+        }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const bool upper = lane & m;
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const float o2 = __shfl_xor_sync(0xffffffffu, x[i], m);
+        x[i] = upper ? o2 - x[i] : x[i] + o2;
+      }
+    }
+    float4 *dst = reinterpret_cast<float4 *>(out + (int64_t)bh * kDim + 8 * lane);
+    dst[0] = make_float4(x[0] * 0.0625f, x[1] * 0.0625f, x[2] * 0.0625f, x[3] * 0.0625f);
+    dst[1] = make_float4(x[4] * 0.0625f, x[5] * 0.0625f, x[6] * 0.0625f, x[7] * 0.0625f);
+  }
 }
 
 }  // namespace
@@ -132,10 +147,25 @@ DecodePlan plan_split_k(int units, int max_len, int slots, int max_splits, int g
 }
 
 DecodePlan plan_decode(int batch, int n_head_groups, int max_seq_len) {
-  // ~3 tiles' worth of per-CTA work (query rotation, ring fill, final merge)
   const int tile = q4_decode_tile_tokens();
-  return plan_split_k(batch * n_head_groups, max_seq_len, kNumSMs * q4_decode_ctas_per_sm(),
-                      kMaxSplitsSmem, tile, 3 * tile);
+  const int units = batch * n_head_groups;
+  const int slots = kNumSMs * q4_decode_ctas_per_sm();
+  if (units * 4 >= slots) {
+    // many independent sequences whose lengths the host does not know: fixed
+    // chunks of 16 tiles, handed out by the block scheduler in order, so short
+    // sequences leave room for long ones (chunks past a length exit at once)
+    DecodePlan p;
+    p.split_tokens = 16 * tile;
+    p.splits = max((max(max_seq_len, 1) + p.split_tokens - 1) / p.split_tokens, 1);
+    while (p.splits > kMaxSplitsSmem) {
+      p.split_tokens *= 2;
+      p.splits = (max_seq_len + p.split_tokens - 1) / p.split_tokens;
+    }
+    return p;
+  }
+  // few sequences: one wave of equal splits (~3 tiles' worth of per-CTA work:
+  // query rotation, ring fill, final merge)
+  return plan_split_k(units, max_seq_len, slots, kMaxSplitsSmem, tile, 3 * tile);
 }
 
 size_t decode_workspace_bytes(int batch, int n_q_heads, const DecodePlan &p) {
@@ -163,7 +193,7 @@ cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int ba
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, q4_decode_combine_kernel, (const float *)ws, seq_lens, n_q_heads,
-                         p.splits, max_seq_len, cap, out);
+                         p.splits, p.split_tokens, max_seq_len, cap, out);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -262,13 +262,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   // inputs may come from the kernel launched just before this one
   grid_dependency_wait();
   launch_dependents();
+  // start the global loads (sequence length; warp w: query head h0 + w, dims
+  // 8 lane .. 8 lane + 7) before the barrier
+  const int len_raw = __ldg(seq_lens + b);
+  float x[8];
+  if (warp < gc) {
+    const int64_t off = ((int64_t)b * n_q_heads + h0 + warp) * kDim + 8 * lane;
+    if (BF16) {
+      const uint4 r = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(q) + off));
+      const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        x[2 * i] = bf16lo(rr[i]);
+        x[2 * i + 1] = bf16hi(rr[i]);
+      }
+    } else {
+      const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(q) + off);
+      const float4 u = __ldg(p), v = __ldg(p + 1);
+      x[0] = u.x, x[1] = u.y, x[2] = u.z, x[3] = u.w;
+      x[4] = v.x, x[5] = v.y, x[6] = v.z, x[7] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; i++) x[i] = 0.f;
+  }
   __syncthreads();
 
   const int cap = c.block_table ? c.max_pages_per_seq * c.page_size : c.max_tokens;
-  const int len = min(max(__ldg(seq_lens + b), 0), min(max_seq_len, cap));
+  const int len = min(max(len_raw, 0), min(max_seq_len, cap));
   const int t0 = s * split_tokens;
   const int t1 = min(len, t0 + split_tokens);
   const int ntiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
+  if (ntiles == 0) return;  // a split past the length writes no record
 
   // first cache row of the 64-token sub-tile starting at token t, -1 if unmapped
   auto sub_row = [&](int t) -> int {
@@ -306,30 +331,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   if (lane == 0 && warp < kStages && warp < ntiles) issue(warp);
 
-  // (1) query: warp w rotates head h0 + w, splits it into fp16 hi + lo and
-  // writes the MMA fragments of its 8 blocks x 2 k-steps
+  // (1) query: warp w rotates head h0 + w (zeros past gc), splits it into
+  // fp16 hi + lo and writes the MMA fragments of its 8 blocks x 2 k-steps
   {
-    float x[8];
-    if (warp < gc) {
-      const int64_t off = ((int64_t)b * n_q_heads + h0 + warp) * kDim + 8 * lane;
-      if (BF16) {
-        const uint4 r = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(q) + off));
-        const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-          x[2 * i] = bf16lo(rr[i]);
-          x[2 * i + 1] = bf16hi(rr[i]);
-        }
-      } else {
-        const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(q) + off);
-        const float4 u = __ldg(p), v = __ldg(p + 1);
-        x[0] = u.x, x[1] = u.y, x[2] = u.z, x[3] = u.w;
-        x[4] = v.x, x[5] = v.y, x[6] = v.z, x[7] = v.w;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; i++) x[i] = 0.f;
-    }
     warp_fwht256(x, lane);
     float hi[8], lo[8], sq = 0.f;
 #pragma unroll

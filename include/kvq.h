@@ -148,7 +148,7 @@ KVQ_API size_t kvq_decode_attn_workspace(const kvq_cache *cache, int32_t batch,
  *   d_seq_lens: device int32[batch]; values are clamped to
  *   [0, min(max_seq_len, capacity)]; a sequence of length 0 gives a zero row.
  *   max_seq_len: host upper bound of the lengths (sizes the grid).
- *   out: device, [batch][num_q_heads][256] fp32.
+ *   out: device, [batch][num_q_heads][256] fp32, 16-byte aligned.
  *   workspace: device, >= kvq_decode_attn_workspace(...) bytes, 16-byte
  *   aligned; its contents are scratch.
  * num_q_heads must be a multiple of num_kv_heads with a group size of 1, 2,
