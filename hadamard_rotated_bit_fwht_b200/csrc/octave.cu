@@ -65,13 +65,23 @@ struct LutSmem {
   float mid[2][15];
 };
 
+// Number of the 2^BITS - 1 sorted LUT midpoints below y (bucketize with
+// right=False: a tie goes to the lower code), by binary search.
+template <int BITS>
+__device__ __forceinline__ int bucket(float y, const float *mid) {
+  int c = 0;
+#pragma unroll
+  for (int step = 1 << (BITS - 1); step >= 1; step >>= 1)
+    if (mid[c + step - 1] < y) c += step;
+  return c;
+}
+
 // _quantize_lut over n = 64 (two values per lane: dims l, l + 32 of the block)
 // or n = 128 (four values per lane); codes out per value, returns the scale.
-template <int NV>
-__device__ __forceinline__ float quantize_lut(const float (&x)[NV], int bits, float mult,
-                                              const LutSmem &L, int (&code)[NV]) {
-  const int tb = bits == 4 ? 1 : 0;
-  const int nmid = (1 << bits) - 1;
+template <int NV, int BITS>
+__device__ __forceinline__ float quantize_lut(const float (&x)[NV], float mult, const LutSmem &L,
+                                              int (&code)[NV]) {
+  constexpr int tb = BITS == 4 ? 1 : 0;
   float sq[NV];
 #pragma unroll
   for (int k = 0; k < NV; k++) sq[k] = __fmul_rn(x[k], x[k]);
@@ -88,8 +98,7 @@ __device__ __forceinline__ float quantize_lut(const float (&x)[NV], int bits, fl
 #pragma unroll
   for (int k = 0; k < NV; k++) {
     const float y = __fmul_rn(__fdiv_rn(x[k], rms), mult);
-    int c = 0;
-    for (int i = 0; i < nmid; i++) c += (L.mid[tb][i] < y) ? 1 : 0;
+    const int c = bucket<BITS>(y, L.mid[tb]);
     code[k] = c;
     pr[k] = __fmul_rn(x[k], L.lut[tb][c]);
   }
@@ -101,24 +110,27 @@ __device__ __forceinline__ float quantize_lut(const float (&x)[NV], int bits, fl
   return __fmul_rn(dot > 0.f ? q : 0.f, kLutOne);
 }
 
-// Byte p of the packed codes of `n` dims starting at codes[base] (layout of
-// the page's module text).
-__device__ __forceinline__ uint32_t pack_byte(const uint8_t *codes, int n, int bits, int p) {
-  if (bits == 4) {
-    const int w = p >> 2, j = p & 3;
-    return (uint32_t)(codes[8 * w + j] & 15) | ((uint32_t)(codes[8 * w + 4 + j] & 15) << 4);
+// Word w (bytes 4w .. 4w+3) of the packed codes of a region of n dims whose
+// codes (one per byte) start at c32 (layout of the page's module text):
+//   4-bit: byte j of a word holds dim 8w + j (low nibble) and 8w + 4 + j;
+//   3-bit: a 2-bit plane (byte j of word w gathers dims 16w + 4i + j in bits
+//          2i..2i+1) followed by a 1-bit plane (byte j of word w gathers dims
+//          32w + 4i + j in bit i); code = lo + 4 * hi.
+__device__ __forceinline__ uint32_t pack_word(const uint32_t *c32, int n, int bits, int w) {
+  if (bits == 4)
+    return (c32[2 * w] & 0x0F0F0F0Fu) | ((c32[2 * w + 1] & 0x0F0F0F0Fu) << 4);
+  if (w < n / 16) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(c32 + 4 * w);
+    return (v.x & 0x03030303u) | ((v.y & 0x03030303u) << 2) | ((v.z & 0x03030303u) << 4) |
+           ((v.w & 0x03030303u) << 6);
   }
-  uint32_t byte = 0;
-  if (p < n / 4) {  // 2-bit plane
-    const int w = p >> 2, j = p & 3;
-#pragma unroll
-    for (int i = 0; i < 4; i++) byte |= (uint32_t)(codes[16 * w + 4 * i + j] & 3) << (2 * i);
-  } else {          // 1-bit plane
-    const int q = p - n / 4, w = q >> 2, j = q & 3;
-#pragma unroll
-    for (int i = 0; i < 8; i++) byte |= (uint32_t)((codes[32 * w + 4 * i + j] >> 2) & 1) << i;
-  }
-  return byte;
+  const int r = w - n / 16;
+  const uint4 u = *reinterpret_cast<const uint4 *>(c32 + 8 * r);
+  const uint4 v = *reinterpret_cast<const uint4 *>(c32 + 8 * r + 4);
+  return ((u.x >> 2) & 0x01010101u) | (((u.y >> 2) & 0x01010101u) << 1) |
+         (((u.z >> 2) & 0x01010101u) << 2) | (((u.w >> 2) & 0x01010101u) << 3) |
+         (((v.x >> 2) & 0x01010101u) << 4) | (((v.y >> 2) & 0x01010101u) << 5) |
+         (((v.z >> 2) & 0x01010101u) << 6) | (((v.w >> 2) & 0x01010101u) << 7);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -127,8 +139,8 @@ __global__ void __launch_bounds__(kThreads)
                            int n_kv_heads, const int64_t *__restrict__ slot_mapping,
                            uint8_t *__restrict__ cache, int block_size, int64_t num_blocks) {
   __shared__ LutSmem L;
-  __shared__ uint8_t kcodes[kWarps][kHead], vcodes[kWarps][kHead];
-  __shared__ __align__(16) uint8_t slot[kWarps][256];
+  __shared__ __align__(16) uint8_t kcodes[kWarps][kHead];
+  __shared__ __align__(16) uint8_t vcodes[kWarps][kHead];
   for (int i = threadIdx.x; i < 16; i += blockDim.x) {
     L.lut[0][i] = i < 8 ? (float)P.lut3[i] : 0.f;
     L.lut[1][i] = (float)P.lut4[i];
@@ -139,6 +151,10 @@ __global__ void __launch_bounds__(kThreads)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t items = (int64_t)num_tokens * n_kv_heads;
   const float vscale = 0.08838834764831845f;  // fp32(1 / sqrt(128))
+  const int slot_words = P.slot_bytes / 4;
+  const int w_kn = P.off_k_nope / 4, w_v = P.off_v / 4, w_sc = P.off_scales / 4;
+  const uint32_t *kc32 = reinterpret_cast<const uint32_t *>(kcodes[warp]);
+  const uint32_t *vc32 = reinterpret_cast<const uint32_t *>(vcodes[warp]);
   for (int64_t it = (int64_t)blockIdx.x * kWarps + warp; it < items;
        it += (int64_t)gridDim.x * kWarps) {
     const int tok = (int)(it / n_kv_heads), h = (int)(it % n_kv_heads);
@@ -168,10 +184,10 @@ __global__ void __launch_bounds__(kThreads)
     float ks[2];
 #pragma unroll
     for (int kb = 0; kb < 2; kb++) {
-      const int bits = (kb * 64 < P.rope_dim) ? 4 : 3;
       float xb[2] = {x[2 * kb], x[2 * kb + 1]};
       int cb[2];
-      ks[kb] = quantize_lut<2>(xb, bits, bits == 4 ? P.mult4 : P.mult3, L, cb);
+      if (kb * 64 < P.rope_dim) ks[kb] = quantize_lut<2, 4>(xb, P.mult4, L, cb);
+      else ks[kb] = quantize_lut<2, 3>(xb, P.mult3, L, cb);
       kcodes[warp][64 * kb + lane] = (uint8_t)cb[0];
       kcodes[warp][64 * kb + lane + 32] = (uint8_t)cb[1];
     }
@@ -205,34 +221,31 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int k = 0; k < 4; k++) x[k] = __fmul_rn(x[k], vscale);
     int cv[4];
-    const float vs = quantize_lut<4>(x, P.v_bits, P.v_bits == 4 ? P.mult4 : P.mult3, L, cv);
+    const float vs = P.v_bits == 4 ? quantize_lut<4, 4>(x, P.mult4, L, cv)
+                                   : quantize_lut<4, 3>(x, P.mult3, L, cv);
 #pragma unroll
     for (int k = 0; k < 4; k++) vcodes[warp][lane + 32 * k] = (uint8_t)cv[k];
     __syncwarp();
-    // ---- slot bytes
-    uint8_t *sl = slot[warp];
-    for (int p = lane; p < P.slot_bytes; p += 32) {
-      uint32_t byte = 0;
-      if (p < P.off_k_nope) byte = pack_byte(kcodes[warp], P.rope_dim, 4, p);
-      else if (p < P.off_v) byte = pack_byte(kcodes[warp] + P.rope_dim, kHead - P.rope_dim, 3, p - P.off_k_nope);
-      else if (p < P.off_scales) byte = pack_byte(vcodes[warp], kHead, P.v_bits, p - P.off_v);
-      else if (p < P.off_scales + 6) {
-        const int si = (p - P.off_scales) >> 1;
-        const float sv = si == 0 ? ks[0] : (si == 1 ? ks[1] : vs);
-        const uint32_t hb = __half_as_ushort(__float2half_rn(sv));
-        byte = (p - P.off_scales) & 1 ? (hb >> 8) : (hb & 0xFF);
-      }
-      sl[p] = (uint8_t)byte;
-    }
-    __syncwarp();
+    // ---- slot words: lane w builds word w (and w + 32) of the slot
     const int64_t sm = __ldg(slot_mapping + tok);
+    uint32_t *dst = nullptr;
     if (sm >= 0) {
       const int64_t blk = sm / block_size, off = sm % block_size;
-      if (blk < num_blocks) {
-        uint32_t *dst = reinterpret_cast<uint32_t *>(
-            cache + ((blk * n_kv_heads + h) * block_size + off) * P.slot_bytes);
-        for (int w = lane; w < P.slot_bytes / 4; w += 32) dst[w] = reinterpret_cast<const uint32_t *>(sl)[w];
-      }
+      if (blk < num_blocks)
+        dst = reinterpret_cast<uint32_t *>(cache +
+                                           ((blk * n_kv_heads + h) * block_size + off) * P.slot_bytes);
+    }
+    for (int w = lane; w < slot_words; w += 32) {
+      uint32_t word = 0;
+      if (w < w_kn) word = pack_word(kc32, P.rope_dim, 4, w);
+      else if (w < w_v) word = pack_word(kc32 + P.rope_dim / 4, kHead - P.rope_dim, 3, w - w_kn);
+      else if (w < w_sc) word = pack_word(vc32, kHead, P.v_bits, w - w_v);
+      else if (w == w_sc)
+        word = (uint32_t)__half_as_ushort(__float2half_rn(ks[0])) |
+               ((uint32_t)__half_as_ushort(__float2half_rn(ks[1])) << 16);
+      else if (w == w_sc + 1)
+        word = (uint32_t)__half_as_ushort(__float2half_rn(vs));
+      if (dst) dst[w] = word;
     }
     __syncwarp();
   }
