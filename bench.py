@@ -2,10 +2,10 @@
 
 One step = one pass of the whole hot path over one batch.  The default
 workload is the long-context decode (1 sequence, 131072 tokens, 32 query /
-4 kv heads, D = 256, bf16 inputs): kvq_quantize_append of the new token's K
-and V (rotate + Q4_0 + store), then kvq_decode_attn over the whole cache
-(rotate q, stream and dequantize the nibbles, online softmax, split-K
-combine, back-rotation).
+4 kv heads, D = 256, bf16 inputs): one kvq_decode_step call -- quantize-on-
+append of the new token's K and V (rotate + Q4_0 + store) and decode attention
+over the whole cache including it (rotate q, stream and dequantize the
+nibbles, online softmax, split-K combine, back-rotation).
 
 `value` is HBM throughput in GB/s: algorithmic bytes per step (every cache
 byte read once, inputs read and outputs written once) / device time per
@@ -169,9 +169,11 @@ class Workload:
 
 
 class LongDecode(Workload):
-    """Long-context decode: append the new token, decode over 131072 tokens."""
-    launches_per_step = 3  # append + decode split + combine
-    kernel_name = "kvq_decode_attn (q4_decode_mma_kernel + q4_decode_combine_kernel)"
+    """Long-context decode step: append the new token and decode over all
+    131072 tokens in one kvq_decode_step call (the split holding the new
+    position quantizes it in its prologue)."""
+    launches_per_step = 2  # decode split (with the append) + combine
+    kernel_name = "kvq_decode_step (q4_decode_mma_kernel with append + q4_decode_combine_kernel)"
     traffic_key = "q4_decode_long"
 
     def __init__(self, dev, copies=3):
@@ -192,30 +194,27 @@ class LongDecode(Workload):
             self.caches.append(c)
         del kd, vd
         self.q = bf16_tensor(synth.to_bf16_bits(synth.queries(W["seed"], B, Hq, 256)), dev)
-        self.new_k = bf16_tensor(kb[:, T - 1:T], dev)
-        self.new_v = bf16_tensor(vb[:, T - 1:T], dev)
+        self.new_k = bf16_tensor(kb[:, T - 1], dev)  # [B, Hkv, 256]
+        self.new_v = bf16_tensor(vb[:, T - 1], dev)
         self.pos = torch.full((B,), T - 1, dtype=torch.int32, device=dev)
         self.lens = torch.full((B,), T, dtype=torch.int32, device=dev)
         self.out = torch.empty((B, Hq, 256), dtype=torch.float32, device=dev)
         self.ws = torch.empty(kvq.decode_attn_workspace(self.caches[0], B, Hq, T),
                               dtype=torch.uint8, device=dev)
         self.kvq = kvq
-        self.kernel_bytes = B * H * T * 288 + B * Hq * 256 * (2 + 4)
-        self.step_bytes = self.kernel_bytes + 2 * B * H * (512 + 144)
+        # cache read once + the new token's K/V in and its codes out + q in + out
+        self.kernel_bytes = B * H * T * 288 + 2 * B * H * (512 + 144) + B * Hq * 256 * (2 + 4)
+        self.step_bytes = self.kernel_bytes
         self.h2d = [self.new_k, self.new_v, self.q]
         self.d2h = [self.out]
         self.config = {"workload": "long_decode", "batch": B, "n_q_heads": Hq,
                        "n_kv_heads": H, "head_dim": 256, "ctx": T,
-                       "step": "kvq_quantize_append(1 token) + kvq_decode_attn",
+                       "step": "kvq_decode_step: append 1 token + decode (one call)",
                        "l2": "3 cache copies (453 MB) rotated per step, inputs > L2"}
 
-    def pre(self, i):
-        self.kvq.quantize_append(self.caches[i % len(self.caches)], self.new_k, self.new_v,
-                                 self.pos)
-
     def kernel_call(self, i):
-        self.kvq.decode_attn(self.caches[i % len(self.caches)], self.q, self.lens, self.T,
-                             1.0 / 16.0, out=self.out, workspace=self.ws)
+        self.kvq.decode_step(self.caches[i % len(self.caches)], self.new_k, self.new_v, self.q,
+                             self.pos, self.T, 1.0 / 16.0, out=self.out, workspace=self.ws)
 
     def extra(self, call_ms):
         th = self.B * self.H * self.T / call_ms * 1e3

@@ -201,6 +201,31 @@ kvq_status kvq_decode_attn(const kvq_cache *cache, const void *q, kvq_dtype dtyp
                                     as_stream(stream)));
 }
 
+kvq_status kvq_decode_step(const kvq_cache *cache, const void *k_new, const void *v_new,
+                           const void *q, kvq_dtype dtype, int32_t batch, int32_t num_q_heads,
+                           const int32_t *d_pos, int32_t max_seq_len, float scale, float *out,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+  kvq_status st = check_cache(cache);
+  if (st != KVQ_OK) return st;
+  if (batch < 0 || num_q_heads <= 0 || max_seq_len < 0 || (dtype != KVQ_F32 && dtype != KVQ_BF16))
+    return KVQ_ERR_INVALID_ARG;
+  if (num_q_heads % cache->num_kv_heads) return KVQ_ERR_INVALID_ARG;
+  const int group = num_q_heads / cache->num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8 && group != 16) return KVQ_ERR_UNSUPPORTED;
+  if (!cache->block_table && batch > cache->batch_capacity) return KVQ_ERR_INVALID_ARG;
+  if (!isfinite(scale)) return KVQ_ERR_INVALID_ARG;
+  if (batch == 0) return KVQ_OK;
+  if (!q || !k_new || !v_new || !d_pos || !out || !aligned(q, 16) || !aligned(k_new, 16) ||
+      !aligned(v_new, 16) || !aligned(out, 16))
+    return KVQ_ERR_INVALID_ARG;
+  DecodePlan p = plan_decode(batch, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len);
+  const size_t need = decode_workspace_bytes(batch, num_q_heads, p);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return KVQ_ERR_WORKSPACE;
+  return from_cuda(launch_q4_decode(*cache, q, dtype == KVQ_BF16, batch, num_q_heads, nullptr,
+                                    max_seq_len, scale, out, static_cast<float *>(workspace), p,
+                                    as_stream(stream), k_new, v_new, d_pos));
+}
+
 kvq_status kvq_octave_layout_of(const kvq_octave_fmt *fmt, kvq_octave_layout *out) {
   return octave_layout(fmt, out);
 }

@@ -27,8 +27,9 @@ constexpr int kBatch = 48;
 
 __global__ void __launch_bounds__(256, 1)
     q4_decode_combine_kernel(const float *__restrict__ ws, const int32_t *__restrict__ seq_lens,
-                             int n_q_heads, int splits, int split_tokens, int max_seq_len,
-                             int cap, float *__restrict__ out) {
+                             const int32_t *__restrict__ pos, int n_q_heads, int splits,
+                             int split_tokens, int max_seq_len, int cap,
+                             float *__restrict__ out) {
   __shared__ float ob[kDim];
   __shared__ float wgt[kMaxSplitsSmem];
   __shared__ float red[16];
@@ -36,7 +37,8 @@ __global__ void __launch_bounds__(256, 1)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x, j = threadIdx.x, lane = j & 31, warp = j >> 5;
   const int b = bh / n_q_heads;
-  const int len = min(max(__ldg(seq_lens + b), 0), min(max_seq_len, cap));
+  const int len_raw = pos ? __ldg(pos + b) + 1 : __ldg(seq_lens + b);
+  const int len = min(max(len_raw, 0), min(max_seq_len, cap));
   const float *rec = ws + (int64_t)bh * splits * kRec;
   // splits past the length wrote no record
   const int ns = min(min(splits, (len + split_tokens - 1) / split_tokens), kMaxSplitsSmem);
@@ -175,10 +177,11 @@ size_t decode_workspace_bytes(int batch, int n_q_heads, const DecodePlan &p) {
 cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int batch,
                              int n_q_heads, const int32_t *seq_lens, int max_seq_len,
                              float scale, float *out, float *ws, const DecodePlan &p,
-                             cudaStream_t s) {
+                             cudaStream_t s, const void *k_new, const void *v_new,
+                             const int32_t *pos) {
   if (batch == 0) return cudaSuccess;
   cudaError_t e = launch_q4_decode_mma(c, q, bf16, batch, n_q_heads, seq_lens, max_seq_len,
-                                       scale, ws, p, s);
+                                       scale, ws, p, s, k_new, v_new, pos);
   if (e != cudaSuccess) return e;
   const int cap = c.block_table ? c.max_pages_per_seq * c.page_size : c.max_tokens;
   // programmatic dependent launch: scheduled while the split kernel drains,
@@ -192,8 +195,8 @@ cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int ba
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, q4_decode_combine_kernel, (const float *)ws, seq_lens, n_q_heads,
-                         p.splits, p.split_tokens, max_seq_len, cap, out);
+  e = cudaLaunchKernelEx(&cfg, q4_decode_combine_kernel, (const float *)ws, seq_lens, pos,
+                         n_q_heads, p.splits, p.split_tokens, max_seq_len, cap, out);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

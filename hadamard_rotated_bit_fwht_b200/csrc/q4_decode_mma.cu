@@ -39,7 +39,7 @@
 
 #include <mutex>
 
-#include "kvq_internal.cuh"
+#include "q4_vec.cuh"
 
 namespace kvq {
 namespace {
@@ -232,7 +232,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     q4_decode_mma_kernel(const __grid_constant__ TmaMaps maps, kvq_cache c,
                          const void *__restrict__ q, const int32_t *__restrict__ seq_lens,
                          int max_seq_len, int n_q_heads, int group, int gc, float sl2,
-                         int split_tokens, int splits, float *__restrict__ ws) {
+                         int split_tokens, int splits, float *__restrict__ ws,
+                         const void *__restrict__ k_new, const void *__restrict__ v_new,
+                         const int32_t *__restrict__ pos) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int s = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
@@ -264,7 +266,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   launch_dependents();
   // start the global loads (sequence length; warp w: query head h0 + w, dims
   // 8 lane .. 8 lane + 7) before the barrier
-  const int len_raw = __ldg(seq_lens + b);
+  // fused decode step (pos != nullptr): the new token goes to position pos[b]
+  // and the sequence then has pos[b] + 1 tokens
+  const int p_new = pos ? __ldg(pos + b) : -1;
+  const int len_raw = pos ? p_new + 1 : __ldg(seq_lens + b);
   float x[8];
   if (warp < gc) {
     const int64_t off = ((int64_t)b * n_q_heads + h0 + warp) * kDim + 8 * lane;
@@ -294,6 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t1 = min(len, t0 + split_tokens);
   const int ntiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
   if (ntiles == 0) return;  // a split past the length writes no record
+  // fused step: every CTA whose split holds the new token quantizes the
+  // token's K and V rows of its kv head into the cache before it issues a tile
+  // load (CTAs of the same kv head write identical bytes)
+  const bool appender = p_new >= t0 && p_new < t1;
 
   // first cache row of the 64-token sub-tile starting at token t, -1 if unmapped
   auto sub_row = [&](int t) -> int {
@@ -329,7 +338,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     atomicMax(const_cast<int *>(issued), it + 1);
   };
-  if (lane == 0 && warp < kStages && warp < ntiles) issue(warp);
+  if (appender) {
+    if (warp == 0) {
+      const int vg = lane >> 3, i = lane & 7;
+      const bool valid = vg < 2;  // lanes 0-7: K, 8-15: V
+      const void *src =
+          static_cast<const char *>(vg == 1 ? v_new : k_new) +
+          ((int64_t)b * c.num_kv_heads + kvh) * kDim * (BF16 ? 2 : 4);
+      uint4 bytes;
+      uint16_t sc;
+      q4v::quantize_vector<BF16>(valid ? src : k_new, valid, lane,
+                                 reinterpret_cast<float4 *>(smem) + 64 * vg, bytes, sc);
+      const int64_t row = q4_row(c, b, kvh, p_new);
+      if (valid && row >= 0) {
+        *reinterpret_cast<uint4 *>((vg ? c.v_codes : c.k_codes) + row * kRowCodeBytes + 16 * i) =
+            bytes;
+        (vg ? c.v_scales : c.k_scales)[row * kRowScales + i] = sc;
+      }
+      // the rows are read back by TMA (async proxy)
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __syncwarp();
+      if (lane == 0)
+        for (int it = 0; it < kStages && it < ntiles; it++) issue(it);
+    }
+  } else if (lane == 0 && warp < kStages && warp < ntiles) {
+    issue(warp);
+  }
 
   // (1) query: warp w rotates head h0 + w (zeros past gc), splits it into
   // fp16 hi + lo and writes the MMA fragments of its 8 blocks x 2 k-steps
@@ -686,7 +720,8 @@ int q4_decode_tile_tokens() { return kTile; }
 
 cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, int batch,
                                  int n_q_heads, const int32_t *seq_lens, int max_seq_len,
-                                 float scale, float *ws, const DecodePlan &p, cudaStream_t s) {
+                                 float scale, float *ws, const DecodePlan &p, cudaStream_t s,
+                                 const void *k_new, const void *v_new, const int32_t *pos) {
   const int group = n_q_heads / c.num_kv_heads;
   const int gc = group < 8 ? group : 8;
   if (p.split_tokens % kTile) return cudaErrorInvalidValue;
@@ -734,10 +769,12 @@ cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, in
   cfg.numAttrs = 1;
   if (bf16)
     e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<true>, maps, c, q, seq_lens, max_seq_len,
-                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws);
+                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws, k_new, v_new,
+                           pos);
   else
     e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<false>, maps, c, q, seq_lens, max_seq_len,
-                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws);
+                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws, k_new, v_new,
+                           pos);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -25,7 +25,7 @@ EXPORTED = (
     "kvq_status_string", "kvq_version", "kvq_rotate", "kvq_quantize_append",
     "kvq_decode_attn_workspace", "kvq_decode_attn", "kvq_octave_layout_of",
     "kvq_octave_codebook", "kvq_octave_quantize", "kvq_octave_decode_attn_workspace",
-    "kvq_octave_decode_attn", "kvq_decode_attn_noalloc",
+    "kvq_octave_decode_attn", "kvq_decode_attn_noalloc", "kvq_decode_step",
 )
 
 
@@ -95,6 +95,9 @@ def lib():
         L.kvq_decode_attn_noalloc.argtypes = [C.POINTER(CacheDesc), C.c_void_p, C.c_int, C.c_int32,
                                               C.c_int32, C.c_void_p, C.c_int32, C.c_float,
                                               C.c_void_p, C.c_void_p]
+        L.kvq_decode_step.argtypes = [C.POINTER(CacheDesc), C.c_void_p, C.c_void_p, C.c_void_p,
+                                      C.c_int, C.c_int32, C.c_int32, C.c_void_p, C.c_int32,
+                                      C.c_float, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
         _lib = L
     return _lib
 
@@ -243,6 +246,33 @@ def decode_attn(cache: Q4Cache, q: torch.Tensor, seq_lens: torch.Tensor, max_seq
     _check("kvq_decode_attn",
            lib().kvq_decode_attn(C.byref(d), _ptr(q), _dtype_code(q), batch, hq, _ptr(seq_lens),
                                  int(max_seq_len), float(scale), _ptr(out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def decode_step(cache: Q4Cache, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+                pos: torch.Tensor, max_seq_len: int, scale: float,
+                out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """Append one token per sequence (k_new, v_new [batch, Hkv, 256] at pos[b])
+    and decode over pos[b] + 1 tokens in one call (kvq_decode_step)."""
+    for name, t in (("k_new", k_new), ("v_new", v_new), ("q", q), ("pos", pos)):
+        _cuda_contig(name, t)
+    if pos.dtype != torch.int32:
+        raise TypeError("pos must be int32")
+    if not (k_new.dtype == v_new.dtype == q.dtype):
+        raise TypeError("k_new, v_new and q must share one dtype")
+    batch, hq, dim = q.shape
+    if out is None:
+        out = torch.empty((batch, hq, dim), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = decode_attn_workspace(cache, batch, hq, max_seq_len)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    d = cache.desc()
+    _check("kvq_decode_step",
+           lib().kvq_decode_step(C.byref(d), _ptr(k_new), _ptr(v_new), _ptr(q), _dtype_code(q),
+                                 batch, hq, _ptr(pos), int(max_seq_len), float(scale),
+                                 _ptr(out), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
 

@@ -162,6 +162,30 @@ KVQ_API kvq_status kvq_decode_attn(const kvq_cache *cache, const void *q, kvq_dt
                            float *out, void *workspace, size_t workspace_bytes,
                            void *stream);
 
+/* kvq_decode_step -- one decode step of the per-token path in a single call:
+ * quantize-on-append of each sequence's new token, then decode attention over
+ * the sequence including it (Strata PR #21, merge note: the per-token path
+ * rotates the new K/V and the query, attends, and rotates the output back).
+ * Equivalent to kvq_quantize_append(cache, k_new, v_new, dtype, batch, 1,
+ * d_pos) followed by kvq_decode_attn(cache, q, dtype, batch, num_q_heads,
+ * seq_lens = d_pos + 1, max_seq_len, scale, out, ...): the cache bytes and the
+ * output are bit-identical to that pair of calls.  The split of the decode that
+ * holds position d_pos[b] quantizes the token in its prologue, so the append
+ * costs no launch of its own.
+ *   k_new, v_new: device, [batch][num_kv_heads][256] of `dtype`, 16-byte
+ *   aligned.  q: device, [batch][num_q_heads][256] of `dtype`, 16-byte aligned.
+ *   d_pos: device int32[batch], position of the new token; a position outside
+ *   the cache (negative, >= capacity) appends nothing; the attended length is
+ *   d_pos[b] + 1 clamped to [0, min(max_seq_len, capacity)].
+ *   max_seq_len: host upper bound of d_pos[b] + 1.
+ *   out, workspace: as kvq_decode_attn (kvq_decode_attn_workspace sizes it).
+ * Errors as kvq_decode_attn. */
+KVQ_API kvq_status kvq_decode_step(const kvq_cache *cache, const void *k_new, const void *v_new,
+                                   const void *q, kvq_dtype dtype, int32_t batch,
+                                   int32_t num_q_heads, const int32_t *d_pos,
+                                   int32_t max_seq_len, float scale, float *out, void *workspace,
+                                   size_t workspace_bytes, void *stream);
+
 /* kvq_decode_attn_noalloc -- kvq_decode_attn without a caller-provided
  * workspace.  (The pages have no counterpart: this is an interface
  * convenience, not part of the method.)
