@@ -60,7 +60,7 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 5)
     q4_append_kernel(kvq_cache c, const void *__restrict__ k, const void *__restrict__ v,
                      int batch, int t_new, const int32_t *__restrict__ start_pos,
                      FastDiv div_heads, FastDiv div_tnew) {
@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kThreads)
       const bool vnext = gn < ngroups && vn < n_vec;
       fetch_raw<BF16>(vnext ? source(vn) : k, i, vnext, raw);
     }
-    fwht256_warp(i, buf, r);
+    fwht256_warp<false>(i, buf, r);
     QuantOut o;
     q4_quantize_l1(r, lane, i, o);
     uint4 bytes = gather_block_bytes(o, stage, i);

@@ -143,6 +143,9 @@ __device__ __forceinline__ void transpose_l0_l1(float r[32], float4 *buf, int i)
 
 // Full FWHT-256 of the 4 vectors of this warp from layout L0: stages,
 // transpose, stages, end scaling.  Leaves layout L1.
+// SCALE = false leaves the stages' output unscaled (16x the rotation); the
+// quantizer folds the 1/16 into its per-block scale instead.
+template <bool SCALE = true>
 __device__ __forceinline__ void fwht256_warp(int i, float4 *buf, float r[32]) {
   bfly_packed<1>(r);  // h = 1
   bfly_packed<2>(r);  // h = 2
@@ -153,12 +156,14 @@ __device__ __forceinline__ void fwht256_warp(int i, float4 *buf, float r[32]) {
   bfly_packed<4>(r);  // h = 32
   bfly_packed<8>(r);  // h = 64
   bfly16(r);          // h = 128
-  const float2 s = make_float2(0.0625f, 0.0625f);
+  if (SCALE) {
+    const float2 s = make_float2(0.0625f, 0.0625f);
 #pragma unroll
-  for (int k = 0; k < 16; k++) {
-    float2 v = mul2(make_float2(r[k], r[k + 16]), s);
-    r[k] = v.x;
-    r[k + 16] = v.y;
+    for (int k = 0; k < 16; k++) {
+      float2 v = mul2(make_float2(r[k], r[k + 16]), s);
+      r[k] = v.x;
+      r[k + 16] = v.y;
+    }
   }
 }
 
@@ -184,7 +189,11 @@ struct QuantOut {
   uint16_t scale;     // fp16 bits of this lane's block (block index = lane i)
 };
 
-// Quantize the 8 blocks of one vector held in layout L1 (this lane: i).
+// Quantize the 8 blocks of one vector held in layout L1 (this lane: i).  r
+// holds the unscaled stage output w = 16 z.  Scaling by 2^-4 is exact (the
+// bit-exact contract excludes blocks whose max-abs value is below 2^-120), so
+// with w the tie-break order is the same, d = (w_mval / -8) / 16 exactly, and
+// z * RN(1/d) = w * RN(1/(16 d)) is the same real product, rounded once.
 __device__ __forceinline__ void q4_quantize_l1(const float r[32], int lane, int i, QuantOut &o) {
   // register of block B, in-block row m: 4 * (B & 1) + m + 8 * (B >> 1)
   uint32_t key[8];
@@ -196,17 +205,33 @@ __device__ __forceinline__ void q4_quantize_l1(const float r[32], int lane, int 
     const float mz = fmaxf(fmaxf(z0, z1), fmaxf(z2, z3));
     key[B] = (__float_as_uint(am) << 1) | (mz == am ? 1u : 0u);
   }
+  // transposed max-reduction over the 8 lanes of the vector: each xor level
+  // halves the blocks a lane keeps, so lane i ends with the key of block i
 #pragma unroll
-  for (int off = 1; off < 8; off <<= 1)
+  for (int j = 0; j < 4; j++) {  // lanes with bit 2 set keep blocks 4..7
+    const bool up = i & 4;
+    const uint32_t send = up ? key[j] : key[j + 4];
+    const uint32_t keep = up ? key[j + 4] : key[j];
+    key[j] = max(keep, __shfl_xor_sync(kVFull, send, 4));
+  }
 #pragma unroll
-    for (int B = 0; B < 8; B++) key[B] = max(key[B], __shfl_xor_sync(kVFull, key[B], off));
-  uint32_t kmine = key[0];
-#pragma unroll
-  for (int B = 1; B < 8; B++) kmine = (i == B) ? key[B] : kmine;
-  const float mval = key_value(kmine);
-  const float d = __fmul_rn(mval, -0.125f);  // == mval / -8 (exact power-of-two scaling)
-  const float id = (d != 0.f) ? __frcp_rn(d) : 0.f;
-  o.scale = __half_as_ushort(__float2half_rn(d));
+  for (int j = 0; j < 2; j++) {  // bit 1: upper two of the four
+    const bool up = i & 2;
+    const uint32_t send = up ? key[j] : key[j + 2];
+    const uint32_t keep = up ? key[j + 2] : key[j];
+    key[j] = max(keep, __shfl_xor_sync(kVFull, send, 2));
+  }
+  uint32_t kmine;
+  {
+    const bool up = i & 1;
+    const uint32_t send = up ? key[0] : key[1];
+    const uint32_t keep = up ? key[1] : key[0];
+    kmine = max(keep, __shfl_xor_sync(kVFull, send, 1));
+  }
+  const float wval = key_value(kmine);
+  const float dw = __fmul_rn(wval, -0.125f);    // 16 d (exact)
+  const float id = (dw != 0.f) ? __frcp_rn(dw) : 0.f;  // RN(1 / (16 d))
+  o.scale = __half_as_ushort(__float2half_rn(__fmul_rn(dw, 0.0625f)));
   float idb[8];
 #pragma unroll
   for (int B = 0; B < 8; B++) idb[B] = __shfl_sync(kVFull, id, (lane & ~7) | B);
@@ -263,7 +288,7 @@ __device__ __forceinline__ void quantize_vector(const void *src, bool valid, int
   fetch_raw<BF16>(src, i, valid, raw);
   float r[32];
   unpack_l0<BF16>(raw, r);
-  fwht256_warp(i, buf, r);
+  fwht256_warp<false>(i, buf, r);
   QuantOut o;
   q4_quantize_l1(r, lane, i, o);
   bytes = gather_block_bytes(o, reinterpret_cast<uint8_t *>(buf) + 16 * vg, i);
