@@ -201,6 +201,33 @@ kvq_status kvq_decode_attn(const kvq_cache *cache, const void *q, kvq_dtype dtyp
                                     as_stream(stream)));
 }
 
+kvq_status kvq_decode_attn_multi(const kvq_cache *cache, const void *q, kvq_dtype dtype,
+                                 int32_t n_q, int32_t num_q_heads, const int32_t *d_q_to_seq,
+                                 const int32_t *d_q_lens, int32_t num_seqs, int32_t max_seq_len,
+                                 float scale, float *out, void *workspace, size_t workspace_bytes,
+                                 void *stream) {
+  kvq_status st = check_cache(cache);
+  if (st != KVQ_OK) return st;
+  if (n_q < 0 || num_q_heads <= 0 || max_seq_len < 0 || num_seqs < 0 ||
+      (dtype != KVQ_F32 && dtype != KVQ_BF16))
+    return KVQ_ERR_INVALID_ARG;
+  if (num_q_heads % cache->num_kv_heads) return KVQ_ERR_INVALID_ARG;
+  const int group = num_q_heads / cache->num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8 && group != 16) return KVQ_ERR_UNSUPPORTED;
+  if (!cache->block_table && num_seqs > cache->batch_capacity) return KVQ_ERR_INVALID_ARG;
+  if (!isfinite(scale)) return KVQ_ERR_INVALID_ARG;
+  if (n_q == 0) return KVQ_OK;
+  if (!q || !d_q_to_seq || !d_q_lens || !out || !aligned(q, 16) || !aligned(out, 16))
+    return KVQ_ERR_INVALID_ARG;
+  DecodePlan p = plan_decode(n_q, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len);
+  const size_t need = decode_workspace_bytes(n_q, num_q_heads, p);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return KVQ_ERR_WORKSPACE;
+  return from_cuda(launch_q4_decode(*cache, q, dtype == KVQ_BF16, n_q, num_q_heads, d_q_lens,
+                                    max_seq_len, scale, out, static_cast<float *>(workspace), p,
+                                    as_stream(stream), nullptr, nullptr, nullptr, d_q_to_seq,
+                                    num_seqs));
+}
+
 kvq_status kvq_decode_step(const kvq_cache *cache, const void *k_new, const void *v_new,
                            const void *q, kvq_dtype dtype, int32_t batch, int32_t num_q_heads,
                            const int32_t *d_pos, int32_t max_seq_len, float scale, float *out,

@@ -83,18 +83,22 @@ DecodePlan plan_decode(int batch, int n_head_groups, int max_seq_len);
 int q4_decode_ctas_per_sm();
 int q4_decode_tile_tokens();
 // k_new, v_new, pos: fused decode step (append one token per sequence at
-// pos[b], then attend over pos[b] + 1 tokens); all nullptr for plain decode
+// pos[b], then attend over pos[b] + 1 tokens); all nullptr for plain decode.
+// q_to_seq: several queries per sequence (batch = number of queries, query b
+// reads sequence q_to_seq[b] < num_seqs with length seq_lens[b]); nullptr: b.
 cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, int batch,
                                  int n_q_heads, const int32_t *seq_lens, int max_seq_len,
                                  float scale, float *ws, const DecodePlan &p, cudaStream_t s,
                                  const void *k_new = nullptr, const void *v_new = nullptr,
-                                 const int32_t *pos = nullptr);
+                                 const int32_t *pos = nullptr, const int32_t *q_to_seq = nullptr,
+                                 int num_seqs = 0);
 size_t decode_workspace_bytes(int batch, int n_q_heads, const DecodePlan &p);
 cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int batch,
                              int n_q_heads, const int32_t *seq_lens, int max_seq_len,
                              float scale, float *out, float *ws, const DecodePlan &p,
                              cudaStream_t s, const void *k_new = nullptr,
-                             const void *v_new = nullptr, const int32_t *pos = nullptr);
+                             const void *v_new = nullptr, const int32_t *pos = nullptr,
+                             const int32_t *q_to_seq = nullptr, int num_seqs = 0);
 
 struct OctaveParams {
   int head_size, rope_dim, v_bits;

@@ -27,9 +27,9 @@ constexpr int kBatch = 48;
 
 __global__ void __launch_bounds__(256, 1)
     q4_decode_combine_kernel(const float *__restrict__ ws, const int32_t *__restrict__ seq_lens,
-                             const int32_t *__restrict__ pos, int n_q_heads, int splits,
-                             int split_tokens, int max_seq_len, int cap,
-                             float *__restrict__ out) {
+                             const int32_t *__restrict__ pos, const int32_t *__restrict__ q_to_seq,
+                             int num_seqs, int n_q_heads, int splits, int split_tokens,
+                             int max_seq_len, int cap, float *__restrict__ out) {
   __shared__ float ob[kDim];
   __shared__ float wgt[kMaxSplitsSmem];
   __shared__ float red[16];
@@ -37,7 +37,9 @@ __global__ void __launch_bounds__(256, 1)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x, j = threadIdx.x, lane = j & 31, warp = j >> 5;
   const int b = bh / n_q_heads;
-  const int len_raw = pos ? __ldg(pos + b) + 1 : __ldg(seq_lens + b);
+  const int bs = q_to_seq ? __ldg(q_to_seq + b) : b;
+  const int len_raw =
+      (bs < 0 || bs >= num_seqs) ? 0 : (pos ? __ldg(pos + b) + 1 : __ldg(seq_lens + b));
   const int len = min(max(len_raw, 0), min(max_seq_len, cap));
   const float *rec = ws + (int64_t)bh * splits * kRec;
   // splits past the length wrote no record
@@ -178,10 +180,10 @@ cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int ba
                              int n_q_heads, const int32_t *seq_lens, int max_seq_len,
                              float scale, float *out, float *ws, const DecodePlan &p,
                              cudaStream_t s, const void *k_new, const void *v_new,
-                             const int32_t *pos) {
+                             const int32_t *pos, const int32_t *q_to_seq, int num_seqs) {
   if (batch == 0) return cudaSuccess;
   cudaError_t e = launch_q4_decode_mma(c, q, bf16, batch, n_q_heads, seq_lens, max_seq_len,
-                                       scale, ws, p, s, k_new, v_new, pos);
+                                       scale, ws, p, s, k_new, v_new, pos, q_to_seq, num_seqs);
   if (e != cudaSuccess) return e;
   const int cap = c.block_table ? c.max_pages_per_seq * c.page_size : c.max_tokens;
   // programmatic dependent launch: scheduled while the split kernel drains,
@@ -196,7 +198,8 @@ cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int ba
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, q4_decode_combine_kernel, (const float *)ws, seq_lens, pos,
-                         n_q_heads, p.splits, p.split_tokens, max_seq_len, cap, out);
+                         q_to_seq, q_to_seq ? num_seqs : batch, n_q_heads, p.splits,
+                         p.split_tokens, max_seq_len, cap, out);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

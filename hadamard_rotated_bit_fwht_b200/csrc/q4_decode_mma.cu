@@ -234,7 +234,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                          int max_seq_len, int n_q_heads, int group, int gc, float sl2,
                          int split_tokens, int splits, float *__restrict__ ws,
                          const void *__restrict__ k_new, const void *__restrict__ v_new,
-                         const int32_t *__restrict__ pos) {
+                         const int32_t *__restrict__ pos, const int32_t *__restrict__ q_to_seq,
+                         int num_seqs) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int s = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
@@ -269,7 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // fused decode step (pos != nullptr): the new token goes to position pos[b]
   // and the sequence then has pos[b] + 1 tokens
   const int p_new = pos ? __ldg(pos + b) : -1;
-  const int len_raw = pos ? p_new + 1 : __ldg(seq_lens + b);
+  // several queries per sequence (q_to_seq != nullptr): query b reads the cache
+  // of sequence bs; a sequence index outside [0, num_seqs) attends to nothing
+  const int bs = q_to_seq ? __ldg(q_to_seq + b) : b;
+  const int len_raw = (bs < 0 || bs >= num_seqs) ? 0 : (pos ? p_new + 1 : __ldg(seq_lens + b));
   float x[8];
   if (warp < gc) {
     const int64_t off = ((int64_t)b * n_q_heads + h0 + warp) * kDim + 8 * lane;
@@ -306,9 +310,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // first cache row of the 64-token sub-tile starting at token t, -1 if unmapped
   auto sub_row = [&](int t) -> int {
-    if (c.block_table == nullptr) return (int)(((int64_t)b * c.num_kv_heads + kvh) * c.max_tokens + t);
+    if (c.block_table == nullptr) return (int)(((int64_t)bs * c.num_kv_heads + kvh) * c.max_tokens + t);
     const int pi = t / c.page_size;
-    const int page = __ldg(c.block_table + (int64_t)b * c.max_pages_per_seq + pi);
+    const int page = __ldg(c.block_table + (int64_t)bs * c.max_pages_per_seq + pi);
     if (page < 0 || page >= c.num_pages) return -1;
     return (int)(((int64_t)page * c.num_kv_heads + kvh) * c.page_size + (t - pi * c.page_size));
   };
@@ -721,7 +725,8 @@ int q4_decode_tile_tokens() { return kTile; }
 cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, int batch,
                                  int n_q_heads, const int32_t *seq_lens, int max_seq_len,
                                  float scale, float *ws, const DecodePlan &p, cudaStream_t s,
-                                 const void *k_new, const void *v_new, const int32_t *pos) {
+                                 const void *k_new, const void *v_new, const int32_t *pos,
+                                 const int32_t *q_to_seq, int num_seqs) {
   const int group = n_q_heads / c.num_kv_heads;
   const int gc = group < 8 ? group : 8;
   if (p.split_tokens % kTile) return cudaErrorInvalidValue;
@@ -770,11 +775,11 @@ cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, in
   if (bf16)
     e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<true>, maps, c, q, seq_lens, max_seq_len,
                            n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws, k_new, v_new,
-                           pos);
+                           pos, q_to_seq, q_to_seq ? num_seqs : batch);
   else
     e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<false>, maps, c, q, seq_lens, max_seq_len,
                            n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws, k_new, v_new,
-                           pos);
+                           pos, q_to_seq, q_to_seq ? num_seqs : batch);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -26,6 +26,7 @@ EXPORTED = (
     "kvq_decode_attn_workspace", "kvq_decode_attn", "kvq_octave_layout_of",
     "kvq_octave_codebook", "kvq_octave_quantize", "kvq_octave_decode_attn_workspace",
     "kvq_octave_decode_attn", "kvq_decode_attn_noalloc", "kvq_decode_step",
+    "kvq_decode_attn_multi",
 )
 
 
@@ -95,6 +96,10 @@ def lib():
         L.kvq_decode_attn_noalloc.argtypes = [C.POINTER(CacheDesc), C.c_void_p, C.c_int, C.c_int32,
                                               C.c_int32, C.c_void_p, C.c_int32, C.c_float,
                                               C.c_void_p, C.c_void_p]
+        L.kvq_decode_attn_multi.argtypes = [C.POINTER(CacheDesc), C.c_void_p, C.c_int, C.c_int32,
+                                            C.c_int32, C.c_void_p, C.c_void_p, C.c_int32,
+                                            C.c_int32, C.c_float, C.c_void_p, C.c_void_p,
+                                            C.c_size_t, C.c_void_p]
         L.kvq_decode_step.argtypes = [C.POINTER(CacheDesc), C.c_void_p, C.c_void_p, C.c_void_p,
                                       C.c_int, C.c_int32, C.c_int32, C.c_void_p, C.c_int32,
                                       C.c_float, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
@@ -247,6 +252,32 @@ def decode_attn(cache: Q4Cache, q: torch.Tensor, seq_lens: torch.Tensor, max_seq
            lib().kvq_decode_attn(C.byref(d), _ptr(q), _dtype_code(q), batch, hq, _ptr(seq_lens),
                                  int(max_seq_len), float(scale), _ptr(out), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def decode_attn_multi(cache: Q4Cache, q: torch.Tensor, q_to_seq: torch.Tensor,
+                      q_lens: torch.Tensor, num_seqs: int, max_seq_len: int, scale: float,
+                      out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """Query i (q [n_q, Hq, 256]) attends over the first q_lens[i] tokens of
+    sequence q_to_seq[i] (kvq_decode_attn_multi)."""
+    for name, t in (("q", q), ("q_to_seq", q_to_seq), ("q_lens", q_lens)):
+        _cuda_contig(name, t)
+    if q_to_seq.dtype != torch.int32 or q_lens.dtype != torch.int32:
+        raise TypeError("q_to_seq and q_lens must be int32")
+    n_q, hq, dim = q.shape
+    if out is None:
+        out = torch.empty((n_q, hq, dim), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = decode_attn_workspace(cache, n_q, hq, max_seq_len)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    d = cache.desc()
+    _check("kvq_decode_attn_multi",
+           lib().kvq_decode_attn_multi(C.byref(d), _ptr(q), _dtype_code(q), n_q, hq,
+                                       _ptr(q_to_seq), _ptr(q_lens), int(num_seqs),
+                                       int(max_seq_len), float(scale), _ptr(out), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(stream)))
     return out
 
 

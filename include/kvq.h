@@ -162,6 +162,29 @@ KVQ_API kvq_status kvq_decode_attn(const kvq_cache *cache, const void *q, kvq_dt
                            float *out, void *workspace, size_t workspace_bytes,
                            void *stream);
 
+/* kvq_decode_attn_multi -- several query tokens per sequence (speculative
+ * verification, multi-token prediction): query i attends over the first
+ * d_q_lens[i] tokens of sequence d_q_to_seq[i] of the Q4_0 cache (the causal
+ * prefix of each drafted token is expressed through its length, as in the
+ * q_to_req / q_to_klen arguments of the Octave page's reference_attention).
+ * Otherwise as kvq_decode_attn with batch = n_q:
+ *   q: device, [n_q][num_q_heads][256] of `dtype`, 16-byte aligned.
+ *   d_q_to_seq: device int32[n_q]; a value outside [0, num_seqs) gives a zero
+ *   row.  num_seqs: sequences in the cache (contiguous: <= batch_capacity;
+ *   paged: rows of the block table).
+ *   d_q_lens: device int32[n_q], clamped to [0, min(max_seq_len, capacity)].
+ *   out: device, [n_q][num_q_heads][256] fp32, 16-byte aligned.
+ *   workspace: >= kvq_decode_attn_workspace(cache, n_q, num_q_heads,
+ *   max_seq_len) bytes.
+ * Each query streams its sequence's cache on its own (no sharing of KV reads
+ * between the queries of one sequence). */
+KVQ_API kvq_status kvq_decode_attn_multi(const kvq_cache *cache, const void *q, kvq_dtype dtype,
+                                         int32_t n_q, int32_t num_q_heads,
+                                         const int32_t *d_q_to_seq, const int32_t *d_q_lens,
+                                         int32_t num_seqs, int32_t max_seq_len, float scale,
+                                         float *out, void *workspace, size_t workspace_bytes,
+                                         void *stream);
+
 /* kvq_decode_step -- one decode step of the per-token path in a single call:
  * quantize-on-append of each sequence's new token, then decode attention over
  * the sequence including it (Strata PR #21, merge note: the per-token path
