@@ -106,10 +106,11 @@ kvq_status octave_params(const kvq_octave_fmt *f, const int32_t *sign_bits, Octa
   kvq_status st = octave_layout(f, &lay);
   if (st != KVQ_OK) return st;
   if (!sign_bits) return KVQ_ERR_INVALID_ARG;
-  if (f->compact || f->head_size != 128 || f->rope_dim > 128) return KVQ_ERR_UNSUPPORTED;
+  if (f->head_size != 128 || f->rope_dim > 128) return KVQ_ERR_UNSUPPORTED;
   memset(&p, 0, sizeof(p));
   p.head_size = f->head_size;
-  p.rope_dim = f->rope_dim;
+  p.rope_dim = f->compact ? 0 : f->rope_dim;
+  p.compact = f->compact ? 1 : 0;
   p.v_bits = f->v_bits;
   p.off_k_nope = lay.off_k_nope;
   p.off_v = lay.off_v;

@@ -101,7 +101,9 @@ cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int ba
                              const int32_t *q_to_seq = nullptr, int num_seqs = 0);
 
 struct OctaveParams {
-  int head_size, rope_dim, v_bits;
+  // rope_dim here is the K dims coded with 4 bits (0 for compact K, whose
+  // codes are all 3-bit over one whole-head rotation with one scale)
+  int head_size, rope_dim, v_bits, compact;
   int off_k_nope, off_v, off_scales, slot_bytes;
   uint32_t sign_words[16];  // up to 512 dims
   int8_t lut3[8];

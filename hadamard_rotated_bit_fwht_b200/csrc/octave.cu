@@ -159,7 +159,8 @@ __global__ void __launch_bounds__(kThreads)
        it += (int64_t)gridDim.x * kWarps) {
     const int tok = (int)(it / n_kv_heads), h = (int)(it % n_kv_heads);
     const int64_t base = it * kHead;
-    // ---- K
+    // ---- K: 64-dim blocks (4-bit RoPE dims, 3-bit others) or, compact, one
+    // whole-head rotation with 3-bit codes and one scale
     float x[4];
 #pragma unroll
     for (int k = 0; k < 4; k++) {
@@ -179,17 +180,34 @@ __global__ void __launch_bounds__(kThreads)
       x[2] = __fadd_rn(a, b);
       x[3] = __fsub_rn(a, b);
     }
-#pragma unroll
-    for (int k = 0; k < 4; k++) x[k] = __fmul_rn(x[k], 0.125f);
     float ks[2];
+    if (P.compact) {
+      float a = x[0], b = x[2];  // h = 64
+      x[0] = __fadd_rn(a, b);
+      x[2] = __fsub_rn(a, b);
+      a = x[1];
+      b = x[3];
+      x[1] = __fadd_rn(a, b);
+      x[3] = __fsub_rn(a, b);
 #pragma unroll
-    for (int kb = 0; kb < 2; kb++) {
-      float xb[2] = {x[2 * kb], x[2 * kb + 1]};
-      int cb[2];
-      if (kb * 64 < P.rope_dim) ks[kb] = quantize_lut<2, 4>(xb, P.mult4, L, cb);
-      else ks[kb] = quantize_lut<2, 3>(xb, P.mult3, L, cb);
-      kcodes[warp][64 * kb + lane] = (uint8_t)cb[0];
-      kcodes[warp][64 * kb + lane + 32] = (uint8_t)cb[1];
+      for (int k = 0; k < 4; k++) x[k] = __fmul_rn(x[k], vscale);
+      int ck[4];
+      ks[0] = quantize_lut<4, 3>(x, P.mult3, L, ck);
+      ks[1] = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; k++) kcodes[warp][lane + 32 * k] = (uint8_t)ck[k];
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; k++) x[k] = __fmul_rn(x[k], 0.125f);
+#pragma unroll
+      for (int kb = 0; kb < 2; kb++) {
+        float xb[2] = {x[2 * kb], x[2 * kb + 1]};
+        int cb[2];
+        if (kb * 64 < P.rope_dim) ks[kb] = quantize_lut<2, 4>(xb, P.mult4, L, cb);
+        else ks[kb] = quantize_lut<2, 3>(xb, P.mult3, L, cb);
+        kcodes[warp][64 * kb + lane] = (uint8_t)cb[0];
+        kcodes[warp][64 * kb + lane + 32] = (uint8_t)cb[1];
+      }
     }
     // ---- V
 #pragma unroll
@@ -240,10 +258,10 @@ __global__ void __launch_bounds__(kThreads)
       if (w < w_kn) word = pack_word(kc32, P.rope_dim, 4, w);
       else if (w < w_v) word = pack_word(kc32 + P.rope_dim / 4, kHead - P.rope_dim, 3, w - w_kn);
       else if (w < w_sc) word = pack_word(vc32, kHead, P.v_bits, w - w_v);
-      else if (w == w_sc)
+      else if (w == w_sc)  // fp16 scales, K first then V
         word = (uint32_t)__half_as_ushort(__float2half_rn(ks[0])) |
-               ((uint32_t)__half_as_ushort(__float2half_rn(ks[1])) << 16);
-      else if (w == w_sc + 1)
+               ((uint32_t)__half_as_ushort(__float2half_rn(P.compact ? vs : ks[1])) << 16);
+      else if (w == w_sc + 1 && !P.compact)
         word = (uint32_t)__half_as_ushort(__float2half_rn(vs));
       if (dst) dst[w] = word;
     }
@@ -283,28 +301,31 @@ __global__ void __launch_bounds__(kThreads)
   if (req < 0 || req >= num_reqs) klen = 0;
   const int t0 = s * split_tokens, t1 = min(klen, t0 + split_tokens);
 
-  // query: signs, FWHT over 64-dim blocks, x 1/8, x scale*log2(e)
+  // query: signs, FWHT over the K rotation blocks (64 dims, or the whole
+  // head for compact K), x fp32(1 / sqrt(block)), x scale*log2(e)
+  const int kb_size = P.compact ? kHead : 64;
   for (int p = threadIdx.x; p < GC * kHead; p += blockDim.x) {
     const int hh = p / kHead, d = p % kHead;
     qs[hh][d] = load_in(query, BF16, ((int64_t)qi * n_q_heads + h0 + hh) * kHead + d) * sign_of(P, d);
   }
-  for (int h = 1; h < 64; h <<= 1) {
+  for (int h = 1; h < kb_size; h <<= 1) {
     __syncthreads();
     for (int p = threadIdx.x; p < GC * 64; p += blockDim.x) {
-      const int vv = p / 64, pi = p % 64;  // 2 blocks x 32 pairs per head
-      const int blk = pi / 32, pj = pi % 32;
-      const int i0 = blk * 64 + (pj / h) * 2 * h + (pj % h);
+      const int vv = p / 64, pi = p % 64;  // 64 pairs per head
+      const int blk = pi / (kb_size / 2), pj = pi % (kb_size / 2);
+      const int i0 = blk * kb_size + (pj / h) * 2 * h + (pj % h);
       const float a = qs[vv][i0], b = qs[vv][i0 + h];
       qs[vv][i0] = a + b;
       qs[vv][i0 + h] = a - b;
     }
   }
   __syncthreads();
+  const float qscale = (P.compact ? 0.08838834764831845f : 0.125f) * scale_log2;
   float qr[GC][4];
 #pragma unroll
   for (int hh = 0; hh < GC; hh++)
 #pragma unroll
-    for (int k = 0; k < 4; k++) qr[hh][k] = qs[hh][lane + 32 * k] * (0.125f * scale_log2);
+    for (int k = 0; k < 4; k++) qr[hh][k] = qs[hh][lane + 32 * k] * qscale;
 
   float m[GC], l[GC], o[GC][4];
 #pragma unroll
@@ -324,9 +345,10 @@ __global__ void __launch_bounds__(kThreads)
     const uint32_t s01 = slot_byte(myword, P.off_scales) | (slot_byte(myword, P.off_scales + 1) << 8);
     const uint32_t s23 = slot_byte(myword, P.off_scales + 2) | (slot_byte(myword, P.off_scales + 3) << 8);
     const uint32_t s45 = slot_byte(myword, P.off_scales + 4) | (slot_byte(myword, P.off_scales + 5) << 8);
+    // scales: K per 64-block then V, or (compact) one K scale then V
     const float sk0 = __half2float(__ushort_as_half((uint16_t)s01)) / kLutOne;
-    const float sk1 = __half2float(__ushort_as_half((uint16_t)s23)) / kLutOne;
-    const float sv = __half2float(__ushort_as_half((uint16_t)s45)) / kLutOne;
+    const float sk1 = P.compact ? sk0 : __half2float(__ushort_as_half((uint16_t)s23)) / kLutOne;
+    const float sv = __half2float(__ushort_as_half((uint16_t)(P.compact ? s23 : s45))) / kLutOne;
     float kd[4], vd[4];
 #pragma unroll
     for (int k = 0; k < 4; k++) {

@@ -499,7 +499,8 @@ __global__ void __launch_bounds__(kThreads, 4)
 }  // namespace
 
 bool octave_mma_supported(const OctaveParams &P) {
-  return P.head_size == kHead && P.rope_dim == 64 && P.v_bits == 4 && P.slot_bytes == 128;
+  return P.head_size == kHead && !P.compact && P.rope_dim == 64 && P.v_bits == 4 &&
+         P.slot_bytes == 128;
 }
 
 cudaError_t launch_octave_decode_mma(const OctaveParams &P, const void *query, int bf16, int num_q,

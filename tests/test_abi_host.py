@@ -92,9 +92,9 @@ def test_validation_without_launch(L):
     # paged cache needs a page size that is a multiple of 64
     d2 = kvq.CacheDesc(p16, p16, p16, p16, 2, 256, 0, 0, p16, 48, 4, 8)
     assert L.kvq_quantize_append(C.byref(d2), p16, p16, 1, 1, 1, p16, None) == kvq.KVQ_ERR_INVALID_ARG
-    # octave: compact K is a valid format this build does not implement
-    f = kvq.OctaveFormat(128, 64, 3, True).desc()
-    sb = np.zeros(4, np.int32)
+    # octave: head 256 is a valid format this build does not implement
+    f = kvq.OctaveFormat(256, 64, 3, True).desc()
+    sb = np.zeros(8, np.int32)
     assert L.kvq_octave_quantize(C.byref(f), p16, p16, 1, 1, 1, p16, p16, 16, 1,
                                  sb.ctypes.data_as(C.c_void_p), None) == kvq.KVQ_ERR_UNSUPPORTED
 

@@ -186,3 +186,51 @@ def test_octave_workload_sampled():
                                  kvq.sign_words(signs)).cpu().numpy()
     want = oracle.octave_attention(q, c, bt, q_to_req, q_to_klen, fmt, 128 ** -0.5, signs)
     assert np.abs(got - want).max() <= ATOL
+
+
+# ------------------------------------------------------------------ compact K
+@pytest.mark.parametrize("v_bits", [3, 4])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_compact_quantize_bitexact(v_bits, dt):
+    """Compact K (octave_k3v3_compact and its 4-bit-V sibling): one whole-head
+    rotation of K with 3-bit codes and a single scale; 4-byte slot padding."""
+    fmt = (128, 64, v_bits, 1)
+    F = kvq.OctaveFormat(128, 64, v_bits, True)
+    slot_bytes = F.layout()["slot_bytes"]
+    T, Hkv, bs = 257, 2, 16
+    k, v, slot, nblk = make_cache(fmt, T, Hkv, bs, 90 + v_bits, dt)
+    signs = synth.sign_pattern(128)
+    cache = torch.zeros((nblk, Hkv, bs, slot_bytes), dtype=torch.uint8, device="cuda")
+    kvq.octave_quantize(F, to_dev(k), to_dev(v), to_dev(slot), cache, kvq.sign_words(signs))
+    want = oracle.octave_quantize(k, v, fmt, signs)
+    got = cache.cpu().numpy().transpose(0, 2, 1, 3).reshape(-1, Hkv, slot_bytes)[slot]
+    bad = np.nonzero(np.any(got != want, axis=-1))
+    assert bad[0].size == 0, f"{bad[0].size} slots differ, first token {bad[0][:3]}"
+
+
+@pytest.mark.parametrize("v_bits", [3, 4])
+@pytest.mark.parametrize("G", [1, 4, 8])
+def test_compact_decode_vs_oracle(v_bits, G):
+    fmt = (128, 64, v_bits, 1)
+    F = kvq.OctaveFormat(128, 64, v_bits, True)
+    slot_bytes = F.layout()["slot_bytes"]
+    Hkv, bs, T = 2, 16, 600
+    k, v, slot, nblk = make_cache(fmt, T, Hkv, bs, 95 + G)
+    signs = synth.sign_pattern(128)
+    cache = torch.zeros((nblk, Hkv, bs, slot_bytes), dtype=torch.uint8, device="cuda")
+    kvq.octave_quantize(F, to_dev(k), to_dev(v), to_dev(slot), cache, kvq.sign_words(signs))
+    nreq, span = 3, 192
+    maxb = -(-span // bs)
+    bt = np.zeros((nreq, maxb), np.int32)
+    for r in range(nreq):
+        for j in range(maxb):
+            bt[r, j] = slot[min(span * r + j * bs, T - 1)] // bs
+    q = synth.to_bf16_bits(synth.queries(97 + G, 4, Hkv * G, 128))
+    q_to_req = np.array([0, 1, 2, 0], np.int32)
+    q_to_klen = np.array([192, 45, 0, 129], np.int32)
+    got = kvq.octave_decode_attn(F, to_dev(q), cache, to_dev(bt), to_dev(q_to_req),
+                                 to_dev(q_to_klen), 192, 128 ** -0.5,
+                                 kvq.sign_words(signs)).cpu().numpy()
+    want = oracle.octave_attention(q, cache.cpu().numpy(), bt, q_to_req, q_to_klen, fmt,
+                                   128 ** -0.5, signs)
+    assert np.abs(got - want).max() <= ATOL
