@@ -136,18 +136,50 @@ def q4_quantize_vectors(x):
     return codes, scales
 
 
-class Q4Cache:
-    """Oracle-side Q4_0 cache with the documented structure-of-arrays layout."""
+# ---------------------------------------------------------------- Q8_0
+def q8_0_block(z):
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    assert z.shape == (32,)
+    qs = np.zeros(32, np.int8)
+    d = C.c_uint16(0)
+    _check(lib().orc_q8_0_block(_p(z), _p(qs), C.byref(d)), "q8_0_block")
+    return qs, int(d.value)
 
-    def __init__(self, n_rows, n_kv_heads, max_tokens=0, block_table=None, page_size=0):
+
+def q8_0_dequant_block(qs, d_bits):
+    qs = np.ascontiguousarray(qs, dtype=np.int8)
+    out = np.zeros(32, np.float64)
+    _check(lib().orc_q8_0_dequant_block(_p(qs), C.c_uint16(d_bits), _p(out)), "q8 dequant")
+    return out
+
+
+def q8_quantize_vectors(x):
+    """x: (..., 256) float32 or bf16 bits -> codes (..., 256) int8, scales (..., 8) u16."""
+    x = np.ascontiguousarray(x)
+    n = x.size // 256
+    codes = np.zeros(x.shape[:-1] + (256,), np.int8)
+    scales = np.zeros(x.shape[:-1] + (8,), np.uint16)
+    _check(lib().orc_q8_quantize_vectors(_p(x), _dtype_code(x), C.c_int64(n), _p(codes),
+                                         _p(scales)), "q8_quantize_vectors")
+    return codes, scales
+
+
+class Q4Cache:
+    """Oracle-side Q4_0 cache with the documented structure-of-arrays layout
+    (bits = 8: the Q8_0 cache, 256 int8 code bytes per row)."""
+
+    def __init__(self, n_rows, n_kv_heads, max_tokens=0, block_table=None, page_size=0,
+                 bits=4):
         self.n_kv_heads = n_kv_heads
         self.max_tokens = max_tokens
         self.block_table = (None if block_table is None else
                             np.ascontiguousarray(block_table, dtype=np.int32))
         self.page_size = page_size
         self.max_pages = 0 if block_table is None else self.block_table.shape[1]
-        self.k_codes = np.zeros((n_rows, 128), np.uint8)
-        self.v_codes = np.zeros((n_rows, 128), np.uint8)
+        self.bits = bits
+        cdt, cw = (np.int8, 256) if bits == 8 else (np.uint8, 128)
+        self.k_codes = np.zeros((n_rows, cw), cdt)
+        self.v_codes = np.zeros((n_rows, cw), cdt)
         self.k_scales = np.zeros((n_rows, 8), np.uint16)
         self.v_scales = np.zeros((n_rows, 8), np.uint16)
 
@@ -170,16 +202,17 @@ class Q4Cache:
         batch, t_new, hkv, d = k.shape
         assert hkv == self.n_kv_heads and d == 256
         sp = np.ascontiguousarray(start_pos, dtype=np.int32)
-        _check(lib().orc_q4_append(*self._args(), _p(k), _p(v), _dtype_code(k), batch, t_new,
-                                   _p(sp)), "q4_append")
+        fn = lib().orc_q8_append if self.bits == 8 else lib().orc_q4_append
+        _check(fn(*self._args(), _p(k), _p(v), _dtype_code(k), batch, t_new, _p(sp)), "append")
 
     def decode_attn(self, q, seq_lens, scale):
         q = np.ascontiguousarray(q)
         batch, hq, d = q.shape
         sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
         out = np.zeros((batch, hq, d), np.float64)
-        _check(lib().orc_q4_decode_attn(*self._args(), _p(q), _dtype_code(q), batch, hq,
-                                        _p(sl), C.c_double(scale), _p(out)), "q4_decode_attn")
+        fn = lib().orc_q8_decode_attn if self.bits == 8 else lib().orc_q4_decode_attn
+        _check(fn(*self._args(), _p(q), _dtype_code(q), batch, hq, _p(sl), C.c_double(scale),
+                  _p(out)), "decode_attn")
         return out
 
 

@@ -192,9 +192,40 @@ int orc_q4_0_dequant_block(const uint8_t qs[16], uint16_t d_bits, double out[32]
   return 0;
 }
 
-/* FWHT-256 (fp32) then Q4_0 over the 8 consecutive 32-value blocks of the
- * rotated vector [P1 How 1-2: rotate before quantization]. */
-static int q4_quantize_one(const void *x, int dtype, int64_t base, uint8_t *codes,
+/* ---------------- Q8_0 ----------------
+ * The 8-bit variant the pages compare Q4_0 against ("int8 KV", "Q8_0").
+ * Reading (the pages name the type but not its steps; the name is GGML's, so
+ * its convention is taken): amax = max |z_j|;  d = amax / 127;
+ * id = d != 0 ? 1/d : 0;  code_j = roundf(z_j * id) (product rounded to fp32,
+ * then rounded to the nearest integer, halves away from zero), stored as int8;
+ * stored scale = fp16(d); dequantized value = code * fp16(d). */
+int orc_q8_0_block(const float z[32], int8_t qs[32], uint16_t *d_bits) {
+  float amax = 0.0f;
+  for (int j = 0; j < Q4_BLK; j++) {
+    if (!finite_f(z[j])) return -2;
+    float a = fabsf(z[j]);
+    if (a > amax) amax = a;
+  }
+  float d = amax / 127.0f;
+  float id = (d != 0.0f) ? 1.0f / d : 0.0f;
+  for (int j = 0; j < Q4_BLK; j++) {
+    float t = z[j] * id;
+    qs[j] = (int8_t)roundf(t);
+  }
+  *d_bits = orc_f32_to_f16(d);
+  return 0;
+}
+
+int orc_q8_0_dequant_block(const int8_t qs[32], uint16_t d_bits, double out[32]) {
+  double d = (double)orc_f16_to_f32(d_bits);
+  for (int j = 0; j < Q4_BLK; j++) out[j] = (double)qs[j] * d;
+  return 0;
+}
+
+/* FWHT-256 (fp32) then Q4_0 (bits 4) or Q8_0 (bits 8) over the 8
+ * consecutive 32-value blocks of the rotated vector [P1 How 1-2: rotate
+ * before quantization].  Code row: 128 (Q4_0) or 256 (Q8_0) bytes. */
+static int kv_quantize_one(int bits, const void *x, int dtype, int64_t base, uint8_t *codes,
                            uint16_t *scales) {
   float y[Q4_DIM];
   for (int j = 0; j < Q4_DIM; j++) {
@@ -203,17 +234,30 @@ static int q4_quantize_one(const void *x, int dtype, int64_t base, uint8_t *code
   }
   fwht_block_f32(y, Q4_DIM);
   for (int b = 0; b < Q4_DIM / Q4_BLK; b++) {
-    int r = orc_q4_0_block(y + b * Q4_BLK, codes + b * 16, scales + b);
+    int r = bits == 8 ? orc_q8_0_block(y + b * Q4_BLK, (int8_t *)codes + b * 32, scales + b)
+                      : orc_q4_0_block(y + b * Q4_BLK, codes + b * 16, scales + b);
     if (r) return r;
   }
   return 0;
 }
 
+static int row_bytes(int bits) { return bits == 8 ? 256 : 128; }
+
 int orc_q4_quantize_vectors(const void *x, int dtype, int64_t n_vec, uint8_t *codes,
                             uint16_t *scales) {
   if (!x || !codes || !scales || n_vec < 0 || (dtype != 0 && dtype != 1)) return -1;
   for (int64_t v = 0; v < n_vec; v++) {
-    int r = q4_quantize_one(x, dtype, v * Q4_DIM, codes + v * 128, scales + v * 8);
+    int r = kv_quantize_one(4, x, dtype, v * Q4_DIM, codes + v * 128, scales + v * 8);
+    if (r) return r;
+  }
+  return 0;
+}
+
+int orc_q8_quantize_vectors(const void *x, int dtype, int64_t n_vec, int8_t *codes,
+                            uint16_t *scales) {
+  if (!x || !codes || !scales || n_vec < 0 || (dtype != 0 && dtype != 1)) return -1;
+  for (int64_t v = 0; v < n_vec; v++) {
+    int r = kv_quantize_one(8, x, dtype, v * Q4_DIM, (uint8_t *)codes + v * 256, scales + v * 8);
     if (r) return r;
   }
   return 0;
@@ -227,7 +271,7 @@ static int64_t q4_row(int b, int h, int t, int n_kv_heads, int max_tokens,
   return ((int64_t)page * n_kv_heads + h) * page_size + (t % page_size);
 }
 
-int orc_q4_append(uint8_t *k_codes, uint16_t *k_scales, uint8_t *v_codes,
+static int kv_append(int bits, uint8_t *k_codes, uint16_t *k_scales, uint8_t *v_codes,
                   uint16_t *v_scales, int n_kv_heads, int max_tokens,
                   const int32_t *block_table, int page_size, int max_pages,
                   const void *k, const void *v, int dtype, int batch, int t_new,
@@ -247,9 +291,10 @@ int orc_q4_append(uint8_t *k_codes, uint16_t *k_scales, uint8_t *v_codes,
         int64_t row = q4_row(b, h, t, n_kv_heads, max_tokens, block_table,
                              page_size, max_pages);
         if (row < 0) return -1;
-        int r = q4_quantize_one(k, dtype, src, k_codes + row * 128, k_scales + row * 8);
+        const int rb = row_bytes(bits);
+        int r = kv_quantize_one(bits, k, dtype, src, k_codes + row * rb, k_scales + row * 8);
         if (r) return r;
-        r = q4_quantize_one(v, dtype, src, v_codes + row * 128, v_scales + row * 8);
+        r = kv_quantize_one(bits, v, dtype, src, v_codes + row * rb, v_scales + row * 8);
         if (r) return r;
       }
     }
@@ -257,19 +302,42 @@ int orc_q4_append(uint8_t *k_codes, uint16_t *k_scales, uint8_t *v_codes,
   return 0;
 }
 
+int orc_q4_append(uint8_t *k_codes, uint16_t *k_scales, uint8_t *v_codes,
+                  uint16_t *v_scales, int n_kv_heads, int max_tokens,
+                  const int32_t *block_table, int page_size, int max_pages,
+                  const void *k, const void *v, int dtype, int batch, int t_new,
+                  const int32_t *start_pos) {
+  return kv_append(4, k_codes, k_scales, v_codes, v_scales, n_kv_heads, max_tokens, block_table,
+                   page_size, max_pages, k, v, dtype, batch, t_new, start_pos);
+}
+
+int orc_q8_append(int8_t *k_codes, uint16_t *k_scales, int8_t *v_codes,
+                  uint16_t *v_scales, int n_kv_heads, int max_tokens,
+                  const int32_t *block_table, int page_size, int max_pages,
+                  const void *k, const void *v, int dtype, int batch, int t_new,
+                  const int32_t *start_pos) {
+  return kv_append(8, (uint8_t *)k_codes, k_scales, (uint8_t *)v_codes, v_scales, n_kv_heads,
+                   max_tokens, block_table, page_size, max_pages, k, v, dtype, batch, t_new,
+                   start_pos);
+}
+
 /* Dequantize one cached row and rotate it back to the original basis in fp64
  * (H is symmetric and orthonormal, so H^-1 = H). */
-static void q4_row_unrotated(const uint8_t *codes, const uint16_t *scales, int64_t row,
-                             double *out) {
-  for (int b = 0; b < Q4_DIM / Q4_BLK; b++)
-    orc_q4_0_dequant_block(codes + row * 128 + b * 16, scales[row * 8 + b],
-                           out + b * Q4_BLK);
+static void kv_row_unrotated(int bits, const uint8_t *codes, const uint16_t *scales,
+                             int64_t row, double *out) {
+  for (int b = 0; b < Q4_DIM / Q4_BLK; b++) {
+    if (bits == 8)
+      orc_q8_0_dequant_block((const int8_t *)codes + row * 256 + b * 32, scales[row * 8 + b],
+                             out + b * Q4_BLK);
+    else
+      orc_q4_0_dequant_block(codes + row * 128 + b * 16, scales[row * 8 + b], out + b * Q4_BLK);
+  }
   fwht_block_f64(out, Q4_DIM);
 }
 
 /* Attention in the original basis: by the score invariance <Hq, Hk> = <q, k>
  * [P1 What] this is the quantity the rotated-space kernel computes. */
-int orc_q4_decode_attn(const uint8_t *k_codes, const uint16_t *k_scales,
+static int kv_decode_attn(int bits, const uint8_t *k_codes, const uint16_t *k_scales,
                        const uint8_t *v_codes, const uint16_t *v_scales,
                        int n_kv_heads, int max_tokens, const int32_t *block_table,
                        int page_size, int max_pages, const void *q, int dtype,
@@ -307,7 +375,7 @@ int orc_q4_decode_attn(const uint8_t *k_codes, const uint16_t *k_scales,
         int64_t row = q4_row(b, g, t, n_kv_heads, max_tokens, block_table, page_size,
                              max_pages);
         if (row < 0) { free(sc); free(qv); return -1; }
-        q4_row_unrotated(k_codes, k_scales, row, kd);
+        kv_row_unrotated(bits, k_codes, k_scales, row, kd);
         for (int hh = 0; hh < group; hh++) {
           double s = 0.0;
           for (int j = 0; j < Q4_DIM; j++) s += qv[hh * Q4_DIM + j] * kd[j];
@@ -330,7 +398,7 @@ int orc_q4_decode_attn(const uint8_t *k_codes, const uint16_t *k_scales,
         int64_t row = q4_row(b, g, t, n_kv_heads, max_tokens, block_table, page_size,
                              max_pages);
         if (row < 0) { free(sc); free(qv); return -1; }
-        q4_row_unrotated(v_codes, v_scales, row, kd);
+        kv_row_unrotated(bits, v_codes, v_scales, row, kd);
         for (int hh = 0; hh < group; hh++) {
           double p = sc[(int64_t)t * group + hh];
           double *o = out + ((int64_t)b * n_q_heads + g * group + hh) * Q4_DIM;
@@ -342,6 +410,28 @@ int orc_q4_decode_attn(const uint8_t *k_codes, const uint16_t *k_scales,
     free(qv);
   }
   return 0;
+}
+
+int orc_q4_decode_attn(const uint8_t *k_codes, const uint16_t *k_scales,
+                       const uint8_t *v_codes, const uint16_t *v_scales,
+                       int n_kv_heads, int max_tokens, const int32_t *block_table,
+                       int page_size, int max_pages, const void *q, int dtype,
+                       int batch, int n_q_heads, const int32_t *seq_lens,
+                       double scale, double *out) {
+  return kv_decode_attn(4, k_codes, k_scales, v_codes, v_scales, n_kv_heads, max_tokens,
+                        block_table, page_size, max_pages, q, dtype, batch, n_q_heads, seq_lens,
+                        scale, out);
+}
+
+int orc_q8_decode_attn(const int8_t *k_codes, const uint16_t *k_scales,
+                       const int8_t *v_codes, const uint16_t *v_scales,
+                       int n_kv_heads, int max_tokens, const int32_t *block_table,
+                       int page_size, int max_pages, const void *q, int dtype,
+                       int batch, int n_q_heads, const int32_t *seq_lens,
+                       double scale, double *out) {
+  return kv_decode_attn(8, (const uint8_t *)k_codes, k_scales, (const uint8_t *)v_codes,
+                        v_scales, n_kv_heads, max_tokens, block_table, page_size, max_pages, q,
+                        dtype, batch, n_q_heads, seq_lens, scale, out);
 }
 
 /* ===================================================================== */

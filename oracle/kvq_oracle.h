@@ -53,6 +53,16 @@ int orc_fwht_f64(double *x, int64_t n_vec, int dim, int block);
 int orc_q4_0_block(const float z[32], uint8_t qs[16], uint16_t *d_bits);
 int orc_q4_0_dequant_block(const uint8_t qs[16], uint16_t d_bits, double out[32]);
 
+/* ---------------- Q8_0 ----------------
+ * The 8-bit KV variant the pages compare Q4_0 against; GGML's Q8_0 steps:
+ * d = amax / 127, id = d ? 1/d : 0, code = roundf(z * id) (int8), fp16(d). */
+int orc_q8_0_block(const float z[32], int8_t qs[32], uint16_t *d_bits);
+int orc_q8_0_dequant_block(const int8_t qs[32], uint16_t d_bits, double out[32]);
+/* Rotate + Q8_0-quantize n_vec vectors: codes n_vec x 256 int8, scales
+ * n_vec x 8 fp16 bit patterns. */
+int orc_q8_quantize_vectors(const void *x, int dtype, int64_t n_vec, int8_t *codes,
+                            uint16_t *scales);
+
 /* Rotate (fp32 FWHT-256) + Q4_0-quantize n_vec vectors of 256 values.
  * dtype: 0 = fp32 input, 1 = bf16 input (raw uint16 bits).
  * codes: n_vec x 128 bytes; scales: n_vec x 8 fp16 bit patterns. */
@@ -82,6 +92,20 @@ int orc_q4_append(uint8_t *k_codes, uint16_t *k_scales, uint8_t *v_codes,
  * reference_attention] */
 int orc_q4_decode_attn(const uint8_t *k_codes, const uint16_t *k_scales,
                        const uint8_t *v_codes, const uint16_t *v_scales,
+                       int n_kv_heads, int max_tokens,
+                       const int32_t *block_table, int page_size,
+                       int max_pages, const void *q, int dtype, int batch,
+                       int n_q_heads, const int32_t *seq_lens, double scale,
+                       double *out);
+
+/* The same two calls over a Q8_0 cache (256 int8 code bytes per row). */
+int orc_q8_append(int8_t *k_codes, uint16_t *k_scales, int8_t *v_codes,
+                  uint16_t *v_scales, int n_kv_heads, int max_tokens,
+                  const int32_t *block_table, int page_size, int max_pages,
+                  const void *k, const void *v, int dtype, int batch,
+                  int t_new, const int32_t *start_pos);
+int orc_q8_decode_attn(const int8_t *k_codes, const uint16_t *k_scales,
+                       const int8_t *v_codes, const uint16_t *v_scales,
                        int n_kv_heads, int max_tokens,
                        const int32_t *block_table, int page_size,
                        int max_pages, const void *q, int dtype, int batch,
