@@ -1,0 +1,217 @@
+// decode_common.cuh -- device and host helpers shared by the split-K decode
+// kernels (q4_decode_mma.cu, q8_decode_mma.cu): bounded mbarrier waits, TMA
+// loads and tensor maps, ldmatrix / mma.sync wrappers, the fp16 hi/lo split,
+// programmatic-dependent-launch controls and the in-register FWHT-256.
+// Nothing here is part of the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace dec {
+
+constexpr unsigned kFullMask = 0xffffffffu;
+
+// bounded waits: ~2^20 polls of up to ~1 us each, abandoned early once any
+// thread of the CTA has given up
+constexpr int kWaitPolls = 1 << 20;
+
+struct TmaMaps {
+  CUtensorMap kc, vc, ks, vs;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(1000u)
+      : "memory");
+  return done != 0;
+}
+// true once the phase with this parity has completed; false after the poll
+// limit or once *abort is set (by any thread of the CTA)
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          const volatile int *abort) {
+  if (mbar_try(bar, parity)) return true;
+  for (int i = 0; i < kWaitPolls; i++) {
+    if (mbar_try(bar, parity)) return true;
+    if (*abort) return false;
+  }
+  return false;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// d += A(16 x 16, f16, row) * B(16 x 8, f16, col) in fp32
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint4 &a, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// d = A * B + c with the accumulator input c kept intact
+__device__ __forceinline__ void mma16816c(float (&d)[4], const uint4 &a, uint32_t b0, uint32_t b1,
+                                          float c0, float c1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%11,%11};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
+}
+
+// nibbles at bits 4..7 and 20..23 of x -> half2 (64 + c) exactly
+__device__ __forceinline__ uint32_t nib64(uint32_t x) {
+  uint32_t h;
+  asm("lop3.b32 %0, %1, 0x00F000F0, 0x54005400, 0xEA;" : "=r"(h) : "r"(x));  // (x & m) | c
+  return h;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// fp32 pair -> fp16 hi + lo pairs (w ~= hi + lo to ~22 bits)
+__device__ __forceinline__ void split_hilo(float2 w, uint32_t &hi, uint32_t &lo) {
+  hi = pack_f16x2(w.x, w.y);
+  const float2 hf = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+  lo = pack_f16x2(w.x - hf.x, w.y - hf.y);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// in-register FWHT-256 of one vector held as 8 consecutive values per lane
+// (lane L: dims 8L .. 8L+7); stages h = 1, 2, ..., 128 in order, no scaling
+__device__ __forceinline__ void warp_fwht256(float (&x)[8], int lane) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+      if ((i & h) == 0) {
+        const float a = x[i], c = x[i + h];
+        x[i] = a + c;
+        x[i + h] = a - c;
+      }
+  }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = lane & m;  // this lane holds the i + h half of each pair
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const float o = __shfl_xor_sync(kFullMask, x[i], m);
+      x[i] = upper ? o - x[i] : x[i] + o;
+    }
+  }
+}
+
+
+// ---- host: 2-D tensor maps over the cache planes (cached per plane)
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// rows x row_bytes uint8 plane, boxes of box_rows rows x box_cols bytes (the
+// maps are cached per plane and box)
+inline bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t row_bytes,
+                     uint32_t box_cols, uint32_t box_rows, bool swizzle) {
+  struct Entry {
+    const void *base;
+    uint64_t rows;
+    uint32_t row_bytes, box_cols, box_rows;
+    CUtensorMap map;
+  };
+  static Entry cache[16];
+  static int next = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry &e : cache)
+    if (e.base == base && e.rows == rows && e.row_bytes == row_bytes && e.box_cols == box_cols &&
+        e.box_rows == box_rows) {
+      *m = e.map;
+      return true;
+    }
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  cache[next] = Entry{base, rows, row_bytes, box_cols, box_rows, *m};
+  next = (next + 1) % 16;
+  return true;
+}
+
+}  // namespace dec
+}  // namespace kvq

@@ -21,6 +21,7 @@ kvq_status check_cache(const kvq_cache *c) {
   if (!c || !c->k_codes || !c->k_scales || !c->v_codes || !c->v_scales) return KVQ_ERR_INVALID_ARG;
   if (c->num_kv_heads < 1 || c->head_dim <= 0) return KVQ_ERR_INVALID_ARG;
   if (c->head_dim != kDim) return KVQ_ERR_UNSUPPORTED;
+  if (c->code_bits != 0 && c->code_bits != 4 && c->code_bits != 8) return KVQ_ERR_INVALID_ARG;
   if (!aligned(c->k_codes, 16) || !aligned(c->v_codes, 16) || !aligned(c->k_scales, 16) ||
       !aligned(c->v_scales, 16))
     return KVQ_ERR_INVALID_ARG;
@@ -163,7 +164,7 @@ kvq_status kvq_quantize_append(const kvq_cache *cache, const void *k, const void
   // the kernel indexes the 2 * batch * t_new * heads vectors with 31-bit counts
   if (2LL * batch * t_new * cache->num_kv_heads >= (1LL << 31)) return KVQ_ERR_UNSUPPORTED;
   return from_cuda(launch_q4_append(*cache, k, v, dtype == KVQ_BF16, batch, t_new, d_start_pos,
-                                    as_stream(stream)));
+                                    as_stream(stream), cache->code_bits == 8 ? 8 : 4));
 }
 
 // CTAs per (sequence, split): q heads in groups of at most 8 per kv head

@@ -68,8 +68,10 @@ __device__ __forceinline__ int64_t q4_row(const kvq_cache &c, int b, int h, int 
 
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_rotate(const void *x, int bf16, float *y, int64_t n_vec, cudaStream_t s);
+// code_bits 4: Q4_0 (128-byte code rows), 8: Q8_0 (256-byte code rows)
 cudaError_t launch_q4_append(const kvq_cache &c, const void *k, const void *v, int bf16,
-                             int batch, int t_new, const int32_t *start_pos, cudaStream_t s);
+                             int batch, int t_new, const int32_t *start_pos, cudaStream_t s,
+                             int code_bits = 4);
 
 struct DecodePlan {
   int splits;       // splits per (sequence, kv head)
@@ -87,6 +89,13 @@ int q4_decode_tile_tokens();
 // q_to_seq: several queries per sequence (batch = number of queries, query b
 // reads sequence q_to_seq[b] < num_seqs with length seq_lens[b]); nullptr: b.
 cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, int batch,
+                                 int n_q_heads, const int32_t *seq_lens, int max_seq_len,
+                                 float scale, float *ws, const DecodePlan &p, cudaStream_t s,
+                                 const void *k_new = nullptr, const void *v_new = nullptr,
+                                 const int32_t *pos = nullptr, const int32_t *q_to_seq = nullptr,
+                                 int num_seqs = 0);
+// the same over a Q8_0 cache (c.code_bits == 8); p.split_tokens a multiple of 64
+cudaError_t launch_q8_decode_mma(const kvq_cache &c, const void *q, int bf16, int batch,
                                  int n_q_heads, const int32_t *seq_lens, int max_seq_len,
                                  float scale, float *ws, const DecodePlan &p, cudaStream_t s,
                                  const void *k_new = nullptr, const void *v_new = nullptr,

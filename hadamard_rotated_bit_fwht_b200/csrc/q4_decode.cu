@@ -182,8 +182,12 @@ cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int ba
                              cudaStream_t s, const void *k_new, const void *v_new,
                              const int32_t *pos, const int32_t *q_to_seq, int num_seqs) {
   if (batch == 0) return cudaSuccess;
-  cudaError_t e = launch_q4_decode_mma(c, q, bf16, batch, n_q_heads, seq_lens, max_seq_len,
-                                       scale, ws, p, s, k_new, v_new, pos, q_to_seq, num_seqs);
+  cudaError_t e =
+      c.code_bits == 8
+          ? launch_q8_decode_mma(c, q, bf16, batch, n_q_heads, seq_lens, max_seq_len, scale, ws, p,
+                                 s, k_new, v_new, pos, q_to_seq, num_seqs)
+          : launch_q4_decode_mma(c, q, bf16, batch, n_q_heads, seq_lens, max_seq_len, scale, ws, p,
+                                 s, k_new, v_new, pos, q_to_seq, num_seqs);
   if (e != cudaSuccess) return e;
   const int cap = c.block_table ? c.max_pages_per_seq * c.page_size : c.max_tokens;
   // programmatic dependent launch: scheduled while the split kernel drains,

@@ -16,7 +16,6 @@ constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kVecPerWarp = 4;
 constexpr int kVecPerCta = kWarps * kVecPerWarp;
-constexpr unsigned kFull = 0xffffffffu;
 
 // ------------------------------------------------------------------ rotate
 template <bool BF16>
@@ -59,7 +58,8 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
   return (uint32_t)(((uint64_t)n * f.m) >> f.shift);
 }
 
-template <bool BF16>
+// Q8: Q8_0 codes (256-byte code rows) instead of Q4_0 (128-byte rows)
+template <bool BF16, bool Q8>
 __global__ void __launch_bounds__(kThreads, 5)
     q4_append_kernel(kvq_cache c, const void *__restrict__ k, const void *__restrict__ v,
                      int batch, int t_new, const int32_t *__restrict__ start_pos,
@@ -101,9 +101,16 @@ __global__ void __launch_bounds__(kThreads, 5)
       fetch_raw<BF16>(vnext ? source(vn) : k, i, vnext, raw);
     }
     fwht256_warp<false>(i, buf, r);
-    QuantOut o;
-    q4_quantize_l1(r, lane, i, o);
-    uint4 bytes = gather_block_bytes(o, stage, i);
+    uint4 bytes[2];
+    uint16_t sc;
+    if (Q8) {
+      q8_quantize_l1(r, lane, i, reinterpret_cast<uint32_t *>(buf), bytes, sc);
+    } else {
+      QuantOut o;
+      q4_quantize_l1(r, lane, i, o);
+      bytes[0] = gather_block_bytes(o, stage, i);
+      sc = o.scale;
+    }
     if (valid) {
       const bool is_v = vid >= per_tensor;
       const uint32_t e = is_v ? vid - per_tensor : vid;
@@ -113,10 +120,16 @@ __global__ void __launch_bounds__(kThreads, 5)
       const int tok = (int)(bt - b * div_tnew.d);
       const int64_t row = q4_row(c, (int)b, h, __ldg(start_pos + b) + tok);
       if (row >= 0) {
-        uint8_t *codes = (is_v ? c.v_codes : c.k_codes) + row * kRowCodeBytes;
         uint16_t *scales = (is_v ? c.v_scales : c.k_scales) + row * kRowScales;
-        *reinterpret_cast<uint4 *>(codes + 16 * i) = bytes;
-        scales[i] = o.scale;
+        if (Q8) {
+          uint8_t *codes = (is_v ? c.v_codes : c.k_codes) + row * 256;
+          *reinterpret_cast<uint4 *>(codes + 32 * i) = bytes[0];
+          *reinterpret_cast<uint4 *>(codes + 32 * i + 16) = bytes[1];
+        } else {
+          uint8_t *codes = (is_v ? c.v_codes : c.k_codes) + row * kRowCodeBytes;
+          *reinterpret_cast<uint4 *>(codes + 16 * i) = bytes[0];
+        }
+        scales[i] = sc;
       }
     }
   }
@@ -148,15 +161,23 @@ cudaError_t launch_rotate(const void *x, int bf16, float *y, int64_t n_vec, cuda
 }
 
 cudaError_t launch_q4_append(const kvq_cache &c, const void *k, const void *v, int bf16,
-                             int batch, int t_new, const int32_t *start_pos, cudaStream_t s) {
+                             int batch, int t_new, const int32_t *start_pos, cudaStream_t s,
+                             int code_bits) {
   const int64_t n_vec = 2LL * batch * t_new * c.num_kv_heads;
   if (n_vec == 0) return cudaSuccess;
   const int grid = grid_for((n_vec + kVecPerCta - 1) / kVecPerCta);
   const FastDiv dh = make_fastdiv((uint32_t)c.num_kv_heads), dt = make_fastdiv((uint32_t)t_new);
-  if (bf16)
-    q4_append_kernel<true><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
-  else
-    q4_append_kernel<false><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
+  if (code_bits == 8) {
+    if (bf16)
+      q4_append_kernel<true, true><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
+    else
+      q4_append_kernel<false, true><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
+  } else {
+    if (bf16)
+      q4_append_kernel<true, false><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
+    else
+      q4_append_kernel<false, false><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
+  }
   return cudaGetLastError();
 }
 

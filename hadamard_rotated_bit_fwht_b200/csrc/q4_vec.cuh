@@ -275,6 +275,99 @@ __device__ __forceinline__ uint4 gather_block_bytes(const QuantOut &o, uint8_t *
 }
 
 
+// ------------------------------------------------------------------ Q8_0
+// Q8_0 of the 8 blocks of one vector in layout L1 (unscaled stage output
+// w = 16 z, this lane: i): amax = max |z|, d = amax / 127, id = d ? 1/d : 0,
+// code = roundf(z * id) (product rounded to fp32, halves away from zero),
+// stored as int8 with fp16(d).  As for Q4_0, the 1/16 folds exactly:
+// RN(16a / 127) = 16 RN(a / 127), RN(1 / (16 d)) = RN(1/d) / 16, and
+// w * RN(1/(16 d)) is the same real product as z * RN(1/d).
+// Lane i returns the 32 code bytes of block i (elements 0..31 in order) and
+// the fp16 bits of its scale; stage: 256 bytes of shared memory per vector.
+__device__ __forceinline__ void q8_quantize_l1(const float r[32], int lane, int i,
+                                               uint32_t *stage, uint4 (&bytes)[2],
+                                               uint16_t &scale) {
+  uint32_t key[8];  // |.| bits: non-negative floats order like unsigned ints
+#pragma unroll
+  for (int B = 0; B < 8; B++) {
+    const int r0 = 4 * (B & 1) + 8 * (B >> 1);
+    const float am = fmaxf(fmaxf(fabsf(r[r0]), fabsf(r[r0 + 1])), fmaxf(fabsf(r[r0 + 2]), fabsf(r[r0 + 3])));
+    key[B] = __float_as_uint(am);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; j++) {
+    const bool up = i & 4;
+    const uint32_t send = up ? key[j] : key[j + 4];
+    const uint32_t keep = up ? key[j + 4] : key[j];
+    key[j] = max(keep, __shfl_xor_sync(kVFull, send, 4));
+  }
+#pragma unroll
+  for (int j = 0; j < 2; j++) {
+    const bool up = i & 2;
+    const uint32_t send = up ? key[j] : key[j + 2];
+    const uint32_t keep = up ? key[j + 2] : key[j];
+    key[j] = max(keep, __shfl_xor_sync(kVFull, send, 2));
+  }
+  uint32_t kmine;
+  {
+    const bool up = i & 1;
+    const uint32_t send = up ? key[0] : key[1];
+    const uint32_t keep = up ? key[1] : key[0];
+    kmine = max(keep, __shfl_xor_sync(kVFull, send, 1));
+  }
+  const float dw = __fdiv_rn(__uint_as_float(kmine), 127.f);  // 16 d
+  const float id = (dw != 0.f) ? __frcp_rn(dw) : 0.f;         // RN(1 / (16 d))
+  scale = __half_as_ushort(__float2half_rn(__fmul_rn(dw, 0.0625f)));
+  float idb[8];
+#pragma unroll
+  for (int B = 0; B < 8; B++) idb[B] = __shfl_sync(kVFull, id, (lane & ~7) | B);
+  // lane i holds elements i, i + 8, i + 16, i + 24 of each block: one word each
+#pragma unroll
+  for (int B = 0; B < 8; B++) {
+    const int r0 = 4 * (B & 1) + 8 * (B >> 1);
+    uint32_t w = 0;
+#pragma unroll
+    for (int m = 0; m < 4; m++) {
+      const int c = (int)roundf(__fmul_rn(r[r0 + m], idb[B]));
+      w |= (uint32_t)(c & 0xFF) << (8 * m);
+    }
+    stage[B * 8 + i] = w;
+  }
+  __syncwarp();
+  // block i: word u (from lane u) holds elements u, u + 8, u + 16, u + 24
+  uint32_t wv[8];
+#pragma unroll
+  for (int u = 0; u < 8; u++) wv[u] = stage[i * 8 + u];
+  __syncwarp();
+  uint32_t ow[8];  // output word k: elements 4k .. 4k + 3
+#pragma unroll
+  for (int k = 0; k < 8; k++) {
+    const int u0 = (4 * k) & 7, m = (4 * k) >> 3;  // elements 4k + j: word u0 + j, byte m
+    // selector: result byte 0 <- byte m of the first word, byte 1 <- byte m of the second
+    const uint32_t lo = __byte_perm(wv[u0], wv[u0 + 1], 0x40 + 0x11 * m);
+    const uint32_t hi = __byte_perm(wv[u0 + 2], wv[u0 + 3], 0x40 + 0x11 * m);
+    ow[k] = __byte_perm(lo, hi, 0x5410);
+  }
+  bytes[0] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+  bytes[1] = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+}
+
+// One warp Q8_0-quantizes up to 4 vectors (as quantize_vector); lane i % 8
+// returns the 32 code bytes of block i and its fp16 scale.  buf: 64 float4 of
+// shared memory per vector.
+template <bool BF16>
+__device__ __forceinline__ void quantize_vector_q8(const void *src, bool valid, int lane,
+                                                   float4 *buf, uint4 (&bytes)[2],
+                                                   uint16_t &scale) {
+  const int i = lane & 7;
+  Raw<BF16> raw;
+  fetch_raw<BF16>(src, i, valid, raw);
+  float r[32];
+  unpack_l0<BF16>(raw, r);
+  fwht256_warp<false>(i, buf, r);
+  q8_quantize_l1(r, lane, i, reinterpret_cast<uint32_t *>(buf), bytes, scale);
+}
+
 // One warp quantizes up to 4 vectors (vector vg = lane / 8): FWHT-256 of the
 // input vector `src` (bf16 or fp32, 256 values; ignored when !valid), Q4_0 of
 // its 8 blocks.  Lane i = lane % 8 returns the 16 code bytes of block i and its

@@ -44,6 +44,7 @@ class CacheDesc(C.Structure):
         ("max_tokens", C.c_int32), ("batch_capacity", C.c_int32),
         ("block_table", C.c_void_p), ("page_size", C.c_int32),
         ("max_pages_per_seq", C.c_int32), ("num_pages", C.c_int32),
+        ("code_bits", C.c_int32),
     ]
 
 
@@ -142,32 +143,36 @@ def _cuda_contig(name, t):
 # Q4_0 + FWHT-256
 # --------------------------------------------------------------------------
 class Q4Cache:
-    """Caller-owned structure-of-arrays Q4_0 cache (layout in include/kvq.h)."""
+    """Caller-owned structure-of-arrays Q4_0 (bits=4) or Q8_0 (bits=8) cache
+    (layout in include/kvq.h)."""
 
     def __init__(self, n_rows, num_kv_heads, device, *, max_tokens=0, batch_capacity=0,
-                 block_table=None, page_size=0, num_pages=0):
+                 block_table=None, page_size=0, num_pages=0, bits=4):
+        if bits not in (4, 8):
+            raise ValueError("bits must be 4 (Q4_0) or 8 (Q8_0)")
         dev = torch.device(device)
+        self.bits = bits
         self.num_kv_heads = num_kv_heads
         self.max_tokens = max_tokens
         self.batch_capacity = batch_capacity
         self.block_table = block_table
         self.page_size = page_size
         self.num_pages = num_pages
-        self.k_codes = torch.zeros((n_rows, 128), dtype=torch.uint8, device=dev)
-        self.v_codes = torch.zeros((n_rows, 128), dtype=torch.uint8, device=dev)
+        self.k_codes = torch.zeros((n_rows, 32 * bits), dtype=torch.uint8, device=dev)
+        self.v_codes = torch.zeros((n_rows, 32 * bits), dtype=torch.uint8, device=dev)
         self.k_scales = torch.zeros((n_rows, 8), dtype=torch.int16, device=dev)
         self.v_scales = torch.zeros((n_rows, 8), dtype=torch.int16, device=dev)
 
     @classmethod
-    def contiguous(cls, batch, num_kv_heads, max_tokens, device="cuda"):
+    def contiguous(cls, batch, num_kv_heads, max_tokens, device="cuda", bits=4):
         return cls(batch * num_kv_heads * max_tokens, num_kv_heads, device,
-                   max_tokens=max_tokens, batch_capacity=batch)
+                   max_tokens=max_tokens, batch_capacity=batch, bits=bits)
 
     @classmethod
-    def paged(cls, num_pages, num_kv_heads, page_size, block_table, device="cuda"):
+    def paged(cls, num_pages, num_kv_heads, page_size, block_table, device="cuda", bits=4):
         bt = block_table.to(device=device, dtype=torch.int32).contiguous()
         return cls(num_pages * num_kv_heads * page_size, num_kv_heads, device,
-                   block_table=bt, page_size=page_size, num_pages=num_pages)
+                   block_table=bt, page_size=page_size, num_pages=num_pages, bits=bits)
 
     def with_block_table(self, block_table: torch.Tensor) -> "Q4Cache":
         """The same planes seen through another block table (e.g. one row, to
@@ -190,10 +195,10 @@ class Q4Cache:
                          self.v_codes.data_ptr(), self.v_scales.data_ptr(),
                          self.num_kv_heads, 256, self.max_tokens, self.batch_capacity,
                          None if bt is None else bt.data_ptr(), self.page_size,
-                         0 if bt is None else bt.shape[1], self.num_pages)
+                         0 if bt is None else bt.shape[1], self.num_pages, self.bits)
 
     def nbytes_per_row(self):
-        return 2 * (128 + 16)
+        return 2 * (32 * self.bits + 16)
 
 
 def rotate(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

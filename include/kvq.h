@@ -71,11 +71,15 @@ KVQ_API int kvq_version(void);
 /* Q4_0 + FWHT-256 cache                                                      */
 /* ------------------------------------------------------------------------ */
 
-/* Q4_0 cache descriptor (structure of arrays, all planes in device memory).
- * A "row" is one (sequence, kv head, token) vector of 256 values:
- *   k_codes / v_codes   row * 128 bytes: the 8 Q4_0 blocks of the rotated
- *                       vector, block b at bytes 16b..16b+15, byte j of a block
+/* Q4_0 / Q8_0 cache descriptor (structure of arrays, all planes in device
+ * memory).  A "row" is one (sequence, kv head, token) vector of 256 values,
+ * rotated by FWHT-256 and cut into 8 blocks of 32:
+ *   k_codes / v_codes   code_bits 0 or 4 (Q4_0): row * 128 bytes, block b at
+ *                       bytes 16b..16b+15, byte j of a block
  *                       = code_j | code_{j+16} << 4 (Strata PR #21, How 2);
+ *                       code_bits 8 (Q8_0, the 8-bit variant the same pages
+ *                       measure Q4_0 against): row * 256 bytes, element j of
+ *                       block b at byte 32b + j as a two's-complement int8;
  *   k_scales / v_scales row * 8 fp16 bit patterns, the scale of block b at b.
  * Row index of (sequence b, kv head h, token t):
  *   contiguous (block_table == NULL):
@@ -98,6 +102,7 @@ typedef struct {
   int32_t page_size;           /* paged: tokens per page, a multiple of 64 */
   int32_t max_pages_per_seq;   /* paged: columns of block_table */
   int32_t num_pages;           /* paged: physical pages in the planes */
+  int32_t code_bits;           /* 0 or 4: Q4_0 rows as above; 8: Q8_0 rows */
 } kvq_cache;
 
 /* kvq_rotate -- y = H x for n_vec vectors of `dim` values, H the orthonormal
@@ -111,7 +116,7 @@ typedef struct {
 KVQ_API kvq_status kvq_rotate(const void *x, kvq_dtype dtype, float *y, int64_t n_vec,
                       int32_t dim, void *stream);
 
-/* kvq_quantize_append -- rotate and Q4_0-quantize t_new new tokens of K and V
+/* kvq_quantize_append -- rotate and Q4_0- (or Q8_0-) quantize t_new new tokens of K and V
  * per sequence and store them in the cache (Strata PR #21, How 1-2 and the
  * merge note's deterministic tie-break a > amax || (a == amax && v > mval)).
  *   k, v: device, [batch][t_new][num_kv_heads][256] of `dtype`.
@@ -122,7 +127,9 @@ KVQ_API kvq_status kvq_rotate(const void *x, kvq_dtype dtype, float *y, int64_t 
  * Codes and scales are bit-identical to: fp32 FWHT-256 as in kvq_rotate, then
  * per 32-value block d = mval / -8, id = d ? 1/d : 0,
  * code = min(15, trunc(z * id + 8.5)) (product and sum rounded separately),
- * scale = fp16(d) (round to nearest even).
+ * scale = fp16(d) (round to nearest even).  Q8_0 (code_bits 8): per block
+ * amax = max |z|, d = amax / 127, id = d ? 1/d : 0, code = round(z * id)
+ * (product rounded to fp32, halves away from zero), scale = fp16(d).
  * batch must be <= batch_capacity for a contiguous cache; one call handles
  * fewer than 2^30 vectors per tensor (batch * t_new * num_kv_heads),
  * KVQ_ERR_UNSUPPORTED otherwise. */
@@ -134,11 +141,14 @@ KVQ_API kvq_status kvq_quantize_append(const kvq_cache *cache, const void *k, co
 KVQ_API size_t kvq_decode_attn_workspace(const kvq_cache *cache, int32_t batch,
                                  int32_t num_q_heads, int32_t max_seq_len);
 
-/* kvq_decode_attn -- one query token per sequence over the Q4_0 cache
- * (Strata PR #21, How 2; merge note: the per-token path rotates Q and the
- * output).  For query head h (kv head h / (num_q_heads / num_kv_heads)):
+/* kvq_decode_attn -- one query token per sequence over the Q4_0 or Q8_0
+ * cache (Strata PR #21, How 2; merge note: the per-token path rotates Q and
+ * the output).  For query head h (kv head h / (num_q_heads / num_kv_heads)):
  *   out[b][h] = H . sum_t softmax_t(scale * <H q[b][h], k_t>) v_t,
  *   t < seq_len[b], with k_t, v_t the dequantized cached rows.
+ * Over a Q8_0 cache the rotated query of each head is rounded to integers at
+ * a step of max|H q| / (127 * 2^14) (about 2^-21 of its largest element)
+ * before the integer tensor-core products with the codes.
  * Split-K flash decoding: partial (max, sum, accumulator) per split in the
  * workspace, then a log-sum-exp combine that also applies the back-rotation.
  * Both kernels are launched with programmatic stream serialization: they may

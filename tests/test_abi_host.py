@@ -89,6 +89,12 @@ def test_validation_without_launch(L):
     need = L.kvq_decode_attn_workspace(C.byref(d), 1, 8, 64)
     assert need > 0
     assert L.kvq_decode_attn(C.byref(d), p16, 1, 1, 8, p16, 64, C.c_float(0.1), p16, p16, need - 1, None) == kvq.KVQ_ERR_WORKSPACE
+    # code_bits other than 0, 4 or 8 is rejected
+    d.code_bits = 5
+    assert L.kvq_quantize_append(C.byref(d), p16, p16, 1, 1, 1, p16, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_decode_attn(C.byref(d), p16, 1, 1, 8, p16, 64, C.c_float(0.1), p16, p16, need, None) == kvq.KVQ_ERR_INVALID_ARG
+    d.code_bits = 8
+    assert L.kvq_decode_attn(C.byref(d), p16, 1, 1, 6, p16, 64, C.c_float(0.1), p16, None, 0, None) == kvq.KVQ_ERR_UNSUPPORTED
     # paged cache needs a page size that is a multiple of 64
     d2 = kvq.CacheDesc(p16, p16, p16, p16, 2, 256, 0, 0, p16, 48, 4, 8)
     assert L.kvq_quantize_append(C.byref(d2), p16, p16, 1, 1, 1, p16, None) == kvq.KVQ_ERR_INVALID_ARG
