@@ -16,7 +16,7 @@ that steps rotate through.  The other workloads are timed per call (with a
 under "workloads"; `--workload NAME` makes one of them the main line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
-                    [--workload long_decode|quantize|paged_decode|octave]
+                    [--workload long_decode|long_decode_q8|quantize|paged_decode|octave]
 """
 from __future__ import annotations
 
@@ -176,6 +176,8 @@ class LongDecode(Workload):
     kernel_name = "kvq_decode_step (q4_decode_mma_kernel with append + q4_decode_combine_kernel)"
     traffic_key = "q4_decode_long"
 
+    bits = 4
+
     def __init__(self, dev, copies=3):
         import torch
         from hadamard_rotated_bit_fwht_b200 import kvq
@@ -189,7 +191,7 @@ class LongDecode(Workload):
         self.caches = []
         zero = torch.zeros(B, dtype=torch.int32, device=dev)
         for _ in range(copies):
-            c = kvq.Q4Cache.contiguous(B, H, T, device=dev)
+            c = kvq.Q4Cache.contiguous(B, H, T, device=dev, bits=self.bits)
             kvq.quantize_append(c, kd, vd, zero)
             self.caches.append(c)
         del kd, vd
@@ -203,14 +205,17 @@ class LongDecode(Workload):
                               dtype=torch.uint8, device=dev)
         self.kvq = kvq
         # cache read once + the new token's K/V in and its codes out + q in + out
-        self.kernel_bytes = B * H * T * 288 + 2 * B * H * (512 + 144) + B * Hq * 256 * (2 + 4)
+        row = 32 * self.bits + 16  # code bytes + 8 fp16 scales per row
+        self.kernel_bytes = B * H * T * 2 * row + 2 * B * H * (512 + row) + B * Hq * 256 * (2 + 4)
         self.step_bytes = self.kernel_bytes
         self.h2d = [self.new_k, self.new_v, self.q]
         self.d2h = [self.out]
-        self.config = {"workload": "long_decode", "batch": B, "n_q_heads": Hq,
-                       "n_kv_heads": H, "head_dim": 256, "ctx": T,
+        self.config = {"workload": "long_decode" if self.bits == 4 else "long_decode_q8",
+                       "batch": B, "n_q_heads": Hq, "n_kv_heads": H, "head_dim": 256, "ctx": T,
+                       "cache": "Q4_0" if self.bits == 4 else "Q8_0",
                        "step": "kvq_decode_step: append 1 token + decode (one call)",
-                       "l2": "3 cache copies (453 MB) rotated per step, inputs > L2"}
+                       "l2": f"{copies} cache copies ({copies * B * H * T * 2 * row / 1e6:.0f} MB) "
+                             "rotated per step, inputs > L2"}
 
     def kernel_call(self, i):
         self.kvq.decode_step(self.caches[i % len(self.caches)], self.new_k, self.new_v, self.q,
@@ -219,6 +224,14 @@ class LongDecode(Workload):
     def extra(self, call_ms):
         th = self.B * self.H * self.T / call_ms * 1e3
         return {"tok_head_per_s": th, "tok_qhead_per_s": th * self.Hq / self.H}
+
+
+class LongDecodeQ8(LongDecode):
+    """The long-context decode step over a Q8_0 cache (the 8-bit variant):
+    544 bytes per token and kv head instead of 288."""
+    bits = 8
+    kernel_name = "kvq_decode_step (q8_decode_mma_kernel with append + q4_decode_combine_kernel)"
+    traffic_key = "q8_decode_long"
 
 
 class QuantizePrefill(Workload):
@@ -424,7 +437,8 @@ class OctaveDecode(Workload):
         return {"tok_head_per_s": self.B * self.ctx * self.H / call_ms * 1e3}
 
 
-WORKLOAD_CLASSES = {"long_decode": LongDecode, "quantize": QuantizePrefill,
+WORKLOAD_CLASSES = {"long_decode": LongDecode, "long_decode_q8": LongDecodeQ8,
+                    "quantize": QuantizePrefill,
                     "paged_decode": PagedDecode, "octave": OctaveDecode}
 
 

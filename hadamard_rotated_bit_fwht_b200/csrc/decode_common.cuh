@@ -21,8 +21,9 @@ constexpr unsigned kFullMask = 0xffffffffu;
 // thread of the CTA has given up
 constexpr int kWaitPolls = 1 << 20;
 
+// code planes; scale rows are contiguous and come by 1-D bulk copies
 struct TmaMaps {
-  CUtensorMap kc, vc, ks, vs;
+  CUtensorMap kc, vc;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -66,6 +67,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+// 1-D bulk copy of `bytes` bytes (a multiple of 16; both addresses 16-byte
+// aligned) onto the barrier's transaction count
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
       : "memory");
 }
 __device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {

@@ -17,11 +17,12 @@ namespace {
 constexpr int kRec = 260;  // floats per partial record: m, l, pad, pad, o[256]
 
 // Log-sum-exp combine of the splits and back-rotation; one CTA of 256 threads
-// per (sequence, q head).  Thread j owns dimension j: the split maxima and sums
-// are reduced cooperatively, then each thread issues all its loads of o_s[j]
-// (up to kBatch at a time, so a split count of up to kBatch costs one L2 round
-// trip) before accumulating.  Warp 0 applies the FWHT-256 (8 values per lane:
-// strides 1, 2, 4 in registers, 8 .. 128 across lanes) and the 1/16.
+// per (sequence, q head).  Thread j owns dimension j and issues its loads of
+// o_s[j] (up to kBatch splits at a time) first; meanwhile warp 0 reduces the
+// split maxima and sums (lane-strided, shuffles) and publishes the weights, so
+// a split count of up to kBatch costs one L2 round trip.  Warp 0 then applies
+// the FWHT-256 (8 values per lane: strides 1, 2, 4 in registers, 8 .. 128
+// across lanes) and the 1/16.
 constexpr int kMaxSplitsSmem = 1024;
 constexpr int kBatch = 48;
 
@@ -32,7 +33,7 @@ __global__ void __launch_bounds__(256, 1)
                              int max_seq_len, int cap, float *__restrict__ out) {
   __shared__ float ob[kDim];
   __shared__ float wgt[kMaxSplitsSmem];
-  __shared__ float red[16];
+  __shared__ float lsum;
   // the partial records come from the split kernel launched just before
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x, j = threadIdx.x, lane = j & 31, warp = j >> 5;
@@ -44,39 +45,37 @@ __global__ void __launch_bounds__(256, 1)
   const float *rec = ws + (int64_t)bh * splits * kRec;
   // splits past the length wrote no record
   const int ns = min(min(splits, (len + split_tokens - 1) / split_tokens), kMaxSplitsSmem);
-  // split maxima and sums (one pass: thread s < ns holds split s, more if ns > 256)
-  float M = -INFINITY;
-  for (int s = j; s < ns; s += 256) M = fmaxf(M, __ldg(rec + (int64_t)s * kRec));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  if (lane == 0) red[warp] = M;
-  __syncthreads();
-  M = red[0];
-#pragma unroll
-  for (int w = 1; w < 8; w++) M = fmaxf(M, red[w]);
-  float L = 0.f;
-  for (int s = j; s < ns; s += 256) {
-    const float ms = __ldg(rec + (int64_t)s * kRec);
-    const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M);
-    wgt[s] = f;
-    L += f * __ldg(rec + (int64_t)s * kRec + 1);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-  if (lane == 0) red[8 + warp] = L;
-  __syncthreads();
-  L = 0.f;
-#pragma unroll
-  for (int w = 0; w < 8; w++) L += red[8 + w];
-  float O = 0.f;
-  for (int s0 = 0; s0 < ns; s0 += kBatch) {
-    float v[kBatch];
+  float v[kBatch];
+  auto fetch = [&](int s0) {
     // volatile asm keeps all kBatch loads ahead of the first use
 #pragma unroll
     for (int k = 0; k < kBatch; k++) {
       const float *src = rec + (int64_t)min(s0 + k, ns - 1) * kRec + 4 + j;
       asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v[k]) : "l"(src));
     }
+  };
+  if (ns > 0) fetch(0);
+  if (warp == 0) {
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldg(rec + (int64_t)s * kRec));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+    for (int s = lane; s < ns; s += 32) {
+      const float ms = __ldg(rec + (int64_t)s * kRec);
+      const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M);
+      wgt[s] = f;
+      L += f * __ldg(rec + (int64_t)s * kRec + 1);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    if (lane == 0) lsum = L;
+  }
+  __syncthreads();
+  const float L = lsum;
+  float O = 0.f;
+  for (int s0 = 0; s0 < ns; s0 += kBatch) {
+    if (s0 > 0) fetch(s0);
 #pragma unroll
     for (int k = 0; k < kBatch; k++) {
       const float w = s0 + k < ns ? wgt[s0 + k] : 0.f;

@@ -6,13 +6,13 @@
 // S = Q_rot K^T (G x T) and O = P V (G x 256), G <= 8 heads per CTA.  One CTA
 // per SM (8 warps, ~200 KB of shared memory):
 //   * 128-token tiles of the split (codes and fp16 scales of K and V, 36 KB)
-//     stream by TMA (2-D maps over the 128-byte code rows and 16-byte scale
-//     rows, hardware 128-byte swizzle) into a ring of 5 stages, each guarded by
-//     a full mbarrier.  The first 5 tiles are issued at kernel start, before
-//     the query is prepared; afterwards the last warp to release a stage (a
-//     shared-memory counter per stage) issues its refill, so no warp is spent
-//     on producing and every warp keeps the full register budget.  Every wait
-//     is bounded.
+//     stream into a ring of 4 stages, each guarded by a full mbarrier: code
+//     rows by TMA (2-D maps over the 128-byte rows, hardware 128-byte
+//     swizzle), scale rows by 1-D bulk copies.  The first 4 tiles are issued
+//     before the query is prepared; afterwards the last warp to release a
+//     stage (a shared-memory counter per stage) issues its refill, so no warp
+//     is spent on producing and every warp keeps the full register budget.
+//     Every wait is bounded.
 //   * warp w owns tokens 16w .. 16w+15 of every tile and runs its own online
 //     softmax over them (no CTA-wide barrier per tile).  The 8 running states
 //     are merged once at the end of the split.
@@ -113,8 +113,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     prefetch_map(&maps.kc);
     prefetch_map(&maps.vc);
-    prefetch_map(&maps.ks);
-    prefetch_map(&maps.vs);
   }
   // inputs may come from the kernel launched just before this one
   grid_dependency_wait();
@@ -170,28 +168,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (page < 0 || page >= c.num_pages) return -1;
     return (int)(((int64_t)page * c.num_kv_heads + kvh) * c.page_size + (t - pi * c.page_size));
   };
-  // one thread: tile `it` (both 64-token halves that hold tokens of the split)
-  // onto its stage's full barrier
+  // one thread: tile `it` onto its stage's full barrier.  Contiguous cache:
+  // the tile's rows are consecutive, one 128-row box per code plane and one
+  // bulk copy of the scale rows of this (sequence, head) per scale plane.
+  // Paged: each 64-token half that holds tokens of the split on its own.
+  // (A tile of 8 copies with 16-byte scale boxes kept the issuing thread busy
+  // about twice as long.)
   auto issue = [&](int it) {
     const int st = it % kStages;
     const int tstart = t0 + it * kTile;
-    const int r0 = sub_row(tstart);
-    const int r1 = tstart + kSub < t1 ? sub_row(tstart + kSub) : -1;
     const uint32_t bar = full0 + 8 * st;
-    const int n = (r0 >= 0) + (r1 >= 0);
-    if (n == 0) {
-      mbar_arrive(bar);
+    const uint32_t dst = smem_u32(smem + st * kStageBytes);
+    if (c.block_table == nullptr) {
+      const int r = sub_row(tstart);
+      const int nrows = min(kTile, c.max_tokens - tstart);
+      mbar_arrive_tx(bar, 2 * kTile * 128 + 2 * nrows * 16);
+      tma_load_2d(dst + kOffKC, &maps.kc, 0, r, bar);
+      tma_load_2d(dst + kOffVC, &maps.vc, 0, r, bar);
+      bulk_load(dst + kOffKS, c.k_scales + (int64_t)r * kRowScales, nrows * 16, bar);
+      bulk_load(dst + kOffVS, c.v_scales + (int64_t)r * kRowScales, nrows * 16, bar);
     } else {
-      mbar_arrive_tx(bar, n * kSubBytes);
-      const uint32_t dst = smem_u32(smem + st * kStageBytes);
+      const int r0 = sub_row(tstart);
+      const int r1 = tstart + kSub < t1 ? sub_row(tstart + kSub) : -1;
+      const int n = (r0 >= 0) + (r1 >= 0);
+      if (n == 0) {
+        mbar_arrive(bar);
+      } else {
+        mbar_arrive_tx(bar, n * kSubBytes);
 #pragma unroll
-      for (int j = 0; j < 2; j++) {
-        const int r = j ? r1 : r0;
-        if (r < 0) continue;
-        tma_load_2d(dst + kOffKC + j * kSub * 128, &maps.kc, 0, r, bar);
-        tma_load_2d(dst + kOffVC + j * kSub * 128, &maps.vc, 0, r, bar);
-        tma_load_2d(dst + kOffKS + j * kSub * 16, &maps.ks, 0, r, bar);
-        tma_load_2d(dst + kOffVS + j * kSub * 16, &maps.vs, 0, r, bar);
+        for (int j = 0; j < 2; j++) {
+          const int r = j ? r1 : r0;
+          if (r < 0) continue;
+          tma_load_2d(dst + kOffKC + j * kSub * 128, &maps.kc, 0, r, bar);
+          tma_load_2d(dst + kOffVC + j * kSub * 128, &maps.vc, 0, r, bar);
+          bulk_load(dst + kOffKS + j * kSub * 16, c.k_scales + (int64_t)r * kRowScales, kSub * 16, bar);
+          bulk_load(dst + kOffVS + j * kSub * 16, c.v_scales + (int64_t)r * kRowScales, kSub * 16, bar);
+        }
       }
     }
     atomicMax(const_cast<int *>(issued), it + 1);
@@ -544,10 +556,9 @@ cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, in
                             : (uint64_t)c.batch_capacity * c.num_kv_heads * c.max_tokens;
   if (rows >= (1ull << 31)) return cudaErrorInvalidValue;  // TMA row coordinates are 32-bit
   TmaMaps maps;
-  if (!make_map(&maps.kc, c.k_codes, rows, 128, 128, kSub, true) ||
-      !make_map(&maps.vc, c.v_codes, rows, 128, 128, kSub, true) ||
-      !make_map(&maps.ks, c.k_scales, rows, 16, 16, kSub, false) ||
-      !make_map(&maps.vs, c.v_scales, rows, 16, 16, kSub, false))
+  const uint32_t box = c.block_table ? kSub : kTile;  // rows per code box
+  if (!make_map(&maps.kc, c.k_codes, rows, 128, 128, box, true) ||
+      !make_map(&maps.vc, c.v_codes, rows, 128, 128, box, true))
     return cudaErrorInvalidValue;
   // opt in to the large dynamic shared-memory carve-out once per device
   static std::mutex mu;

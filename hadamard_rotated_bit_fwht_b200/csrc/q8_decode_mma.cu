@@ -14,10 +14,10 @@
 //     S = 127 * 2^14 / max|q|, rounded to integers n and split exactly into
 //     int8 digits n = 2^14 H + 2^7 M + L (|M|, |L| <= 64); one MMA takes H and
 //     M (rows 0-7, 8-15), a second one L.  Both accumulators start at the bits
-//     of 1.5 * 2^23, so an exact integer block dot becomes an fp32 by one
-//     subtraction (H, M) or carries the offset into the score, which starts at
-//     -1.5 * 2^23 * sum of the token's block scales (L).  1 / (16 S) joins the
-//     softmax scale.
+//     of 1.5 * 2^23, so each exact integer block dot becomes an fp32 by one
+//     subtraction; the three are combined with their weights and the block's
+//     scale, read straight from the staged fp16 scale rows.  1 / (16 S) joins
+//     the softmax scale.
 //   * PV on the fp16 path (m16n8k16, fp32 accumulation): A = V^T codes
 //     (ldmatrix.trans) as exact fp16 values: sign bit flipped, each byte paired
 //     with the exponent byte of 1024 (1152 + c), 1152 subtracted; B = p * d_v
@@ -49,21 +49,16 @@ constexpr float kQRange = 2080768.f;  // 127 * 2^14
 constexpr uint32_t kMagicBits = 0x4B400000u;  // bits of 1.5 * 2^23
 constexpr float kMagic = 12582912.f;
 // stage: K codes as two 64-row x 128-byte boxes (dims 0-127, 128-255; 128B
-// swizzle), V codes likewise, then K and V scales (64 rows x 16 bytes)
+// swizzle), V codes likewise, then K and V scale rows (64 x 16 bytes, 1-D bulk
+// copies)
 constexpr int kBox = kTile * 128;
 constexpr int kOffKC = 0;
 constexpr int kOffVC = kOffKC + 2 * kBox;
 constexpr int kOffKS = kOffVC + 2 * kBox;
 constexpr int kOffVS = kOffKS + kTile * 16;
 constexpr int kStageBytes = kOffVS + kTile * 16;  // 34 KB
-// after the ring, per warp: K scales fp32 [block][16 pos], score starts [16],
-// V scales fp16 [block][16 pos]
-constexpr int kFsK = 8 * 16 * 4;
-constexpr int kFsB = 16 * 4;
-constexpr int kFsV = 8 * 16 * 2;
-constexpr int kFsWarp = kFsK + kFsB + kFsV;
-constexpr int kOffFs = kStages * kStageBytes;
-constexpr int kOffQ = kOffFs + kWarps * kFsWarp;   // query digits int8 [level][head][256]
+// after the ring
+constexpr int kOffQ = kStages * kStageBytes;       // query digits int8 [level][head][256]
 constexpr int kOffQS = kOffQ + 3 * 8 * 256;        // per-head 1 / (16 S), fp32 [8]
 constexpr int kOffQT = kOffQS + 128;               // query fragment table [8][32] x 32 B
 constexpr int kOffBar = kOffQT + 8 * 32 * 32;      // full[kStages]
@@ -90,6 +85,11 @@ __device__ __forceinline__ void imma16832(uint32_t (&d)[4], uint32_t a0, uint32_
       : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(kMagicBits));
 }
+
+__device__ __forceinline__ uint32_t word(const uint4 &v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+__device__ __forceinline__ __half2 as_h2(uint32_t x) { return *reinterpret_cast<const __half2 *>(&x); }
 
 __device__ __forceinline__ float2 as_f2(uint32_t a, uint32_t b) {
   return make_float2(__uint_as_float(a), __uint_as_float(b));
@@ -141,8 +141,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     prefetch_map(&maps.kc);
     prefetch_map(&maps.vc);
-    prefetch_map(&maps.ks);
-    prefetch_map(&maps.vs);
   }
   grid_dependency_wait();
   launch_dependents();
@@ -195,14 +193,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (r < 0) {
       mbar_arrive(bar);
     } else {
-      mbar_arrive_tx(bar, kStageBytes);
+      // scale rows of this (sequence, head) only: contiguous caches end each
+      // head's rows at max_tokens, pages hold whole 64-token tiles
+      const int nrows = c.block_table ? kTile : min(kTile, c.max_tokens - (t0 + it * kTile));
+      mbar_arrive_tx(bar, 4 * kBox + 2 * nrows * 16);
       const uint32_t dst = smem_u32(smem + st * kStageBytes);
       tma_load_2d(dst + kOffKC, &maps.kc, 0, r, bar);
       tma_load_2d(dst + kOffKC + kBox, &maps.kc, 128, r, bar);
       tma_load_2d(dst + kOffVC, &maps.vc, 0, r, bar);
       tma_load_2d(dst + kOffVC + kBox, &maps.vc, 128, r, bar);
-      tma_load_2d(dst + kOffKS, &maps.ks, 0, r, bar);
-      tma_load_2d(dst + kOffVS, &maps.vs, 0, r, bar);
+      bulk_load(dst + kOffKS, c.k_scales + (int64_t)r * kRowScales, nrows * 16, bar);
+      bulk_load(dst + kOffVS, c.v_scales + (int64_t)r * kRowScales, nrows * 16, bar);
     }
     atomicMax(const_cast<int *>(issued), it + 1);
   };
@@ -281,6 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     sf = sl2 * reinterpret_cast<const float *>(smem + kOffQS)[g];
   }
   __syncthreads();
+  uint4 qhm_r[8];
+#pragma unroll
+  for (int bb = 0; bb < 8; bb++) qhm_r[bb] = qtab[2 * (bb * 32 + lane)];
 
   // (2) the split: warp group gq = warp / 4 takes the tiles it with it % 2 == gq,
   // warp wi = warp % 4 tokens 16wi .. 16wi + 15 of each of them
@@ -291,10 +295,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int m = 0; m < 2; m++) o[bb][m][0] = o[bb][m][1] = o[bb][m][2] = o[bb][m][3] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;  // head g
-  uint8_t *fsw = smem + kOffFs + warp * kFsWarp;
-  float *fsk = reinterpret_cast<float *>(fsw);
-  float *fsb = reinterpret_cast<float *>(fsw + kFsK);
-  uint16_t *fsv = reinterpret_cast<uint16_t *>(fsw + kFsK + kFsB);
   // ldmatrix rows: lanes 8j .. 8j + 7 address matrix j = (token half j & 1,
   // 16-byte chunk 2bb + (j >> 1)); the chunk is swizzled by the row (128B mode)
   const int tr = 16 * wi + (lane & 7) + 8 * ((lane >> 3) & 1);
@@ -313,49 +313,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool live = nvalid > 0;
     if (live && c.block_table != nullptr) live = tile_row(ttile) >= 0;
     if (live) {
-      {  // widen the scales: lanes 0-15 K, 16-31 V (lane & 15 = token);
-         // pos 4tg + 2T + e for token 8T + 2tg + e; invalid tokens -> 0
-        const int t = lane & 15;
-        const bool is_v = lane >= 16;
-        const uint4 w = *reinterpret_cast<const uint4 *>(stage + (is_v ? kOffVS : kOffKS) +
-                                                         (16 * wi + t) * 16);
-        const int ps = 4 * ((t >> 1) & 3) + 2 * (t >> 3) + (t & 1);
-        const bool ok = t < nvalid;
-        const uint32_t ww[4] = {ok ? w.x : 0u, ok ? w.y : 0u, ok ? w.z : 0u, ok ? w.w : 0u};
-        if (is_v) {
-#pragma unroll
-          for (int k2 = 0; k2 < 4; k2++) {
-            fsv[(2 * k2) * 16 + ps] = (uint16_t)(ww[k2] & 0xffffu);
-            fsv[(2 * k2 + 1) * 16 + ps] = (uint16_t)(ww[k2] >> 16);
-          }
-        } else {
-          float sum = 0.f;
-#pragma unroll
-          for (int k2 = 0; k2 < 4; k2++) {
-            const float2 d2 = __half22float2(*reinterpret_cast<const __half2 *>(&ww[k2]));
-            fsk[(2 * k2) * 16 + ps] = d2.x;
-            fsk[(2 * k2 + 1) * 16 + ps] = d2.y;
-            sum += d2.x + d2.y;
-          }
-          fsb[ps] = -kMagic * sum;
-        }
-      }
-      __syncwarp();
+      // scale rows of tokens 2tg, 2tg + 1, 8 + 2tg, 9 + 2tg of this warp: 8 fp16
+      // each, the scale of block bb in half bb
+      const uint8_t *ksr = stage + kOffKS + (16 * wi + 2 * tg) * 16;
+      const uint4 kq0 = *reinterpret_cast<const uint4 *>(ksr);
+      const uint4 kq1 = *reinterpret_cast<const uint4 *>(ksr + 16);
+      const uint4 kq8 = *reinterpret_cast<const uint4 *>(ksr + 128);
+      const uint4 kq9 = *reinterpret_cast<const uint4 *>(ksr + 144);
       const uint32_t kbase = smem_u32(stage + kOffKC) + lrow, vbase = smem_u32(stage + kOffVC) + lrow;
 
       // ---- QK: head g, tokens 8T + 2tg + {0, 1}, T = 0, 1
-      float2 sacc[2];
-      {
-        const float4 sb = *reinterpret_cast<const float4 *>(fsb + 4 * tg);
-        sacc[0] = make_float2(sb.x, sb.y);
-        sacc[1] = make_float2(sb.z, sb.w);
-      }
+      float2 sacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int bb = 0; bb < 8; bb++) {
-        const uint4 qhm = qtab[2 * (bb * 32 + lane)], ql = qtab[2 * (bb * 32 + lane) + 1];
+        const uint4 qhm = qhm_r[bb];
+        const uint2 ql = *reinterpret_cast<const uint2 *>(qtab + 2 * (bb * 32 + lane) + 1);
         uint32_t kr[4];  // (tokens 0-7, dims 0-15 of block bb), (8-15, 0-15), (0-7, 16-31), (8-15, 16-31)
         ldsm_x4(kbase + (bb >> 2) * kBox + ((((2 * bb) & 7) << 4) ^ lz), kr);
-        const float4 dk = *reinterpret_cast<const float4 *>(fsk + bb * 16 + 4 * tg);
+        const uint32_t sel = (bb & 1) ? 0x7632u : 0x5410u;
+        const float2 dk0 = __half22float2(as_h2(__byte_perm(word(kq0, bb >> 1), word(kq1, bb >> 1), sel)));
+        const float2 dk1 = __half22float2(as_h2(__byte_perm(word(kq8, bb >> 1), word(kq9, bb >> 1), sel)));
 #pragma unroll
         for (int T = 0; T < 2; T++) {
           uint32_t a1[4], a2[4];
@@ -364,9 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 mg = make_float2(-kMagic, -kMagic);
           const float2 hH = __fadd2_rn(as_f2(a1[0], a1[1]), mg);   // 2^14-digit dot, exact
           const float2 hM = __fadd2_rn(as_f2(a1[2], a1[3]), mg);   // 2^7-digit dot, exact
-          const float2 t = __ffma2_rn(hM, make_float2(128.f, 128.f), as_f2(a2[0], a2[1]));
-          const float2 v = __ffma2_rn(hH, make_float2(16384.f, 16384.f), t);  // dot + magic
-          const float2 d = T ? make_float2(dk.z, dk.w) : make_float2(dk.x, dk.y);
+          const float2 hL = __fadd2_rn(as_f2(a2[0], a2[1]), mg);   // 1-digit dot, exact
+          const float2 t = __ffma2_rn(hM, make_float2(128.f, 128.f), hL);
+          const float2 v = __ffma2_rn(hH, make_float2(16384.f, 16384.f), t);
+          const float2 d = T ? dk1 : dk0;
           sacc[T] = __ffma2_rn(d, v, sacc[T]);
         }
       }
@@ -405,6 +383,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         split_hilo(make_float2(p0, p1), ph[T], pl[T]);
       }
       // ---- PV over the 16 tokens (one k-step)
+      const uint8_t *vsr = stage + kOffVS + (16 * wi + 2 * tg) * 16;
+      uint4 vq0 = *reinterpret_cast<const uint4 *>(vsr);
+      uint4 vq1 = *reinterpret_cast<const uint4 *>(vsr + 16);
+      uint4 vq8 = *reinterpret_cast<const uint4 *>(vsr + 128);
+      uint4 vq9 = *reinterpret_cast<const uint4 *>(vsr + 144);
+      if (nvalid < 16) {  // tokens past the end: zero scales (their rows may hold anything)
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        if (2 * tg >= nvalid) vq0 = z;
+        if (2 * tg + 1 >= nvalid) vq1 = z;
+        if (8 + 2 * tg >= nvalid) vq8 = z;
+        if (9 + 2 * tg >= nvalid) vq9 = z;
+      }
       const __half2 ph0 = *reinterpret_cast<const __half2 *>(&ph[0]);
       const __half2 ph1 = *reinterpret_cast<const __half2 *>(&ph[1]);
       const __half2 pl0 = *reinterpret_cast<const __half2 *>(&pl[0]);
@@ -413,9 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int bb = 0; bb < 8; bb++) {
         uint32_t vr[4];  // (tokens 0-7, dims 0-15), (8-15, 0-15), (0-7, 16-31), (8-15, 16-31)
         ldsm_x4_t(vbase + (bb >> 2) * kBox + ((((2 * bb) & 7) << 4) ^ lz), vr);
-        const uint2 dvp = *reinterpret_cast<const uint2 *>(fsv + bb * 16 + 4 * tg);
-        const __half2 d01 = *reinterpret_cast<const __half2 *>(&dvp.x);
-        const __half2 d89 = *reinterpret_cast<const __half2 *>(&dvp.y);
+        const uint32_t vsel = (bb & 1) ? 0x7632u : 0x5410u;
+        const __half2 d01 = as_h2(__byte_perm(word(vq0, bb >> 1), word(vq1, bb >> 1), vsel));
+        const __half2 d89 = as_h2(__byte_perm(word(vq8, bb >> 1), word(vq9, bb >> 1), vsel));
         // w = p d_v exactly as hi + lo (TwoProduct with fp16 FMA)
         const __half2 wh0 = __hmul2_rn(ph0, d01), wh1 = __hmul2_rn(ph1, d89);
         const __half2 wl0 = __hfma2(pl0, d01, __hfma2(ph0, d01, __hneg2(wh0)));
@@ -543,9 +533,7 @@ cudaError_t launch_q8_decode_mma(const kvq_cache &c, const void *q, int bf16, in
   if (rows >= (1ull << 31)) return cudaErrorInvalidValue;  // TMA row coordinates are 32-bit
   TmaMaps maps;
   if (!make_map(&maps.kc, c.k_codes, rows, kCodeRow, 128, kTile, true) ||
-      !make_map(&maps.vc, c.v_codes, rows, kCodeRow, 128, kTile, true) ||
-      !make_map(&maps.ks, c.k_scales, rows, 16, 16, kTile, false) ||
-      !make_map(&maps.vs, c.v_scales, rows, 16, 16, kTile, false))
+      !make_map(&maps.vc, c.v_codes, rows, kCodeRow, 128, kTile, true))
     return cudaErrorInvalidValue;
   static std::mutex mu;
   static unsigned configured[2] = {0u, 0u};
