@@ -9,7 +9,9 @@ nibbles, online softmax, split-K combine, back-rotation).
 
 `value` is HBM throughput in GB/s: algorithmic bytes per step (every cache
 byte read once, inputs read and outputs written once) / device time per
-step, summed over ranks.  Every workload's data is larger than the 126 MB L2;
+step, summed over ranks.  The timed steps replay CUDA graphs of the step back
+to back, as a decode loop drives it; `e2e` calls the public API eagerly with
+host copies in and out.  Every workload's data is larger than the 126 MB L2;
 the long-decode cache (151 MB) is additionally kept in three copies (453 MB)
 that steps rotate through.  The other workloads are timed per call (with a
 512 MB L2 flush before each call, outside the timed events) and reported
@@ -153,6 +155,7 @@ class Workload:
     launches_per_step = 0
     kernel_name = ""
     traffic_key = ""
+    cycle = 1  # steps rotate through this many input copies
 
     def pre(self, i):
         pass
@@ -190,6 +193,7 @@ class LongDecode(Workload):
         kd, vd = bf16_tensor(kb, dev), bf16_tensor(vb, dev)
         self.caches = []
         zero = torch.zeros(B, dtype=torch.int32, device=dev)
+        self.cycle = copies
         for _ in range(copies):
             c = kvq.Q4Cache.contiguous(B, H, T, device=dev, bits=self.bits)
             kvq.quantize_append(c, kd, vd, zero)
@@ -443,34 +447,68 @@ WORKLOAD_CLASSES = {"long_decode": LongDecode, "long_decode_q8": LongDecodeQ8,
 
 
 # ----------------------------------------------------------------- timing
+def capture_graphs(wl, fn):
+    """One CUDA graph of fn(i) per distinct step (i mod wl.cycle: the steps of
+    a workload rotate through wl.cycle cache copies), captured on a side stream
+    after one eager run of each."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graphs = []
+    with torch.cuda.stream(s):
+        for i in range(wl.cycle):
+            fn(i)
+        s.synchronize()
+        for i in range(wl.cycle):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                fn(i)
+            graphs.append(g)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return graphs
+
+
 def time_steps(wl, steps, warmup, dist=None):
-    """Device time of `steps` steps (CUDA events on the launching stream around
-    the region, barrier + synchronize on both sides) and the mean device time
-    of the dominant call inside those steps (events around each call)."""
+    """Device time of `steps` steps and the mean device time of the dominant
+    call.  Steps replay CUDA graphs of pre(i) + kernel_call(i) back to back
+    (the way a decode loop is driven), with CUDA events on the launching stream
+    around the whole region only and barrier + synchronize on both sides.  The
+    call time comes from a second pass that replays graphs of kernel_call(i)
+    alone with events around each replay."""
     import torch
     for i in range(warmup):
         wl.step(i)
+    torch.cuda.synchronize()
+    step_g = capture_graphs(wl, wl.step)
+    call_g = capture_graphs(wl, wl.kernel_call)
+    n = wl.cycle
+    for i in range(warmup):
+        step_g[i % n].replay()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     s = torch.cuda.current_stream()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(s)
     for i in range(steps):
-        wl.pre(i)
-        ev[i][0].record(s)
-        wl.kernel_call(i)
-        ev[i][1].record(s)
+        step_g[i % n].replay()
     t1.record(s)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     total_ms = t0.elapsed_time(t1)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        ev[i][0].record(s)
+        call_g[i % n].replay()
+        ev[i][1].record(s)
+    torch.cuda.synchronize()
     call_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    del step_g, call_g
     return total_ms, call_ms
 
 
@@ -693,7 +731,9 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {**info["config"], "parallelism": f"replicas x{world}"},
+            "config": {**info["config"], "parallelism": f"replicas x{world}",
+                       "timing": "steps replay CUDA graphs back to back (one per input copy); "
+                                 "e2e runs the public API eagerly"},
             "frac_of_peak": value / world / peak,
             **info["extra"],
             "roofline": {"bound": "hbm", "kernel": info["kernel"], "achieved": achieved,

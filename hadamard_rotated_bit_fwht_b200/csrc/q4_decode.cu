@@ -34,14 +34,16 @@ __global__ void __launch_bounds__(256, 1)
   __shared__ float ob[kDim];
   __shared__ float wgt[kMaxSplitsSmem];
   __shared__ float lsum;
-  // the partial records come from the split kernel launched just before
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x, j = threadIdx.x, lane = j & 31, warp = j >> 5;
   const int b = bh / n_q_heads;
+  // the lengths are inputs of the call: the split kernel releases this grid
+  // only after its own dependency wait, so they are final here
   const int bs = q_to_seq ? __ldg(q_to_seq + b) : b;
   const int len_raw =
       (bs < 0 || bs >= num_seqs) ? 0 : (pos ? __ldg(pos + b) + 1 : __ldg(seq_lens + b));
   const int len = min(max(len_raw, 0), min(max_seq_len, cap));
+  // the partial records come from the split kernel launched just before
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const float *rec = ws + (int64_t)bh * splits * kRec;
   // splits past the length wrote no record
   const int ns = min(min(splits, (len + split_tokens - 1) / split_tokens), kMaxSplitsSmem);
@@ -54,8 +56,27 @@ __global__ void __launch_bounds__(256, 1)
       asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v[k]) : "l"(src));
     }
   };
+  // warp 0 fetches the split maxima and sums (lane s: splits s and s + 32)
+  // ahead of its record loads
+  float2 r0 = make_float2(-INFINITY, 0.f), r1 = make_float2(-INFINITY, 0.f);
+  if (warp == 0 && ns <= 64) {
+    if (lane < ns) r0 = __ldg(reinterpret_cast<const float2 *>(rec + (int64_t)lane * kRec));
+    if (lane + 32 < ns) r1 = __ldg(reinterpret_cast<const float2 *>(rec + (int64_t)(lane + 32) * kRec));
+  }
   if (ns > 0) fetch(0);
-  if (warp == 0) {
+  if (warp == 0 && ns <= 64) {
+    float M = fmaxf(r0.x, r1.x);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float f0 = (M == -INFINITY || r0.x == -INFINITY) ? 0.f : exp2f(r0.x - M);
+    const float f1 = (M == -INFINITY || r1.x == -INFINITY) ? 0.f : exp2f(r1.x - M);
+    if (lane < ns) wgt[lane] = f0;
+    if (lane + 32 < ns) wgt[lane + 32] = f1;
+    float L = f0 * r0.y + f1 * r1.y;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    if (lane == 0) lsum = L;
+  } else if (warp == 0) {
     float M = -INFINITY;
     for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldg(rec + (int64_t)s * kRec));
 #pragma unroll
