@@ -72,10 +72,10 @@ constexpr int kSmemBytes = kSmemUsed + 1024;   // slack for the 1024-byte alignm
 // (head stride 264 floats spreads the 4 heads a warp writes at once over banks)
 constexpr int kMergeHead = 264;
 constexpr int kMergeWarpFloats = 16 + 8 * kMergeHead;
-constexpr int kOffMergeF = kWarps * kMergeWarpFloats * 4;  // exp2 factors [warp][8], then M, L
+constexpr int kOffMergeF = kWarps * kMergeWarpFloats * 4;  // per-warp m, l [warp][8], then M, L
 static_assert(kStages % 2 == 0, "each stage must serve one warp group");
 static_assert(kStageBytes % 1024 == 0, "stages must keep the swizzle atoms aligned");
-static_assert(kOffMergeF + (kWarps + 2) * 8 * 4 <= kStages * kStageBytes, "merge fits the ring");
+static_assert(kOffMergeF + (2 * kWarps + 2) * 8 * 4 <= kStages * kStageBytes, "merge fits the ring");
 static_assert(kOffBar % 8 == 0, "mbarrier alignment");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
@@ -476,48 +476,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
   }
-  float *mw = reinterpret_cast<float *>(smem) + warp * kMergeWarpFloats;
-  if (!abort_all) {
-    if (tg == 0) {
-      mw[g] = m_run;
-      mw[8 + g] = l_run;
-    }
-#pragma unroll
-    for (int bb = 0; bb < 8; bb++) {
-      // wsum of (head h, block bb) lives in lane 4h + bb/2, as wA (bb even) or wB (odd)
-      const float sA = __shfl_sync(kFull, (bb & 1) ? wB : wA, 8 * tg + (bb >> 1));
-      const float sB = __shfl_sync(kFull, (bb & 1) ? wB : wA, 8 * tg + 4 + (bb >> 1));
-      const float cA = kBias * sA, cB = kBias * sB;
-#pragma unroll
-      for (int m = 0; m < 2; m++) {
-        const int d0 = 32 * bb + 16 * m + 2 * g;  // row g; row g + 8 is d0 + 1
-        float *oa = mw + 16 + (2 * tg) * kMergeHead + d0;
-        float *ob = oa + kMergeHead;
-        oa[0] = o[bb][m][0] - cA;
-        ob[0] = o[bb][m][1] - cB;
-        oa[1] = o[bb][m][2] - cA;
-        ob[1] = o[bb][m][3] - cB;
-      }
-    }
+  // per-warp (m, l) of each head, then every warp scales its accumulators to
+  // the CTA maximum before storing them, so the final pass only adds
+  float *ml = reinterpret_cast<float *>(smem + kOffMergeF);  // m [warp][head], l [warp][head]
+  float *mh = ml + 2 * kWarps * 8;                            // M, L per head
+  if (!abort_all && tg == 0) {
+    ml[warp * 8 + g] = m_run;
+    ml[kWarps * 8 + warp * 8 + g] = l_run;
   }
   __syncthreads();
-  float *fac = reinterpret_cast<float *>(smem + kOffMergeF);  // [warp][head] exp2 factors
-  float *mh = fac + kWarps * 8;                                // M, L per head
-  if (!abort_all && tid < 8) {
-    const float *m0 = reinterpret_cast<const float *>(smem);
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; w++) M = fmaxf(M, m0[w * kMergeWarpFloats + tid]);
-    float L = 0.f;
+  if (!abort_all) {
+    // this thread's accumulator columns are heads 2tg and 2tg + 1
+    const int ha = 2 * tg, hb = ha + 1;
+    float Ma = -INFINITY, Mb = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kWarps; w++) {
-      const float mwv = m0[w * kMergeWarpFloats + tid];
-      const float f = mwv == -INFINITY ? 0.f : ex2(mwv - M);
-      fac[w * 8 + tid] = f;
-      L += f * m0[w * kMergeWarpFloats + 8 + tid];
+      Ma = fmaxf(Ma, ml[w * 8 + ha]);
+      Mb = fmaxf(Mb, ml[w * 8 + hb]);
     }
-    mh[tid] = M;
-    mh[8 + tid] = L;
+    const float ma = ml[warp * 8 + ha], mb = ml[warp * 8 + hb];
+    const float fa = ma == -INFINITY ? 0.f : ex2(ma - Ma);
+    const float fb = mb == -INFINITY ? 0.f : ex2(mb - Mb);
+    float *mw = reinterpret_cast<float *>(smem) + warp * kMergeWarpFloats + 16;
+#pragma unroll
+      for (int bb = 0; bb < 8; bb++) {
+        // wsum of (head h, block bb) lives in lane 4h + bb/2, as wA (bb even) or wB (odd)
+        const float sA = __shfl_sync(kFull, (bb & 1) ? wB : wA, 8 * tg + (bb >> 1));
+        const float sB = __shfl_sync(kFull, (bb & 1) ? wB : wA, 8 * tg + 4 + (bb >> 1));
+        const float cA = kBias * sA, cB = kBias * sB;
+#pragma unroll
+        for (int m = 0; m < 2; m++) {
+          const int d0 = 32 * bb + 16 * m + 2 * g;  // row g; row g + 8 is d0 + 1
+          *reinterpret_cast<float2 *>(mw + ha * kMergeHead + d0) =
+              make_float2((o[bb][m][0] - cA) * fa, (o[bb][m][2] - cA) * fa);
+          *reinterpret_cast<float2 *>(mw + hb * kMergeHead + d0) =
+              make_float2((o[bb][m][1] - cB) * fb, (o[bb][m][3] - cB) * fb);
+        }
+      }
+    if (tid < 8) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kWarps; w++) M = fmaxf(M, ml[w * 8 + tid]);
+      float L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; w++) {
+        const float mwv = ml[w * 8 + tid];
+        L += (mwv == -INFINITY ? 0.f : ex2(mwv - M)) * ml[kWarps * 8 + w * 8 + tid];
+      }
+      mh[tid] = M;
+      mh[8 + tid] = L;
+    }
   }
   __syncthreads();
   const float nan = __int_as_float(0x7fc00000);
@@ -527,8 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!abort_all) {
 #pragma unroll
       for (int w = 0; w < kWarps; w++)
-        acc += fac[w * 8 + hh] *
-               reinterpret_cast<const float *>(smem)[w * kMergeWarpFloats + 16 + hh * kMergeHead + tid];
+        acc += reinterpret_cast<const float *>(smem)[w * kMergeWarpFloats + 16 + hh * kMergeHead + tid];
     }
     rec[4 + tid] = abort_all ? nan : acc;
     if (tid == 0) {
