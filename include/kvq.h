@@ -291,9 +291,10 @@ KVQ_API kvq_status kvq_octave_codebook(int32_t bits, int8_t *lut, float *lut_mul
  * one FWHT over the head (power-of-two heads), v_bits codes.  Each scale is
  * fp16(|x|^2 / (x . LUT[c]) * LUT_ONE) (0 when that dot is not positive) with
  * LUT_ONE = 64; sums run in the fixed pairwise order v[i] + v[i + n/2],
- * halving n.  Bit-identical to that fp32 sequence.  This build implements
- * head_size 128 with v_bits 3 or 4 and non-compact K; other valid formats
- * return KVQ_ERR_UNSUPPORTED. */
+ * halving n.  Bit-identical to that fp32 sequence.  Compact K (kernel code
+ * 16 + v_bits): K x signs, one FWHT over the whole head, 3-bit codes and one
+ * scale for the head.  This build implements head_size 128 with v_bits 3 or
+ * 4, compact or not; other valid formats return KVQ_ERR_UNSUPPORTED. */
 KVQ_API kvq_status kvq_octave_quantize(const kvq_octave_fmt *fmt, const void *key,
                                const void *value, kvq_dtype dtype, int32_t num_tokens,
                                int32_t num_kv_heads, const int64_t *d_slot_mapping,
