@@ -172,6 +172,92 @@ __device__ __forceinline__ void warp_fwht256(float (&x)[8], int lane) {
 }
 
 
+// ---- work schedule shared by the split and combine kernels
+// Attended length of query row b of a decode call: the fused step attends
+// pos[b] + 1 tokens, several queries per sequence read sequence q_to_seq[b]
+// (outside [0, num_seqs): nothing), clamped to [0, min(max_seq_len, cap)].
+__device__ __forceinline__ int decode_len(int b, const int32_t *seq_lens, const int32_t *pos,
+                                          const int32_t *q_to_seq, int num_seqs, int max_seq_len,
+                                          int cap) {
+  const int bs = q_to_seq ? __ldg(q_to_seq + b) : b;
+  const int raw =
+      (bs < 0 || bs >= num_seqs) ? 0 : (pos ? __ldg(pos + b) + 1 : __ldg(seq_lens + b));
+  return min(max(raw, 0), min(max_seq_len, cap));
+}
+
+// Balanced schedule over all (query row, head group) units of a call: unit
+// u = b * n_hg + hg holds ceil(len_b / tile) tiles; the units' tiles are laid
+// end to end and CTA c of G' = min(G, T) takes tiles [c T / G', (c + 1) T / G')
+// (at least one each; CTAs c >= G' have none).  A CTA may cross unit
+// boundaries; each (unit, CTA) overlap is one segment, whose partial records
+// sit at slot u + c (u + c grows strictly along the tiles, so slots are unique
+// and below n_units + G).
+// tokens of work the fused append of the new token is counted as when the
+// stream schedule shares a unit's tiles (it costs its CTA a few microseconds)
+constexpr int kAppendTokens = 256;
+
+struct StreamLoc {
+  int total;   // T
+  int unit;    // unit holding the probed tile (-1 if none)
+  int start;   // first tile of that unit
+  int want;    // first tile of the unit asked for (0 if none asked)
+};
+// the CTA of G' owning tile t
+__device__ __forceinline__ int cta_of_tile(int t, int total, int ctas) {
+  return (int)(((int64_t)(t + 1) * ctas - 1) / total);
+}
+// Block-wide (kThreads threads, all must call): T, the unit holding tile
+// probe(T) (a functor of T, e.g. this CTA's first tile) and the first tile of
+// unit want_unit.  sm: 2 * warps + 4 ints of shared memory.
+template <int kThreads, class TilesFn, class ProbeFn>
+__device__ StreamLoc stream_locate(int n_units, TilesFn tiles, ProbeFn probe, int want_unit,
+                                   int *sm) {
+  constexpr int kW = kThreads / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (n_units + kThreads - 1) / kThreads;
+  const int u0 = min(n_units, tid * per), u1 = min(n_units, u0 + per);
+  int local = 0;
+  for (int u = u0; u < u1; u++) local += tiles(u);
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(kFullMask, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) sm[warp] = incl;
+  if (tid == 0) {
+    sm[2 * kW] = -1;
+    sm[2 * kW + 1] = 0;
+    sm[2 * kW + 2] = 0;
+  }
+  __syncthreads();
+  int base = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < kW; w++) {
+    base += w < warp ? sm[w] : 0;
+    total += sm[w];
+  }
+  const int p = probe(total);
+  int S = base + incl - local;  // first tile of unit u0
+  for (int u = u0; u < u1; u++) {
+    const int n = tiles(u);
+    if (n > 0 && S <= p && p < S + n) {
+      sm[2 * kW] = u;
+      sm[2 * kW + 1] = S;
+    }
+    if (u == want_unit) sm[2 * kW + 2] = S;
+    S += n;
+  }
+  __syncthreads();
+  StreamLoc r;
+  r.total = total;
+  r.unit = sm[2 * kW];
+  r.start = sm[2 * kW + 1];
+  r.want = sm[2 * kW + 2];
+  __syncthreads();  // sm may be reused
+  return r;
+}
+
 // ---- host: 2-D tensor maps over the cache planes (cached per plane)
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;

@@ -168,6 +168,9 @@ kvq_status kvq_quantize_append(const kvq_cache *cache, const void *k, const void
 }
 
 // CTAs per (sequence, split): q heads in groups of at most 8 per kv head
+// tokens per tile of the split kernel (the stream schedule's granule)
+static int decode_tile(const kvq_cache *c) { return c->code_bits == 8 ? 64 : 128; }
+
 static int head_groups(int num_q_heads, int num_kv_heads) {
   const int group = num_q_heads / num_kv_heads;
   return num_q_heads / (group < 8 ? (group > 0 ? group : 1) : 8);
@@ -176,7 +179,8 @@ static int head_groups(int num_q_heads, int num_kv_heads) {
 size_t kvq_decode_attn_workspace(const kvq_cache *cache, int32_t batch, int32_t num_q_heads,
                                  int32_t max_seq_len) {
   if (!cache || batch <= 0 || num_q_heads <= 0 || cache->num_kv_heads <= 0) return 0;
-  DecodePlan p = plan_decode(batch, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len);
+  DecodePlan p = plan_decode(batch, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len,
+                             decode_tile(cache));
   return decode_workspace_bytes(batch, num_q_heads, p);
 }
 
@@ -195,7 +199,8 @@ kvq_status kvq_decode_attn(const kvq_cache *cache, const void *q, kvq_dtype dtyp
   if (!isfinite(scale)) return KVQ_ERR_INVALID_ARG;
   if (batch == 0) return KVQ_OK;
   if (!q || !d_seq_lens || !out || !aligned(q, 16) || !aligned(out, 16)) return KVQ_ERR_INVALID_ARG;
-  DecodePlan p = plan_decode(batch, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len);
+  DecodePlan p = plan_decode(batch, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len,
+                             decode_tile(cache));
   const size_t need = decode_workspace_bytes(batch, num_q_heads, p);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return KVQ_ERR_WORKSPACE;
   return from_cuda(launch_q4_decode(*cache, q, dtype == KVQ_BF16, batch, num_q_heads, d_seq_lens,
@@ -221,7 +226,8 @@ kvq_status kvq_decode_attn_multi(const kvq_cache *cache, const void *q, kvq_dtyp
   if (n_q == 0) return KVQ_OK;
   if (!q || !d_q_to_seq || !d_q_lens || !out || !aligned(q, 16) || !aligned(out, 16))
     return KVQ_ERR_INVALID_ARG;
-  DecodePlan p = plan_decode(n_q, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len);
+  DecodePlan p = plan_decode(n_q, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len,
+                             decode_tile(cache));
   const size_t need = decode_workspace_bytes(n_q, num_q_heads, p);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return KVQ_ERR_WORKSPACE;
   return from_cuda(launch_q4_decode(*cache, q, dtype == KVQ_BF16, n_q, num_q_heads, d_q_lens,
@@ -247,7 +253,8 @@ kvq_status kvq_decode_step(const kvq_cache *cache, const void *k_new, const void
   if (!q || !k_new || !v_new || !d_pos || !out || !aligned(q, 16) || !aligned(k_new, 16) ||
       !aligned(v_new, 16) || !aligned(out, 16))
     return KVQ_ERR_INVALID_ARG;
-  DecodePlan p = plan_decode(batch, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len);
+  DecodePlan p = plan_decode(batch, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len,
+                             decode_tile(cache));
   const size_t need = decode_workspace_bytes(batch, num_q_heads, p);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return KVQ_ERR_WORKSPACE;
   return from_cuda(launch_q4_decode(*cache, q, dtype == KVQ_BF16, batch, num_q_heads, nullptr,

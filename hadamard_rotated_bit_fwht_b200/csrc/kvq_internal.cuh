@@ -74,14 +74,18 @@ cudaError_t launch_q4_append(const kvq_cache &c, const void *k, const void *v, i
                              int code_bits = 4);
 
 struct DecodePlan {
-  int splits;       // splits per (sequence, kv head)
-  int split_tokens; // tokens per split (multiple of 64)
+  int splits;       // split mode: splits per (query row, head group)
+  int split_tokens; // split mode: tokens per split (multiple of 64)
+  int stream;       // 1: balanced stream schedule over all units (see decode_common.cuh)
+  int ctas;         // stream mode: CTAs of the split kernel
+  int n_units;      // query rows x head groups
+  int tile;         // stream mode: tokens per tile of the split kernel
 };
 // split-K plan over `units` independent problems with `slots` resident CTAs
 DecodePlan plan_split_k(int units, int max_len, int slots, int max_splits, int granule = 64,
                         int overhead_tokens = 0);
-// n_head_groups: q heads / min(group, 8), the CTAs per sequence and split
-DecodePlan plan_decode(int batch, int n_head_groups, int max_seq_len);
+// n_head_groups: q heads / min(group, 8); tile: 128 (Q4_0) or 64 (Q8_0)
+DecodePlan plan_decode(int batch, int n_head_groups, int max_seq_len, int tile = 128);
 int q4_decode_ctas_per_sm();
 int q4_decode_tile_tokens();
 // k_new, v_new, pos: fused decode step (append one token per sequence at

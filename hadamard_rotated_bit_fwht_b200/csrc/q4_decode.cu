@@ -9,7 +9,7 @@
 // writes one partial record (m, l, o[256]) per (sequence, q head, split); the
 // combine kernel here merges the splits with a log-sum-exp and applies the
 // back-rotation H o (FWHT-256) -- once per query head, after the combine.
-#include "kvq_internal.cuh"
+#include "decode_common.cuh"
 
 namespace kvq {
 namespace {
@@ -24,35 +24,65 @@ constexpr int kRec = 260;  // floats per partial record: m, l, pad, pad, o[256]
 // the FWHT-256 (8 values per lane: strides 1, 2, 4 in registers, 8 .. 128
 // across lanes) and the 1/16.
 constexpr int kMaxSplitsSmem = 1024;
+constexpr int kMaxStreamUnits = 4096;  // units scanned by every CTA of a stream schedule
 constexpr int kBatch = 48;
 
 __global__ void __launch_bounds__(256, 1)
     q4_decode_combine_kernel(const float *__restrict__ ws, const int32_t *__restrict__ seq_lens,
                              const int32_t *__restrict__ pos, const int32_t *__restrict__ q_to_seq,
                              int num_seqs, int n_q_heads, int splits, int split_tokens,
+                             int stream, int n_hg, int n_units, int ctas, int gc, int tile,
+                             int append_tiles,
                              int max_seq_len, int cap, float *__restrict__ out) {
   __shared__ float ob[kDim];
   __shared__ float wgt[kMaxSplitsSmem];
   __shared__ float lsum;
+  __shared__ int scan[2 * 8 + 4];
   const int bh = blockIdx.x, j = threadIdx.x, lane = j & 31, warp = j >> 5;
   const int b = bh / n_q_heads;
   // the lengths are inputs of the call: the split kernel releases this grid
   // only after its own dependency wait, so they are final here
-  const int bs = q_to_seq ? __ldg(q_to_seq + b) : b;
-  const int len_raw =
-      (bs < 0 || bs >= num_seqs) ? 0 : (pos ? __ldg(pos + b) + 1 : __ldg(seq_lens + b));
-  const int len = min(max(len_raw, 0), min(max_seq_len, cap));
+  auto row_len = [&](int row) {
+    return dec::decode_len(row, seq_lens, pos, q_to_seq, num_seqs, max_seq_len, cap);
+  };
+  const int len = row_len(b);
+  // this head's partial records: rec + s * rstride, s < ns
+  const float *rec = ws;
+  int64_t rstride = kRec;
+  int ns = 0;
+  if (stream) {
+    // the segments of unit u are the CTAs its tiles fall to (slots u + c)
+    const int h = bh % n_q_heads, hg = h / gc, hh = h % gc, u = b * n_hg + hg;
+    const dec::StreamLoc L = dec::stream_locate<256>(
+        n_units,
+        [&](int uu) {
+          const int l = row_len(uu / n_hg);
+          return l > 0 ? (l + tile - 1) / tile + append_tiles : 0;
+        },
+        [](int) { return -1; }, u, scan);
+    const int n = (len + tile - 1) / tile;
+    if (n > 0) {
+      // the split kernel shares the T tiles over min(ctas, T) CTAs
+      const int ge = min(ctas, L.total);
+      const int c0 = dec::cta_of_tile(L.want, L.total, ge);
+      const int c1 = dec::cta_of_tile(L.want + n - 1, L.total, ge);
+      ns = c1 - c0 + 1;
+      rec = ws + ((int64_t)(u + c0) * gc + hh) * kRec;
+      rstride = (int64_t)gc * kRec;
+    }
+  } else {
+    rec = ws + (int64_t)bh * splits * kRec;
+    // splits past the length wrote no record
+    ns = min(min(splits, (len + split_tokens - 1) / split_tokens), kMaxSplitsSmem);
+  }
   // the partial records come from the split kernel launched just before
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const float *rec = ws + (int64_t)bh * splits * kRec;
-  // splits past the length wrote no record
-  const int ns = min(min(splits, (len + split_tokens - 1) / split_tokens), kMaxSplitsSmem);
   float v[kBatch];
   auto fetch = [&](int s0) {
     // volatile asm keeps all kBatch loads ahead of the first use
 #pragma unroll
     for (int k = 0; k < kBatch; k++) {
-      const float *src = rec + (int64_t)min(s0 + k, ns - 1) * kRec + 4 + j;
+      const float *src = rec + min(s0 + k, ns - 1) * rstride + 4 + j;
       asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v[k]) : "l"(src));
     }
   };
@@ -60,8 +90,8 @@ __global__ void __launch_bounds__(256, 1)
   // ahead of its record loads
   float2 r0 = make_float2(-INFINITY, 0.f), r1 = make_float2(-INFINITY, 0.f);
   if (warp == 0 && ns <= 64) {
-    if (lane < ns) r0 = __ldg(reinterpret_cast<const float2 *>(rec + (int64_t)lane * kRec));
-    if (lane + 32 < ns) r1 = __ldg(reinterpret_cast<const float2 *>(rec + (int64_t)(lane + 32) * kRec));
+    if (lane < ns) r0 = __ldg(reinterpret_cast<const float2 *>(rec + lane * rstride));
+    if (lane + 32 < ns) r1 = __ldg(reinterpret_cast<const float2 *>(rec + (lane + 32) * rstride));
   }
   if (ns > 0) fetch(0);
   if (warp == 0 && ns <= 64) {
@@ -78,15 +108,15 @@ __global__ void __launch_bounds__(256, 1)
     if (lane == 0) lsum = L;
   } else if (warp == 0) {
     float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldg(rec + (int64_t)s * kRec));
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldg(rec + s * rstride));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     float L = 0.f;
     for (int s = lane; s < ns; s += 32) {
-      const float ms = __ldg(rec + (int64_t)s * kRec);
+      const float ms = __ldg(rec + s * rstride);
       const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M);
       wgt[s] = f;
-      L += f * __ldg(rec + (int64_t)s * kRec + 1);
+      L += f * __ldg(rec + s * rstride + 1);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
@@ -145,7 +175,7 @@ DecodePlan plan_split_k(int units, int max_len, int slots, int max_splits, int g
   const int len = max(max_len, 1);
   const int tiles = (len + granule - 1) / granule;
   units = max(units, 1);
-  DecodePlan best;
+  DecodePlan best = {};
   const int min_tiles = max(256 / granule, 1);
   best.split_tokens = max(tiles, min_tiles) * granule;
   best.splits = 1;
@@ -170,29 +200,47 @@ DecodePlan plan_split_k(int units, int max_len, int slots, int max_splits, int g
   return best;
 }
 
-DecodePlan plan_decode(int batch, int n_head_groups, int max_seq_len) {
-  const int tile = q4_decode_tile_tokens();
-  const int units = batch * n_head_groups;
+DecodePlan plan_decode(int batch, int n_head_groups, int max_seq_len, int tile) {
+  DecodePlan p = {};
+  p.n_units = batch * n_head_groups;
+  p.tile = tile;
   const int slots = kNumSMs * q4_decode_ctas_per_sm();
-  if (units * 4 >= slots) {
-    // many independent sequences whose lengths the host does not know: fixed
-    // chunks of 16 tiles, handed out by the block scheduler in order, so short
-    // sequences leave room for long ones (chunks past a length exit at once)
-    DecodePlan p;
-    p.split_tokens = 16 * tile;
-    p.splits = max((max(max_seq_len, 1) + p.split_tokens - 1) / p.split_tokens, 1);
-    while (p.splits > kMaxSplitsSmem) {
-      p.split_tokens *= 2;
-      p.splits = (max_seq_len + p.split_tokens - 1) / p.split_tokens;
-    }
+  if (p.n_units * 4 < slots) {
+    // few long rows: one wave of equal splits (~3 tiles' worth of per-CTA work:
+    // query rotation, ring fill, final merge); as even as the stream schedule
+    // without its length scan
+    DecodePlan q = plan_split_k(p.n_units, max_seq_len, slots, kMaxSplitsSmem, 128, 3 * 128);
+    q.n_units = p.n_units;
+    q.tile = tile;
+    return q;
+  }
+  if (p.n_units <= kMaxStreamUnits) {
+    // stream schedule: every CTA takes an equal share of all units' tiles,
+    // whatever the (device-side) lengths; at most one CTA per tile
+    const int64_t tiles_max = (int64_t)p.n_units * ((max(max_seq_len, 1) + tile - 1) / tile);
+    p.stream = 1;
+    p.ctas = tiles_max < slots ? (int)(tiles_max > 0 ? tiles_max : 1) : slots;
+    p.splits = 0;
+    p.split_tokens = tile;
     return p;
   }
-  // few sequences: one wave of equal splits (~3 tiles' worth of per-CTA work:
-  // query rotation, ring fill, final merge)
-  return plan_split_k(units, max_seq_len, slots, kMaxSplitsSmem, tile, 3 * tile);
+  // very many rows: fixed chunks of 16 tiles, handed out by the block
+  // scheduler in order, so short sequences leave room for long ones (chunks
+  // past a length exit at once)
+  p.split_tokens = 16 * 128;
+  p.splits = max((max(max_seq_len, 1) + p.split_tokens - 1) / p.split_tokens, 1);
+  while (p.splits > kMaxSplitsSmem) {
+    p.split_tokens *= 2;
+    p.splits = (max_seq_len + p.split_tokens - 1) / p.split_tokens;
+  }
+  return p;
 }
 
 size_t decode_workspace_bytes(int batch, int n_q_heads, const DecodePlan &p) {
+  if (p.stream) {
+    const int gc = n_q_heads / max(p.n_units / max(batch, 1), 1);
+    return (size_t)(p.n_units + p.ctas) * gc * kRec * sizeof(float);
+  }
   return (size_t)batch * n_q_heads * p.splits * kRec * sizeof(float);
 }
 
@@ -221,9 +269,12 @@ cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int ba
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  const int n_hg = p.n_units / batch;
   e = cudaLaunchKernelEx(&cfg, q4_decode_combine_kernel, (const float *)ws, seq_lens, pos,
                          q_to_seq, q_to_seq ? num_seqs : batch, n_q_heads, p.splits,
-                         p.split_tokens, max_seq_len, cap, out);
+                         p.split_tokens, p.stream, n_hg, p.n_units, p.ctas, n_q_heads / n_hg,
+                         p.tile, p.stream && pos ? dec::kAppendTokens / p.tile : 0, max_seq_len, cap,
+                         out);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

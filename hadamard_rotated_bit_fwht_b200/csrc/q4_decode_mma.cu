@@ -81,19 +81,20 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 using namespace dec;
 
-template <bool BF16>
+// STREAM: the balanced schedule over all units (gridDim.x CTAs) instead of
+// one split per CTA (a separate instance, so the split path keeps its code)
+template <bool BF16, bool STREAM>
 __global__ void __launch_bounds__(kThreads, 1)
     q4_decode_mma_kernel(const __grid_constant__ TmaMaps maps, kvq_cache c,
                          const void *__restrict__ q, const int32_t *__restrict__ seq_lens,
                          int max_seq_len, int n_q_heads, int group, int gc, float sl2,
-                         int split_tokens, int splits, float *__restrict__ ws,
+                         int split_tokens, int splits, int n_hg, int n_units,
+                         int append_tiles, float *__restrict__ ws,
                          const void *__restrict__ k_new, const void *__restrict__ v_new,
                          const int32_t *__restrict__ pos, const int32_t *__restrict__ q_to_seq,
                          int num_seqs) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  const int s = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-  const int h0 = hg * gc, kvh = h0 / group;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tg = lane & 3;
   const uint32_t full0 = smem_u32(smem + kOffBar);
@@ -102,447 +103,520 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *issued = abort_flag + 1;  // tiles issued so far (in order)
 
   if (tid == 0) {
-#pragma unroll
-    for (int i = 0; i < kStages; i++) {
-      mbar_init(full0 + 8 * i, 1);
-      rel[i] = 0;
-    }
-    *abort_flag = 0;
-    *issued = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     prefetch_map(&maps.kc);
     prefetch_map(&maps.vc);
   }
   // inputs may come from the kernel launched just before this one
   grid_dependency_wait();
   launch_dependents();
-  // start the global loads (sequence length; warp w: query head h0 + w, dims
-  // 8 lane .. 8 lane + 7) before the barrier
-  // fused decode step (pos != nullptr): the new token goes to position pos[b]
-  // and the sequence then has pos[b] + 1 tokens
-  const int p_new = pos ? __ldg(pos + b) : -1;
-  // several queries per sequence (q_to_seq != nullptr): query b reads the cache
-  // of sequence bs; a sequence index outside [0, num_seqs) attends to nothing
-  const int bs = q_to_seq ? __ldg(q_to_seq + b) : b;
-  const int len_raw = (bs < 0 || bs >= num_seqs) ? 0 : (pos ? p_new + 1 : __ldg(seq_lens + b));
-  float x[8];
-  if (warp < gc) {
-    const int64_t off = ((int64_t)b * n_q_heads + h0 + warp) * kDim + 8 * lane;
-    if (BF16) {
-      const uint4 r = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(q) + off));
-      const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-      for (int i = 0; i < 4; i++) {
-        x[2 * i] = bf16lo(rr[i]);
-        x[2 * i + 1] = bf16hi(rr[i]);
-      }
-    } else {
-      const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(q) + off);
-      const float4 u = __ldg(p), v = __ldg(p + 1);
-      x[0] = u.x, x[1] = u.y, x[2] = u.z, x[3] = u.w;
-      x[4] = v.x, x[5] = v.y, x[6] = v.z, x[7] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; i++) x[i] = 0.f;
-  }
-  __syncthreads();
-
   const int cap = c.block_table ? c.max_pages_per_seq * c.page_size : c.max_tokens;
-  const int len = min(max(len_raw, 0), min(max_seq_len, cap));
-  const int t0 = s * split_tokens;
-  const int t1 = min(len, t0 + split_tokens);
-  const int ntiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
-  if (ntiles == 0) return;  // a split past the length writes no record
-  // fused step: every CTA whose split holds the new token quantizes the
-  // token's K and V rows of its kv head into the cache before it issues a tile
-  // load (CTAs of the same kv head write identical bytes)
-  const bool appender = p_new >= t0 && p_new < t1;
-
-  // first cache row of the 64-token sub-tile starting at token t, -1 if unmapped
-  auto sub_row = [&](int t) -> int {
-    if (c.block_table == nullptr) return (int)(((int64_t)bs * c.num_kv_heads + kvh) * c.max_tokens + t);
-    const int pi = t / c.page_size;
-    const int page = __ldg(c.block_table + (int64_t)bs * c.max_pages_per_seq + pi);
-    if (page < 0 || page >= c.num_pages) return -1;
-    return (int)(((int64_t)page * c.num_kv_heads + kvh) * c.page_size + (t - pi * c.page_size));
+  auto row_len = [&](int row) {
+    return decode_len(row, seq_lens, pos, q_to_seq, num_seqs, max_seq_len, cap);
   };
-  // one thread: tile `it` onto its stage's full barrier.  Contiguous cache:
-  // the tile's rows are consecutive, one 128-row box per code plane and one
-  // bulk copy of the scale rows of this (sequence, head) per scale plane.
-  // Paged: each 64-token half that holds tokens of the split on its own.
-  // (A tile of 8 copies with 16-byte scale boxes kept the issuing thread busy
-  // about twice as long.)
-  auto issue = [&](int it) {
-    const int st = it % kStages;
-    const int tstart = t0 + it * kTile;
-    const uint32_t bar = full0 + 8 * st;
-    const uint32_t dst = smem_u32(smem + st * kStageBytes);
-    if (c.block_table == nullptr) {
-      const int r = sub_row(tstart);
-      const int nrows = min(kTile, c.max_tokens - tstart);
-      mbar_arrive_tx(bar, 2 * kTile * 128 + 2 * nrows * 16);
-      tma_load_2d(dst + kOffKC, &maps.kc, 0, r, bar);
-      tma_load_2d(dst + kOffVC, &maps.vc, 0, r, bar);
-      bulk_load(dst + kOffKS, c.k_scales + (int64_t)r * kRowScales, nrows * 16, bar);
-      bulk_load(dst + kOffVS, c.v_scales + (int64_t)r * kRowScales, nrows * 16, bar);
+  // a unit's tiles, plus append_tiles that stand for the fused append of the
+  // new token (the schedule gives the CTA holding it correspondingly fewer
+  // real tiles; tiles past the length hold no work)
+  auto unit_tiles = [&](int u) {
+    const int l = row_len(u / n_hg);
+    return l > 0 ? (l + kTile - 1) / kTile + append_tiles : 0;
+  };
+  // this CTA's segments: stream mode walks the (query row, head group) units
+  // its share of the concatenated tiles crosses; split mode has the one split
+  // (blockIdx.x of row blockIdx.z, head group blockIdx.y)
+  int seg_unit = -1, seg_start = 0, t_cur = 0, t_end = 0;
+  if constexpr (STREAM) {
+    // min(CTAs, T) CTAs share the tiles, so every one of them owns at least one
+    auto share = [&](int c, int total) {
+      return (int)((int64_t)c * total / min((int)gridDim.x, total));
+    };
+    const StreamLoc L = stream_locate<kThreads>(
+        n_units, unit_tiles,
+        [&](int total) { return (int)blockIdx.x < min((int)gridDim.x, total) ? share(blockIdx.x, total) : -1; },
+        -1, reinterpret_cast<int *>(smem));
+    if ((int)blockIdx.x < min((int)gridDim.x, L.total)) {
+      t_cur = share(blockIdx.x, L.total);
+      t_end = share(blockIdx.x + 1, L.total);
+      seg_unit = L.unit;
+      seg_start = L.start;
+    }
+  }
+  const float nan = __int_as_float(0x7fc00000);
+  bool dead = false;  // a load never arrived: the remaining segments write NaN
+  for (int seg = 0; STREAM || seg < 1; seg++) {
+    int b, hg, t0, t1;
+    int64_t rec_base, rec_hstride;  // record of head h0 + hh: ws + (rec_base + hh * rec_hstride) * kRec
+    if constexpr (STREAM) {
+      if (seg_unit < 0 || seg_unit >= n_units || t_cur >= t_end) break;
+      int n = unit_tiles(seg_unit);
+      while (n == 0 && seg_unit + 1 < n_units) n = unit_tiles(++seg_unit);  // units without tiles hold none of the range
+      if (n == 0) break;
+      b = seg_unit / n_hg;
+      hg = seg_unit % n_hg;
+      const int hi = min(t_end, seg_start + n) - seg_start;
+      t0 = (t_cur - seg_start) * kTile;
+      t1 = min(row_len(b), hi * kTile);
+      rec_base = ((int64_t)seg_unit + blockIdx.x) * gc;
+      rec_hstride = 1;
+      t_cur = seg_start + hi;
+      seg_start += n;
+      seg_unit++;
     } else {
-      const int r0 = sub_row(tstart);
-      const int r1 = tstart + kSub < t1 ? sub_row(tstart + kSub) : -1;
-      const int n = (r0 >= 0) + (r1 >= 0);
-      if (n == 0) {
-        mbar_arrive(bar);
+      b = blockIdx.z;
+      hg = blockIdx.y;
+      t0 = blockIdx.x * split_tokens;
+      t1 = min(row_len(b), t0 + split_tokens);
+      rec_base = ((int64_t)b * n_q_heads + hg * gc) * splits + blockIdx.x;
+      rec_hstride = splits;
+    }
+    const int h0 = hg * gc, kvh = h0 / group;
+    // this segment's global inputs first: their latency overlaps the sizing
+    // and the barrier set-up below
+    // fused decode step (pos != nullptr): the new token goes to position pos[b]
+    // and the sequence then has pos[b] + 1 tokens
+    const int p_new = pos ? __ldg(pos + b) : -1;
+    // several queries per sequence (q_to_seq != nullptr): query b reads the cache
+    // of sequence bs
+    const int bs = q_to_seq ? __ldg(q_to_seq + b) : b;
+    float x[8];  // warp w: query head h0 + w, dims 8 lane .. 8 lane + 7
+    if (warp < gc) {
+      const int64_t off = ((int64_t)b * n_q_heads + h0 + warp) * kDim + 8 * lane;
+      if (BF16) {
+        const uint4 r = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(q) + off));
+        const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
+        #pragma unroll
+        for (int i = 0; i < 4; i++) {
+          x[2 * i] = bf16lo(rr[i]);
+          x[2 * i + 1] = bf16hi(rr[i]);
+        }
       } else {
-        mbar_arrive_tx(bar, n * kSubBytes);
-#pragma unroll
-        for (int j = 0; j < 2; j++) {
-          const int r = j ? r1 : r0;
-          if (r < 0) continue;
-          tma_load_2d(dst + kOffKC + j * kSub * 128, &maps.kc, 0, r, bar);
-          tma_load_2d(dst + kOffVC + j * kSub * 128, &maps.vc, 0, r, bar);
-          bulk_load(dst + kOffKS + j * kSub * 16, c.k_scales + (int64_t)r * kRowScales, kSub * 16, bar);
-          bulk_load(dst + kOffVS + j * kSub * 16, c.v_scales + (int64_t)r * kRowScales, kSub * 16, bar);
-        }
+        const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(q) + off);
+        const float4 u = __ldg(p), v = __ldg(p + 1);
+        x[0] = u.x, x[1] = u.y, x[2] = u.z, x[3] = u.w;
+        x[4] = v.x, x[5] = v.y, x[6] = v.z, x[7] = v.w;
       }
+    } else {
+      #pragma unroll
+      for (int i = 0; i < 8; i++) x[i] = 0.f;
     }
-    atomicMax(const_cast<int *>(issued), it + 1);
-  };
-  if (appender) {
-    if (warp == 0) {
-      const int vg = lane >> 3, i = lane & 7;
-      const bool valid = vg < 2;  // lanes 0-7: K, 8-15: V
-      const void *src =
-          static_cast<const char *>(vg == 1 ? v_new : k_new) +
-          ((int64_t)b * c.num_kv_heads + kvh) * kDim * (BF16 ? 2 : 4);
-      uint4 bytes;
-      uint16_t sc;
-      q4v::quantize_vector<BF16>(valid ? src : k_new, valid, lane,
-                                 reinterpret_cast<float4 *>(smem) + 64 * vg, bytes, sc);
-      const int64_t row = q4_row(c, b, kvh, p_new);
-      if (valid && row >= 0) {
-        *reinterpret_cast<uint4 *>((vg ? c.v_codes : c.k_codes) + row * kRowCodeBytes + 16 * i) =
-            bytes;
-        (vg ? c.v_scales : c.k_scales)[row * kRowScales + i] = sc;
+    const int ntiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
+    if (ntiles == 0) continue;  // a split past the length writes no record
+    if (dead) {
+      for (int hh = 0; hh < gc; hh++) {
+        float *rec = ws + (rec_base + hh * rec_hstride) * kRec;
+        rec[4 + tid] = nan;
+        if (tid == 0) rec[0] = rec[1] = nan;
       }
-      // the rows are read back by TMA (async proxy), which also overwrites the
-      // shared-memory buffers the quantizer used
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0)
-        for (int it = 0; it < kStages && it < ntiles; it++) issue(it);
+      continue;
     }
-  } else if (lane == 0 && warp < kStages && warp < ntiles) {
-    issue(warp);
-  }
-
-  // (1) query: warp w rotates head h0 + w (zeros past gc), splits it into
-  // fp16 hi + lo and writes the MMA fragments of its 8 blocks x 2 k-steps
-  {
-    warp_fwht256(x, lane);
-    float hi[8], lo[8], sq = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-      const float v = x[i] * 0.0625f;  // the FWHT's 1/16 (exact)
-      hi[i] = __half2float(__float2half_rn(v));
-      lo[i] = __half2float(__float2half_rn(v - hi[i]));
-      sq += hi[i] + lo[i];
-    }
-    // lane L holds dims 8L..8L+7 = block L/4, k-step (L/2)&1, tg 2(L&1) and 2(L&1)+1
-    uint4 *qf = reinterpret_cast<uint4 *>(smem + kOffQF) + (warp * 8 + (lane >> 2)) * 8 +
-                ((lane >> 1) & 1) * 4 + 2 * (lane & 1);
-#pragma unroll
-    for (int e = 0; e < 2; e++) {
-      const int i = 4 * e;
-      qf[e] = make_uint4(pack_f16x2(hi[i], hi[i + 2]), pack_f16x2(lo[i], lo[i + 2]),
-                         pack_f16x2(hi[i + 1], hi[i + 3]), pack_f16x2(lo[i + 1], lo[i + 3]));
-    }
-    sq += __shfl_xor_sync(kFull, sq, 1);
-    sq += __shfl_xor_sync(kFull, sq, 2);
-    if ((lane & 3) == 0)
-      reinterpret_cast<float *>(smem + kOffQB)[warp * 8 + (lane >> 2)] = -kBias * sq;
-  }
-  __syncthreads();
-  uint4 qa[8][2];
-  float cb[8];  // accumulator start of the hi rows: -72 * sum over the block of (hi + lo)
-  {
-    const uint4 *qf = reinterpret_cast<const uint4 *>(smem + kOffQF) + g * 64 + tg;
-#pragma unroll
-    for (int bb = 0; bb < 8; bb++) {
-      qa[bb][0] = qf[bb * 8];
-      qa[bb][1] = qf[bb * 8 + 4];
-      cb[bb] = reinterpret_cast<const float *>(smem + kOffQB)[g * 8 + bb];
-    }
-  }
-
-  // (2) the split: warp group gq = warp / 4 takes the tiles it with it % 2 == gq,
-  // warp wi = warp % 4 tokens 32wi .. 32wi + 31 of each of them
-  const int gq = warp >> 2, wi = warp & 3;
-  float o[8][2][4];  // [block][M-tile X (dims 2g, 2g+1) / Y (16 + 2g, 17 + 2g)][reg]
-#pragma unroll
-  for (int bb = 0; bb < 8; bb++)
-#pragma unroll
-    for (int m = 0; m < 2; m++) o[bb][m][0] = o[bb][m][1] = o[bb][m][2] = o[bb][m][3] = 0.f;
-  float wacc[4] = {0.f, 0.f, 0.f, 0.f};  // sum_t p d_v: head g (hi, lo rows) x blocks 2tg, 2tg+1
-  float m_run = -INFINITY, l_run = 0.f;  // head g
-  float *fsk = reinterpret_cast<float *>(smem + kOffFs + warp * (kFsK + kFsV));
-  __half *fsv = reinterpret_cast<__half *>(smem + kOffFs + warp * (kFsK + kFsV) + kFsK);
-  const int row_l = 32 * wi + 8 * ((lane >> 3) & 1) + (lane & 7);  // ldmatrix row (T = 0/1)
-  const int blk_l = lane >> 4;
-
-  for (int it = gq; it < ntiles; it += 2) {
-    const int st = it % kStages;
-    if (!mbar_wait(full0 + 8 * st, (it / kStages) & 1, abort_flag)) {
-      *abort_flag = 1;
-      break;
-    }
-    const uint8_t *stage = smem + st * kStageBytes;
-    const int tw = t0 + it * kTile + 32 * wi;  // first token of this warp
-    const int nvalid = min(32, t1 - tw);
-    bool live = nvalid > 0;
-    if (live && c.block_table != nullptr) live = sub_row(tw & ~(kSub - 1)) >= 0;
-    if (live) {
-      {  // widen: lane = token; K scales -> fp32, V scales fp16, [block][pos]; invalid -> 0
-        const int t = lane;
-        const uint4 wk = *reinterpret_cast<const uint4 *>(stage + kOffKS + (32 * wi + t) * 16);
-        const uint4 wv = *reinterpret_cast<const uint4 *>(stage + kOffVS + (32 * wi + t) * 16);
-        // pos: 16 * (T >> 1) + 4 * tg + 2 * (T & 1) + e for t = 8T + 2tg + e
-        const int T = t >> 3, tg2 = (t >> 1) & 3, e = t & 1;
-        const int pos = 16 * (T >> 1) + 4 * tg2 + 2 * (T & 1) + e;
-        const bool ok = t < nvalid;
-        const uint32_t kk[4] = {wk.x, wk.y, wk.z, wk.w}, vv[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-        for (int k2 = 0; k2 < 4; k2++) {
-          const float2 pk2 = __half22float2(*reinterpret_cast<const __half2 *>(&kk[k2]));
-          fsk[(2 * k2) * 32 + pos] = ok ? pk2.x : 0.f;
-          fsk[(2 * k2 + 1) * 32 + pos] = ok ? pk2.y : 0.f;
-          const uint32_t v2 = ok ? vv[k2] : 0u;
-          reinterpret_cast<uint16_t *>(fsv)[(2 * k2) * 32 + pos] = (uint16_t)(v2 & 0xffffu);
-          reinterpret_cast<uint16_t *>(fsv)[(2 * k2 + 1) * 32 + pos] = (uint16_t)(v2 >> 16);
-        }
-      }
-      __syncwarp();
-      const uint32_t kbase = smem_u32(stage + kOffKC), vbase = smem_u32(stage + kOffVC);
-
-      // ---- QK: head g, tokens 8T + 2tg + {0, 1}, T = 0..3
-      float2 sacc[4];
-#pragma unroll
-      for (int T = 0; T < 4; T++) sacc[T] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int bp = 0; bp < 4; bp++) {
-#pragma unroll
-        for (int tp = 0; tp < 2; tp++) {  // token groups 2tp, 2tp + 1
-          uint32_t kr[4];  // (T0, block 2bp), (T1, 2bp), (T0, 2bp + 1), (T1, 2bp + 1)
-          ldsm_x4(kbase + (row_l + 16 * tp) * 128 + (((2 * bp + blk_l) ^ (lane & 7)) << 4), kr);
-#pragma unroll
-          for (int half = 0; half < 2; half++) {
-            const int bb = 2 * bp + half;
-            const float4 dk = *reinterpret_cast<const float4 *>(fsk + bb * 32 + 16 * tp + 4 * tg);
-#pragma unroll
-            for (int T = 0; T < 2; T++) {
-              const uint32_t w = kr[2 * half + T];
-              float acc[4];
-              mma16816c(acc, qa[bb][0], nib64(w << 4), nib64(w >> 4), cb[bb], 0.f);
-              mma16816(acc, qa[bb][1], nib64(w), nib64(w >> 8));
-              const float2 d = T ? make_float2(dk.z, dk.w) : make_float2(dk.x, dk.y);
-              sacc[2 * tp + T] = __ffma2_rn(
-                  d, __fadd2_rn(make_float2(acc[0], acc[1]), make_float2(acc[2], acc[3])), sacc[2 * tp + T]);
-            }
-          }
-        }
-      }
-      // ---- online softmax of head g over this warp's 32 tokens
-      float x[8];
-#pragma unroll
-      for (int T = 0; T < 4; T++) {
-        x[2 * T] = sacc[T].x * sl2;
-        x[2 * T + 1] = sacc[T].y * sl2;
-      }
-      if (nvalid < 32) {
-#pragma unroll
-        for (int e2 = 0; e2 < 8; e2++)
-          if (8 * (e2 >> 1) + 2 * tg + (e2 & 1) >= nvalid) x[e2] = -INFINITY;
-      }
-      float mx = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-      if (__any_sync(kFull, mx > m_run)) {
-        const float mn = fmaxf(m_run, mx);
-        const float alpha = mn == m_run ? 1.f : ex2(m_run - mn);
-        m_run = mn;
-        l_run *= alpha;
-#pragma unroll
-        for (int k = 0; k < 4; k++) wacc[k] *= alpha;  // rows of head g
-        const float a0 = __shfl_sync(kFull, alpha, 8 * tg);
-        const float a1 = __shfl_sync(kFull, alpha, 8 * tg + 4);
-#pragma unroll
-        for (int bb = 0; bb < 8; bb++)
-#pragma unroll
-          for (int m = 0; m < 2; m++) {
-            o[bb][m][0] *= a0;
-            o[bb][m][1] *= a1;
-            o[bb][m][2] *= a0;
-            o[bb][m][3] *= a1;
-          }
-      }
-      uint32_t ph[4], pl[4];  // p of head g as fp16 hi + lo pairs, token groups T
-#pragma unroll
-      for (int T = 0; T < 4; T++) {
-        const float p0 = ex2(x[2 * T] - m_run), p1 = ex2(x[2 * T + 1] - m_run);
-        l_run += p0 + p1;
-        split_hilo(make_float2(p0, p1), ph[T], pl[T]);
-      }
-      // ---- PV: k-steps of 16 tokens (token groups 2ks, 2ks + 1)
-#pragma unroll
-      for (int ks = 0; ks < 2; ks++) {
-        {  // sum_t p d_v for blocks 2tg, 2tg+1 on the tensor cores (d_v exact in fp16)
-          const uint2 dvb = *reinterpret_cast<const uint2 *>(fsv + g * 32 + 16 * ks + 4 * tg);
-          const uint32_t a[4] = {ph[2 * ks], pl[2 * ks], ph[2 * ks + 1], pl[2 * ks + 1]};
-          mma16816(wacc, a, dvb.x, dvb.y);
-        }
-#pragma unroll
-        for (int bp = 0; bp < 4; bp++) {
-          uint32_t vr[4];  // (tokens 0-7, block 2bp), (8-15, 2bp), (0-7, 2bp + 1), (8-15, 2bp + 1)
-          ldsm_x4_t(vbase + (row_l + 16 * ks) * 128 + (((2 * bp + blk_l) ^ (lane & 7)) << 4), vr);
-#pragma unroll
-          for (int half = 0; half < 2; half++) {
-            const int bb = 2 * bp + half;
-            const uint2 dvp = *reinterpret_cast<const uint2 *>(fsv + bb * 32 + 16 * ks + 4 * tg);
-            const __half2 d01 = *reinterpret_cast<const __half2 *>(&dvp.x);
-            const __half2 d89 = *reinterpret_cast<const __half2 *>(&dvp.y);
-            // w = p d_v exactly as hi + lo (TwoProduct with fp16 FMA)
-            const __half2 ph0 = *reinterpret_cast<const __half2 *>(&ph[2 * ks]);
-            const __half2 ph1 = *reinterpret_cast<const __half2 *>(&ph[2 * ks + 1]);
-            const __half2 pl0 = *reinterpret_cast<const __half2 *>(&pl[2 * ks]);
-            const __half2 pl1 = *reinterpret_cast<const __half2 *>(&pl[2 * ks + 1]);
-            const __half2 wh0 = __hmul2_rn(ph0, d01), wh1 = __hmul2_rn(ph1, d89);
-            const __half2 wl0 = __hfma2(pl0, d01, __hfma2(ph0, d01, __hneg2(wh0)));
-            const __half2 wl1 = __hfma2(pl1, d89, __hfma2(ph1, d89, __hneg2(wh1)));
-            const uint32_t bh0 = *reinterpret_cast<const uint32_t *>(&wh0);
-            const uint32_t bh1 = *reinterpret_cast<const uint32_t *>(&wh1);
-            const uint32_t bl0 = *reinterpret_cast<const uint32_t *>(&wl0);
-            const uint32_t bl1 = *reinterpret_cast<const uint32_t *>(&wl1);
-            const uint32_t r0 = vr[2 * half], r1 = vr[2 * half + 1];
-            {
-              const uint32_t a[4] = {nib64(r0 << 4), nib64(r0 >> 4), nib64(r1 << 4), nib64(r1 >> 4)};
-              mma16816(o[bb][0], a, bh0, bh1);
-              mma16816(o[bb][0], a, bl0, bl1);
-            }
-            {
-              const uint32_t a[4] = {nib64(r0), nib64(r0 >> 8), nib64(r1), nib64(r1 >> 8)};
-              mma16816(o[bb][1], a, bh0, bh1);
-              mma16816(o[bb][1], a, bl0, bl1);
-            }
-          }
-        }
-      }
-    }
-    // release the stage; the last of its 4 warps refills it with tile it + kStages
-    // (same warp group: kStages is even)
-    __syncwarp();
-    if (lane == 0) {
-      int old;
-      asm volatile("atom.release.cta.shared::cta.add.s32 %0, [%1], 1;"
-                   : "=r"(old)
-                   : "r"(smem_u32(rel + st))
-                   : "memory");
-      if (old == 3) {
-        asm volatile("fence.acq_rel.cta;" ::: "memory");
-        rel[st] = 0;
-        if (it + kStages < ntiles && !*abort_flag) {
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          issue(it + kStages);
-        }
-      }
-    }
-  }
-
-  // (3) merge the 8 warps' states into this split's records
-  l_run += __shfl_xor_sync(kFull, l_run, 1);
-  l_run += __shfl_xor_sync(kFull, l_run, 2);
-  // wacc: head g, blocks 2tg (hi + lo rows: [0] + [2]) and 2tg + 1 ([1] + [3])
-  const float wA = wacc[0] + wacc[2], wB = wacc[1] + wacc[3];
-  __syncthreads();  // every warp is done with the ring
-  const bool abort_all = *abort_flag != 0;
-  if (abort_all) {
-    // a load never arrived: let every load still in flight land (bounded,
-    // ignoring the flag) before the CTA's shared memory goes away
+    // the previous segment is done with shared memory; its generic writes
+    // (the merge) precede the copies that will overwrite the ring
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
     if (tid == 0) {
-      const int n = *issued;
-      for (int it = n > kStages ? n - kStages : 0; it < n; it++)
-        for (int i = 0; i < kWaitPolls && !mbar_try(full0 + 8 * (it % kStages), (it / kStages) & 1); i++) {
-        }
+      #pragma unroll
+      for (int i = 0; i < kStages; i++) {
+        if (seg > 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(full0 + 8 * i) : "memory");
+        mbar_init(full0 + 8 * i, 1);
+        rel[i] = 0;
+      }
+      *abort_flag = 0;
+      *issued = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     __syncthreads();
-  }
-  // per-warp (m, l) of each head, then every warp scales its accumulators to
-  // the CTA maximum before storing them, so the final pass only adds
-  float *ml = reinterpret_cast<float *>(smem + kOffMergeF);  // m [warp][head], l [warp][head]
-  float *mh = ml + 2 * kWarps * 8;                            // M, L per head
-  if (!abort_all && tg == 0) {
-    ml[warp * 8 + g] = m_run;
-    ml[kWarps * 8 + warp * 8 + g] = l_run;
-  }
-  __syncthreads();
-  if (!abort_all) {
-    // this thread's accumulator columns are heads 2tg and 2tg + 1
-    const int ha = 2 * tg, hb = ha + 1;
-    float Ma = -INFINITY, Mb = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; w++) {
-      Ma = fmaxf(Ma, ml[w * 8 + ha]);
-      Mb = fmaxf(Mb, ml[w * 8 + hb]);
-    }
-    const float ma = ml[warp * 8 + ha], mb = ml[warp * 8 + hb];
-    const float fa = ma == -INFINITY ? 0.f : ex2(ma - Ma);
-    const float fb = mb == -INFINITY ? 0.f : ex2(mb - Mb);
-    float *mw = reinterpret_cast<float *>(smem) + warp * kMergeWarpFloats + 16;
-#pragma unroll
-      for (int bb = 0; bb < 8; bb++) {
-        // wsum of (head h, block bb) lives in lane 4h + bb/2, as wA (bb even) or wB (odd)
-        const float sA = __shfl_sync(kFull, (bb & 1) ? wB : wA, 8 * tg + (bb >> 1));
-        const float sB = __shfl_sync(kFull, (bb & 1) ? wB : wA, 8 * tg + 4 + (bb >> 1));
-        const float cA = kBias * sA, cB = kBias * sB;
-#pragma unroll
-        for (int m = 0; m < 2; m++) {
-          const int d0 = 32 * bb + 16 * m + 2 * g;  // row g; row g + 8 is d0 + 1
-          *reinterpret_cast<float2 *>(mw + ha * kMergeHead + d0) =
-              make_float2((o[bb][m][0] - cA) * fa, (o[bb][m][2] - cA) * fa);
-          *reinterpret_cast<float2 *>(mw + hb * kMergeHead + d0) =
-              make_float2((o[bb][m][1] - cB) * fb, (o[bb][m][3] - cB) * fb);
+    // fused step: every CTA whose split holds the new token quantizes the
+    // token's K and V rows of its kv head into the cache before it issues a tile
+    // load (CTAs of the same kv head write identical bytes)
+    const bool appender = p_new >= t0 && p_new < t1;
+
+    // first cache row of the 64-token sub-tile starting at token t, -1 if unmapped
+    auto sub_row = [&](int t) -> int {
+      if (c.block_table == nullptr) return (int)(((int64_t)bs * c.num_kv_heads + kvh) * c.max_tokens + t);
+      const int pi = t / c.page_size;
+      const int page = __ldg(c.block_table + (int64_t)bs * c.max_pages_per_seq + pi);
+      if (page < 0 || page >= c.num_pages) return -1;
+      return (int)(((int64_t)page * c.num_kv_heads + kvh) * c.page_size + (t - pi * c.page_size));
+    };
+    // one thread: tile `it` onto its stage's full barrier.  Contiguous cache:
+    // the tile's rows are consecutive, one 128-row box per code plane and one
+    // bulk copy of the scale rows of this (sequence, head) per scale plane.
+    // Paged: each 64-token half that holds tokens of the split on its own.
+    // (A tile of 8 copies with 16-byte scale boxes kept the issuing thread busy
+    // about twice as long.)
+    auto issue = [&](int it) {
+      const int st = it % kStages;
+      const int tstart = t0 + it * kTile;
+      const uint32_t bar = full0 + 8 * st;
+      const uint32_t dst = smem_u32(smem + st * kStageBytes);
+      if (c.block_table == nullptr) {
+        const int r = sub_row(tstart);
+        const int nrows = min(kTile, c.max_tokens - tstart);
+        mbar_arrive_tx(bar, 2 * kTile * 128 + 2 * nrows * 16);
+        tma_load_2d(dst + kOffKC, &maps.kc, 0, r, bar);
+        tma_load_2d(dst + kOffVC, &maps.vc, 0, r, bar);
+        bulk_load(dst + kOffKS, c.k_scales + (int64_t)r * kRowScales, nrows * 16, bar);
+        bulk_load(dst + kOffVS, c.v_scales + (int64_t)r * kRowScales, nrows * 16, bar);
+      } else {
+        const int r0 = sub_row(tstart);
+        const int r1 = tstart + kSub < t1 ? sub_row(tstart + kSub) : -1;
+        const int n = (r0 >= 0) + (r1 >= 0);
+        if (n == 0) {
+          mbar_arrive(bar);
+        } else {
+          mbar_arrive_tx(bar, n * kSubBytes);
+          #pragma unroll
+          for (int j = 0; j < 2; j++) {
+            const int r = j ? r1 : r0;
+            if (r < 0) continue;
+            tma_load_2d(dst + kOffKC + j * kSub * 128, &maps.kc, 0, r, bar);
+            tma_load_2d(dst + kOffVC + j * kSub * 128, &maps.vc, 0, r, bar);
+            bulk_load(dst + kOffKS + j * kSub * 16, c.k_scales + (int64_t)r * kRowScales, kSub * 16, bar);
+            bulk_load(dst + kOffVS + j * kSub * 16, c.v_scales + (int64_t)r * kRowScales, kSub * 16, bar);
+          }
         }
       }
-    if (tid < 8) {
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kWarps; w++) M = fmaxf(M, ml[w * 8 + tid]);
-      float L = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; w++) {
-        const float mwv = ml[w * 8 + tid];
-        L += (mwv == -INFINITY ? 0.f : ex2(mwv - M)) * ml[kWarps * 8 + w * 8 + tid];
+      atomicMax(const_cast<int *>(issued), it + 1);
+    };
+    // initial tiles: warp w issues tile w, except the tile holding the new
+    // token of a fused step, which the appending warp issues once the token's
+    // rows are in the cache (a later tile holding it is refilled inside the
+    // loop, after the barrier that follows the append)
+    const int it_new = appender ? (p_new - t0) / kTile : -1;
+    if (lane == 0 && warp < kStages && warp < ntiles && warp != it_new) issue(warp);
+    if (appender && warp == 0) {
+      // scratch outside the ring (the per-warp scale areas of warps 0 and 1,
+      // used only inside the tile loop)
+      float4 *scratch = reinterpret_cast<float4 *>(smem + kOffFs);
+      {
+        const int vg = lane >> 3, i = lane & 7;
+        const bool valid = vg < 2;  // lanes 0-7: K, 8-15: V
+        const void *src =
+            static_cast<const char *>(vg == 1 ? v_new : k_new) +
+            ((int64_t)b * c.num_kv_heads + kvh) * kDim * (BF16 ? 2 : 4);
+          uint4 bytes;
+        uint16_t sc;
+        q4v::quantize_vector<BF16>(valid ? src : k_new, valid, lane, scratch + 64 * vg, bytes, sc);
+        const int64_t row = q4_row(c, bs, kvh, p_new);
+        if (valid && row >= 0) {
+          *reinterpret_cast<uint4 *>((vg ? c.v_codes : c.k_codes) + row * kRowCodeBytes + 16 * i) =
+              bytes;
+          (vg ? c.v_scales : c.k_scales)[row * kRowScales + i] = sc;
+        }
       }
-      mh[tid] = M;
-      mh[8 + tid] = L;
+      // the rows are read back by TMA (async proxy)
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __syncwarp();
+      if (lane == 0 && it_new < kStages) issue(it_new);
     }
-  }
-  __syncthreads();
-  const float nan = __int_as_float(0x7fc00000);
-  for (int hh = 0; hh < gc; hh++) {
-    float *rec = ws + (((int64_t)b * n_q_heads + h0 + hh) * splits + s) * kRec;
-    float acc = 0.f;
+
+    // (1) query: warp w rotates head h0 + w (zeros past gc), splits it into
+    // fp16 hi + lo and writes the MMA fragments of its 8 blocks x 2 k-steps
+    {
+      warp_fwht256(x, lane);
+      float hi[8], lo[8], sq = 0.f;
+      #pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const float v = x[i] * 0.0625f;  // the FWHT's 1/16 (exact)
+        hi[i] = __half2float(__float2half_rn(v));
+        lo[i] = __half2float(__float2half_rn(v - hi[i]));
+        sq += hi[i] + lo[i];
+      }
+      // lane L holds dims 8L..8L+7 = block L/4, k-step (L/2)&1, tg 2(L&1) and 2(L&1)+1
+      uint4 *qf = reinterpret_cast<uint4 *>(smem + kOffQF) + (warp * 8 + (lane >> 2)) * 8 +
+                  ((lane >> 1) & 1) * 4 + 2 * (lane & 1);
+      #pragma unroll
+      for (int e = 0; e < 2; e++) {
+        const int i = 4 * e;
+        qf[e] = make_uint4(pack_f16x2(hi[i], hi[i + 2]), pack_f16x2(lo[i], lo[i + 2]),
+                           pack_f16x2(hi[i + 1], hi[i + 3]), pack_f16x2(lo[i + 1], lo[i + 3]));
+      }
+      sq += __shfl_xor_sync(kFull, sq, 1);
+      sq += __shfl_xor_sync(kFull, sq, 2);
+      if ((lane & 3) == 0)
+        reinterpret_cast<float *>(smem + kOffQB)[warp * 8 + (lane >> 2)] = -kBias * sq;
+    }
+    __syncthreads();
+    uint4 qa[8][2];
+    float cb[8];  // accumulator start of the hi rows: -72 * sum over the block of (hi + lo)
+    {
+      const uint4 *qf = reinterpret_cast<const uint4 *>(smem + kOffQF) + g * 64 + tg;
+      #pragma unroll
+      for (int bb = 0; bb < 8; bb++) {
+        qa[bb][0] = qf[bb * 8];
+        qa[bb][1] = qf[bb * 8 + 4];
+        cb[bb] = reinterpret_cast<const float *>(smem + kOffQB)[g * 8 + bb];
+      }
+    }
+
+    // (2) the split: warp group gq = warp / 4 takes the tiles it with it % 2 == gq,
+    // warp wi = warp % 4 tokens 32wi .. 32wi + 31 of each of them
+    const int gq = warp >> 2, wi = warp & 3;
+    float o[8][2][4];  // [block][M-tile X (dims 2g, 2g+1) / Y (16 + 2g, 17 + 2g)][reg]
+    #pragma unroll
+    for (int bb = 0; bb < 8; bb++)
+      #pragma unroll
+      for (int m = 0; m < 2; m++) o[bb][m][0] = o[bb][m][1] = o[bb][m][2] = o[bb][m][3] = 0.f;
+    float wacc[4] = {0.f, 0.f, 0.f, 0.f};  // sum_t p d_v: head g (hi, lo rows) x blocks 2tg, 2tg+1
+    float m_run = -INFINITY, l_run = 0.f;  // head g
+    float *fsk = reinterpret_cast<float *>(smem + kOffFs + warp * (kFsK + kFsV));
+    __half *fsv = reinterpret_cast<__half *>(smem + kOffFs + warp * (kFsK + kFsV) + kFsK);
+    const int row_l = 32 * wi + 8 * ((lane >> 3) & 1) + (lane & 7);  // ldmatrix row (T = 0/1)
+    const int blk_l = lane >> 4;
+
+    for (int it = gq; it < ntiles; it += 2) {
+      const int st = it % kStages;
+      if (!mbar_wait(full0 + 8 * st, (it / kStages) & 1, abort_flag)) {
+        *abort_flag = 1;
+        break;
+      }
+      const uint8_t *stage = smem + st * kStageBytes;
+      const int tw = t0 + it * kTile + 32 * wi;  // first token of this warp
+      const int nvalid = min(32, t1 - tw);
+      bool live = nvalid > 0;
+      if (live && c.block_table != nullptr) live = sub_row(tw & ~(kSub - 1)) >= 0;
+      if (live) {
+        {  // widen: lane = token; K scales -> fp32, V scales fp16, [block][pos]; invalid -> 0
+          const int t = lane;
+          const uint4 wk = *reinterpret_cast<const uint4 *>(stage + kOffKS + (32 * wi + t) * 16);
+          const uint4 wv = *reinterpret_cast<const uint4 *>(stage + kOffVS + (32 * wi + t) * 16);
+          // pos: 16 * (T >> 1) + 4 * tg + 2 * (T & 1) + e for t = 8T + 2tg + e
+          const int T = t >> 3, tg2 = (t >> 1) & 3, e = t & 1;
+          const int pos = 16 * (T >> 1) + 4 * tg2 + 2 * (T & 1) + e;
+          const bool ok = t < nvalid;
+          const uint32_t kk[4] = {wk.x, wk.y, wk.z, wk.w}, vv[4] = {wv.x, wv.y, wv.z, wv.w};
+          #pragma unroll
+          for (int k2 = 0; k2 < 4; k2++) {
+            const float2 pk2 = __half22float2(*reinterpret_cast<const __half2 *>(&kk[k2]));
+            fsk[(2 * k2) * 32 + pos] = ok ? pk2.x : 0.f;
+            fsk[(2 * k2 + 1) * 32 + pos] = ok ? pk2.y : 0.f;
+            const uint32_t v2 = ok ? vv[k2] : 0u;
+            reinterpret_cast<uint16_t *>(fsv)[(2 * k2) * 32 + pos] = (uint16_t)(v2 & 0xffffu);
+            reinterpret_cast<uint16_t *>(fsv)[(2 * k2 + 1) * 32 + pos] = (uint16_t)(v2 >> 16);
+          }
+        }
+        __syncwarp();
+        const uint32_t kbase = smem_u32(stage + kOffKC), vbase = smem_u32(stage + kOffVC);
+
+        // ---- QK: head g, tokens 8T + 2tg + {0, 1}, T = 0..3
+        float2 sacc[4];
+        #pragma unroll
+        for (int T = 0; T < 4; T++) sacc[T] = make_float2(0.f, 0.f);
+        #pragma unroll
+        for (int bp = 0; bp < 4; bp++) {
+          #pragma unroll
+          for (int tp = 0; tp < 2; tp++) {  // token groups 2tp, 2tp + 1
+            uint32_t kr[4];  // (T0, block 2bp), (T1, 2bp), (T0, 2bp + 1), (T1, 2bp + 1)
+            ldsm_x4(kbase + (row_l + 16 * tp) * 128 + (((2 * bp + blk_l) ^ (lane & 7)) << 4), kr);
+            #pragma unroll
+            for (int half = 0; half < 2; half++) {
+              const int bb = 2 * bp + half;
+              const float4 dk = *reinterpret_cast<const float4 *>(fsk + bb * 32 + 16 * tp + 4 * tg);
+              #pragma unroll
+              for (int T = 0; T < 2; T++) {
+                const uint32_t w = kr[2 * half + T];
+                float acc[4];
+                mma16816c(acc, qa[bb][0], nib64(w << 4), nib64(w >> 4), cb[bb], 0.f);
+                mma16816(acc, qa[bb][1], nib64(w), nib64(w >> 8));
+                const float2 d = T ? make_float2(dk.z, dk.w) : make_float2(dk.x, dk.y);
+                sacc[2 * tp + T] = __ffma2_rn(
+                    d, __fadd2_rn(make_float2(acc[0], acc[1]), make_float2(acc[2], acc[3])), sacc[2 * tp + T]);
+              }
+            }
+          }
+        }
+        // ---- online softmax of head g over this warp's 32 tokens
+        float x[8];
+        #pragma unroll
+        for (int T = 0; T < 4; T++) {
+          x[2 * T] = sacc[T].x * sl2;
+          x[2 * T + 1] = sacc[T].y * sl2;
+        }
+        if (nvalid < 32) {
+          #pragma unroll
+          for (int e2 = 0; e2 < 8; e2++)
+            if (8 * (e2 >> 1) + 2 * tg + (e2 & 1) >= nvalid) x[e2] = -INFINITY;
+        }
+        float mx = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        if (__any_sync(kFull, mx > m_run)) {
+          const float mn = fmaxf(m_run, mx);
+          const float alpha = mn == m_run ? 1.f : ex2(m_run - mn);
+          m_run = mn;
+          l_run *= alpha;
+          #pragma unroll
+          for (int k = 0; k < 4; k++) wacc[k] *= alpha;  // rows of head g
+          const float a0 = __shfl_sync(kFull, alpha, 8 * tg);
+          const float a1 = __shfl_sync(kFull, alpha, 8 * tg + 4);
+          #pragma unroll
+          for (int bb = 0; bb < 8; bb++)
+            #pragma unroll
+            for (int m = 0; m < 2; m++) {
+              o[bb][m][0] *= a0;
+              o[bb][m][1] *= a1;
+              o[bb][m][2] *= a0;
+              o[bb][m][3] *= a1;
+            }
+        }
+        uint32_t ph[4], pl[4];  // p of head g as fp16 hi + lo pairs, token groups T
+        #pragma unroll
+        for (int T = 0; T < 4; T++) {
+          const float p0 = ex2(x[2 * T] - m_run), p1 = ex2(x[2 * T + 1] - m_run);
+          l_run += p0 + p1;
+          split_hilo(make_float2(p0, p1), ph[T], pl[T]);
+        }
+        // ---- PV: k-steps of 16 tokens (token groups 2ks, 2ks + 1)
+        #pragma unroll
+        for (int ks = 0; ks < 2; ks++) {
+          {  // sum_t p d_v for blocks 2tg, 2tg+1 on the tensor cores (d_v exact in fp16)
+            const uint2 dvb = *reinterpret_cast<const uint2 *>(fsv + g * 32 + 16 * ks + 4 * tg);
+            const uint32_t a[4] = {ph[2 * ks], pl[2 * ks], ph[2 * ks + 1], pl[2 * ks + 1]};
+            mma16816(wacc, a, dvb.x, dvb.y);
+          }
+          #pragma unroll
+          for (int bp = 0; bp < 4; bp++) {
+            uint32_t vr[4];  // (tokens 0-7, block 2bp), (8-15, 2bp), (0-7, 2bp + 1), (8-15, 2bp + 1)
+            ldsm_x4_t(vbase + (row_l + 16 * ks) * 128 + (((2 * bp + blk_l) ^ (lane & 7)) << 4), vr);
+            #pragma unroll
+            for (int half = 0; half < 2; half++) {
+              const int bb = 2 * bp + half;
+              const uint2 dvp = *reinterpret_cast<const uint2 *>(fsv + bb * 32 + 16 * ks + 4 * tg);
+              const __half2 d01 = *reinterpret_cast<const __half2 *>(&dvp.x);
+              const __half2 d89 = *reinterpret_cast<const __half2 *>(&dvp.y);
+              // w = p d_v exactly as hi + lo (TwoProduct with fp16 FMA)
+              const __half2 ph0 = *reinterpret_cast<const __half2 *>(&ph[2 * ks]);
+              const __half2 ph1 = *reinterpret_cast<const __half2 *>(&ph[2 * ks + 1]);
+              const __half2 pl0 = *reinterpret_cast<const __half2 *>(&pl[2 * ks]);
+              const __half2 pl1 = *reinterpret_cast<const __half2 *>(&pl[2 * ks + 1]);
+              const __half2 wh0 = __hmul2_rn(ph0, d01), wh1 = __hmul2_rn(ph1, d89);
+              const __half2 wl0 = __hfma2(pl0, d01, __hfma2(ph0, d01, __hneg2(wh0)));
+              const __half2 wl1 = __hfma2(pl1, d89, __hfma2(ph1, d89, __hneg2(wh1)));
+              const uint32_t bh0 = *reinterpret_cast<const uint32_t *>(&wh0);
+              const uint32_t bh1 = *reinterpret_cast<const uint32_t *>(&wh1);
+              const uint32_t bl0 = *reinterpret_cast<const uint32_t *>(&wl0);
+              const uint32_t bl1 = *reinterpret_cast<const uint32_t *>(&wl1);
+              const uint32_t r0 = vr[2 * half], r1 = vr[2 * half + 1];
+              {
+                const uint32_t a[4] = {nib64(r0 << 4), nib64(r0 >> 4), nib64(r1 << 4), nib64(r1 >> 4)};
+                mma16816(o[bb][0], a, bh0, bh1);
+                mma16816(o[bb][0], a, bl0, bl1);
+              }
+              {
+                const uint32_t a[4] = {nib64(r0), nib64(r0 >> 8), nib64(r1), nib64(r1 >> 8)};
+                mma16816(o[bb][1], a, bh0, bh1);
+                mma16816(o[bb][1], a, bl0, bl1);
+              }
+            }
+          }
+        }
+      }
+      // release the stage; the last of its 4 warps refills it with tile it + kStages
+      // (same warp group: kStages is even)
+      __syncwarp();
+      if (lane == 0) {
+        int old;
+        asm volatile("atom.release.cta.shared::cta.add.s32 %0, [%1], 1;"
+                     : "=r"(old)
+                     : "r"(smem_u32(rel + st))
+                     : "memory");
+        if (old == 3) {
+          asm volatile("fence.acq_rel.cta;" ::: "memory");
+          rel[st] = 0;
+          if (it + kStages < ntiles && !*abort_flag) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(it + kStages);
+          }
+        }
+      }
+    }
+
+    // (3) merge the 8 warps' states into this split's records
+    l_run += __shfl_xor_sync(kFull, l_run, 1);
+    l_run += __shfl_xor_sync(kFull, l_run, 2);
+    // wacc: head g, blocks 2tg (hi + lo rows: [0] + [2]) and 2tg + 1 ([1] + [3])
+    const float wA = wacc[0] + wacc[2], wB = wacc[1] + wacc[3];
+    __syncthreads();  // every warp is done with the ring
+    const bool abort_all = *abort_flag != 0;
+    if (abort_all) {
+      // a load never arrived: let every load still in flight land (bounded,
+      // ignoring the flag) before the CTA's shared memory goes away
+      if (tid == 0) {
+        const int n = *issued;
+        for (int it = n > kStages ? n - kStages : 0; it < n; it++)
+          for (int i = 0; i < kWaitPolls && !mbar_try(full0 + 8 * (it % kStages), (it / kStages) & 1); i++) {
+          }
+      }
+      __syncthreads();
+    }
+    // per-warp (m, l) of each head, then every warp scales its accumulators to
+    // the CTA maximum before storing them, so the final pass only adds
+    float *ml = reinterpret_cast<float *>(smem + kOffMergeF);  // m [warp][head], l [warp][head]
+    float *mh = ml + 2 * kWarps * 8;                            // M, L per head
+    if (!abort_all && tg == 0) {
+      ml[warp * 8 + g] = m_run;
+      ml[kWarps * 8 + warp * 8 + g] = l_run;
+    }
+    __syncthreads();
     if (!abort_all) {
-#pragma unroll
-      for (int w = 0; w < kWarps; w++)
-        acc += reinterpret_cast<const float *>(smem)[w * kMergeWarpFloats + 16 + hh * kMergeHead + tid];
+      // this thread's accumulator columns are heads 2tg and 2tg + 1
+      const int ha = 2 * tg, hb = ha + 1;
+      float Ma = -INFINITY, Mb = -INFINITY;
+      #pragma unroll
+      for (int w = 0; w < kWarps; w++) {
+        Ma = fmaxf(Ma, ml[w * 8 + ha]);
+        Mb = fmaxf(Mb, ml[w * 8 + hb]);
+      }
+      const float ma = ml[warp * 8 + ha], mb = ml[warp * 8 + hb];
+      const float fa = ma == -INFINITY ? 0.f : ex2(ma - Ma);
+      const float fb = mb == -INFINITY ? 0.f : ex2(mb - Mb);
+      float *mw = reinterpret_cast<float *>(smem) + warp * kMergeWarpFloats + 16;
+        #pragma unroll
+        for (int bb = 0; bb < 8; bb++) {
+          // wsum of (head h, block bb) lives in lane 4h + bb/2, as wA (bb even) or wB (odd)
+          const float sA = __shfl_sync(kFull, (bb & 1) ? wB : wA, 8 * tg + (bb >> 1));
+          const float sB = __shfl_sync(kFull, (bb & 1) ? wB : wA, 8 * tg + 4 + (bb >> 1));
+          const float cA = kBias * sA, cB = kBias * sB;
+          #pragma unroll
+          for (int m = 0; m < 2; m++) {
+            const int d0 = 32 * bb + 16 * m + 2 * g;  // row g; row g + 8 is d0 + 1
+            *reinterpret_cast<float2 *>(mw + ha * kMergeHead + d0) =
+                make_float2((o[bb][m][0] - cA) * fa, (o[bb][m][2] - cA) * fa);
+            *reinterpret_cast<float2 *>(mw + hb * kMergeHead + d0) =
+                make_float2((o[bb][m][1] - cB) * fb, (o[bb][m][3] - cB) * fb);
+          }
+        }
+      if (tid < 8) {
+        float M = -INFINITY;
+        #pragma unroll
+        for (int w = 0; w < kWarps; w++) M = fmaxf(M, ml[w * 8 + tid]);
+        float L = 0.f;
+        #pragma unroll
+        for (int w = 0; w < kWarps; w++) {
+          const float mwv = ml[w * 8 + tid];
+          L += (mwv == -INFINITY ? 0.f : ex2(mwv - M)) * ml[kWarps * 8 + w * 8 + tid];
+        }
+        mh[tid] = M;
+        mh[8 + tid] = L;
+      }
     }
-    rec[4 + tid] = abort_all ? nan : acc;
-    if (tid == 0) {
-      rec[0] = abort_all ? nan : mh[hh];
-      rec[1] = abort_all ? nan : mh[8 + hh];
+    __syncthreads();
+    for (int hh = 0; hh < gc; hh++) {
+      float *rec = ws + (rec_base + hh * rec_hstride) * kRec;
+      float acc = 0.f;
+      if (!abort_all) {
+        #pragma unroll
+        for (int w = 0; w < kWarps; w++)
+          acc += reinterpret_cast<const float *>(smem)[w * kMergeWarpFloats + 16 + hh * kMergeHead + tid];
+      }
+      rec[4 + tid] = abort_all ? nan : acc;
+      if (tid == 0) {
+        rec[0] = abort_all ? nan : mh[hh];
+        rec[1] = abort_all ? nan : mh[8 + hh];
+      }
     }
-  }
+    if (abort_all) dead = true;
+  }  // segments
 }
 }  // namespace
 
@@ -556,7 +630,9 @@ cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, in
                                  const int32_t *q_to_seq, int num_seqs) {
   const int group = n_q_heads / c.num_kv_heads;
   const int gc = group < 8 ? group : 8;
-  if (p.split_tokens % kTile) return cudaErrorInvalidValue;
+  if (p.stream ? p.tile != kTile : p.split_tokens % kTile) return cudaErrorInvalidValue;
+  const int n_hg = n_q_heads / gc;
+  const int append_tiles = p.stream && pos ? kAppendTokens / kTile : 0;
   const float sl2 = scale * kLog2e;
   const uint64_t rows = c.block_table
                             ? (uint64_t)c.num_pages * c.num_kv_heads * c.page_size
@@ -569,27 +645,29 @@ cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, in
     return cudaErrorInvalidValue;
   // opt in to the large dynamic shared-memory carve-out once per device
   static std::mutex mu;
-  static unsigned configured[2] = {0u, 0u};
+  static unsigned configured[4] = {0u, 0u, 0u, 0u};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  const int variant = bf16 + 2 * p.stream;
   {
     std::lock_guard<std::mutex> lock(mu);
     const unsigned bit = 1u << (dev & 31);
-    if (!(configured[bf16] & bit)) {
-      e = bf16 ? cudaFuncSetAttribute(q4_decode_mma_kernel<true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)
-               : cudaFuncSetAttribute(q4_decode_mma_kernel<false>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (!(configured[variant] & bit)) {
+      const void *fn = variant == 0   ? (const void *)q4_decode_mma_kernel<false, false>
+                       : variant == 1 ? (const void *)q4_decode_mma_kernel<true, false>
+                       : variant == 2 ? (const void *)q4_decode_mma_kernel<false, true>
+                                      : (const void *)q4_decode_mma_kernel<true, true>;
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
       if (e != cudaSuccess) return e;
-      configured[bf16] |= bit;
+      configured[variant] |= bit;
     }
   }
   // programmatic dependent launch: this grid may be scheduled while the
   // previous kernel on the stream finishes; it waits for it (griddepcontrol)
   // before touching global memory
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.splits, n_q_heads / gc, batch);
+  cfg.gridDim = p.stream ? dim3(p.ctas) : dim3(p.splits, n_q_heads / gc, batch);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = s;
@@ -598,14 +676,31 @@ cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, in
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (bf16)
-    e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<true>, maps, c, q, seq_lens, max_seq_len,
-                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws, k_new, v_new,
+  switch (variant) {
+    case 0:
+      e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<false, false>, maps, c, q, seq_lens, max_seq_len,
+                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, n_hg,
+                           p.n_units, append_tiles, ws, k_new, v_new,
                            pos, q_to_seq, q_to_seq ? num_seqs : batch);
-  else
-    e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<false>, maps, c, q, seq_lens, max_seq_len,
-                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, ws, k_new, v_new,
+      break;
+    case 1:
+      e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<true, false>, maps, c, q, seq_lens, max_seq_len,
+                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, n_hg,
+                           p.n_units, append_tiles, ws, k_new, v_new,
                            pos, q_to_seq, q_to_seq ? num_seqs : batch);
+      break;
+    case 2:
+      e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<false, true>, maps, c, q, seq_lens, max_seq_len,
+                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, n_hg,
+                           p.n_units, append_tiles, ws, k_new, v_new,
+                           pos, q_to_seq, q_to_seq ? num_seqs : batch);
+      break;
+    default:
+      e = cudaLaunchKernelEx(&cfg, q4_decode_mma_kernel<true, true>, maps, c, q, seq_lens, max_seq_len,
+                           n_q_heads, group, gc, sl2, p.split_tokens, p.splits, n_hg,
+                           p.n_units, append_tiles, ws, k_new, v_new,
+                           pos, q_to_seq, q_to_seq ? num_seqs : batch);
+  }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
