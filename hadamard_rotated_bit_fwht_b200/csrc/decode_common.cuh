@@ -21,9 +21,11 @@ constexpr unsigned kFullMask = 0xffffffffu;
 // thread of the CTA has given up
 constexpr int kWaitPolls = 1 << 20;
 
-// code planes; scale rows are contiguous and come by 1-D bulk copies
+// code planes; scale rows are contiguous and come by 1-D bulk copies.  kc2,
+// vc2: the same planes with boxes of twice the rows (paged Q4_0 tiles whose
+// two halves are consecutive rows of one page)
 struct TmaMaps {
-  CUtensorMap kc, vc;
+  CUtensorMap kc, vc, kc2, vc2;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

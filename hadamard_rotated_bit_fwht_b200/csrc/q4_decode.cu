@@ -18,16 +18,17 @@ constexpr int kRec = 260;  // floats per partial record: m, l, pad, pad, o[256]
 
 // Log-sum-exp combine of the splits and back-rotation; one CTA of 256 threads
 // per (sequence, q head).  Thread j owns dimension j and issues its loads of
-// o_s[j] (up to kBatch splits at a time) first; meanwhile warp 0 reduces the
+// o_s[j] (up to kB splits at a time) first; meanwhile warp 0 reduces the
 // split maxima and sums (lane-strided, shuffles) and publishes the weights, so
-// a split count of up to kBatch costs one L2 round trip.  Warp 0 then applies
+// a split count of up to kB costs one L2 round trip.  Warp 0 then applies
 // the FWHT-256 (8 values per lane: strides 1, 2, 4 in registers, 8 .. 128
 // across lanes) and the 1/16.
 constexpr int kMaxSplitsSmem = 1024;
 constexpr int kMaxStreamUnits = 4096;  // units scanned by every CTA of a stream schedule
-constexpr int kBatch = 48;
-
-__global__ void __launch_bounds__(256, 1)
+// kB: records loaded per round trip.  48 for few heads with many splits; 16
+// (4 CTAs per SM) for many heads with few records each
+template <int kB>
+__global__ void __launch_bounds__(256, kB <= 16 ? 4 : 1)
     q4_decode_combine_kernel(const float *__restrict__ ws, const int32_t *__restrict__ seq_lens,
                              const int32_t *__restrict__ pos, const int32_t *__restrict__ q_to_seq,
                              int num_seqs, int n_q_heads, int splits, int split_tokens,
@@ -77,11 +78,11 @@ __global__ void __launch_bounds__(256, 1)
   }
   // the partial records come from the split kernel launched just before
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  float v[kBatch];
+  float v[kB];
   auto fetch = [&](int s0) {
-    // volatile asm keeps all kBatch loads ahead of the first use
+    // volatile asm keeps all kB loads ahead of the first use
 #pragma unroll
-    for (int k = 0; k < kBatch; k++) {
+    for (int k = 0; k < kB; k++) {
       const float *src = rec + min(s0 + k, ns - 1) * rstride + 4 + j;
       asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v[k]) : "l"(src));
     }
@@ -125,10 +126,10 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   const float L = lsum;
   float O = 0.f;
-  for (int s0 = 0; s0 < ns; s0 += kBatch) {
+  for (int s0 = 0; s0 < ns; s0 += kB) {
     if (s0 > 0) fetch(s0);
 #pragma unroll
-    for (int k = 0; k < kBatch; k++) {
+    for (int k = 0; k < kB; k++) {
       const float w = s0 + k < ns ? wgt[s0 + k] : 0.f;
       asm volatile("fma.rn.f32 %0, %1, %2, %0;" : "+f"(O) : "f"(w), "f"(v[k]));
     }
@@ -270,7 +271,11 @@ cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int ba
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int n_hg = p.n_units / batch;
-  e = cudaLaunchKernelEx(&cfg, q4_decode_combine_kernel, (const float *)ws, seq_lens, pos,
+  // records per head: the splits, or the CTAs one unit's tiles spread over
+  const int per_head = p.stream ? p.ctas / max(p.n_units, 1) + 2 : p.splits;
+  e = cudaLaunchKernelEx(&cfg,
+                         per_head <= 16 ? q4_decode_combine_kernel<16> : q4_decode_combine_kernel<48>,
+                         (const float *)ws, seq_lens, pos,
                          q_to_seq, q_to_seq ? num_seqs : batch, n_q_heads, p.splits,
                          p.split_tokens, p.stream, n_hg, p.n_units, p.ctas, n_q_heads / n_hg,
                          p.tile, p.stream && pos ? dec::kAppendTokens / p.tile : 0, max_seq_len, cap,

@@ -105,6 +105,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     prefetch_map(&maps.kc);
     prefetch_map(&maps.vc);
+    if (c.block_table) {
+      prefetch_map(&maps.kc2);
+      prefetch_map(&maps.vc2);
+    }
   }
   // inputs may come from the kernel launched just before this one
   grid_dependency_wait();
@@ -241,7 +245,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // one thread: tile `it` onto its stage's full barrier.  Contiguous cache:
     // the tile's rows are consecutive, one 128-row box per code plane and one
     // bulk copy of the scale rows of this (sequence, head) per scale plane.
-    // Paged: each 64-token half that holds tokens of the split on its own.
+    // Paged: the same when the tile's two 64-token halves are consecutive rows
+    // of one page, else each half that holds tokens of the split on its own.
     // (A tile of 8 copies with 16-byte scale boxes kept the issuing thread busy
     // about twice as long.)
     auto issue = [&](int it) {
@@ -263,6 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = (r0 >= 0) + (r1 >= 0);
         if (n == 0) {
           mbar_arrive(bar);
+        } else if (r0 >= 0 && r1 == r0 + kSub) {
+          // both halves on one page, consecutive rows: copies as for a contiguous cache
+          mbar_arrive_tx(bar, 2 * kSubBytes);
+          tma_load_2d(dst + kOffKC, &maps.kc2, 0, r0, bar);
+          tma_load_2d(dst + kOffVC, &maps.vc2, 0, r0, bar);
+          bulk_load(dst + kOffKS, c.k_scales + (int64_t)r0 * kRowScales, kTile * 16, bar);
+          bulk_load(dst + kOffVS, c.v_scales + (int64_t)r0 * kRowScales, kTile * 16, bar);
         } else {
           mbar_arrive_tx(bar, n * kSubBytes);
           #pragma unroll
@@ -643,6 +655,14 @@ cudaError_t launch_q4_decode_mma(const kvq_cache &c, const void *q, int bf16, in
   if (!make_map(&maps.kc, c.k_codes, rows, 128, 128, box, true) ||
       !make_map(&maps.vc, c.v_codes, rows, 128, 128, box, true))
     return cudaErrorInvalidValue;
+  if (c.block_table) {
+    if (!make_map(&maps.kc2, c.k_codes, rows, 128, 128, kTile, true) ||
+        !make_map(&maps.vc2, c.v_codes, rows, 128, 128, kTile, true))
+      return cudaErrorInvalidValue;
+  } else {
+    maps.kc2 = maps.kc;
+    maps.vc2 = maps.vc;
+  }
   // opt in to the large dynamic shared-memory carve-out once per device
   static std::mutex mu;
   static unsigned configured[4] = {0u, 0u, 0u, 0u};

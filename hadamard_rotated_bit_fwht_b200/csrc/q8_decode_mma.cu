@@ -610,6 +610,8 @@ cudaError_t launch_q8_decode_mma(const kvq_cache &c, const void *q, int bf16, in
   if (!make_map(&maps.kc, c.k_codes, rows, kCodeRow, 128, kTile, true) ||
       !make_map(&maps.vc, c.v_codes, rows, kCodeRow, 128, kTile, true))
     return cudaErrorInvalidValue;
+  maps.kc2 = maps.kc;  // a 64-token tile is one box already
+  maps.vc2 = maps.vc;
   static std::mutex mu;
   static unsigned configured[4] = {0u, 0u, 0u, 0u};
   int dev = 0;
