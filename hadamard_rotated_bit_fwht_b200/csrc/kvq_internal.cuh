@@ -44,6 +44,19 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
   return __fadd2_rn(a, make_float2(-b.x, -b.y));
 }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+// a * b + 0, rounded once: the same value as RN(a * b) except that a -0
+// product comes out +0.  Unlike a plain multiply, ptxas cannot rewrite it into
+// a multiply and contract that with a following add.
+__device__ __forceinline__ float2 mul2_rn_p0(float2 a, float2 b) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)), "l"(0ull));
+  return upk(r);
+}
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));
+  return upk(r);
+}
 __device__ __forceinline__ float2 add2_rz(float2 a, float2 b) {
   uint64_t r;
   asm("add.rz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a)), "l"(pk(b)));

@@ -241,15 +241,17 @@ __device__ __forceinline__ void q4_quantize_l1(const float r[32], int lane, int 
 #pragma unroll
   for (int B = 0; B < 8; B++) {
     const int r0 = 4 * (B & 1) + 8 * (B >> 1);
-    // z * id and + 8.5 round separately: scalar __fmul_rn / __fadd_rn are
-    // never merged into a multiply-add (the packed fp32x2 forms were observed
-    // to be, which moves a value sitting on a rounding tie).
-    float t[4];
-#pragma unroll
-    for (int m = 0; m < 4; m++) t[m] = __fadd_rn(__fmul_rn(r[r0 + m], idb[B]), 8.5f);
+    // z * id and + 8.5 round separately.  A packed multiply followed by a
+    // packed add was observed to be merged into one multiply-add (which moves
+    // a value sitting on a rounding tie); the product is therefore a packed
+    // fma with a +0 addend, which has the product's rounding and cannot be
+    // merged.
+    const float2 idv = make_float2(idb[B], idb[B]), half8 = make_float2(8.5f, 8.5f);
+    const float2 t02 = add2_rn(mul2_rn_p0(make_float2(r[r0], r[r0 + 2]), idv), half8);
+    const float2 t13 = add2_rn(mul2_rn_p0(make_float2(r[r0 + 1], r[r0 + 3]), idv), half8);
     // 2^23 + floor(t) for t >= 0; the low 16 bits are floor(t) in 0..16
-    const float2 f02 = add2_rz(make_float2(t[0], t[2]), magic);
-    const float2 f13 = add2_rz(make_float2(t[1], t[3]), magic);
+    const float2 f02 = add2_rz(t02, magic);
+    const float2 f13 = add2_rz(t13, magic);
     // element-in-block i + 8m: byte i = c0 | c2 << 4, byte i + 8 = c1 | c3 << 4
     const uint32_t x02 = min_u16x2(__byte_perm(__float_as_uint(f02.x), __float_as_uint(f02.y), 0x5410), fifteen);
     const uint32_t x13 = min_u16x2(__byte_perm(__float_as_uint(f13.x), __float_as_uint(f13.y), 0x5410), fifteen);
@@ -325,10 +327,15 @@ __device__ __forceinline__ void q8_quantize_l1(const float r[32], int lane, int 
 #pragma unroll
   for (int B = 0; B < 8; B++) {
     const int r0 = 4 * (B & 1) + 8 * (B >> 1);
+    // products rounded once each (packed, as in q4_quantize_l1)
+    const float2 idv = make_float2(idb[B], idb[B]);
+    const float2 p01 = mul2_rn_p0(make_float2(r[r0], r[r0 + 1]), idv);
+    const float2 p23 = mul2_rn_p0(make_float2(r[r0 + 2], r[r0 + 3]), idv);
+    const float p[4] = {p01.x, p01.y, p23.x, p23.y};
     uint32_t w = 0;
 #pragma unroll
     for (int m = 0; m < 4; m++) {
-      const int c = (int)roundf(__fmul_rn(r[r0 + m], idb[B]));
+      const int c = (int)roundf(p[m]);
       w |= (uint32_t)(c & 0xFF) << (8 * m);
     }
     stage[B * 8 + i] = w;
