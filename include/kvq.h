@@ -151,6 +151,10 @@ KVQ_API size_t kvq_decode_attn_workspace(const kvq_cache *cache, int32_t batch,
  * before the integer tensor-core products with the codes.
  * Split-K flash decoding: partial (max, sum, accumulator) per split in the
  * workspace, then a log-sum-exp combine that also applies the back-rotation.
+ * Few rows: equal splits of each row.  Many rows (at least 37 (row, head
+ * group) units): every SM's CTA takes an equal run of all rows' tiles, found
+ * on the device from d_seq_lens, and writes one partial per row it touches.
+ * Either way the result depends only on the inputs (run to run identical).
  * Both kernels are launched with programmatic stream serialization: they may
  * be scheduled while the previous kernel on the stream drains and wait for it
  * on the device before reading any input.
@@ -201,10 +205,13 @@ KVQ_API kvq_status kvq_decode_attn_multi(const kvq_cache *cache, const void *q, 
  * rotates the new K/V and the query, attends, and rotates the output back).
  * Equivalent to kvq_quantize_append(cache, k_new, v_new, dtype, batch, 1,
  * d_pos) followed by kvq_decode_attn(cache, q, dtype, batch, num_q_heads,
- * seq_lens = d_pos + 1, max_seq_len, scale, out, ...): the cache bytes and the
- * output are bit-identical to that pair of calls.  The split of the decode that
- * holds position d_pos[b] quantizes the token in its prologue, so the append
- * costs no launch of its own.
+ * seq_lens = d_pos + 1, max_seq_len, scale, out, ...): the cache bytes are
+ * bit-identical to that pair of calls, and so is the output when the batch
+ * has few rows (fewer than 37 (row, head group) units: one split per CTA).
+ * Larger batches use the balanced schedule, in which the CTA appending a
+ * token is given fewer tiles; the output then matches the pair of calls to
+ * fp32 rounding.  The CTA whose tiles hold position d_pos[b] quantizes the
+ * token in its prologue, so the append costs no launch of its own.
  *   k_new, v_new: device, [batch][num_kv_heads][256] of `dtype`, 16-byte
  *   aligned.  q: device, [batch][num_q_heads][256] of `dtype`, 16-byte aligned.
  *   d_pos: device int32[batch], position of the new token; a position outside
