@@ -151,7 +151,8 @@ class Workload:
     """One step of the hot path on a synthetic batch: pre(i) (the append of
     the step's new tokens, if any) then kernel_call(i) (the dominant call).
     Subclasses set step_bytes / kernel_bytes (algorithmic), launches_per_step,
-    kernel_name, traffic_key, config, and h2d / d2h tensors for e2e."""
+    kernel_name, traffic_key, config, and for e2e the names of the step's
+    input tensors (h2d) and the output tensors (d2h)."""
     launches_per_step = 0
     kernel_name = ""
     traffic_key = ""
@@ -212,7 +213,7 @@ class LongDecode(Workload):
         row = 32 * self.bits + 16  # code bytes + 8 fp16 scales per row
         self.kernel_bytes = B * H * T * 2 * row + 2 * B * H * (512 + row) + B * Hq * 256 * (2 + 4)
         self.step_bytes = self.kernel_bytes
-        self.h2d = [self.new_k, self.new_v, self.q]
+        self.h2d = ["new_k", "new_v", "q"]
         self.d2h = [self.out]
         self.config = {"workload": "long_decode" if self.bits == 4 else "long_decode_q8",
                        "batch": B, "n_q_heads": Hq, "n_kv_heads": H, "head_dim": 256, "ctx": T,
@@ -264,7 +265,7 @@ class QuantizePrefill(Workload):
         self.zero = torch.zeros(B, dtype=torch.int32, device=dev)
         self.kvq = kvq
         self.kernel_bytes = self.step_bytes = 2 * B * P * H * (512 + 144)
-        self.h2d = [self.k, self.v]
+        self.h2d = ["k", "v"]
         self.d2h = [self.cache.k_scales[:1]]
         self.config = {"workload": "quantize", "batch": B, "n_kv_heads": H, "head_dim": 256,
                        "prefill": P, "dtype_in": "bf16",
@@ -354,7 +355,7 @@ class PagedDecode(Workload):
         self.total = int(lens.sum())
         self.kernel_bytes = self.total * H * 288 + B * Hq * 256 * 6
         self.step_bytes = self.kernel_bytes + 2 * B * H * (512 + 144)
-        self.h2d = [self.new_k, self.new_v, self.q]
+        self.h2d = ["new_k", "new_v", "q"]
         self.d2h = [self.out]
         self.config = {"workload": "paged_decode", "batch": B, "n_q_heads": Hq,
                        "n_kv_heads": H, "head_dim": 256, "tokens": self.total,
@@ -418,7 +419,7 @@ class OctaveDecode(Workload):
         self.kernel_bytes = B * ctx * H * 128 + B * Hq * 128 * 6
         self.step_bytes = self.kernel_bytes + B * H * (2 * 256 + 128)
         self.quant_bytes = ctx * H * (2 * 256 + 128)
-        self.h2d = [self.new_k, self.new_v, self.q]
+        self.h2d = ["new_k", "new_v", "q"]
         self.d2h = [self.out]
         self.config = {"workload": "octave", "format": "k3v4", "head_size": 128, "rope_dim": 64,
                        "batch": B, "n_q_heads": Hq, "n_kv_heads": H, "ctx": ctx,
@@ -514,14 +515,26 @@ def time_steps(wl, steps, warmup, dist=None):
 
 def time_e2e(wl, steps, warmup):
     """The same step with its inputs copied host -> device from pinned memory
-    and its output copied back, inside the timed region."""
+    and its output copied back, inside the timed region.  The step's inputs
+    (the attributes named in wl.h2d) are moved into one device staging buffer
+    so that one copy per step brings all of them."""
     import torch
-    hin = [t.cpu().pin_memory() for t in wl.h2d]
+    dev = getattr(wl, wl.h2d[0]).device
+    sizes = [getattr(wl, n).numel() * getattr(wl, n).element_size() for n in wl.h2d]
+    offs = [sum((s + 255) // 256 * 256 for s in sizes[:i]) for i in range(len(sizes))]
+    total = offs[-1] + (sizes[-1] + 255) // 256 * 256
+    stage_d = torch.empty(total, dtype=torch.uint8, device=dev)
+    stage_h = torch.empty(total, dtype=torch.uint8).pin_memory()
+    for name, off, size in zip(wl.h2d, offs, sizes):
+        t = getattr(wl, name)
+        view = stage_d[off:off + size].view(t.dtype).view(t.shape)
+        view.copy_(t)
+        stage_h[off:off + size].copy_(view.view(torch.uint8).reshape(-1).cpu())
+        setattr(wl, name, view)
     hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in wl.d2h]
 
     def one(i):
-        for d, h in zip(wl.h2d, hin):
-            d.copy_(h, non_blocking=True)
+        stage_d.copy_(stage_h, non_blocking=True)
         wl.step(i)
         for d, h in zip(wl.d2h, hout):
             h.copy_(d, non_blocking=True)
@@ -536,7 +549,7 @@ def time_e2e(wl, steps, warmup):
         one(i)
     b.record(s)
     torch.cuda.synchronize()
-    h2d = sum(t.numel() * t.element_size() for t in hin)
+    h2d = sum(sizes)
     d2h = sum(t.numel() * t.element_size() for t in hout)
     return a.elapsed_time(b) / steps, h2d, d2h
 
