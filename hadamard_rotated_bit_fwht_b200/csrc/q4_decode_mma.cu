@@ -4,7 +4,7 @@
 //
 // With GQA the decode step is a small dense contraction per kv head:
 // S = Q_rot K^T (G x T) and O = P V (G x 256), G <= 8 heads per CTA.  One CTA
-// per SM (8 warps, ~200 KB of shared memory):
+// per SM (8 warps, ~170 KB of shared memory):
 //   * 128-token tiles of the split (codes and fp16 scales of K and V, 36 KB)
 //     stream into a ring of 4 stages, each guarded by a full mbarrier: code
 //     rows by TMA (2-D maps over the 128-byte rows, hardware 128-byte
@@ -13,9 +13,10 @@
 //     stage (a shared-memory counter per stage) issues its refill, so no warp
 //     is spent on producing and every warp keeps the full register budget.
 //     Every wait is bounded.
-//   * warp w owns tokens 16w .. 16w+15 of every tile and runs its own online
-//     softmax over them (no CTA-wide barrier per tile).  The 8 running states
-//     are merged once at the end of the split.
+//   * warp group gq = warp / 4 takes the tiles it with it % 2 == gq, warp
+//     wi = warp % 4 tokens 32 wi .. 32 wi + 31 of each, with its own online
+//     softmax (no CTA-wide barrier per tile).  The 8 running states are
+//     merged once at the end of the split.
 //   * QK on mma.sync m16n8k16 (f16 x f16 -> f32): A = the rotated query of the
 //     8 heads split exactly into fp16 hi (rows 0-7) and lo (rows 8-15), held in
 //     registers for the whole split; B = K codes of 8 tokens as the exact fp16
@@ -32,8 +33,9 @@
 //     removed at the end.
 //   * The QK accumulator layout (head g = lane / 4, tokens 2(lane % 4) + {0,1},
 //     + 8) is the PV B-fragment layout, so p never leaves registers.
-// Split-K partials (m, l, o[256]) per (sequence, q head, split) go to the
-// combine + back-rotation kernel (q4_decode.cu).
+// Split-K partials (m, l, o[256]) per (query row, q head, split) -- or, under
+// the balanced stream schedule, per (unit, CTA) segment -- go to the combine +
+// back-rotation kernel (q4_decode.cu).
 #include "decode_common.cuh"
 #include "q4_vec.cuh"
 

@@ -27,8 +27,9 @@
 //     exactly computed weight sums would turn that rounding into an error
 //     shared by all 32 dims of a block, which the back-rotation collects into
 //     single output dims, so the codes enter without bias.
-// Split-K partial records (m, l, o[256]) go to the Q4_0 path's combine and
-// back-rotation kernel.
+// The work schedule (one split per CTA, or the balanced stream schedule over
+// all units) is the Q4_0 kernel's; the partial records (m, l, o[256]) go to
+// the same combine and back-rotation kernel.
 #include "decode_common.cuh"
 #include "q4_vec.cuh"
 
