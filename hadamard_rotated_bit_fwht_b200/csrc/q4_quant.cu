@@ -19,7 +19,7 @@ constexpr int kVecPerCta = kWarps * kVecPerWarp;
 
 // ------------------------------------------------------------------ rotate
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads) rotate_kernel(const void *__restrict__ x,
+__global__ void __launch_bounds__(kThreads, 4) rotate_kernel(const void *__restrict__ x,
                                                           float *__restrict__ y, int64_t n_vec) {
   __shared__ float4 smem[kWarps][kVecPerWarp][64];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
