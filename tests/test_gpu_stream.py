@@ -159,3 +159,18 @@ def test_stream_multi_token(bits):
         lens = np.zeros(B, np.int32)
         lens[s] = q_lens[i]
         assert np.abs(got[i] - oc.decode_attn(qb, lens, 1 / 16)[s]).max() <= ATOL
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_chunked_fallback_many_rows(bits):
+    """More than 4096 (row, head group) units: fixed 2048-token chunks handed
+    out by the block scheduler."""
+    B, H, G, T = 4100, 1, 4, 256
+    lens = np.random.default_rng(750).integers(0, T + 1, B).astype(np.int32)
+    lens[:4] = [0, 1, 128, T]
+    gc, oc, _, _ = contiguous(751 + bits, B, H, T, bits)
+    q = synth.to_bf16_bits(synth.queries(752, B, H * G, 256))
+    got = kvq.decode_attn(gc, to_dev(q), to_dev(lens), T, 1 / 16).cpu().numpy()
+    want = oc.decode_attn(q, lens, 1 / 16)
+    assert np.abs(got - want).max() <= ATOL
+    assert not np.any(got[lens == 0])
