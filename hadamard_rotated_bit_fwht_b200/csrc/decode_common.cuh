@@ -71,6 +71,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
 // 1-D bulk copy of `bytes` bytes (a multiple of 16; both addresses 16-byte
 // aligned) onto the barrier's transaction count
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
@@ -277,12 +285,17 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // rows x row_bytes uint8 plane, boxes of box_rows rows x box_cols bytes (the
 // maps are cached per plane and box)
+// planes > 1: the rows are cut into `planes` column planes of box_cols bytes
+// (box_cols * planes == row_bytes), and one box brings box_rows rows of every
+// plane, laid out plane after plane (a 3-D map whose outer dimension steps
+// box_cols bytes along the row), the same shared-memory image as `planes`
+// 2-D boxes at consecutive column offsets
 inline bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t row_bytes,
-                     uint32_t box_cols, uint32_t box_rows, bool swizzle) {
+                     uint32_t box_cols, uint32_t box_rows, bool swizzle, uint32_t planes = 1) {
   struct Entry {
     const void *base;
     uint64_t rows;
-    uint32_t row_bytes, box_cols, box_rows;
+    uint32_t row_bytes, box_cols, box_rows, planes;
     CUtensorMap map;
   };
   static Entry cache[16];
@@ -291,22 +304,23 @@ inline bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint32_t r
   std::lock_guard<std::mutex> lock(mu);
   for (const Entry &e : cache)
     if (e.base == base && e.rows == rows && e.row_bytes == row_bytes && e.box_cols == box_cols &&
-        e.box_rows == box_rows) {
+        e.box_rows == box_rows && e.planes == planes) {
       *m = e.map;
       return true;
     }
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[2] = {row_bytes, rows};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_cols, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+  if (planes < 1 || (planes > 1 && box_cols * planes != row_bytes)) return false;
+  const cuuint64_t dims[3] = {planes > 1 ? box_cols : row_bytes, rows, planes};
+  const cuuint64_t strides[2] = {row_bytes, box_cols};
+  const cuuint32_t box[3] = {box_cols, box_rows, planes};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, planes > 1 ? 3 : 2, const_cast<void *>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return false;
-  cache[next] = Entry{base, rows, row_bytes, box_cols, box_rows, *m};
+  cache[next] = Entry{base, rows, row_bytes, box_cols, box_rows, planes, *m};
   next = (next + 1) % 16;
   return true;
 }

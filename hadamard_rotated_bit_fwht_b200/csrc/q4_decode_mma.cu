@@ -204,6 +204,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       #pragma unroll
       for (int i = 0; i < 8; i++) x[i] = 0.f;
     }
+    // the barriers are set up before the length is needed, so that this
+    // overlaps the length load; the previous segment is done with shared
+    // memory and its generic writes (the merge) precede the copies that
+    // will overwrite the ring (a dead CTA may still have copies in flight
+    // and leaves its barriers alone)
+    if (!dead) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncthreads();
+      if (tid == 0) {
+        #pragma unroll
+        for (int i = 0; i < kStages; i++) {
+          if (seg > 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(full0 + 8 * i) : "memory");
+          mbar_init(full0 + 8 * i, 1);
+          rel[i] = 0;
+        }
+        *abort_flag = 0;
+        *issued = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      __syncthreads();
+    }
     const int ntiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
     if (ntiles == 0) continue;  // a split past the length writes no record
     if (dead) {
@@ -214,23 +236,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       continue;
     }
-    // the previous segment is done with shared memory; its generic writes
-    // (the merge) precede the copies that will overwrite the ring
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-    if (tid == 0) {
-      #pragma unroll
-      for (int i = 0; i < kStages; i++) {
-        if (seg > 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(full0 + 8 * i) : "memory");
-        mbar_init(full0 + 8 * i, 1);
-        rel[i] = 0;
-      }
-      *abort_flag = 0;
-      *issued = 0;
-      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
-    __syncthreads();
     // fused step: every CTA whose split holds the new token quantizes the
     // token's K and V rows of its kv head into the cache before it issues a tile
     // load (CTAs of the same kv head write identical bytes)

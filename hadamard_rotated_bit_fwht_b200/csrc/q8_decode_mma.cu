@@ -49,9 +49,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kQRange = 2080768.f;  // 127 * 2^14
 constexpr uint32_t kMagicBits = 0x4B400000u;  // bits of 1.5 * 2^23
 constexpr float kMagic = 12582912.f;
-// stage: K codes as two 64-row x 128-byte boxes (dims 0-127, 128-255; 128B
-// swizzle), V codes likewise, then K and V scale rows (64 x 16 bytes, 1-D bulk
-// copies)
+// stage: K codes as two 64-row x 128-byte planes (dims 0-127, 128-255; 128B
+// swizzle) brought by one 3-D box, V codes likewise, then K and V scale rows
+// (64 x 16 bytes, 1-D bulk copies)
 constexpr int kBox = kTile * 128;
 constexpr int kOffKC = 0;
 constexpr int kOffVC = kOffKC + 2 * kBox;
@@ -221,6 +221,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       #pragma unroll
       for (int i = 0; i < 8; i++) x[i] = 0.f;
     }
+    // the barriers are set up before the length is needed, so that this
+    // overlaps the length load; the previous segment is done with shared
+    // memory and its generic writes (the merge) precede the copies that
+    // will overwrite the ring (a dead CTA may still have copies in flight
+    // and leaves its barriers alone)
+    if (!dead) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncthreads();
+      if (tid == 0) {
+        #pragma unroll
+        for (int i = 0; i < kStages; i++) {
+          if (seg > 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(full0 + 8 * i) : "memory");
+          mbar_init(full0 + 8 * i, 1);
+          rel[i] = 0;
+        }
+        *abort_flag = 0;
+        *issued = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      __syncthreads();
+    }
     const int ntiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
     if (ntiles == 0) continue;  // a split past the length writes no record
     if (dead) {
@@ -231,23 +253,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       continue;
     }
-    // the previous segment is done with shared memory; its generic writes
-    // (the merge) precede the copies that will overwrite the ring
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-    if (tid == 0) {
-      #pragma unroll
-      for (int i = 0; i < kStages; i++) {
-        if (seg > 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(full0 + 8 * i) : "memory");
-        mbar_init(full0 + 8 * i, 1);
-        rel[i] = 0;
-      }
-      *abort_flag = 0;
-      *issued = 0;
-      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
-    __syncthreads();
     const bool appender = p_new >= t0 && p_new < t1;
 
     // first cache row of the 64-token tile starting at token t, -1 if unmapped
@@ -270,10 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nrows = c.block_table ? kTile : min(kTile, c.max_tokens - (t0 + it * kTile));
         mbar_arrive_tx(bar, 4 * kBox + 2 * nrows * 16);
         const uint32_t dst = smem_u32(smem + st * kStageBytes);
-        tma_load_2d(dst + kOffKC, &maps.kc, 0, r, bar);
-        tma_load_2d(dst + kOffKC + kBox, &maps.kc, 128, r, bar);
-        tma_load_2d(dst + kOffVC, &maps.vc, 0, r, bar);
-        tma_load_2d(dst + kOffVC + kBox, &maps.vc, 128, r, bar);
+        tma_load_3d(dst + kOffKC, &maps.kc, 0, r, 0, bar);
+        tma_load_3d(dst + kOffVC, &maps.vc, 0, r, 0, bar);
         bulk_load(dst + kOffKS, c.k_scales + (int64_t)r * kRowScales, nrows * 16, bar);
         bulk_load(dst + kOffVS, c.v_scales + (int64_t)r * kRowScales, nrows * 16, bar);
       }
@@ -608,8 +611,8 @@ cudaError_t launch_q8_decode_mma(const kvq_cache &c, const void *q, int bf16, in
                             : (uint64_t)c.batch_capacity * c.num_kv_heads * c.max_tokens;
   if (rows >= (1ull << 31)) return cudaErrorInvalidValue;  // TMA row coordinates are 32-bit
   TmaMaps maps;
-  if (!make_map(&maps.kc, c.k_codes, rows, kCodeRow, 128, kTile, true) ||
-      !make_map(&maps.vc, c.v_codes, rows, kCodeRow, 128, kTile, true))
+  if (!make_map(&maps.kc, c.k_codes, rows, kCodeRow, 128, kTile, true, 2) ||
+      !make_map(&maps.vc, c.v_codes, rows, kCodeRow, 128, kTile, true, 2))
     return cudaErrorInvalidValue;
   maps.kc2 = maps.kc;  // a 64-token tile is one box already
   maps.vc2 = maps.vc;
