@@ -47,10 +47,12 @@ __device__ __forceinline__ float sign_of(const OctaveParams &P, int d) {
   return ((P.sign_words[d >> 5] >> (d & 31)) & 1u) ? -1.f : 1.f;
 }
 
-// one cross-lane butterfly stage on lane-index bit h
-__device__ __forceinline__ float xstage(float v, int lane, int h) {
+// one cross-lane butterfly stage on lane-index bit h: v + o on the lower lane,
+// o - v on the upper one, as one FMA with sg = +-1 (sg * v is exact, so the
+// FMA rounds the same sum once)
+__device__ __forceinline__ float xstage(float v, float sg, int h) {
   const float o = __shfl_xor_sync(kFull, v, h);
-  return (lane & h) ? __fsub_rn(o, v) : __fadd_rn(v, o);
+  return __fmaf_rn(sg, v, o);
 }
 
 // sum over the 32 lanes of one value per lane, pairs (i, i + 16), (i, i + 8), ...
@@ -91,8 +93,9 @@ __device__ __forceinline__ float quantize_lut(const float (&x)[NV], float mult, 
   if (NV == 4) ss = __fadd_rn(__fadd_rn(sq[0], sq[2]), __fadd_rn(sq[1], sq[3]));
   else ss = __fadd_rn(sq[0], sq[1]);
   ss = xsum(ss);
-  const float n = (float)(NV * 32);
-  float rms = __fsqrt_rn(__fdiv_rn(ss, n));
+  // ss / n for n = 64, 128: the product with the exact 1 / n is the same
+  // real number, so it rounds the same
+  float rms = __fsqrt_rn(__fmul_rn(ss, 1.f / (float)(NV * 32)));
   rms = rms < 1e-12f ? 1e-12f : rms;
   float pr[NV];
 #pragma unroll
@@ -133,9 +136,10 @@ __device__ __forceinline__ uint32_t pack_word(const uint32_t *c32, int n, int bi
          (((v.z >> 2) & 0x01010101u) << 6) | (((v.w >> 2) & 0x01010101u) << 7);
 }
 
+template <bool BF16>
 __global__ void __launch_bounds__(kThreads)
     octave_quantize_kernel(OctaveParams P, const void *__restrict__ key,
-                           const void *__restrict__ value, int bf16, int num_tokens,
+                           const void *__restrict__ value, int num_tokens,
                            int n_kv_heads, const int64_t *__restrict__ slot_mapping,
                            uint8_t *__restrict__ cache, int block_size, int64_t num_blocks) {
   __shared__ LutSmem L;
@@ -155,9 +159,23 @@ __global__ void __launch_bounds__(kThreads)
   const int w_kn = P.off_k_nope / 4, w_v = P.off_v / 4, w_sc = P.off_scales / 4;
   const uint32_t *kc32 = reinterpret_cast<const uint32_t *>(kcodes[warp]);
   const uint32_t *vc32 = reinterpret_cast<const uint32_t *>(vcodes[warp]);
+  float sg[4];  // signs of dims lane + 32k (K and V share them)
+#pragma unroll
+  for (int k = 0; k < 4; k++) sg[k] = sign_of(P, lane + 32 * k);
+  float bsg[5];  // butterfly signs of stages h = 1 .. 16
+#pragma unroll
+  for (int i = 0; i < 5; i++) bsg[i] = (lane >> i) & 1 ? -1.f : 1.f;
+  const bool idx32 = items <= 0x7fffffff;  // 32-bit index arithmetic suffices
   for (int64_t it = (int64_t)blockIdx.x * kWarps + warp; it < items;
        it += (int64_t)gridDim.x * kWarps) {
-    const int tok = (int)(it / n_kv_heads), h = (int)(it % n_kv_heads);
+    int tok, h;
+    if (idx32) {
+      tok = (int)it / n_kv_heads;
+      h = (int)it - tok * n_kv_heads;
+    } else {
+      tok = (int)(it / n_kv_heads);
+      h = (int)(it - (int64_t)tok * n_kv_heads);
+    }
     const int64_t base = it * kHead;
     // ---- K: 64-dim blocks (4-bit RoPE dims, 3-bit others) or, compact, one
     // whole-head rotation with 3-bit codes and one scale
@@ -165,12 +183,12 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int k = 0; k < 4; k++) {
       const int d = lane + 32 * k;
-      x[k] = __fmul_rn(load_in(key, bf16, base + d), sign_of(P, d));
+      x[k] = __fmul_rn(load_in(key, BF16, base + d), sg[k]);
     }
 #pragma unroll
-    for (int hh = 1; hh < 32; hh <<= 1)
+    for (int i = 0; i < 5; i++)
 #pragma unroll
-      for (int k = 0; k < 4; k++) x[k] = xstage(x[k], lane, hh);
+      for (int k = 0; k < 4; k++) x[k] = xstage(x[k], bsg[i], 1 << i);
     {  // h = 32 inside each 64-block: (l, l+32), (l+64, l+96)
       float a = x[0], b = x[1];
       x[0] = __fadd_rn(a, b);
@@ -213,12 +231,12 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int k = 0; k < 4; k++) {
       const int d = lane + 32 * k;
-      x[k] = __fmul_rn(load_in(value, bf16, base + d), sign_of(P, d));
+      x[k] = __fmul_rn(load_in(value, BF16, base + d), sg[k]);
     }
 #pragma unroll
-    for (int hh = 1; hh < 32; hh <<= 1)
+    for (int i = 0; i < 5; i++)
 #pragma unroll
-      for (int k = 0; k < 4; k++) x[k] = xstage(x[k], lane, hh);
+      for (int k = 0; k < 4; k++) x[k] = xstage(x[k], bsg[i], 1 << i);
     {
       float a = x[0], b = x[1];  // h = 32
       x[0] = __fadd_rn(a, b);
@@ -248,16 +266,27 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t sm = __ldg(slot_mapping + tok);
     uint32_t *dst = nullptr;
     if (sm >= 0) {
-      const int64_t blk = sm / block_size, off = sm % block_size;
+      int64_t blk, off;
+      if (sm <= 0x7fffffff) {
+        blk = (int)sm / block_size;
+        off = (int)sm - (int)blk * block_size;
+      } else {
+        blk = sm / block_size;
+        off = sm - blk * block_size;
+      }
       if (blk < num_blocks)
         dst = reinterpret_cast<uint32_t *>(cache +
                                            ((blk * n_kv_heads + h) * block_size + off) * P.slot_bytes);
     }
     for (int w = lane; w < slot_words; w += 32) {
       uint32_t word = 0;
-      if (w < w_kn) word = pack_word(kc32, P.rope_dim, 4, w);
-      else if (w < w_v) word = pack_word(kc32 + P.rope_dim / 4, kHead - P.rope_dim, 3, w - w_kn);
-      else if (w < w_sc) word = pack_word(vc32, kHead, P.v_bits, w - w_v);
+      // the 4-bit regions (K RoPE dims, 4-bit V) share one path, as do the
+      // 3-bit ones, so that the warp runs each packing once
+      const bool kr = w < w_kn, vr = w >= w_v && w < w_sc;
+      if (kr || (vr && P.v_bits == 4)) word = pack_word(kr ? kc32 : vc32, 0, 4, kr ? w : w - w_v);
+      else if (w < w_sc)
+        word = vr ? pack_word(vc32, kHead, 3, w - w_v)
+                  : pack_word(kc32 + P.rope_dim / 4, kHead - P.rope_dim, 3, w - w_kn);
       else if (w == w_sc)  // fp16 scales, K first then V
         word = (uint32_t)__half_as_ushort(__float2half_rn(ks[0])) |
                ((uint32_t)__half_as_ushort(__float2half_rn(P.compact ? vs : ks[1])) << 16);
@@ -477,10 +506,25 @@ cudaError_t launch_octave_quantize(const OctaveParams &p, const void *key, const
                                    int block_size, int64_t num_blocks, cudaStream_t s) {
   const int64_t items = (int64_t)num_tokens * n_kv_heads;
   if (items == 0) return cudaSuccess;
-  int64_t blocks = (items + kWarps - 1) / kWarps;
-  const int grid = (int)(blocks < kNumSMs * 16 ? blocks : kNumSMs * 16);
-  octave_quantize_kernel<<<grid, kThreads, 0, s>>>(p, key, value, bf16, num_tokens, n_kv_heads,
-                                                  slot_mapping, cache, block_size, num_blocks);
+  // one wave of resident CTAs, each warp striding over the (token, head) items
+  static int resident[2] = {0, 0};
+  int &per_sm = resident[bf16 ? 1 : 0];
+  if (per_sm == 0) {
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &n, bf16 ? octave_quantize_kernel<true> : octave_quantize_kernel<false>, kThreads, 0);
+    if (e != cudaSuccess) return e;
+    per_sm = n > 0 ? n : 1;
+  }
+  const int64_t blocks = (items + kWarps - 1) / kWarps;
+  const int64_t wave = (int64_t)kNumSMs * per_sm;
+  const int grid = (int)(blocks < wave ? blocks : wave);
+  if (bf16)
+    octave_quantize_kernel<true><<<grid, kThreads, 0, s>>>(p, key, value, num_tokens, n_kv_heads,
+                                                          slot_mapping, cache, block_size, num_blocks);
+  else
+    octave_quantize_kernel<false><<<grid, kThreads, 0, s>>>(p, key, value, num_tokens, n_kv_heads,
+                                                           slot_mapping, cache, block_size, num_blocks);
   return cudaGetLastError();
 }
 
