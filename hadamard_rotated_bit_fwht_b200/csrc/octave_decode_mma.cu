@@ -252,16 +252,19 @@ __global__ void __launch_bounds__(kThreads, 4)
 
   // ---- loader: thread tid copies chunks 4 (tid & 1) .. + 3 of row tid / 2
   const int lr = tid >> 1, lc0 = 4 * (tid & 1);
+  // block index of a token: a shift for power-of-two block sizes
+  const int bs_shift = (block_size & (block_size - 1)) == 0 ? __ffs(block_size) - 1 : -1;
   auto issue = [&](int it) {
     uint8_t *st = smem + (it % kStages) * kStageBytes;
     const int t = t0 + it * kTile + lr;
     bool ok = t < t1;
     const uint8_t *src = cache;
     if (ok) {
-      const int blk = __ldg(block_table + (int64_t)req * max_blocks + t / block_size);
+      const int bi = bs_shift >= 0 ? t >> bs_shift : t / block_size;
+      const int blk = __ldg(block_table + (int64_t)req * max_blocks + bi);
       ok = blk >= 0 && blk < num_blocks;
       if (ok)
-        src = cache + (((int64_t)blk * n_kv_heads + kvh) * block_size + (t % block_size)) *
+        src = cache + (((int64_t)blk * n_kv_heads + kvh) * block_size + (t - bi * block_size)) *
                           P.slot_bytes;
     }
     if (lc0 == 0) smem[kOffV + (it % kStages) * kTile + lr] = ok ? 1 : 0;

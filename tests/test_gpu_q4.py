@@ -306,3 +306,81 @@ def test_long_decode_full_size_sampled():
     compare_cache(gc, oc, rows=rng.choice(B * H * T, 4096, replace=False))
     want = oc.decode_attn(q, [T], 1 / 16)
     assert np.abs(got - want).max() <= ATOL
+
+
+def test_quantize_workload_full_size():
+    """Quantize-on-append workload at full size (8 sequences x 8 kv heads,
+    bf16): a 4096-token prefill, then 256 single-token appends, as the
+    benchmark drives them; every code and scale row bit-identical to the
+    oracle quantising all 4352 tokens at once."""
+    W = synth.WORKLOADS["quantize"]
+    B, H, P, A, cap = W["batch"], W["n_kv_heads"], W["prefill"], W["appends"], W["capacity"]
+    k, v = synth.kv_tokens(W["seed"], B, P + A, H, 256, W["outlier_frac"], W["outlier_factor"])
+    kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+    del k, v
+    gc = kvq.Q4Cache.contiguous(B, H, cap)
+    kvq.quantize_append(gc, to_dev(kb[:, :P]), to_dev(vb[:, :P]), to_dev(np.zeros(B, np.int32)))
+    for i in range(A):
+        kvq.quantize_append(gc, to_dev(kb[:, P + i:P + i + 1]), to_dev(vb[:, P + i:P + i + 1]),
+                            to_dev(np.full(B, P + i, np.int32)))
+    oc = oracle.Q4Cache(B * H * cap, H, max_tokens=cap)
+    oc.append(kb, vb, np.zeros(B, np.int32))
+    torch.cuda.synchronize()
+    compare_cache(gc, oc)
+
+
+def test_paged_decode_full_size_sampled():
+    """Batched paged workload at full size (32 sequences of U[8192, 32768]
+    tokens, 16 q / 2 kv heads, 256-token shuffled pages, bf16) in the launch
+    configuration the benchmark times (the balanced stream schedule over all
+    64 units): for four sampled sequences (the longest, the shortest, two
+    random ones) every output row within 2e-3 of the oracle and every cache
+    row bit-identical."""
+    W = synth.WORKLOADS["paged_decode"]
+    B, H, Hq, ps = W["batch"], W["n_kv_heads"], W["n_q_heads"], W["page_size"]
+    lens = synth.seq_lens(W["seed"], B, W["ctx_lo"], W["ctx_hi"])
+    npp = (lens + ps - 1) // ps
+    bt, n_pages = synth.page_table(W["seed"], B, npp, int(npp.max()))
+    gc = kvq.Q4Cache.paged(n_pages, H, ps, torch.from_numpy(bt))
+    rng = np.random.default_rng(11)
+    pick = sorted({int(np.argmax(lens)), int(np.argmin(lens))} |
+                  set(rng.choice(B, 2, replace=False).tolist()))
+    kept = {}
+    for b0 in range(0, B, 8):  # the benchmark's generation: 8 sequences at a time
+        Lc = int(lens[b0:b0 + 8].max())
+        k, v = synth.kv_tokens(W["seed"] * 100 + b0, 8, Lc, H, 256, W["outlier_frac"],
+                               W["outlier_factor"])
+        kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+        del k, v
+        for j in range(8):
+            b, L = b0 + j, int(lens[b0 + j])
+            kvq.quantize_append(gc.with_block_table(torch.from_numpy(bt[b:b + 1])),
+                                to_dev(kb[j:j + 1, :L]), to_dev(vb[j:j + 1, :L]),
+                                to_dev(np.zeros(1, np.int32)))
+            if b in pick:
+                kept[b] = (kb[j:j + 1, :L].copy(), vb[j:j + 1, :L].copy())
+        del kb, vb
+    q = synth.to_bf16_bits(synth.queries(W["seed"], B, Hq, 256))
+    got = kvq.decode_attn(gc, to_dev(q), to_dev(lens), int(lens.max()), 1 / 16).cpu().numpy()
+    # the oracle holds the sampled sequences only, on consecutive pages of its own
+    cbt = np.full((len(pick), bt.shape[1]), -1, np.int32)
+    o = 0
+    for i, b in enumerate(pick):
+        cbt[i, :npp[b]] = np.arange(o, o + npp[b])
+        o += int(npp[b])
+    oc = oracle.Q4Cache(o * H * ps, H, block_table=cbt, page_size=ps)
+    for i, b in enumerate(pick):
+        oc.with_block_table(cbt[i:i + 1]).append(kept[b][0], kept[b][1], np.zeros(1, np.int32))
+    want = oc.decode_attn(q[pick], lens[pick], 1 / 16)
+    assert np.abs(got[pick] - want).max() <= ATOL
+    for name in ("k_codes", "v_codes", "k_scales", "v_scales"):
+        g = getattr(gc, name).cpu().numpy()
+        if name.endswith("scales"):
+            g = g.view(np.uint16)
+        for i, b in enumerate(pick):
+            t = np.arange(int(lens[b]))
+            hs = np.arange(H)
+            rg = ((bt[b, t // ps][:, None] * H + hs) * ps + (t % ps)[:, None]).ravel()
+            ro = ((cbt[i, t // ps][:, None] * H + hs) * ps + (t % ps)[:, None]).ravel()
+            bad = np.nonzero(np.any(g[rg] != getattr(oc, name)[ro], axis=-1))[0]
+            assert bad.size == 0, f"{name}, sequence {b}: {bad.size} rows differ"
