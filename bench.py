@@ -50,22 +50,38 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
-def kernel_source_hash():
+# the sources that decide each captured kernel's code and launch shape
+_COMMON = ["kvq_internal.cuh", "kvq_api.cu"]
+_DECODE = _COMMON + ["decode_common.cuh", "q4_vec.cuh", "q4_decode.cu"]
+TRAFFIC_SOURCES = {
+    "q4_decode_long": _DECODE + ["q4_decode_mma.cu"],
+    "q4_decode_paged": _DECODE + ["q4_decode_mma.cu"],
+    "q8_decode_long": _DECODE + ["q8_decode_mma.cu"],
+    "q4_decode_combine": _DECODE,
+    "q4_append_prefill": _COMMON + ["q4_vec.cuh", "q4_quant.cu"],
+    "octave_decode": _COMMON + ["octave.cu", "octave_decode_mma.cu"],
+    "octave_quantize": _COMMON + ["octave.cu"],
+}
+
+
+def kernel_source_hash(key: str) -> str:
+    """Hash of the CUDA sources behind one traffic entry."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hadamard_rotated_bit_fwht_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(set(TRAFFIC_SOURCES[key])):
+        h.update(f.encode() + b"\0")
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(key: str):
-    """DRAM bytes per call from a committed ncu capture, only if the kernel
+    """DRAM bytes per call from a committed ncu capture, only if the kernel's
     sources are unchanged since it was taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
+    if not os.path.exists(p) or key not in TRAFFIC_SOURCES:
         return None
     e = json.load(open(p)).get(key)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(key):
         return None
     return e.get("bytes_per_call")
 
