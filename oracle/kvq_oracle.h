@@ -1,6 +1,7 @@
 /*
  * kvq_oracle.h -- plain single-threaded CPU oracle for the Hadamard-rotated
- * low-bit KV cache (FWHT-256 + Q4_0, and the Octave block-Hadamard variant).
+ * low-bit KV cache (FWHT-256 + Q4_0, its Q8_0 counterpart, and the Octave
+ * block-Hadamard variant).
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may include, link or
  * call this library: only tests/, __graft_entry__.smoke() and the bench's
