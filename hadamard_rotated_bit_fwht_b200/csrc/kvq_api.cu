@@ -184,10 +184,14 @@ size_t kvq_decode_attn_workspace(const kvq_cache *cache, int32_t batch, int32_t 
   return decode_workspace_bytes(batch, num_q_heads, p);
 }
 
-kvq_status kvq_decode_attn(const kvq_cache *cache, const void *q, kvq_dtype dtype, int32_t batch,
-                           int32_t num_q_heads, const int32_t *d_seq_lens, int32_t max_seq_len,
-                           float scale, float *out, void *workspace, size_t workspace_bytes,
-                           void *stream) {
+}  // extern "C"
+
+// Every argument check of kvq_decode_attn except the workspace ones, in the
+// same order; shared with the allocation-free variant so both report the same
+// status for the same bad argument.
+kvq_status kvq::check_decode_args(const kvq_cache *cache, const void *q, kvq_dtype dtype,
+                                  int32_t batch, int32_t num_q_heads, const int32_t *d_seq_lens,
+                                  int32_t max_seq_len, float scale, const float *out) {
   kvq_status st = check_cache(cache);
   if (st != KVQ_OK) return st;
   if (batch < 0 || num_q_heads <= 0 || max_seq_len < 0 || (dtype != KVQ_F32 && dtype != KVQ_BF16))
@@ -199,6 +203,18 @@ kvq_status kvq_decode_attn(const kvq_cache *cache, const void *q, kvq_dtype dtyp
   if (!isfinite(scale)) return KVQ_ERR_INVALID_ARG;
   if (batch == 0) return KVQ_OK;
   if (!q || !d_seq_lens || !out || !aligned(q, 16) || !aligned(out, 16)) return KVQ_ERR_INVALID_ARG;
+  return KVQ_OK;
+}
+
+extern "C" {
+
+kvq_status kvq_decode_attn(const kvq_cache *cache, const void *q, kvq_dtype dtype, int32_t batch,
+                           int32_t num_q_heads, const int32_t *d_seq_lens, int32_t max_seq_len,
+                           float scale, float *out, void *workspace, size_t workspace_bytes,
+                           void *stream) {
+  kvq_status st = check_decode_args(cache, q, dtype, batch, num_q_heads, d_seq_lens, max_seq_len,
+                                    scale, out);
+  if (st != KVQ_OK || batch == 0) return st;
   DecodePlan p = plan_decode(batch, head_groups(num_q_heads, cache->num_kv_heads), max_seq_len,
                              decode_tile(cache));
   const size_t need = decode_workspace_bytes(batch, num_q_heads, p);

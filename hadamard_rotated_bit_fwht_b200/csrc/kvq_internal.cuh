@@ -119,6 +119,10 @@ cudaError_t launch_q8_decode_mma(const kvq_cache &c, const void *q, int bf16, in
                                  const int32_t *pos = nullptr, const int32_t *q_to_seq = nullptr,
                                  int num_seqs = 0);
 size_t decode_workspace_bytes(int batch, int n_q_heads, const DecodePlan &p);
+// host: the argument checks of kvq_decode_attn that precede its workspace checks
+kvq_status check_decode_args(const kvq_cache *cache, const void *q, kvq_dtype dtype,
+                             int32_t batch, int32_t num_q_heads, const int32_t *d_seq_lens,
+                             int32_t max_seq_len, float scale, const float *out);
 cudaError_t launch_q4_decode(const kvq_cache &c, const void *q, int bf16, int batch,
                              int n_q_heads, const int32_t *seq_lens, int max_seq_len,
                              float scale, float *out, float *ws, const DecodePlan &p,

@@ -13,7 +13,10 @@
 // device address is looked up once per device (cudaGetSymbolAddress) on the
 // first call made with that device current; host code never passes the
 // variable itself to a kernel, since in host code the name is only a host-side
-// stand-in for the device symbol.
+// stand-in for the device symbol.  The cached address belongs to the device's
+// primary context: after cudaDeviceReset the module is loaded again and the
+// address may change, so this entry point must not be used on a device after
+// that device has been reset in the same process.
 #include <mutex>
 
 #include "kvq_internal.cuh"
@@ -50,17 +53,16 @@ KVQ_API kvq_status kvq_decode_attn_noalloc(const kvq_cache *cache, const void *q
                                            int32_t num_q_heads, const int32_t *d_seq_lens,
                                            int32_t max_seq_len, float scale, float *out,
                                            void *stream) {
-  // Same host-side checks as kvq_decode_attn; the scratch size replaces the
-  // caller's workspace size.
-  if (cache == nullptr || batch < 0 || num_q_heads <= 0 || max_seq_len < 0)
-    return KVQ_ERR_INVALID_ARG;
+  // The argument checks of kvq_decode_attn come first, so a bad argument gets
+  // the status kvq_decode_attn would give it; only a valid shape whose
+  // workspace exceeds the array gets KVQ_ERR_WORKSPACE.
+  const kvq_status st = kvq::check_decode_args(cache, q, dtype, batch, num_q_heads, d_seq_lens,
+                                               max_seq_len, scale, out);
+  if (st != KVQ_OK || batch == 0) return st;
   const size_t need = kvq_decode_attn_workspace(cache, batch, num_q_heads, max_seq_len);
-  if (batch > 0 && need > kNoAllocScratchBytes) return KVQ_ERR_WORKSPACE;
-  float *ws = nullptr;
-  if (batch > 0) {
-    ws = scratch_for_current_device();
-    if (ws == nullptr) return KVQ_ERR_CUDA;
-  }
+  if (need > kNoAllocScratchBytes) return KVQ_ERR_WORKSPACE;
+  float *ws = scratch_for_current_device();
+  if (ws == nullptr) return KVQ_ERR_CUDA;
   return kvq_decode_attn(cache, q, dtype, batch, num_q_heads, d_seq_lens, max_seq_len, scale,
                          out, ws, kNoAllocScratchBytes, stream);
 }

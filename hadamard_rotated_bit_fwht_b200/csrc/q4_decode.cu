@@ -232,7 +232,7 @@ DecodePlan plan_decode(int batch, int n_head_groups, int max_seq_len, int tile) 
   p.splits = max((max(max_seq_len, 1) + p.split_tokens - 1) / p.split_tokens, 1);
   while (p.splits > kMaxSplitsSmem) {
     p.split_tokens *= 2;
-    p.splits = (max_seq_len + p.split_tokens - 1) / p.split_tokens;
+    p.splits = (max(max_seq_len, 1) + p.split_tokens - 1) / p.split_tokens;
   }
   return p;
 }

@@ -20,6 +20,9 @@ LIB_PATH = os.path.join(_PKG, "libkvq.so")
 
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA = range(5)
 KVQ_F32, KVQ_BF16 = 0, 1
+# bytes of the fixed scratch array behind kvq_decode_attn_noalloc
+# (KVQ_DECODE_NOALLOC_SCRATCH_BYTES in include/kvq.h)
+KVQ_DECODE_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 EXPORTED = (
     "kvq_status_string", "kvq_version", "kvq_rotate", "kvq_quantize_append",

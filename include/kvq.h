@@ -236,13 +236,17 @@ KVQ_API kvq_status kvq_decode_step(const kvq_cache *cache, const void *k_new, co
  * allocates nothing: its split-K partials live in a fixed device array inside
  * the library, KVQ_DECODE_NOALLOC_SCRATCH_BYTES large, which every GPU that
  * loads the library holds until the process exits.
- *   Arguments, layouts and results are those of kvq_decode_attn.
- *   A shape whose workspace (kvq_decode_attn_workspace) exceeds
- *   KVQ_DECODE_NOALLOC_SCRATCH_BYTES returns KVQ_ERR_WORKSPACE before any
- *   launch; use kvq_decode_attn with a workspace for such shapes.
+ *   Arguments, layouts and results are those of kvq_decode_attn, and so are
+ *   the argument checks and their order: a bad argument returns the status
+ *   kvq_decode_attn would return for it.  A valid shape whose workspace
+ *   (kvq_decode_attn_workspace) exceeds KVQ_DECODE_NOALLOC_SCRATCH_BYTES
+ *   returns KVQ_ERR_WORKSPACE before any launch; use kvq_decode_attn with a
+ *   workspace for such shapes.
  *   The first call on a device looks up the array's device address with that
  *   device current (KVQ_ERR_CUDA if the lookup fails); make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is kept for the life of the
+ *   process: after cudaDeviceReset on a device, do not call this entry point
+ *   on that device again.
  *   All calls on a device share the one array: every call overwrites the
  *   records it reads, so nothing carries over from the previous call, but two
  *   calls whose kernels overlap on the GPU (different streams, no ordering

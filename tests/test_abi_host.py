@@ -111,3 +111,26 @@ def test_sign_words_marshalling():
     w = kvq.sign_words(s)
     assert w.dtype == np.int32 and w.shape == (4,)
     assert w[0] == 1 and w[1] == 2 and w[3] == np.int32(np.uint32(1 << 31).view(np.int32))
+
+
+def test_noalloc_checks_arguments_before_its_size(L):
+    hdr = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    m = re.search(r"#define KVQ_DECODE_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", hdr)
+    assert m and int(m.group(1)) << int(m.group(2)) == kvq.KVQ_DECODE_NOALLOC_SCRATCH_BYTES
+    buf = (C.c_uint8 * 4096)()
+    p16 = (C.addressof(buf) + 15) // 16 * 16
+    # 108 sequences x 8 kv heads, 64 q heads (group 8): valid, but its stream-
+    # schedule workspace is above the fixed array -> refused before any launch
+    d = kvq.CacheDesc(p16, p16, p16, p16, 8, 256, 64, 108, None, 0, 0, 0)
+    assert L.kvq_decode_attn_workspace(C.byref(d), 108, 64, 64) > kvq.KVQ_DECODE_NOALLOC_SCRATCH_BYTES
+
+    def call(dtype=1, hq=64, q=p16, batch=108):
+        return L.kvq_decode_attn_noalloc(C.byref(d), q, dtype, batch, hq, p16, 64, C.c_float(0.1),
+                                         p16, None)
+
+    assert call() == kvq.KVQ_ERR_WORKSPACE
+    assert call(dtype=7) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(q=None) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(hq=8 * 32) == kvq.KVQ_ERR_UNSUPPORTED
+    assert call(batch=109) == kvq.KVQ_ERR_INVALID_ARG  # above the contiguous capacity
+    assert call(batch=0) == kvq.KVQ_OK
