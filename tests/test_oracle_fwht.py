@@ -102,6 +102,41 @@ def test_f16_converter_against_numpy():
     assert np.array_equal(got, want)
 
 
+def test_f16_converter_exhaustive():
+    """Every one of the 2^32 fp32 bit patterns converts exactly as numpy's
+    round-to-nearest-even binary16 conversion does (NaN payloads excepted:
+    non-finite input is outside the quantizers' contract).  Chunks of 2^24
+    patterns run on all host cores (numpy's cast and the ctypes call release
+    the GIL)."""
+    import ctypes as C
+    from concurrent.futures import ThreadPoolExecutor
+
+    L = oracle.lib()
+    n = 1 << 24
+
+    def sweep(chunks):
+        base = np.arange(n, dtype=np.uint32)
+        u = np.empty(n, np.uint32)
+        want = np.empty(n, np.float16)
+        got = np.empty(n, np.uint16)
+        f = u.view(np.float32)
+        bad = 0
+        with np.errstate(over="ignore", invalid="ignore"):
+            for c in chunks:
+                np.add(base, np.uint32(c * n), out=u)
+                np.copyto(want, f, casting="unsafe")
+                L.orc_f32_to_f16_array(f.ctypes.data_as(C.c_void_p),
+                                       got.ctypes.data_as(C.c_void_p), C.c_int64(n))
+                diff = want.view(np.uint16) != got
+                if diff.any():
+                    bad += int((diff & ~np.isnan(f)).sum())
+        return bad
+
+    k = os.cpu_count() or 1
+    with ThreadPoolExecutor(k) as ex:
+        assert sum(ex.map(sweep, [range(i, 256, k) for i in range(k)])) == 0
+
+
 def test_f16_roundtrip_exact():
     h = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
     h = h[np.isfinite(h.view(np.float16))]

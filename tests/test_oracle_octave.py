@@ -176,3 +176,130 @@ def test_attention_bruteforce():
             p = np.exp(sc - sc.max())
             p /= p.sum()
             np.testing.assert_allclose(got[i, h], p @ V[:, g], atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Hand-derived goldens for _quantize_lut and for the slot assembly of
+# reference_quantize, and planted misreadings that each of them catches.
+# ---------------------------------------------------------------------------
+LUT_GOLD = json.load(open(os.path.join(GOLD, "octave_quantize_lut.json")))
+SLOT_GOLD = json.load(open(os.path.join(GOLD, "octave_slot_k3v4.json")))
+
+
+def _bits32(v):
+    return "0x%08x" % int(np.float32(v).view(np.uint32))
+
+
+def test_lut_golden_inputs_are_the_codebook():
+    for bits in (3, 4):
+        lut, mult = oracle.octave_codebook(bits)
+        assert lut.tolist() == LUT_GOLD["inputs"][f"lut{bits}"]
+        assert _bits32(mult) == LUT_GOLD["inputs"][f"lut_mult{bits}_bits"]
+
+
+def _check_lut_case(qlut, f16, case):
+    x = np.array([np.uint32(int(b, 16)).view(np.float32) for b in case["x_bits"]], np.float32)
+    codes, scale = qlut(x, case["bits"])
+    assert list(codes) == case["codes"], "codes"
+    assert _bits32(scale) == case["scale_f32_bits"], "fp32 scale"
+    assert "0x%04x" % f16(scale) == case["scale_f16_bits"], "fp16 scale"
+
+
+@pytest.mark.parametrize("case", LUT_GOLD["cases"], ids=lambda c: c["name"])
+def test_quantize_lut_golden(case):
+    _check_lut_case(oracle.octave_quantize_lut,
+                    lambda s: int(oracle.f32_to_f16_bits(np.array([s], np.float32))[0]), case)
+
+
+def _slot_inputs():
+    s = np.ones(128, np.float32)
+    s[[1, 70, 127]] = -1
+    walsh = lambda i, k: -1.0 if bin(i & k).count("1") % 2 else 1.0
+    k = np.zeros((1, 1, 128), np.float32)
+    v = np.zeros((1, 1, 128), np.float32)
+    for i in range(64):
+        k[0, 0, i] = s[i] * np.float32(3 / 8) * walsh(i, 5)
+        k[0, 0, 64 + i] = s[64 + i] * np.float32(-5 / 8) * walsh(i, 9)
+    for i in range(128):
+        v[0, 0, i] = s[i] * np.float32(0.5) * walsh(i, 100)
+    return k, v, s
+
+
+def test_slot_golden_k3v4():
+    k, v, s = _slot_inputs()
+    slot = oracle.octave_quantize(k, v, tuple(SLOT_GOLD["format"]), s)[0, 0]
+    assert slot.tobytes().hex() == SLOT_GOLD["slot_hex"]
+
+
+# Each entry plants one plausible misreading in a copy of the oracle source
+# (the oracle itself is untouched); at least one golden must then fail.
+PLANTED = {
+    "bucketize right=True": ("if (mid[k] < y) c++;", "if (mid[k] <= y) c++;"),
+    "ss summed left to right": ("float ss = tree_sum_f32(tmp, n);",
+                                "float ss = 0.0f; for (int i = 0; i < n; i++) ss = ss + tmp[i];"),
+    "dot summed left to right": ("float dot = tree_sum_f32(tmp, n);",
+                                 "float dot = 0.0f; for (int i = 0; i < n; i++) dot = dot + tmp[i];"),
+    "y with one rounding": ("float y = x[i] / rms;\n    y = y * mult;", "float y = x[i] * (mult / rms);"),
+    "fp16 half up": ("if (rem > 0x1000u || (rem == 0x1000u && (h & 1u))) h++;",
+                     "if (rem >= 0x1000u) h++;"),
+    "V scale before K scales": ("uint16_t hb = orc_f32_to_f16(scales[s]);",
+                                "uint16_t hb = orc_f32_to_f16(scales[(s + f.num_k_scales) % f.num_scales]);"),
+    "pad bytes not zero": ("memset(slot, 0, (size_t)f.slot_bytes);",
+                           "memset(slot, 0x5a, (size_t)f.slot_bytes);"),
+    "sign flips skipped": ("for (int i = 0; i < d; i++) x[i] = x[i] * signs[i];", ""),
+    "RoPE and NoPE bit widths swapped": (
+        "int bits = kb < f.num_rope_blocks ? OCT_ROPE_BITS : OCT_NOPE_BITS;",
+        "int bits = kb < f.num_rope_blocks ? OCT_NOPE_BITS : OCT_ROPE_BITS;"),
+}
+
+
+def _planted_lib(tmp_path, old, new):
+    import ctypes as C
+    import subprocess
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "kvq_oracle.c")).read()
+    assert src.count(old) == 1, f"pattern not found once in the oracle: {old!r}"
+    path = tmp_path / "planted.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / "planted.so"
+    subprocess.check_call(["gcc", *oracle.CFLAGS, "-I", os.path.dirname(oracle.__file__),
+                           "-o", str(so), str(path), "-lm"])
+    L = C.CDLL(str(so))
+    L.orc_f32_to_f16.restype = C.c_uint16
+    L.orc_f32_to_f16.argtypes = [C.c_float]
+    return L
+
+
+def _goldens_pass(L):
+    import ctypes as C
+
+    def qlut(x, bits):
+        codes = np.zeros(x.size, np.uint8)
+        s = C.c_float(0)
+        r = L.orc_octave_quantize_lut(x.ctypes.data_as(C.c_void_p), x.size, bits,
+                                      codes.ctypes.data_as(C.c_void_p), C.byref(s))
+        assert r == 0
+        return codes, np.float32(s.value)
+
+    ok = True
+    for case in LUT_GOLD["cases"]:
+        try:
+            _check_lut_case(qlut, lambda s: int(L.orc_f32_to_f16(float(s))), case)
+        except AssertionError:
+            ok = False
+    k, v, s = _slot_inputs()
+    out = np.zeros(128, np.uint8)
+    r = L.orc_octave_quantize(128, 64, 4, 0, k.ctypes.data_as(C.c_void_p),
+                              v.ctypes.data_as(C.c_void_p), 0, 1, 1,
+                              s.ctypes.data_as(C.c_void_p), out.ctypes.data_as(C.c_void_p))
+    assert r == 0
+    return ok and out.tobytes().hex() == SLOT_GOLD["slot_hex"]
+
+
+def test_goldens_pass_on_unplanted_copy(tmp_path):
+    assert _goldens_pass(_planted_lib(tmp_path, "#define OCT_HB 64", "#define OCT_HB 64"))
+
+
+@pytest.mark.parametrize("name", sorted(PLANTED))
+def test_goldens_catch_planted_misreading(tmp_path, name):
+    old, new = PLANTED[name]
+    assert not _goldens_pass(_planted_lib(tmp_path, old, new)), f"{name} went unnoticed"
