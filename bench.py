@@ -624,44 +624,151 @@ def other_workloads(dev, main_name, reps, peak):
 
 
 # ----------------------------------------------------------------- CPU oracle leg
-def cpu_oracle_long_decode(steps: int, warmup: int = 0):
-    """Time the oracle on the same workload on the host: the cache of kv head 0
-    (131072 tokens) is built once (untimed), then each step appends the new
-    token and decodes its 8 query heads (`warmup` untimed steps first).
-    Returns (GB/s, seconds, sample)."""
+def cpu_oracle_long_decode(steps: int, warmup: int = 0, threads: int = 1):
+    """Time the oracle on the long-context decode step on the host.  With one
+    thread the sample is kv head 0 (its 8 query heads over all 131072 tokens,
+    1/4 of a step); with more, the whole step (all 4 kv heads, one
+    (sequence, kv head) unit per thread).  The cache is built once (untimed);
+    each step appends the new token and decodes (`warmup` untimed steps
+    first).  Returns (GB/s, seconds, sample, threads used)."""
     import oracle
     W = synth.WORKLOADS["long_decode"]
     T, Hq, H = W["ctx"], W["n_q_heads"], W["n_kv_heads"]
     G = Hq // H
+    nh = 1 if threads <= 1 else H
     k, v = synth.kv_tokens(W["seed"], 1, T, H, 256, W["outlier_frac"], W["outlier_factor"])
-    kb = np.ascontiguousarray(synth.to_bf16_bits(k)[:, :, :1])
-    vb = np.ascontiguousarray(synth.to_bf16_bits(v)[:, :, :1])
+    kb = np.ascontiguousarray(synth.to_bf16_bits(k)[:, :, :nh])
+    vb = np.ascontiguousarray(synth.to_bf16_bits(v)[:, :, :nh])
     del k, v
-    q = synth.to_bf16_bits(synth.queries(W["seed"], 1, Hq, 256))[:, :G].copy()
-    oc = oracle.Q4Cache(T, 1, max_tokens=T)
-    oc.append(kb, vb, [0])
-    for _ in range(warmup):
+    q = synth.to_bf16_bits(synth.queries(W["seed"], 1, Hq, 256))[:, :G * nh].copy()
+    oc = oracle.Q4Cache(T * nh, nh, max_tokens=T)
+    oc.append(kb, vb, [0], threads=threads)
+    used = min(threads, nh)
+
+    def step():
         oc.append(kb[:, T - 1:T], vb[:, T - 1:T], [T - 1])
-        oc.decode_attn(q, [T], 1 / 16)
+        oc.decode_attn(q, [T], 1 / 16, threads=threads)
+
+    for _ in range(warmup):
+        step()
     t = time.perf_counter()
     for _ in range(steps):
-        oc.append(kb[:, T - 1:T], vb[:, T - 1:T], [T - 1])
-        oc.decode_attn(q, [T], 1 / 16)
+        step()
     dt = time.perf_counter() - t
-    bytes_per_step = T * 288 + G * 256 * 6 + 2 * (512 + 144)
-    sample = (f"{steps} steps of the long-context decode step restricted to kv head 0 "
-              f"(its {G} query heads, {T} tokens): 1/{H} of a GPU step")
-    return bytes_per_step * steps / dt / 1e9, dt, sample
+    bytes_per_step = nh * (T * 288 + G * 256 * 6 + 2 * (512 + 144))
+    if nh == 1:
+        sample = (f"{steps} steps of the long-context decode step restricted to kv head 0 "
+                  f"(its {G} query heads, {T} tokens): 1/{H} of a GPU step, 1 thread")
+    else:
+        sample = (f"{steps} whole long-context decode steps ({H} kv heads x {G} query heads, "
+                  f"{T} tokens), one (sequence, kv head) unit per thread")
+    return bytes_per_step * steps / dt / 1e9, dt, sample, used
+
+
+def cpu_oracle_quantize(threads: int):
+    """Oracle quantize-on-append of the whole 4096-token prefill (8 sequences x
+    8 kv heads), (sequence, 512-token chunk) units on threads."""
+    import oracle
+    W = synth.WORKLOADS["quantize"]
+    B, H, P = W["batch"], W["n_kv_heads"], W["prefill"]
+    k, v = synth.kv_tokens(W["seed"], B, P, H, 256, W["outlier_frac"], W["outlier_factor"])
+    kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+    del k, v
+    oc = oracle.Q4Cache(B * H * W["capacity"], H, max_tokens=W["capacity"])
+    t = time.perf_counter()
+    oc.append(kb, vb, np.zeros(B, np.int32), threads=threads)
+    dt = time.perf_counter() - t
+    return {"value": B * P / dt / 1e6, "unit": "Mtok/s", "seconds": dt,
+            "GB_s": 2 * B * P * H * (512 + 144) / dt / 1e9,
+            "cores": min(threads, B * (P // 512)), "kind": "oracle",
+            "sample": f"the whole prefill ({B} sequences x {P} tokens x {H} kv heads)"}
+
+
+def cpu_oracle_paged(threads: int):
+    """Oracle decode of the first 8 of the 32 paged sequences (the benchmark's
+    first generation group; 16 (sequence, kv head) units on threads)."""
+    import oracle
+    W = synth.WORKLOADS["paged_decode"]
+    B, H, Hq, ps = W["batch"], W["n_kv_heads"], W["n_q_heads"], W["page_size"]
+    n = 8
+    lens = synth.seq_lens(W["seed"], B, W["ctx_lo"], W["ctx_hi"])[:n]
+    npp = (lens + ps - 1) // ps
+    bt, n_pages = synth.page_table(W["seed"], n, npp, int(npp.max()))
+    k, v = synth.kv_tokens(W["seed"] * 100, n, int(lens.max()), H, 256, W["outlier_frac"],
+                           W["outlier_factor"])
+    kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+    del k, v
+    oc = oracle.Q4Cache(n_pages * H * ps, H, block_table=bt, page_size=ps)
+    for b in range(n):
+        oc.with_block_table(bt[b:b + 1]).append(kb[b:b + 1, :lens[b]], vb[b:b + 1, :lens[b]],
+                                                np.zeros(1, np.int32), threads=threads)
+    q = synth.to_bf16_bits(synth.queries(W["seed"], B, Hq, 256))[:n]
+    reps = 4
+    t = time.perf_counter()
+    for _ in range(reps):
+        oc.decode_attn(q, lens, 1 / 16, threads=threads)
+    dt = time.perf_counter() - t
+    return {"value": reps * int(lens.sum()) * H * 288 / dt / 1e9, "unit": "GB/s", "seconds": dt,
+            "cores": min(threads, n * H), "kind": "oracle",
+            "sample": f"{reps} decodes of {n} of the {B} sequences ({int(lens.sum())} tokens, "
+                      f"{H} kv heads)"}
+
+
+def cpu_oracle_octave(threads: int):
+    """Oracle Octave k3v4 decode of 4 of the 16 requests (16384 tokens each,
+    all 32 query heads; one query token per thread)."""
+    import oracle
+    W = synth.WORKLOADS["octave"]
+    H, Hq, ctx, bs = W["n_kv_heads"], W["n_q_heads"], W["ctx"], W["block_size"]
+    n = 4
+    fmt = (W["head_size"], W["rope_dim"], W["v_bits"], 0)
+    signs = synth.sign_pattern(128)
+    cache = np.zeros((n * ctx // bs, H, bs, 128), np.uint8)
+    bt = np.arange(n * ctx // bs, dtype=np.int32).reshape(n, ctx // bs)
+    for r in range(n):
+        k, v = synth.kv_tokens(W["seed"] * 100 + r, 1, ctx, H, 128, W["outlier_frac"],
+                               W["outlier_factor"])
+        slots = oracle.octave_quantize(synth.to_bf16_bits(k[0]), synth.to_bf16_bits(v[0]), fmt,
+                                       signs, threads=threads)
+        del k, v
+        cache[r * ctx // bs:(r + 1) * ctx // bs] = slots.reshape(ctx // bs, bs, H, 128).transpose(0, 2, 1, 3)
+    q = synth.to_bf16_bits(synth.queries(W["seed"], W["batch"], Hq, 128))[:n]
+    t = time.perf_counter()
+    oracle.octave_attention(q, cache, bt, np.arange(n, dtype=np.int32), np.full(n, ctx, np.int32),
+                            fmt, 128 ** -0.5, signs, threads=threads)
+    dt = time.perf_counter() - t
+    return {"value": n * ctx * H * 128 / dt / 1e9, "unit": "GB/s", "seconds": dt,
+            "cores": min(threads, n), "kind": "oracle",
+            "sample": f"decode of {n} of the {W['batch']} requests ({ctx} tokens, {Hq} q heads)"}
+
+
+def cpu_baselines(threads: int):
+    """The headline (long-context decode) oracle figure on all cores and on one,
+    plus bounded multi-core samples of the other workloads."""
+    gbs1, dt1, sample1, _ = cpu_oracle_long_decode(steps=3, threads=1)
+    gbs, dt, sample, used = cpu_oracle_long_decode(steps=2, threads=threads)
+    per = {"long_decode": {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle",
+                           "sample": sample, "seconds": dt},
+           "long_decode_1_core": {"value": gbs1, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                  "sample": sample1, "seconds": dt1},
+           "quantize": cpu_oracle_quantize(threads),
+           "paged_decode": cpu_oracle_paged(threads),
+           "octave": cpu_oracle_octave(threads)}
+    return {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle", "sample": sample,
+            "seconds": dt, "host_threads": threads, "single_core": per["long_decode_1_core"],
+            "workloads": per}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    # bounded sample: at most 8 timed and 2 warm-up oracle steps (~0.5 s each)
-    steps = max(1, min(args.steps, 8))
+    import oracle
+    threads = oracle.host_threads()
+    # bounded sample: at most 4 timed and 2 warm-up whole oracle steps
+    steps = max(1, min(args.steps, 4))
     warm = max(0, min(args.warmup, 2))
-    gbs, dt, sample = cpu_oracle_long_decode(steps, warm)
+    gbs, dt, sample, used = cpu_oracle_long_decode(steps, warm, threads=threads)
     W = synth.WORKLOADS["long_decode"]
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s",
@@ -673,8 +780,8 @@ def run_reference(args):
                    "cache": "Q4_0",
                    "step": "kvq_decode_step: append 1 token + decode (one call)",
                    "parallelism": f"replicas x{args.gpus}"},
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle",
+                         "sample": sample, "host_threads": threads},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -760,9 +867,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "long_decode":
-        gbs, dt, sample = cpu_oracle_long_decode(steps=5)
-        cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
-               "seconds": dt}
+        import oracle
+        cpu = cpu_baselines(oracle.host_threads())
 
     if rank == 0:
         line = {

@@ -47,11 +47,33 @@ def gaussian(seed: int, shape) -> np.ndarray:
     return out.reshape(shape)
 
 
+def _chunked(n: int, fn) -> None:
+    """fn(lo, hi) over [0, n) in _CHUNK pieces, on threads for large n."""
+    spans = [(lo, min(n, lo + _CHUNK)) for lo in range(0, n, _CHUNK)]
+    if len(spans) <= 1:
+        for lo, hi in spans:
+            fn(lo, hi)
+        return
+    with ThreadPoolExecutor(min(len(spans), os.cpu_count() or 1)) as ex:
+        list(ex.map(lambda sp: fn(*sp), spans))
+
+
 def to_bf16_bits(x32: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest-even bf16; return the uint16 bits."""
-    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32)
-    r = ((u >> 16) & 1) + np.uint32(0x7FFF)
-    return ((u + r) >> 16).astype(np.uint16)
+    x = np.ascontiguousarray(x32, dtype=np.float32)
+    u = x.view(np.uint32).reshape(-1)
+    out = np.empty(u.size, np.uint16)
+
+    def conv(lo, hi):
+        t = u[lo:hi] >> np.uint32(16)
+        t &= np.uint32(1)
+        t += np.uint32(0x7FFF)
+        t += u[lo:hi]
+        t >>= np.uint32(16)
+        out[lo:hi] = t
+
+    _chunked(u.size, conv)
+    return out.reshape(x.shape)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -68,13 +90,21 @@ def outlier_channels(seed: int, n_heads: int, dim: int, frac: float = 0.01) -> n
 def apply_outliers(x: np.ndarray, channels: np.ndarray, factor: float) -> np.ndarray:
     """Scale the given channels of the last dim; x is (..., H, D), channels (H, k)
     or (k,) for the same channels on every head."""
-    x = x.copy()
     if channels.ndim == 1:
-        x[..., channels] *= np.float32(factor)
+        scale = np.ones(x.shape[-1], np.float32)
+        scale[channels] = np.float32(factor)
     else:
+        scale = np.ones(x.shape[-2:], np.float32)
         for h in range(channels.shape[0]):
-            x[..., h, channels[h]] *= np.float32(factor)
-    return x
+            scale[h, channels[h]] = np.float32(factor)
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty_like(x)
+    rows = scale.size
+    xf, of = x.reshape(-1, rows), out.reshape(-1, rows)
+    step = max(1, _CHUNK // rows)
+    for r0 in range(0, xf.shape[0], step):
+        np.multiply(xf[r0:r0 + step], scale.reshape(-1), out=of[r0:r0 + step])
+    return out
 
 
 def seq_lens(seed: int, batch: int, lo: int, hi: int) -> np.ndarray:

@@ -15,6 +15,7 @@ from __future__ import annotations
 import ctypes as C
 import os
 import subprocess
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -164,6 +165,33 @@ def q8_quantize_vectors(x):
     return codes, scales
 
 
+# ---------------------------------------------------------------- threads
+# The oracle itself is single-threaded C.  For large workloads the calls below
+# can split the work into independent units -- (sequence, kv head) for decode,
+# (sequence, token range) for append, query tokens for Octave attention, token
+# ranges for Octave quantize -- and run the unchanged C function on each unit
+# from a pool of host threads (ctypes releases the GIL during the call).  Each
+# unit performs exactly the operations, in the same order, that the whole call
+# performs for it, so the results are bit-identical to the single call.
+def host_threads() -> int:
+    """Cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_units(fn, units, threads):
+    """fn(unit) for each unit on up to `threads` host threads, results in order."""
+    if threads <= 1 or len(units) <= 1:
+        return [fn(u) for u in units]
+    # fill the oracle's lazily computed codebook cache before any thread runs
+    octave_codebook(3)
+    octave_codebook(4)
+    with ThreadPoolExecutor(min(threads, len(units))) as ex:
+        return list(ex.map(fn, units))
+
+
 class Q4Cache:
     """Oracle-side Q4_0 cache with the documented structure-of-arrays layout
     (bits = 8: the Q8_0 cache, 256 int8 code bytes per row)."""
@@ -195,7 +223,43 @@ class Q4Cache:
                 self.n_kv_heads, self.max_tokens, _p(self.block_table), self.page_size,
                 self.max_pages)
 
-    def append(self, k, v, start_pos):
+    def _seq_view_args(self, b):
+        """Arguments that make sequence b of this cache sequence 0 of a cache
+        (same rows, same kv heads)."""
+        if self.block_table is None:
+            row0 = b * self.n_kv_heads * self.max_tokens
+            bt, ps, mp, mt = None, 0, 0, self.max_tokens
+            keep = None
+        else:
+            row0 = 0
+            keep = np.ascontiguousarray(self.block_table[b:b + 1])
+            bt, ps, mp, mt = keep, self.page_size, self.max_pages, 0
+        planes = [a[row0:] for a in (self.k_codes, self.k_scales, self.v_codes, self.v_scales)]
+        args = (*[_p(a) for a in planes], self.n_kv_heads, mt, _p(bt), ps, mp)
+        return args, (planes, keep)
+
+    def _unit_view_args(self, b, g):
+        """Arguments that make (sequence b, kv head g) the only sequence and kv
+        head of a paged cache over the same rows: a one-entry block table
+        holding page 0 of a view whose base is the unit's first row
+        (contiguous), or the sequence's pages times the kv head count with the
+        base moved by g pages' worth of rows (paged)."""
+        if self.block_table is None:
+            row0 = (b * self.n_kv_heads + g) * self.max_tokens
+            bt = np.zeros((1, 1), np.int32)
+            ps, mp = self.max_tokens, 1
+        else:
+            row0 = g * self.page_size
+            pages = self.block_table[b:b + 1].astype(np.int64)
+            bt = np.where(pages < 0, -1, pages * self.n_kv_heads).astype(np.int32)
+            ps, mp = self.page_size, self.max_pages
+        planes = [a[row0:] for a in (self.k_codes, self.k_scales, self.v_codes, self.v_scales)]
+        args = (*[_p(a) for a in planes], 1, 0, _p(bt), ps, mp)
+        return args, (planes, bt)
+
+    def append(self, k, v, start_pos, threads=1, chunk=512):
+        """Quantize k, v ([batch, t_new, Hkv, 256]) into the cache; with
+        threads > 1, (sequence, chunk of tokens) units run in parallel."""
         k = np.ascontiguousarray(k)
         v = np.ascontiguousarray(v)
         assert k.shape == v.shape and k.dtype == v.dtype
@@ -203,16 +267,50 @@ class Q4Cache:
         assert hkv == self.n_kv_heads and d == 256
         sp = np.ascontiguousarray(start_pos, dtype=np.int32)
         fn = lib().orc_q8_append if self.bits == 8 else lib().orc_q4_append
-        _check(fn(*self._args(), _p(k), _p(v), _dtype_code(k), batch, t_new, _p(sp)), "append")
+        if threads <= 1:
+            _check(fn(*self._args(), _p(k), _p(v), _dtype_code(k), batch, t_new, _p(sp)),
+                   "append")
+            return
 
-    def decode_attn(self, q, seq_lens, scale):
+        def unit(u):
+            b, i0 = u
+            args, keep = self._seq_view_args(b)
+            ku = np.ascontiguousarray(k[b:b + 1, i0:i0 + chunk])
+            vu = np.ascontiguousarray(v[b:b + 1, i0:i0 + chunk])
+            spu = np.array([sp[b] + i0], np.int32)
+            return fn(*args, _p(ku), _p(vu), _dtype_code(ku), 1, ku.shape[1], _p(spu))
+
+        units = [(b, i0) for b in range(batch) for i0 in range(0, t_new, chunk)]
+        for r in run_units(unit, units, threads):
+            _check(r, "append")
+
+    def decode_attn(self, q, seq_lens, scale, threads=1):
+        """fp64 decode attention; with threads > 1, (sequence, kv head) units
+        run in parallel."""
         q = np.ascontiguousarray(q)
         batch, hq, d = q.shape
         sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
         out = np.zeros((batch, hq, d), np.float64)
         fn = lib().orc_q8_decode_attn if self.bits == 8 else lib().orc_q4_decode_attn
-        _check(fn(*self._args(), _p(q), _dtype_code(q), batch, hq, _p(sl), C.c_double(scale),
-                  _p(out)), "decode_attn")
+        if threads <= 1:
+            _check(fn(*self._args(), _p(q), _dtype_code(q), batch, hq, _p(sl),
+                      C.c_double(scale), _p(out)), "decode_attn")
+            return out
+        G = hq // self.n_kv_heads
+
+        def unit(u):
+            b, g = u
+            args, keep = self._unit_view_args(b, g)
+            qu = np.ascontiguousarray(q[b:b + 1, g * G:(g + 1) * G])
+            ou = np.zeros((1, G, d), np.float64)
+            r = fn(*args, _p(qu), _dtype_code(qu), 1, G, _p(sl[b:b + 1].copy()),
+                   C.c_double(scale), _p(ou))
+            return r, ou
+
+        units = [(b, g) for b in range(batch) for g in range(self.n_kv_heads)]
+        for (b, g), (r, ou) in zip(units, run_units(unit, units, threads)):
+            _check(r, "decode_attn")
+            out[b, g * G:(g + 1) * G] = ou[0]
         return out
 
 
@@ -274,16 +372,27 @@ def octave_unrotate(y, signs, block):
     return z
 
 
-def octave_quantize(key, value, fmt, signs):
-    """fmt: (head_size, rope_dim, v_bits, compact). key/value: (T, H, D)."""
+def octave_quantize(key, value, fmt, signs, threads=1, chunk=1024):
+    """fmt: (head_size, rope_dim, v_bits, compact). key/value: (T, H, D).
+    With threads > 1, chunks of tokens run in parallel."""
     key = np.ascontiguousarray(key)
     value = np.ascontiguousarray(value)
     T, H, D = key.shape
     info = octave_format(*fmt)
     out = np.zeros((T, H, info["slot_bytes"]), np.uint8)
     s = np.ascontiguousarray(signs, dtype=np.float32)
-    _check(lib().orc_octave_quantize(*fmt, _p(key), _p(value), _dtype_code(key), T, H, _p(s),
-                                     _p(out)), "octave_quantize")
+
+    def unit(t0):
+        t1 = min(T, t0 + chunk)
+        return lib().orc_octave_quantize(*fmt, _p(key[t0:t1]), _p(value[t0:t1]),
+                                         _dtype_code(key), t1 - t0, H, _p(s), _p(out[t0:t1]))
+
+    if threads <= 1:
+        _check(lib().orc_octave_quantize(*fmt, _p(key), _p(value), _dtype_code(key), T, H, _p(s),
+                                         _p(out)), "octave_quantize")
+        return out
+    for r in run_units(unit, list(range(0, T, chunk)), threads):
+        _check(r, "octave_quantize")
     return out
 
 
@@ -299,7 +408,10 @@ def octave_dequantize(slots, fmt, signs, rotated=False):
     return k, v
 
 
-def octave_attention(query, cache, block_table, q_to_req, q_to_klen, fmt, scale, signs):
+def octave_attention(query, cache, block_table, q_to_req, q_to_klen, fmt, scale, signs,
+                     threads=1):
+    """reference_attention in fp64; with threads > 1, query tokens run in
+    parallel."""
     query = np.ascontiguousarray(query)
     cache = np.ascontiguousarray(cache, dtype=np.uint8)
     nq, hq, d = query.shape
@@ -309,7 +421,19 @@ def octave_attention(query, cache, block_table, q_to_req, q_to_klen, fmt, scale,
     ql = np.ascontiguousarray(q_to_klen, dtype=np.int32)
     s = np.ascontiguousarray(signs, dtype=np.float32)
     out = np.zeros((nq, hq, d), np.float64)
-    _check(lib().orc_octave_attention(*fmt, _p(query), _dtype_code(query), nq, hq, _p(cache),
-                                      C.c_int64(cache.shape[0]), hkv, bs, _p(bt), bt.shape[1], _p(qr), _p(ql),
-                                      C.c_double(scale), _p(s), _p(out)), "octave_attention")
+
+    def unit(i):
+        return lib().orc_octave_attention(*fmt, _p(query[i:i + 1]), _dtype_code(query), 1, hq,
+                                          _p(cache), C.c_int64(cache.shape[0]), hkv, bs, _p(bt),
+                                          bt.shape[1], _p(qr[i:i + 1]), _p(ql[i:i + 1]),
+                                          C.c_double(scale), _p(s), _p(out[i:i + 1]))
+
+    if threads <= 1:
+        _check(lib().orc_octave_attention(*fmt, _p(query), _dtype_code(query), nq, hq, _p(cache),
+                                          C.c_int64(cache.shape[0]), hkv, bs, _p(bt), bt.shape[1],
+                                          _p(qr), _p(ql), C.c_double(scale), _p(s), _p(out)),
+               "octave_attention")
+        return out
+    for r in run_units(unit, list(range(nq)), threads):
+        _check(r, "octave_attention")
     return out

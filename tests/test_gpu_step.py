@@ -109,3 +109,22 @@ def test_step_paged_and_out_of_range_positions():
     assert_planes_equal(f, a)
     assert torch.equal(got, want_gpu)
     assert torch.count_nonzero(got[1]) == 0
+    # the oracle over the same paged layout: the new tokens of sequences 0 and
+    # 2 appended, none for sequence 1 (position -1, zero row) or sequence 3
+    # (no page for its position: its length is clamped to the 256 tokens its
+    # pages hold)
+    oc = oracle.Q4Cache(n_pages * H * ps, H, block_table=bt, page_size=ps)
+    for b in range(B):
+        L = int(lens[b])
+        oc.with_block_table(bt[b:b + 1]).append(k[b:b + 1, :L], v[b:b + 1, :L],
+                                                np.zeros(1, np.int32))
+    for b in (0, 2):
+        oc.with_block_table(bt[b:b + 1]).append(new_k[b:b + 1, None], new_v[b:b + 1, None],
+                                                pos[b:b + 1])
+    for name in PLANES:
+        g = getattr(f, name).cpu().numpy()
+        assert np.array_equal(g.view(np.uint16) if name.endswith("scales") else g,
+                              getattr(oc, name)), name
+    olens = np.array([pos[0] + 1, 0, pos[2] + 1, npp[3] * ps], np.int32)
+    want = oc.decode_attn(q, olens, 1 / 16)
+    assert np.abs(got.cpu().numpy() - want).max() <= ATOL

@@ -126,3 +126,51 @@ def test_paged_equals_contiguous():
     pc.append(k, v, [0, 0])
     sl = [70, 33]
     np.testing.assert_array_equal(cc.decode_attn(q, sl, 0.0625), pc.decode_attn(q, sl, 0.0625))
+
+
+@pytest.mark.parametrize("paged", [False, True])
+@pytest.mark.parametrize("bits", [4, 8])
+def test_threaded_units_bit_identical(paged, bits):
+    """The threaded harness (independent (sequence, kv head) decode units and
+    (sequence, token chunk) append units of the unchanged C oracle) gives
+    exactly the single-call results."""
+    B, Hkv, Hq, T, ps = 3, 2, 8, 300, 64
+    k, v = synth.kv_tokens(77, B, T, Hkv, 256, 0.01, 16.0)
+    kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+    q = synth.to_bf16_bits(synth.queries(78, B, Hq, 256))
+    lens = np.array([300, 0, 129], np.int32)
+    if paged:
+        npp = -(-T // ps)
+        bt, n_pages = synth.page_table(79, B, np.full(B, npp), npp)
+
+        def mk():
+            return oracle.Q4Cache(n_pages * Hkv * ps, Hkv, block_table=bt, page_size=ps, bits=bits)
+    else:
+        def mk():
+            return oracle.Q4Cache(B * Hkv * T, Hkv, max_tokens=T, bits=bits)
+    one, many = mk(), mk()
+    one.append(kb, vb, np.zeros(B, np.int32))
+    many.append(kb, vb, np.zeros(B, np.int32), threads=4, chunk=37)
+    for a in ("k_codes", "k_scales", "v_codes", "v_scales"):
+        assert np.array_equal(getattr(one, a), getattr(many, a)), a
+    want = one.decode_attn(q, lens, 1 / 16)
+    got = one.decode_attn(q, lens, 1 / 16, threads=4)
+    assert np.array_equal(got, want)
+
+
+def test_threaded_octave_bit_identical():
+    fmt = (128, 64, 4, 0)
+    s = synth.sign_pattern(128)
+    nblk, Hkv, Hq, bs = 8, 2, 8, 16
+    k = synth.to_bf16_bits(synth.gaussian(21, (nblk * bs, Hkv, 128)))
+    v = synth.to_bf16_bits(synth.gaussian(22, (nblk * bs, Hkv, 128)))
+    slots = oracle.octave_quantize(k, v, fmt, s)
+    assert np.array_equal(oracle.octave_quantize(k, v, fmt, s, threads=3, chunk=10), slots)
+    cache = slots.reshape(nblk, bs, Hkv, 128).transpose(0, 2, 1, 3).copy()
+    bt = np.array([[5, 2, 7, 0], [1, 3, 4, 6]], np.int32)
+    q = synth.to_bf16_bits(synth.gaussian(23, (3, Hq, 128)))
+    q2r = np.array([0, 1, 1], np.int32)
+    q2l = np.array([50, 64, 0], np.int32)
+    want = oracle.octave_attention(q, cache, bt, q2r, q2l, fmt, 0.09, s)
+    got = oracle.octave_attention(q, cache, bt, q2r, q2l, fmt, 0.09, s, threads=3)
+    assert np.array_equal(got, want)
