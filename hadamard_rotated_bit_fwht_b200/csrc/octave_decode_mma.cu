@@ -12,12 +12,16 @@
 //     a time from nibble-packed codes (two 8-entry halves plus a
 //     sign-replicated mask for 4-bit codes, one prmt for 3-bit codes), and
 //     those bytes are B-fragment registers as they stand.  The rotated query
-//     of each head is scaled by S = 127 * 128 / max|q| and split exactly into
-//     int8 H and L (S q = 128 H + L, |L| <= 64), rows 0-7 H and rows 8-15 L;
-//     its columns are stored in the order the codes arrive in.  Per (block,
-//     8 tokens) 128 d_H + d_L is the exact integer dot product, converted to
-//     fp32 once and multiplied by the block scale; 1 / S joins the softmax
-//     scale.  The query is thereby carried to 3e-5 of its largest element.
+//     of each head is scaled by S = 127 * 2^14 / max|q|, rounded to an
+//     integer and split exactly into three int8 digits
+//     (S q = 2^14 H + 2^7 M + L, |M|, |L| <= 64): one A tile holds H (rows
+//     0-7) and M (rows 8-15), a second one L (rows 0-7); their columns are
+//     stored in the order the codes arrive in.  Per (block, 8 tokens) the
+//     digit dot products are combined in fp32 (2^14 d_H + (2^7 d_M + d_L))
+//     and multiplied by the block scale; 1 / S joins the softmax scale.  The
+//     query is thereby carried to 2.4e-7 of its largest element.  (Two
+//     digits, 14 bits, left up to 2.3e-3 of error in the outputs of the
+//     16 x 16384-token workload, whose keys carry x16 outlier channels.)
 //   * PV on the fp16 path (m16n8k16, fp32 accumulation): A = V^T codes through
 //     the biased table (each byte u becomes the exact fp16 1024 + u by pairing
 //     it with 0x64; one half2 subtract of 1152 leaves LUT[c]), read by
@@ -42,13 +46,13 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kHead = 128;
 constexpr int kORec = 132;  // m, l, pad, pad, o[128]
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kQRange = 16256.f;  // 127 * 128
+constexpr float kQRange = 2080768.f;  // 127 * 2^14
 constexpr int kStageBytes = kTile * 128;
 constexpr int kOffF = kStages * kStageBytes;  // fp32 scales [3][64] of the current tile
 constexpr int kOffV = kOffF + 3 * kTile * 4;  // per stage, per token: 1 if its block is mapped
 constexpr int kQStride = 144;                 // int8 query row: 128 B + 16 B pad
-constexpr int kOffQ = kOffV + kStages * kTile;  // int8 query rows (0-7 H, 8-15 L)
-constexpr int kSmemBytes = kOffQ + 16 * kQStride;
+constexpr int kOffQ = kOffV + kStages * kTile;  // int8 query rows: 0-7 H, 8-15 M, 16-23 L, 24-31 zero
+constexpr int kSmemBytes = kOffQ + 32 * kQStride;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -183,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     T3hi = c[4] | c[5] << 8 | c[6] << 16 | c[7] << 24;
   }
 
-  // ---- query: signs, FWHT over the two 64-dim blocks; int8 H / L rows
+  // ---- query: signs, FWHT over the two 64-dim blocks; int8 H / M / L rows
   float *qs = reinterpret_cast<float *>(smem);  // [8][128]
   {
     // thread tid always holds dim tid: sign bit (tid & 31) of word tid / 32
@@ -232,19 +236,28 @@ __global__ void __launch_bounds__(kThreads, 4)
     const int hh = p >> 7, col = p & 127;
     const float m = qmax[hh];
     const int dim = qcol_dim(col >> 5, col & 31);
+    // |x| <= 127 * 2^14 < 2^21, so x is a multiple of 2^-3 at worst and every
+    // difference below is exact; the digits sum to rint(x)
     const float x = m > 0.f ? qs[hh * kHead + dim] * (kQRange / m) : 0.f;
-    const float hi = rintf(x * 0.0078125f);
-    const float lo = rintf(x - 128.f * hi);  // exact difference, |lo| <= 64
+    const float hi = rintf(x * (1.f / 16384.f));
+    const float r1 = x - 16384.f * hi;  // |r1| <= 2^13
+    const float mid = rintf(r1 * 0.0078125f);
+    const float lo = rintf(r1 - 128.f * mid);  // |lo| <= 64
     qrow[hh * kQStride + col] = (uint8_t)(int8_t)(int)hi;
-    qrow[(8 + hh) * kQStride + col] = (uint8_t)(int8_t)(int)lo;
+    qrow[(8 + hh) * kQStride + col] = (uint8_t)(int8_t)(int)mid;
+    qrow[(16 + hh) * kQStride + col] = (uint8_t)(int8_t)(int)lo;
+    qrow[(24 + hh) * kQStride + col] = 0;
   }
   __syncthreads();
-  uint32_t qa[4][4];  // A fragments of the virtual chunks
+  uint32_t qa[4][4], qb[4][4];  // A fragments of the virtual chunks: (H, M) and (L, 0)
   {
     const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
     const uint32_t qaddr = smem_u32(qrow) + row * kQStride + 16 * (lane >> 4);
 #pragma unroll
-    for (int vc = 0; vc < 4; vc++) ldsm_x4(qaddr + 32 * vc, qa[vc]);
+    for (int vc = 0; vc < 4; vc++) {
+      ldsm_x4(qaddr + 32 * vc, qa[vc]);
+      ldsm_x4(qaddr + 16 * kQStride + 32 * vc, qb[vc]);
+    }
   }
   // FWHT-64 blocks carry 1 / 8; the query ints carry S
   const float sl = scale_log2 * (qmax[g] * (0.125f / kQRange));
@@ -319,8 +332,9 @@ __global__ void __launch_bounds__(kThreads, 4)
       auto chunk_addr = [&](int ch) -> uint32_t {
         return base + mr * 128 + ((ch ^ (mr & 7)) << 4);
       };
-      // ---- QK: integer MMAs, one accumulator per (block, 8 tokens)
-      int accr[2][4] = {}, accn[2][4] = {};
+      // ---- QK: integer MMAs, accumulators per (block, 8 tokens): (H, M) rows
+      // and L rows
+      int accr[2][4] = {}, accn[2][4] = {}, accrl[2][4] = {}, accnl[2][4] = {};
       {  // RoPE: chunks 0, 1 (4-bit)
         uint32_t kr[4];
         ldsm_x4(chunk_addr(mc), kr);  // (T0, c0), (T1, c0), (T0, c1), (T1, c1)
@@ -328,7 +342,9 @@ __global__ void __launch_bounds__(kThreads, 4)
         for (int m = 0; m < 4; m++) {
           const int T = m & 1, c = m >> 1;
           const uint32_t w = kr[m];
-          imma16832(accr[T], qa[c], lut4_bytes(w & 0xFFFFu, T4), lut4_bytes(w >> 16, T4));
+          const uint32_t b0 = lut4_bytes(w & 0xFFFFu, T4), b1 = lut4_bytes(w >> 16, T4);
+          imma16832(accr[T], qa[c], b0, b1);
+          imma16832(accrl[T], qb[c], b0, b1);
         }
       }
       {  // NoPE: 2-bit plane chunk 2, 1-bit plane in chunk 3 (words 0, 1)
@@ -356,6 +372,8 @@ __global__ void __launch_bounds__(kThreads, 4)
           }
           imma16832(accn[T], qa[2], R[0], R[1]);
           imma16832(accn[T], qa[3], R[2], R[3]);
+          imma16832(accnl[T], qb[2], R[0], R[1]);
+          imma16832(accnl[T], qb[3], R[2], R[3]);
         }
       }
       float2 sacc[2];
@@ -364,10 +382,13 @@ __global__ void __launch_bounds__(kThreads, 4)
         const float2 dr = *reinterpret_cast<const float2 *>(fsc + 16 * warp + 8 * T + 2 * tg);
         const float2 dn =
             *reinterpret_cast<const float2 *>(fsc + kTile + 16 * warp + 8 * T + 2 * tg);
-        sacc[T].x = fmaf(dr.x, (float)(accr[T][0] * 128 + accr[T][2]),
-                         dn.x * (float)(accn[T][0] * 128 + accn[T][2]));
-        sacc[T].y = fmaf(dr.y, (float)(accr[T][1] * 128 + accr[T][3]),
-                         dn.y * (float)(accn[T][1] * 128 + accn[T][3]));
+        // digit dots: H in [0..1], M in [2..3] (rows g + 8), L in the second tile's [0..1]
+        const float r0 = fmaf((float)accr[T][0], 16384.f, (float)(accr[T][2] * 128 + accrl[T][0]));
+        const float r1 = fmaf((float)accr[T][1], 16384.f, (float)(accr[T][3] * 128 + accrl[T][1]));
+        const float n0 = fmaf((float)accn[T][0], 16384.f, (float)(accn[T][2] * 128 + accnl[T][0]));
+        const float n1 = fmaf((float)accn[T][1], 16384.f, (float)(accn[T][3] * 128 + accnl[T][1]));
+        sacc[T].x = fmaf(dr.x, r0, dn.x * n0);
+        sacc[T].y = fmaf(dr.y, r1, dn.y * n1);
       }
       // ---- online softmax (base 2), head g, this warp's 16 tokens
       float sc[4] = {sacc[0].x * sl, sacc[0].y * sl, sacc[1].x * sl, sacc[1].y * sl};
