@@ -36,16 +36,37 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
+OBJ_DIR = os.path.join(ROOT, "_build", "kvq")
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every .cu to an object in parallel (relocatable device code is
+    not needed: no kernel calls across files), then link libkvq.so."""
     if not force and not _stale():
         return LIB
+    from concurrent.futures import ThreadPoolExecutor
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    compile_flags = [f for f in FLAGS if f not in ("--shared",)]
+    tag = f".{os.getpid()}"
+
+    def compile_one(src):
+        obj = os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + tag + ".o")
+        cmd = [NVCC, *compile_flags, "-I", INCLUDE, "-c", src, "-o", obj]
+        if verbose:
+            cmd += ["-Xptxas", "-v"]
+            print(" ".join(cmd))
+        subprocess.check_call(cmd)
+        return obj
+
+    srcs = sources()
+    with ThreadPoolExecutor(min(len(srcs), os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(compile_one, srcs))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *FLAGS, "-I", INCLUDE, "-o", tmp, *sources()]
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
-        print(" ".join(cmd))
-    subprocess.check_call(cmd)
+    subprocess.check_call([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "--shared",
+                           "-Xcompiler", "-fPIC", "-o", tmp, *objs])
     os.replace(tmp, LIB)
+    for o in objs:
+        os.remove(o)
     return LIB
 
 

@@ -52,16 +52,33 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return done != 0;
 }
-// true once the phase with this parity has completed; false after the poll
-// limit or once *abort is set (by any thread of the CTA)
+// non-blocking test of the phase with this parity
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+// true once the phase with this parity has completed; false after `polls`
+// polls (0: one non-blocking test) or once *abort is set (by any thread of
+// the CTA)
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          const volatile int *abort) {
+                                          const volatile int *abort, int polls) {
+  if (polls <= 0) return mbar_test(bar, parity);
   if (mbar_try(bar, parity)) return true;
-  for (int i = 0; i < kWaitPolls; i++) {
+  for (int i = 0; i < polls; i++) {
     if (mbar_try(bar, parity)) return true;
     if (*abort) return false;
   }
   return false;
+}
+// record a condition in the library's device error word (see kvq_device_errors)
+__device__ __forceinline__ void report(uint32_t *err, uint32_t flag) {
+  if (err != nullptr) atomicOr(err, flag);
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint32_t bar) {

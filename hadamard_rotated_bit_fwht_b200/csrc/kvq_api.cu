@@ -301,7 +301,9 @@ kvq_status kvq_octave_quantize(const kvq_octave_fmt *fmt, const void *key, const
       (dtype != KVQ_F32 && dtype != KVQ_BF16))
     return KVQ_ERR_INVALID_ARG;
   if (num_tokens == 0) return KVQ_OK;
-  if (!key || !value || !d_slot_mapping || !cache || !aligned(cache, 4)) return KVQ_ERR_INVALID_ARG;
+  if (!key || !value || !d_slot_mapping || !cache || !aligned(cache, 4) || !aligned(key, 16) ||
+      !aligned(value, 16))
+    return KVQ_ERR_INVALID_ARG;
   return from_cuda(launch_octave_quantize(p, key, value, dtype == KVQ_BF16, num_tokens,
                                           num_kv_heads, d_slot_mapping, cache, block_size,
                                           num_blocks, as_stream(stream)));

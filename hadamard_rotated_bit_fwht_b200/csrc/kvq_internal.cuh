@@ -79,6 +79,13 @@ __device__ __forceinline__ int64_t q4_row(const kvq_cache &c, int b, int h, int 
   return ((int64_t)page * c.num_kv_heads + h) * c.page_size + (t - pi * c.page_size);
 }
 
+// ---------------------------------------------------------------- errors
+// Device address of the library's error word on the current device (nullptr
+// if the lookup fails), and the mbarrier poll limit of the decode kernels'
+// bounded waits (kvq_set_wait_limit; 1 << 20 by default).
+uint32_t *device_error_word();
+int wait_poll_limit();
+
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_rotate(const void *x, int bf16, float *y, int64_t n_vec, cudaStream_t s);
 // code_bits 4: Q4_0 (128-byte code rows), 8: Q8_0 (256-byte code rows)

@@ -1,24 +1,9 @@
 // octave.cu -- the Octave KV-cache variant (vLLM API page
-// "vllm.v1.attention.ops.rocm_octave"): quantize into per-(token, head) byte
-// slots, and decode attention over the paged slot cache.
+// "vllm.v1.attention.ops.rocm_octave"): decode attention over the paged slot
+// cache (the SIMT split kernel for the formats the tensor-core kernel does not
+// take, the split-K combine and the back-rotation).
 //
-// Quantize (reference_quantize): one warp per (token, kv head); lane l holds
-// dims l, l+32, l+64, l+96 of the 128-dim head.
-//   K: x * signs, FWHT over each 64-dim block (stages h = 1..16 across lanes
-//      with xor-shuffles, h = 32 in registers, then x 1/8), then per block
-//      _quantize_lut with 4-bit codes for RoPE blocks and 3-bit codes for NoPE
-//      blocks.
-//   V: x * signs, FWHT-128 over the head (h = 32, 64 in registers), x
-//      fp32(1/sqrt(128)), _quantize_lut with v_bits codes.
-//   _quantize_lut: ss = sum x^2 and dot = sum x * LUT[c] in the fixed pairwise
-//      order (v[i] + v[i + n/2], halving n: in-register levels first, then
-//      xor-shuffles 16, 8, 4, 2, 1, which add exactly the same pairs);
-//      rms = max(sqrt(ss / n), 1e-12); y = x / rms * LUT_MULT; code = number
-//      of LUT midpoints below y (ties go to the lower code);
-//      scale = (dot > 0 ? ss / max(dot, 1e-30) : 0) * LUT_ONE, LUT_ONE = 64,
-//      stored as fp16.
-//   The slot is assembled in shared memory (bit packing of the page's module
-//   text / _pack) and written with one 128-byte warp store.
+// Quantize (reference_quantize) lives in octave_quant.cu.
 // Decode (reference_attention, computed in the rotated space): one CTA per
 //   (split, q-head group, query token); the query is rotated like K (signs +
 //   64-dim blocks), each warp streams slots (one 32-bit word per lane,
@@ -45,257 +30,6 @@ __device__ __forceinline__ float load_in(const void *p, int bf16, int64_t idx) {
 
 __device__ __forceinline__ float sign_of(const OctaveParams &P, int d) {
   return ((P.sign_words[d >> 5] >> (d & 31)) & 1u) ? -1.f : 1.f;
-}
-
-// one cross-lane butterfly stage on lane-index bit h: v + o on the lower lane,
-// o - v on the upper one, as one FMA with sg = +-1 (sg * v is exact, so the
-// FMA rounds the same sum once)
-__device__ __forceinline__ float xstage(float v, float sg, int h) {
-  const float o = __shfl_xor_sync(kFull, v, h);
-  return __fmaf_rn(sg, v, o);
-}
-
-// sum over the 32 lanes of one value per lane, pairs (i, i + 16), (i, i + 8), ...
-__device__ __forceinline__ float xsum(float v) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(kFull, v, off));
-  return v;
-}
-
-struct LutSmem {
-  float lut[2][16];  // [0]: 3-bit (8 entries), [1]: 4-bit
-  float mid[2][15];
-};
-
-// Number of the 2^BITS - 1 sorted LUT midpoints below y (bucketize with
-// right=False: a tie goes to the lower code), by binary search.
-template <int BITS>
-__device__ __forceinline__ int bucket(float y, const float *mid) {
-  int c = 0;
-#pragma unroll
-  for (int step = 1 << (BITS - 1); step >= 1; step >>= 1)
-    if (mid[c + step - 1] < y) c += step;
-  return c;
-}
-
-// _quantize_lut over n = 64 (two values per lane: dims l, l + 32 of the block)
-// or n = 128 (four values per lane); codes out per value, returns the scale.
-template <int NV, int BITS>
-__device__ __forceinline__ float quantize_lut(const float (&x)[NV], float mult, const LutSmem &L,
-                                              int (&code)[NV]) {
-  constexpr int tb = BITS == 4 ? 1 : 0;
-  float sq[NV];
-#pragma unroll
-  for (int k = 0; k < NV; k++) sq[k] = __fmul_rn(x[k], x[k]);
-  // in-register levels: NV = 4 holds (l, l+32, l+64, l+96): first (l, l+64),
-  // (l+32, l+96) [n = 128 -> 64], then their sum [64 -> 32]; NV = 2: (l, l+32).
-  float ss;
-  if (NV == 4) ss = __fadd_rn(__fadd_rn(sq[0], sq[2]), __fadd_rn(sq[1], sq[3]));
-  else ss = __fadd_rn(sq[0], sq[1]);
-  ss = xsum(ss);
-  // ss / n for n = 64, 128: the product with the exact 1 / n is the same
-  // real number, so it rounds the same
-  float rms = __fsqrt_rn(__fmul_rn(ss, 1.f / (float)(NV * 32)));
-  rms = rms < 1e-12f ? 1e-12f : rms;
-  float pr[NV];
-#pragma unroll
-  for (int k = 0; k < NV; k++) {
-    const float y = __fmul_rn(__fdiv_rn(x[k], rms), mult);
-    const int c = bucket<BITS>(y, L.mid[tb]);
-    code[k] = c;
-    pr[k] = __fmul_rn(x[k], L.lut[tb][c]);
-  }
-  float dot;
-  if (NV == 4) dot = __fadd_rn(__fadd_rn(pr[0], pr[2]), __fadd_rn(pr[1], pr[3]));
-  else dot = __fadd_rn(pr[0], pr[1]);
-  dot = xsum(dot);
-  const float q = __fdiv_rn(ss, dot > 1e-30f ? dot : 1e-30f);
-  return __fmul_rn(dot > 0.f ? q : 0.f, kLutOne);
-}
-
-// Word w (bytes 4w .. 4w+3) of the packed codes of a region of n dims whose
-// codes (one per byte) start at c32 (layout of the page's module text):
-//   4-bit: byte j of a word holds dim 8w + j (low nibble) and 8w + 4 + j;
-//   3-bit: a 2-bit plane (byte j of word w gathers dims 16w + 4i + j in bits
-//          2i..2i+1) followed by a 1-bit plane (byte j of word w gathers dims
-//          32w + 4i + j in bit i); code = lo + 4 * hi.
-__device__ __forceinline__ uint32_t pack_word(const uint32_t *c32, int n, int bits, int w) {
-  if (bits == 4)
-    return (c32[2 * w] & 0x0F0F0F0Fu) | ((c32[2 * w + 1] & 0x0F0F0F0Fu) << 4);
-  if (w < n / 16) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(c32 + 4 * w);
-    return (v.x & 0x03030303u) | ((v.y & 0x03030303u) << 2) | ((v.z & 0x03030303u) << 4) |
-           ((v.w & 0x03030303u) << 6);
-  }
-  const int r = w - n / 16;
-  const uint4 u = *reinterpret_cast<const uint4 *>(c32 + 8 * r);
-  const uint4 v = *reinterpret_cast<const uint4 *>(c32 + 8 * r + 4);
-  return ((u.x >> 2) & 0x01010101u) | (((u.y >> 2) & 0x01010101u) << 1) |
-         (((u.z >> 2) & 0x01010101u) << 2) | (((u.w >> 2) & 0x01010101u) << 3) |
-         (((v.x >> 2) & 0x01010101u) << 4) | (((v.y >> 2) & 0x01010101u) << 5) |
-         (((v.z >> 2) & 0x01010101u) << 6) | (((v.w >> 2) & 0x01010101u) << 7);
-}
-
-template <bool BF16>
-__global__ void __launch_bounds__(kThreads)
-    octave_quantize_kernel(OctaveParams P, const void *__restrict__ key,
-                           const void *__restrict__ value, int num_tokens,
-                           int n_kv_heads, const int64_t *__restrict__ slot_mapping,
-                           uint8_t *__restrict__ cache, int block_size, int64_t num_blocks) {
-  __shared__ LutSmem L;
-  __shared__ __align__(16) uint8_t kcodes[kWarps][kHead];
-  __shared__ __align__(16) uint8_t vcodes[kWarps][kHead];
-  for (int i = threadIdx.x; i < 16; i += blockDim.x) {
-    L.lut[0][i] = i < 8 ? (float)P.lut3[i] : 0.f;
-    L.lut[1][i] = (float)P.lut4[i];
-    if (i < 7) L.mid[0][i] = ((float)P.lut3[i + 1] + (float)P.lut3[i]) / 2.0f;
-    if (i < 15) L.mid[1][i] = ((float)P.lut4[i + 1] + (float)P.lut4[i]) / 2.0f;
-  }
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t items = (int64_t)num_tokens * n_kv_heads;
-  const float vscale = 0.08838834764831845f;  // fp32(1 / sqrt(128))
-  const int slot_words = P.slot_bytes / 4;
-  const int w_kn = P.off_k_nope / 4, w_v = P.off_v / 4, w_sc = P.off_scales / 4;
-  const uint32_t *kc32 = reinterpret_cast<const uint32_t *>(kcodes[warp]);
-  const uint32_t *vc32 = reinterpret_cast<const uint32_t *>(vcodes[warp]);
-  float sg[4];  // signs of dims lane + 32k (K and V share them)
-#pragma unroll
-  for (int k = 0; k < 4; k++) sg[k] = sign_of(P, lane + 32 * k);
-  float bsg[5];  // butterfly signs of stages h = 1 .. 16
-#pragma unroll
-  for (int i = 0; i < 5; i++) bsg[i] = (lane >> i) & 1 ? -1.f : 1.f;
-  const bool idx32 = items <= 0x7fffffff;  // 32-bit index arithmetic suffices
-  for (int64_t it = (int64_t)blockIdx.x * kWarps + warp; it < items;
-       it += (int64_t)gridDim.x * kWarps) {
-    int tok, h;
-    if (idx32) {
-      tok = (int)it / n_kv_heads;
-      h = (int)it - tok * n_kv_heads;
-    } else {
-      tok = (int)(it / n_kv_heads);
-      h = (int)(it - (int64_t)tok * n_kv_heads);
-    }
-    const int64_t base = it * kHead;
-    // ---- K: 64-dim blocks (4-bit RoPE dims, 3-bit others) or, compact, one
-    // whole-head rotation with 3-bit codes and one scale
-    float x[4];
-#pragma unroll
-    for (int k = 0; k < 4; k++) {
-      const int d = lane + 32 * k;
-      x[k] = __fmul_rn(load_in(key, BF16, base + d), sg[k]);
-    }
-#pragma unroll
-    for (int i = 0; i < 5; i++)
-#pragma unroll
-      for (int k = 0; k < 4; k++) x[k] = xstage(x[k], bsg[i], 1 << i);
-    {  // h = 32 inside each 64-block: (l, l+32), (l+64, l+96)
-      float a = x[0], b = x[1];
-      x[0] = __fadd_rn(a, b);
-      x[1] = __fsub_rn(a, b);
-      a = x[2];
-      b = x[3];
-      x[2] = __fadd_rn(a, b);
-      x[3] = __fsub_rn(a, b);
-    }
-    float ks[2];
-    if (P.compact) {
-      float a = x[0], b = x[2];  // h = 64
-      x[0] = __fadd_rn(a, b);
-      x[2] = __fsub_rn(a, b);
-      a = x[1];
-      b = x[3];
-      x[1] = __fadd_rn(a, b);
-      x[3] = __fsub_rn(a, b);
-#pragma unroll
-      for (int k = 0; k < 4; k++) x[k] = __fmul_rn(x[k], vscale);
-      int ck[4];
-      ks[0] = quantize_lut<4, 3>(x, P.mult3, L, ck);
-      ks[1] = 0.f;
-#pragma unroll
-      for (int k = 0; k < 4; k++) kcodes[warp][lane + 32 * k] = (uint8_t)ck[k];
-    } else {
-#pragma unroll
-      for (int k = 0; k < 4; k++) x[k] = __fmul_rn(x[k], 0.125f);
-#pragma unroll
-      for (int kb = 0; kb < 2; kb++) {
-        float xb[2] = {x[2 * kb], x[2 * kb + 1]};
-        int cb[2];
-        if (kb * 64 < P.rope_dim) ks[kb] = quantize_lut<2, 4>(xb, P.mult4, L, cb);
-        else ks[kb] = quantize_lut<2, 3>(xb, P.mult3, L, cb);
-        kcodes[warp][64 * kb + lane] = (uint8_t)cb[0];
-        kcodes[warp][64 * kb + lane + 32] = (uint8_t)cb[1];
-      }
-    }
-    // ---- V
-#pragma unroll
-    for (int k = 0; k < 4; k++) {
-      const int d = lane + 32 * k;
-      x[k] = __fmul_rn(load_in(value, BF16, base + d), sg[k]);
-    }
-#pragma unroll
-    for (int i = 0; i < 5; i++)
-#pragma unroll
-      for (int k = 0; k < 4; k++) x[k] = xstage(x[k], bsg[i], 1 << i);
-    {
-      float a = x[0], b = x[1];  // h = 32
-      x[0] = __fadd_rn(a, b);
-      x[1] = __fsub_rn(a, b);
-      a = x[2];
-      b = x[3];
-      x[2] = __fadd_rn(a, b);
-      x[3] = __fsub_rn(a, b);
-      a = x[0];                  // h = 64
-      b = x[2];
-      x[0] = __fadd_rn(a, b);
-      x[2] = __fsub_rn(a, b);
-      a = x[1];
-      b = x[3];
-      x[1] = __fadd_rn(a, b);
-      x[3] = __fsub_rn(a, b);
-    }
-#pragma unroll
-    for (int k = 0; k < 4; k++) x[k] = __fmul_rn(x[k], vscale);
-    int cv[4];
-    const float vs = P.v_bits == 4 ? quantize_lut<4, 4>(x, P.mult4, L, cv)
-                                   : quantize_lut<4, 3>(x, P.mult3, L, cv);
-#pragma unroll
-    for (int k = 0; k < 4; k++) vcodes[warp][lane + 32 * k] = (uint8_t)cv[k];
-    __syncwarp();
-    // ---- slot words: lane w builds word w (and w + 32) of the slot
-    const int64_t sm = __ldg(slot_mapping + tok);
-    uint32_t *dst = nullptr;
-    if (sm >= 0) {
-      int64_t blk, off;
-      if (sm <= 0x7fffffff) {
-        blk = (int)sm / block_size;
-        off = (int)sm - (int)blk * block_size;
-      } else {
-        blk = sm / block_size;
-        off = sm - blk * block_size;
-      }
-      if (blk < num_blocks)
-        dst = reinterpret_cast<uint32_t *>(cache +
-                                           ((blk * n_kv_heads + h) * block_size + off) * P.slot_bytes);
-    }
-    for (int w = lane; w < slot_words; w += 32) {
-      uint32_t word = 0;
-      // the 4-bit regions (K RoPE dims, 4-bit V) share one path, as do the
-      // 3-bit ones, so that the warp runs each packing once
-      const bool kr = w < w_kn, vr = w >= w_v && w < w_sc;
-      if (kr || (vr && P.v_bits == 4)) word = pack_word(kr ? kc32 : vc32, 0, 4, kr ? w : w - w_v);
-      else if (w < w_sc)
-        word = vr ? pack_word(vc32, kHead, 3, w - w_v)
-                  : pack_word(kc32 + P.rope_dim / 4, kHead - P.rope_dim, 3, w - w_kn);
-      else if (w == w_sc)  // fp16 scales, K first then V
-        word = (uint32_t)__half_as_ushort(__float2half_rn(ks[0])) |
-               ((uint32_t)__half_as_ushort(__float2half_rn(P.compact ? vs : ks[1])) << 16);
-      else if (w == w_sc + 1 && !P.compact)
-        word = (uint32_t)__half_as_ushort(__float2half_rn(vs));
-      if (dst) dst[w] = word;
-    }
-    __syncwarp();
-  }
 }
 
 // ------------------------------------------------------------------ decode
@@ -499,34 +233,6 @@ __global__ void __launch_bounds__(kHead)
 }
 
 }  // namespace
-
-cudaError_t launch_octave_quantize(const OctaveParams &p, const void *key, const void *value,
-                                   int bf16, int num_tokens, int n_kv_heads,
-                                   const int64_t *slot_mapping, uint8_t *cache,
-                                   int block_size, int64_t num_blocks, cudaStream_t s) {
-  const int64_t items = (int64_t)num_tokens * n_kv_heads;
-  if (items == 0) return cudaSuccess;
-  // one wave of resident CTAs, each warp striding over the (token, head) items
-  static int resident[2] = {0, 0};
-  int &per_sm = resident[bf16 ? 1 : 0];
-  if (per_sm == 0) {
-    int n = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-        &n, bf16 ? octave_quantize_kernel<true> : octave_quantize_kernel<false>, kThreads, 0);
-    if (e != cudaSuccess) return e;
-    per_sm = n > 0 ? n : 1;
-  }
-  const int64_t blocks = (items + kWarps - 1) / kWarps;
-  const int64_t wave = (int64_t)kNumSMs * per_sm;
-  const int grid = (int)(blocks < wave ? blocks : wave);
-  if (bf16)
-    octave_quantize_kernel<true><<<grid, kThreads, 0, s>>>(p, key, value, num_tokens, n_kv_heads,
-                                                          slot_mapping, cache, block_size, num_blocks);
-  else
-    octave_quantize_kernel<false><<<grid, kThreads, 0, s>>>(p, key, value, num_tokens, n_kv_heads,
-                                                           slot_mapping, cache, block_size, num_blocks);
-  return cudaGetLastError();
-}
 
 DecodePlan plan_octave_decode(int num_q, int n_head_groups, int max_klen) {
   return plan_split_k(num_q * n_head_groups, max_klen, kNumSMs * 4, 1 << 20);

@@ -134,7 +134,8 @@ __global__ void __launch_bounds__(256, kB <= 16 ? 4 : 1)
       asm volatile("fma.rn.f32 %0, %1, %2, %0;" : "+f"(O) : "f"(w), "f"(v[k]));
     }
   }
-  ob[j] = L > 0.f ? O / L : 0.f;
+  // L = 0: no token (zero row); L NaN: a split that gave up (its record is NaN)
+  ob[j] = L > 0.f ? O / L : (L == 0.f ? 0.f : __int_as_float(0x7fc00000));
   __syncthreads();
   if (warp == 0) {
     float x[8];

@@ -5,6 +5,8 @@
 // Method: Strata PR #21 "Q4_0 KV cache + FWHT-256", How 1 and How 2, with the
 // maintainer's tie-break; stage order and end scaling: vLLM rocm_octave page,
 // fwht_blocks.
+#include <mutex>
+
 #include "q4_vec.cuh"
 
 namespace kvq {
@@ -145,8 +147,24 @@ FastDiv make_fastdiv(uint32_t d) {
   return f;
 }
 
+// Grid of a grid-stride kernel: one wave of the CTAs that fit on the SMs at
+// once (queried once per kernel), or fewer when there is less work.  A second,
+// partial wave would leave most SMs idle while it runs.
+template <auto Kernel>
 int grid_for(int64_t groups) {
-  int64_t cap = (int64_t)kNumSMs * 8;
+  static std::mutex mu;
+  static int per_sm = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (per_sm == 0) {
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, kThreads, 0) != cudaSuccess ||
+          n <= 0)
+        n = 1;
+      per_sm = n;
+    }
+  }
+  const int64_t cap = (int64_t)kNumSMs * per_sm;
   return (int)(groups < cap ? (groups > 0 ? groups : 1) : cap);
 }
 
@@ -154,9 +172,9 @@ int grid_for(int64_t groups) {
 
 cudaError_t launch_rotate(const void *x, int bf16, float *y, int64_t n_vec, cudaStream_t s) {
   if (n_vec == 0) return cudaSuccess;
-  const int grid = grid_for((n_vec + kVecPerCta - 1) / kVecPerCta);
-  if (bf16) rotate_kernel<true><<<grid, kThreads, 0, s>>>(x, y, n_vec);
-  else rotate_kernel<false><<<grid, kThreads, 0, s>>>(x, y, n_vec);
+  const int64_t groups = (n_vec + kVecPerCta - 1) / kVecPerCta;
+  if (bf16) rotate_kernel<true><<<grid_for<rotate_kernel<true>>(groups), kThreads, 0, s>>>(x, y, n_vec);
+  else rotate_kernel<false><<<grid_for<rotate_kernel<false>>(groups), kThreads, 0, s>>>(x, y, n_vec);
   return cudaGetLastError();
 }
 
@@ -165,19 +183,19 @@ cudaError_t launch_q4_append(const kvq_cache &c, const void *k, const void *v, i
                              int code_bits) {
   const int64_t n_vec = 2LL * batch * t_new * c.num_kv_heads;
   if (n_vec == 0) return cudaSuccess;
-  const int grid = grid_for((n_vec + kVecPerCta - 1) / kVecPerCta);
+  const int64_t groups = (n_vec + kVecPerCta - 1) / kVecPerCta;
   const FastDiv dh = make_fastdiv((uint32_t)c.num_kv_heads), dt = make_fastdiv((uint32_t)t_new);
+#define KVQ_APPEND(B, Q)                                                                     \
+  q4_append_kernel<B, Q><<<grid_for<q4_append_kernel<B, Q>>(groups), kThreads, 0, s>>>(      \
+      c, k, v, batch, t_new, start_pos, dh, dt)
   if (code_bits == 8) {
-    if (bf16)
-      q4_append_kernel<true, true><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
-    else
-      q4_append_kernel<false, true><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
+    if (bf16) KVQ_APPEND(true, true);
+    else KVQ_APPEND(false, true);
   } else {
-    if (bf16)
-      q4_append_kernel<true, false><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
-    else
-      q4_append_kernel<false, false><<<grid, kThreads, 0, s>>>(c, k, v, batch, t_new, start_pos, dh, dt);
+    if (bf16) KVQ_APPEND(true, false);
+    else KVQ_APPEND(false, false);
   }
+#undef KVQ_APPEND
   return cudaGetLastError();
 }
 

@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          int append_tiles, float *__restrict__ ws,
                          const void *__restrict__ k_new, const void *__restrict__ v_new,
                          const int32_t *__restrict__ pos, const int32_t *__restrict__ q_to_seq,
-                         int num_seqs) {
+                         int num_seqs, uint32_t *__restrict__ err, int wait_polls) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -378,8 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int it = gq; it < ntiles; it += 2) {
       const int st = it % kStages;
-      if (!mbar_wait(full0 + 8 * st, (it / kStages) & 1, abort_flag)) {
+      if (!mbar_wait(full0 + 8 * st, (it / kStages) & 1, abort_flag, wait_polls)) {
         *abort_flag = 1;
+        report(err, KVQ_DEVERR_WAIT_TIMEOUT);
         break;
       }
       const uint8_t *stage = smem + st * kStageBytes;
@@ -635,6 +636,8 @@ cudaError_t launch_q8_decode_mma(const kvq_cache &c, const void *q, int bf16, in
       configured[variant] |= bit;
     }
   }
+  uint32_t *err = device_error_word();
+  const int polls = wait_poll_limit();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = p.stream ? dim3(p.ctas) : dim3(p.splits, n_q_heads / gc, batch);
   cfg.blockDim = dim3(kThreads);
@@ -650,25 +653,25 @@ cudaError_t launch_q8_decode_mma(const kvq_cache &c, const void *q, int bf16, in
       e = cudaLaunchKernelEx(&cfg, q8_decode_mma_kernel<false, false>, maps, c, q, seq_lens, max_seq_len,
                            n_q_heads, group, gc, sl2, p.split_tokens, p.splits, n_hg,
                            p.n_units, append_tiles, ws, k_new, v_new,
-                           pos, q_to_seq, q_to_seq ? num_seqs : batch);
+                           pos, q_to_seq, q_to_seq ? num_seqs : batch, err, polls);
       break;
     case 1:
       e = cudaLaunchKernelEx(&cfg, q8_decode_mma_kernel<true, false>, maps, c, q, seq_lens, max_seq_len,
                            n_q_heads, group, gc, sl2, p.split_tokens, p.splits, n_hg,
                            p.n_units, append_tiles, ws, k_new, v_new,
-                           pos, q_to_seq, q_to_seq ? num_seqs : batch);
+                           pos, q_to_seq, q_to_seq ? num_seqs : batch, err, polls);
       break;
     case 2:
       e = cudaLaunchKernelEx(&cfg, q8_decode_mma_kernel<false, true>, maps, c, q, seq_lens, max_seq_len,
                            n_q_heads, group, gc, sl2, p.split_tokens, p.splits, n_hg,
                            p.n_units, append_tiles, ws, k_new, v_new,
-                           pos, q_to_seq, q_to_seq ? num_seqs : batch);
+                           pos, q_to_seq, q_to_seq ? num_seqs : batch, err, polls);
       break;
     default:
       e = cudaLaunchKernelEx(&cfg, q8_decode_mma_kernel<true, true>, maps, c, q, seq_lens, max_seq_len,
                            n_q_heads, group, gc, sl2, p.split_tokens, p.splits, n_hg,
                            p.n_units, append_tiles, ws, k_new, v_new,
-                           pos, q_to_seq, q_to_seq ? num_seqs : batch);
+                           pos, q_to_seq, q_to_seq ? num_seqs : batch, err, polls);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -29,8 +29,9 @@ EXPORTED = (
     "kvq_decode_attn_workspace", "kvq_decode_attn", "kvq_octave_layout_of",
     "kvq_octave_codebook", "kvq_octave_quantize", "kvq_octave_decode_attn_workspace",
     "kvq_octave_decode_attn", "kvq_decode_attn_noalloc", "kvq_decode_step",
-    "kvq_decode_attn_multi",
+    "kvq_decode_attn_multi", "kvq_device_errors", "kvq_set_wait_limit",
 )
+KVQ_DEVERR_WAIT_TIMEOUT, KVQ_DEVERR_BOUNDS = 1, 2
 
 
 class KVQError(RuntimeError):
@@ -107,6 +108,8 @@ def lib():
         L.kvq_decode_step.argtypes = [C.POINTER(CacheDesc), C.c_void_p, C.c_void_p, C.c_void_p,
                                       C.c_int, C.c_int32, C.c_int32, C.c_void_p, C.c_int32,
                                       C.c_float, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
+        L.kvq_device_errors.argtypes = [C.POINTER(C.c_uint32)]
+        L.kvq_set_wait_limit.argtypes = [C.c_int32]
         _lib = L
     return _lib
 
@@ -429,3 +432,20 @@ def octave_decode_attn(fmt: OctaveFormat, query: torch.Tensor, cache: torch.Tens
                sb.ctypes.data_as(C.c_void_p), _ptr(out), _ptr(workspace),
                workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
+
+
+# --------------------------------------------------------------------------
+# Diagnostics
+# --------------------------------------------------------------------------
+def device_errors() -> int:
+    """Flags recorded on the current device since the last call (cleared by
+    reading; synchronizes the device): KVQ_DEVERR_WAIT_TIMEOUT, KVQ_DEVERR_BOUNDS."""
+    f = C.c_uint32(0)
+    _check("kvq_device_errors", lib().kvq_device_errors(C.byref(f)))
+    return int(f.value)
+
+
+def set_wait_limit(polls: int = -1) -> None:
+    """Poll limit of the decode kernels' bounded waits (-1: the default)."""
+    _check("kvq_set_wait_limit", lib().kvq_set_wait_limit(int(polls)))
+

@@ -258,6 +258,41 @@ KVQ_API kvq_status kvq_decode_attn_noalloc(const kvq_cache *cache, const void *q
                                            float scale, float *out, void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* Conditions kernels cannot return as a status                               */
+/* ------------------------------------------------------------------------ */
+
+/* (The pages have no counterpart: these calls are diagnostics of this
+ * library.)  A kernel that meets a condition it cannot report through a
+ * kvq_status -- it runs after the call has returned -- ORs one of these flags
+ * into a 32-bit error word the library keeps on each device:
+ *   KVQ_DEVERR_WAIT_TIMEOUT  a decode kernel's bounded wait for a tile of the
+ *                            cache gave up (the poll limit below); the
+ *                            affected CTAs stop, their partial results are NaN
+ *                            and so are the outputs that include them;
+ *   KVQ_DEVERR_BOUNDS        a build compiled with KVQ_DEBUG_BOUNDS found a
+ *                            computed address outside the buffer it should
+ *                            lie in and skipped the access. */
+#define KVQ_DEVERR_WAIT_TIMEOUT 1u
+#define KVQ_DEVERR_BOUNDS 2u
+
+/* kvq_device_errors -- the error word of the current device: *flags gets the
+ * OR of the flags recorded since the previous call, and the word is cleared.
+ * Unlike every other call this one synchronizes the device (it reads the word
+ * after all work on the device has finished); KVQ_ERR_CUDA if that or the
+ * copy fails.  flags: host pointer. */
+KVQ_API kvq_status kvq_device_errors(uint32_t *flags);
+
+/* kvq_set_wait_limit -- poll limit of the decode kernels' bounded waits on
+ * their tile loads, for kernels launched after the call (process-wide).
+ * Each poll waits up to about 1 us; the default (polls = -1) is 2^20, far
+ * beyond any load that is merely slow.  polls = 0 makes each wait a single
+ * non-blocking test, so that a wait on a tile still in flight gives up: a way
+ * to exercise the timeout path (KVQ_DEVERR_WAIT_TIMEOUT, NaN outputs) without
+ * a fault.  After giving up, a CTA still waits, with the default limit, for
+ * the copies it has issued before it exits.  polls < -1: KVQ_ERR_INVALID_ARG. */
+KVQ_API kvq_status kvq_set_wait_limit(int32_t polls);
+
+/* ------------------------------------------------------------------------ */
 /* Octave variant (vLLM API page "vllm.v1.attention.ops.rocm_octave")        */
 /* ------------------------------------------------------------------------ */
 
@@ -290,7 +325,8 @@ KVQ_API kvq_status kvq_octave_layout_of(const kvq_octave_fmt *fmt, kvq_octave_la
 KVQ_API kvq_status kvq_octave_codebook(int32_t bits, int8_t *lut, float *lut_mult);
 
 /* kvq_octave_quantize -- reference_quantize into a paged cache.
- *   key, value: device, [num_tokens][num_kv_heads][head_size] of `dtype`.
+ *   key, value: device, [num_tokens][num_kv_heads][head_size] of `dtype`,
+ *   16-byte aligned.
  *   d_slot_mapping: device int64[num_tokens]; token i goes to block
  *   slot / block_size, offset slot % block_size; a negative slot or a block
  *   outside [0, num_blocks) skips the token.

@@ -134,3 +134,9 @@ def test_noalloc_checks_arguments_before_its_size(L):
     assert call(hq=8 * 32) == kvq.KVQ_ERR_UNSUPPORTED
     assert call(batch=109) == kvq.KVQ_ERR_INVALID_ARG  # above the contiguous capacity
     assert call(batch=0) == kvq.KVQ_OK
+
+
+def test_device_error_calls_validate_on_host(L):
+    assert L.kvq_device_errors(None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_set_wait_limit(-2) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_set_wait_limit(-1) == kvq.KVQ_OK

@@ -242,3 +242,52 @@ def test_compact_decode_vs_oracle(v_bits, G):
     want = oracle.octave_attention(q, cache.cpu().numpy(), bt, q_to_req, q_to_klen, fmt,
                                    128 ** -0.5, signs)
     assert np.abs(got - want).max() <= ATOL
+
+
+@pytest.mark.parametrize("fmt", [(128, 64, 4, 0), (128, 64, 3, 0), (128, 0, 4, 0),
+                                 (128, 128, 3, 0), (128, 64, 3, 1), (128, 64, 4, 1)],
+                         ids=lambda f: "-".join(map(str, f)))
+def test_quantize_stress_bitexact(fmt):
+    """2^20 (token, head) vectors for k3v4 (2^16 for the other formats) whose
+    magnitudes span 2^-40 .. 2^40 per vector, with exact zeros, repeated
+    values and single spikes mixed in: every slot bit-identical to the oracle.
+    The kernel takes codes from a floor table of 2 y except within 2^-13 of a
+    doubled midpoint, where it redoes the IEEE division; this drives both
+    paths and the zero / tiny-vector cases."""
+    n_tok, Hkv = (131072, 8) if fmt == (128, 64, 4, 0) else (8192, 8)
+    F = kvq.OctaveFormat(128, fmt[1], fmt[2], bool(fmt[3]))
+    slot_bytes = F.layout()["slot_bytes"]
+    rng = np.random.default_rng(sum(fmt) + fmt[1])
+    k = synth.gaussian(900 + fmt[2], (n_tok, Hkv, 128))
+    v = synth.gaussian(901 + fmt[2], (n_tok, Hkv, 128))
+    scale = np.exp2(rng.integers(-40, 41, size=(n_tok, Hkv, 1))).astype(np.float32)
+    k *= scale
+    v *= scale[::-1]
+    k[rng.random((n_tok, Hkv)) < 0.002] = 0.0          # all-zero vectors
+    v[rng.random((n_tok, Hkv, 128)) < 0.01] = 0.0      # scattered exact zeros
+    rep = rng.random((n_tok, Hkv)) < 0.01              # constant vectors
+    k[rep] = np.float32(1.5)
+    spike = rng.random((n_tok, Hkv)) < 0.01            # one large element
+    k[spike, 3] *= np.float32(1e4)
+    kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+    slot = np.arange(n_tok, dtype=np.int64)
+    bs = 256
+    nblk = n_tok // bs
+    signs = synth.sign_pattern(128)
+    cache = torch.zeros((nblk, Hkv, bs, slot_bytes), dtype=torch.uint8, device="cuda")
+    kvq.octave_quantize(F, to_dev(kb), to_dev(vb), to_dev(slot), cache, kvq.sign_words(signs))
+    want = oracle.octave_quantize(kb, vb, fmt, signs, threads=oracle.host_threads())
+    got = cache.cpu().numpy().transpose(0, 2, 1, 3).reshape(-1, Hkv, slot_bytes)
+    bad = np.nonzero(np.any(got != want, axis=-1))
+    assert bad[0].size == 0, f"{bad[0].size} slots differ, first (token, head) {list(zip(*bad))[:3]}"
+
+
+def test_quantize_rejects_misaligned_inputs():
+    F = kvq.OctaveFormat(128, 64, 4)
+    k = torch.zeros(2 * 128 * 2 + 8, dtype=torch.bfloat16, device="cuda")
+    cache = torch.zeros((1, 2, 16, 128), dtype=torch.uint8, device="cuda")
+    slot = torch.zeros(1, dtype=torch.int64, device="cuda")
+    kk = k[4:4 + 256].view(1, 2, 128)  # 8 bytes past a 16-byte boundary
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.octave_quantize(F, kk, kk, slot, cache, kvq.sign_words(synth.sign_pattern(128)))
+    assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
