@@ -79,6 +79,27 @@ __device__ __forceinline__ int64_t q4_row(const kvq_cache &c, int b, int h, int 
   return ((int64_t)page * c.num_kv_heads + h) * c.page_size + (t - pi * c.page_size);
 }
 
+// ---------------------------------------------------------------- bounds
+// Rows of the cache planes (contiguous or paged).
+__device__ __forceinline__ int64_t cache_rows(const kvq_cache &c) {
+  return c.block_table ? (int64_t)c.num_pages * c.num_kv_heads * c.page_size
+                       : (int64_t)c.batch_capacity * c.num_kv_heads * c.max_tokens;
+}
+// Debug builds (compiled with KVQ_DEBUG_BOUNDS): true if [lo, hi) lies
+// inside [0, n); otherwise KVQ_DEVERR_BOUNDS goes into the error word and the
+// caller skips or redirects the access.  Release builds: always true (the
+// index arithmetic keeps every access inside the buffers the call describes).
+__device__ __forceinline__ bool in_bounds(int64_t lo, int64_t hi, int64_t n, uint32_t *err) {
+#ifdef KVQ_DEBUG_BOUNDS
+  if (lo >= 0 && lo <= hi && hi <= n) return true;
+  if (err != nullptr) atomicOr(err, KVQ_DEVERR_BOUNDS);
+  return false;
+#else
+  (void)lo, (void)hi, (void)n, (void)err;
+  return true;
+#endif
+}
+
 // ---------------------------------------------------------------- errors
 // Device address of the library's error word on the current device (nullptr
 // if the lookup fails), and the mbarrier poll limit of the decode kernels'

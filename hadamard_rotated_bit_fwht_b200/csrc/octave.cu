@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(kThreads)
                                int max_blocks, const int32_t *__restrict__ q_to_req,
                                const int32_t *__restrict__ q_to_klen, int max_klen,
                                float scale_log2, int split_tokens, int splits,
-                               float *__restrict__ ws) {
+                               float *__restrict__ ws, uint32_t *__restrict__ err) {
   __shared__ float qs[GC][kHead];
   __shared__ float lut[2][16];
   __shared__ float red_m[kWarps][GC], red_l[kWarps][GC];
@@ -102,7 +102,9 @@ __global__ void __launch_bounds__(kThreads)
   for (int t = t0 + warp; t < t1; t += kWarps) {
     const int blk = __ldg(block_table + (int64_t)req * max_blocks + t / block_size);
     if (blk < 0 || blk >= num_blocks) continue;
-    const uint8_t *sp = cache + (((int64_t)blk * n_kv_heads + kvh) * block_size + (t % block_size)) * P.slot_bytes;
+    const int64_t si = ((int64_t)blk * n_kv_heads + kvh) * block_size + (t % block_size);
+    if (!in_bounds(si, si + 1, num_blocks * n_kv_heads * block_size, err)) continue;
+    const uint8_t *sp = cache + si * P.slot_bytes;
     const uint32_t myword = lane < P.slot_bytes / 4 ? __ldg(reinterpret_cast<const uint32_t *>(sp) + lane) : 0u;
     // scales
     const uint32_t s01 = slot_byte(myword, P.off_scales) | (slot_byte(myword, P.off_scales + 1) << 8);
@@ -272,13 +274,14 @@ cudaError_t launch_octave_decode(const OctaveParams &P, const void *query, int b
       octave_decode_split_kernel<G, true><<<grid, kThreads, 0, s>>>(                         \
           P, query, n_q_heads, group, cache, n_kv_heads, block_size, num_blocks, block_table, \
           num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2, plan.split_tokens,        \
-          plan.splits, ws);                                                                   \
+          plan.splits, ws, err);                                                              \
     else                                                                                      \
       octave_decode_split_kernel<G, false><<<grid, kThreads, 0, s>>>(                        \
           P, query, n_q_heads, group, cache, n_kv_heads, block_size, num_blocks, block_table, \
           num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2, plan.split_tokens,        \
-          plan.splits, ws);                                                                   \
+          plan.splits, ws, err);                                                              \
   } while (0)
+  uint32_t *err = device_error_word();
   switch (gc) {
     case 1: KVQ_LAUNCH(1); break;
     case 2: KVQ_LAUNCH(2); break;

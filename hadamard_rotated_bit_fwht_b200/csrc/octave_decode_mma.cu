@@ -14,10 +14,13 @@
 //     those bytes are B-fragment registers as they stand.  The rotated query
 //     of each head is scaled by S = 127 * 2^14 / max|q|, rounded to an
 //     integer and split exactly into three int8 digits
-//     (S q = 2^14 H + 2^7 M + L, |M|, |L| <= 64): one A tile holds H (rows
-//     0-7) and M (rows 8-15), a second one L (rows 0-7); their columns are
-//     stored in the order the codes arrive in.  Per (block, 8 tokens) the
-//     digit dot products are combined in fp32 (2^14 d_H + (2^7 d_M + d_L))
+//     (S q = 2^14 H + 2^7 M + L, |M|, |L| <= 64).  Up to 4 heads per CTA, one
+//     A tile holds all three: H in rows 0-3, L in rows 4-7, M in rows 8-11,
+//     and the L dot products come from the lanes 16 apart by one shuffle; with
+//     more heads one A tile holds H (rows 0-7) and M (rows 8-15), a second
+//     one L.  The columns are stored in the order the codes arrive in.  Per
+//     (block, 8 tokens) the digit dot products are combined in fp32
+//     (2^14 d_H + (2^7 d_M + d_L))
 //     and multiplied by the block scale; 1 / S joins the softmax scale.  The
 //     query is thereby carried to 2.4e-7 of its largest element.  (Two
 //     digits, 14 bits, left up to 2.3e-3 of error in the outputs of the
@@ -141,7 +144,8 @@ __device__ __forceinline__ int qcol_dim(int vc, int k) {
                 : 64 + 16 * tg + 8 * (vc - 2) + 4 * hi + j;
 }
 
-template <bool BF16>
+// PACK: gc <= 4, the three query digits in one A tile
+template <bool BF16, bool PACK>
 __global__ void __launch_bounds__(kThreads, 4)
     octave_decode_mma_kernel(OctaveParams P, const void *__restrict__ query, int n_q_heads,
                              int group, int gc, const uint8_t *__restrict__ cache, int n_kv_heads,
@@ -150,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 4)
                              int max_blocks, const int32_t *__restrict__ q_to_req,
                              const int32_t *__restrict__ q_to_klen, int max_klen,
                              float scale_log2, int split_tokens, int splits,
-                             float *__restrict__ ws) {
+                             float *__restrict__ ws, uint32_t *__restrict__ err) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int s = blockIdx.x, hg = blockIdx.y, qi = blockIdx.z;
   const int h0 = hg * gc, kvh = h0 / group;
@@ -243,10 +247,19 @@ __global__ void __launch_bounds__(kThreads, 4)
     const float r1 = x - 16384.f * hi;  // |r1| <= 2^13
     const float mid = rintf(r1 * 0.0078125f);
     const float lo = rintf(r1 - 128.f * mid);  // |lo| <= 64
-    qrow[hh * kQStride + col] = (uint8_t)(int8_t)(int)hi;
-    qrow[(8 + hh) * kQStride + col] = (uint8_t)(int8_t)(int)mid;
-    qrow[(16 + hh) * kQStride + col] = (uint8_t)(int8_t)(int)lo;
-    qrow[(24 + hh) * kQStride + col] = 0;
+    if (PACK) {  // H rows 0-3, L rows 4-7, M rows 8-11, zero rows 12-15
+      if (hh < 4) {
+        qrow[hh * kQStride + col] = (uint8_t)(int8_t)(int)hi;
+        qrow[(4 + hh) * kQStride + col] = (uint8_t)(int8_t)(int)lo;
+        qrow[(8 + hh) * kQStride + col] = (uint8_t)(int8_t)(int)mid;
+        qrow[(12 + hh) * kQStride + col] = 0;
+      }
+    } else {
+      qrow[hh * kQStride + col] = (uint8_t)(int8_t)(int)hi;
+      qrow[(8 + hh) * kQStride + col] = (uint8_t)(int8_t)(int)mid;
+      qrow[(16 + hh) * kQStride + col] = (uint8_t)(int8_t)(int)lo;
+      qrow[(24 + hh) * kQStride + col] = 0;
+    }
   }
   __syncthreads();
   uint32_t qa[4][4], qb[4][4];  // A fragments of the virtual chunks: (H, M) and (L, 0)
@@ -256,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 #pragma unroll
     for (int vc = 0; vc < 4; vc++) {
       ldsm_x4(qaddr + 32 * vc, qa[vc]);
-      ldsm_x4(qaddr + 16 * kQStride + 32 * vc, qb[vc]);
+      if (!PACK) ldsm_x4(qaddr + 16 * kQStride + 32 * vc, qb[vc]);
     }
   }
   // FWHT-64 blocks carry 1 / 8; the query ints carry S
@@ -276,9 +289,9 @@ __global__ void __launch_bounds__(kThreads, 4)
       const int bi = bs_shift >= 0 ? t >> bs_shift : t / block_size;
       const int blk = __ldg(block_table + (int64_t)req * max_blocks + bi);
       ok = blk >= 0 && blk < num_blocks;
-      if (ok)
-        src = cache + (((int64_t)blk * n_kv_heads + kvh) * block_size + (t - bi * block_size)) *
-                          P.slot_bytes;
+      const int64_t si = ((int64_t)blk * n_kv_heads + kvh) * block_size + (t - bi * block_size);
+      ok = ok && in_bounds(si, si + 1, num_blocks * n_kv_heads * block_size, err);
+      if (ok) src = cache + si * P.slot_bytes;
     }
     if (lc0 == 0) smem[kOffV + (it % kStages) * kTile + lr] = ok ? 1 : 0;
     const uint32_t rowa = smem_u32(st) + lr * 128;
@@ -344,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 4)
           const uint32_t w = kr[m];
           const uint32_t b0 = lut4_bytes(w & 0xFFFFu, T4), b1 = lut4_bytes(w >> 16, T4);
           imma16832(accr[T], qa[c], b0, b1);
-          imma16832(accrl[T], qb[c], b0, b1);
+          if (!PACK) imma16832(accrl[T], qb[c], b0, b1);
         }
       }
       {  // NoPE: 2-bit plane chunk 2, 1-bit plane in chunk 3 (words 0, 1)
@@ -372,8 +385,10 @@ __global__ void __launch_bounds__(kThreads, 4)
           }
           imma16832(accn[T], qa[2], R[0], R[1]);
           imma16832(accn[T], qa[3], R[2], R[3]);
-          imma16832(accnl[T], qb[2], R[0], R[1]);
-          imma16832(accnl[T], qb[3], R[2], R[3]);
+          if (!PACK) {
+            imma16832(accnl[T], qb[2], R[0], R[1]);
+            imma16832(accnl[T], qb[3], R[2], R[3]);
+          }
         }
       }
       float2 sacc[2];
@@ -382,7 +397,14 @@ __global__ void __launch_bounds__(kThreads, 4)
         const float2 dr = *reinterpret_cast<const float2 *>(fsc + 16 * warp + 8 * T + 2 * tg);
         const float2 dn =
             *reinterpret_cast<const float2 *>(fsc + kTile + 16 * warp + 8 * T + 2 * tg);
-        // digit dots: H in [0..1], M in [2..3] (rows g + 8), L in the second tile's [0..1]
+        if (PACK) {  // L sits in rows 4-7: the [0..1] of the lanes 16 apart
+#pragma unroll
+          for (int e = 0; e < 2; e++) {
+            accrl[T][e] = __shfl_xor_sync(kFull, accr[T][e], 16);
+            accnl[T][e] = __shfl_xor_sync(kFull, accn[T][e], 16);
+          }
+        }
+        // digit dots: H in [0..1], M in [2..3] (rows g + 8), L in accrl / accnl [0..1]
         const float r0 = fmaf((float)accr[T][0], 16384.f, (float)(accr[T][2] * 128 + accrl[T][0]));
         const float r1 = fmaf((float)accr[T][1], 16384.f, (float)(accr[T][3] * 128 + accrl[T][1]));
         const float n0 = fmaf((float)accn[T][0], 16384.f, (float)(accn[T][2] * 128 + accnl[T][0]));
@@ -539,15 +561,15 @@ cudaError_t launch_octave_decode_mma(const OctaveParams &P, const void *query, i
   dim3 grid(plan.splits, n_q_heads / gc, num_q);
   const float sl2 = scale * kLog2e;
   if (bf16)
-    octave_decode_mma_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(
+    (gc <= 4 ? octave_decode_mma_kernel<true, true> : octave_decode_mma_kernel<true, false>)<<<grid, kThreads, kSmemBytes, s>>>(
         P, query, n_q_heads, group, gc, cache, n_kv_heads, block_size, num_blocks, block_table,
         num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2, plan.split_tokens,
-        plan.splits, ws);
+        plan.splits, ws, device_error_word());
   else
-    octave_decode_mma_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(
+    (gc <= 4 ? octave_decode_mma_kernel<false, true> : octave_decode_mma_kernel<false, false>)<<<grid, kThreads, kSmemBytes, s>>>(
         P, query, n_q_heads, group, gc, cache, n_kv_heads, block_size, num_blocks, block_table,
         num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2, plan.split_tokens,
-        plan.splits, ws);
+        plan.splits, ws, device_error_word());
   return cudaGetLastError();
 }
 

@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     octave_quant_kernel(const __grid_constant__ OctaveParams P, const void *__restrict__ key,
                         const void *__restrict__ value, int64_t items, int n_kv_heads,
                         const int64_t *__restrict__ slot_mapping, uint8_t *__restrict__ cache,
-                        int block_size, int64_t num_blocks) {
+                        int block_size, int64_t num_blocks, uint32_t *__restrict__ err) {
   __shared__ QTables T;
   extern __shared__ float2 xs_all[];  // [64 pairs][kThreads]
   for (int t = threadIdx.x; t < 1024; t += blockDim.x) {
@@ -309,9 +309,9 @@ __global__ void __launch_bounds__(kThreads, 3)
     uint32_t *dst = nullptr;  // the slot, or null for a skipped token
     if (sm >= 0) {
       const int64_t blk = sm / block_size, off = sm - blk * block_size;
-      if (blk < num_blocks)
-        dst = reinterpret_cast<uint32_t *>(cache + ((blk * n_kv_heads + h) * block_size + off) *
-                                                       (int64_t)kSlotBytes);
+      const int64_t si = (blk * n_kv_heads + h) * block_size + off;
+      if (blk < num_blocks && in_bounds(si, si + 1, num_blocks * n_kv_heads * block_size, err))
+        dst = reinterpret_cast<uint32_t *>(cache + si * (int64_t)kSlotBytes);
     }
     const void *krow = static_cast<const char *>(key) + it * kHead * (BF16 ? 2 : 4);
     const void *vrow = static_cast<const char *>(value) + it * kHead * (BF16 ? 2 : 4);
@@ -379,7 +379,7 @@ cudaError_t launch_one(const OctaveParams &p, const void *key, const void *value
   const int64_t wave = (int64_t)kNumSMs * resident;
   const int grid = (int)(blocks < wave ? blocks : wave);
   kern<<<grid, kThreads, kXsBytes, s>>>(p, key, value, items, n_kv_heads, slot_mapping, cache,
-                                        block_size, num_blocks);
+                                        block_size, num_blocks, device_error_word());
   return cudaGetLastError();
 }
 

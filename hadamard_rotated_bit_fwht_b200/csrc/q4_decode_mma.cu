@@ -256,6 +256,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // of one page, else each half that holds tokens of the split on its own.
     // (A tile of 8 copies with 16-byte scale boxes kept the issuing thread busy
     // about twice as long.)
+    // first row of a run of scale rows, inside the planes (debug builds check
+    // and report; release builds use it as is)
+    auto scale_src = [&](int64_t r, int n) -> int64_t {
+      return in_bounds(r, r + n, cache_rows(c), err) ? r : 0;
+    };
     auto issue = [&](int it) {
       const int st = it % kStages;
       const int tstart = t0 + it * kTile;
@@ -267,8 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_tx(bar, 2 * kTile * 128 + 2 * nrows * 16);
         tma_load_2d(dst + kOffKC, &maps.kc, 0, r, bar);
         tma_load_2d(dst + kOffVC, &maps.vc, 0, r, bar);
-        bulk_load(dst + kOffKS, c.k_scales + (int64_t)r * kRowScales, nrows * 16, bar);
-        bulk_load(dst + kOffVS, c.v_scales + (int64_t)r * kRowScales, nrows * 16, bar);
+        bulk_load(dst + kOffKS, c.k_scales + scale_src(r, nrows) * kRowScales, nrows * 16, bar);
+        bulk_load(dst + kOffVS, c.v_scales + scale_src(r, nrows) * kRowScales, nrows * 16, bar);
       } else {
         const int r0 = sub_row(tstart);
         const int r1 = tstart + kSub < t1 ? sub_row(tstart + kSub) : -1;
@@ -280,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_tx(bar, 2 * kSubBytes);
           tma_load_2d(dst + kOffKC, &maps.kc2, 0, r0, bar);
           tma_load_2d(dst + kOffVC, &maps.vc2, 0, r0, bar);
-          bulk_load(dst + kOffKS, c.k_scales + (int64_t)r0 * kRowScales, kTile * 16, bar);
-          bulk_load(dst + kOffVS, c.v_scales + (int64_t)r0 * kRowScales, kTile * 16, bar);
+          bulk_load(dst + kOffKS, c.k_scales + scale_src(r0, kTile) * kRowScales, kTile * 16, bar);
+          bulk_load(dst + kOffVS, c.v_scales + scale_src(r0, kTile) * kRowScales, kTile * 16, bar);
         } else {
           mbar_arrive_tx(bar, n * kSubBytes);
           #pragma unroll
@@ -290,8 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (r < 0) continue;
             tma_load_2d(dst + kOffKC + j * kSub * 128, &maps.kc, 0, r, bar);
             tma_load_2d(dst + kOffVC + j * kSub * 128, &maps.vc, 0, r, bar);
-            bulk_load(dst + kOffKS + j * kSub * 16, c.k_scales + (int64_t)r * kRowScales, kSub * 16, bar);
-            bulk_load(dst + kOffVS + j * kSub * 16, c.v_scales + (int64_t)r * kRowScales, kSub * 16, bar);
+            bulk_load(dst + kOffKS + j * kSub * 16, c.k_scales + scale_src(r, kSub) * kRowScales, kSub * 16, bar);
+            bulk_load(dst + kOffVS + j * kSub * 16, c.v_scales + scale_src(r, kSub) * kRowScales, kSub * 16, bar);
           }
         }
       }
@@ -317,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint16_t sc;
         q4v::quantize_vector<BF16>(valid ? src : k_new, valid, lane, scratch + 64 * vg, bytes, sc);
         const int64_t row = q4_row(c, bs, kvh, p_new);
-        if (valid && row >= 0) {
+        if (valid && row >= 0 && in_bounds(row, row + 1, cache_rows(c), err)) {
           *reinterpret_cast<uint4 *>((vg ? c.v_codes : c.k_codes) + row * kRowCodeBytes + 16 * i) =
               bytes;
           (vg ? c.v_scales : c.k_scales)[row * kRowScales + i] = sc;

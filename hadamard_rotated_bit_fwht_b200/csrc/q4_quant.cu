@@ -65,7 +65,7 @@ template <bool BF16, bool Q8>
 __global__ void __launch_bounds__(kThreads, 5)
     q4_append_kernel(kvq_cache c, const void *__restrict__ k, const void *__restrict__ v,
                      int batch, int t_new, const int32_t *__restrict__ start_pos,
-                     FastDiv div_heads, FastDiv div_tnew) {
+                     FastDiv div_heads, FastDiv div_tnew, uint32_t *__restrict__ err) {
   __shared__ float4 smem[kWarps][kVecPerWarp][64];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int vg = lane >> 3, i = lane & 7;
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 5)
       const uint32_t b = fdiv(bt, div_tnew);
       const int tok = (int)(bt - b * div_tnew.d);
       const int64_t row = q4_row(c, (int)b, h, __ldg(start_pos + b) + tok);
-      if (row >= 0) {
+      if (row >= 0 && in_bounds(row, row + 1, cache_rows(c), err)) {
         uint16_t *scales = (is_v ? c.v_scales : c.k_scales) + row * kRowScales;
         if (Q8) {
           uint8_t *codes = (is_v ? c.v_codes : c.k_codes) + row * 256;
@@ -185,9 +185,10 @@ cudaError_t launch_q4_append(const kvq_cache &c, const void *k, const void *v, i
   if (n_vec == 0) return cudaSuccess;
   const int64_t groups = (n_vec + kVecPerCta - 1) / kVecPerCta;
   const FastDiv dh = make_fastdiv((uint32_t)c.num_kv_heads), dt = make_fastdiv((uint32_t)t_new);
+  uint32_t *err = device_error_word();
 #define KVQ_APPEND(B, Q)                                                                     \
   q4_append_kernel<B, Q><<<grid_for<q4_append_kernel<B, Q>>(groups), kThreads, 0, s>>>(      \
-      c, k, v, batch, t_new, start_pos, dh, dt)
+      c, k, v, batch, t_new, start_pos, dh, dt, err)
   if (code_bits == 8) {
     if (bf16) KVQ_APPEND(true, true);
     else KVQ_APPEND(false, true);

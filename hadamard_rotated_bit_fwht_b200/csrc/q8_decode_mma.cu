@@ -263,6 +263,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (page < 0 || page >= c.num_pages) return -1;
       return (int)(((int64_t)page * c.num_kv_heads + kvh) * c.page_size + (t - pi * c.page_size));
     };
+    // first row of a run of scale rows, inside the planes (debug builds check
+    // and report; release builds use it as is)
+    auto scale_src = [&](int64_t r, int n) -> int64_t {
+      return in_bounds(r, r + n, cache_rows(c), err) ? r : 0;
+    };
     auto issue = [&](int it) {
       const int st = it % kStages;
       const int r = tile_row(t0 + it * kTile);
@@ -277,8 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t dst = smem_u32(smem + st * kStageBytes);
         tma_load_3d(dst + kOffKC, &maps.kc, 0, r, 0, bar);
         tma_load_3d(dst + kOffVC, &maps.vc, 0, r, 0, bar);
-        bulk_load(dst + kOffKS, c.k_scales + (int64_t)r * kRowScales, nrows * 16, bar);
-        bulk_load(dst + kOffVS, c.v_scales + (int64_t)r * kRowScales, nrows * 16, bar);
+        bulk_load(dst + kOffKS, c.k_scales + scale_src(r, nrows) * kRowScales, nrows * 16, bar);
+        bulk_load(dst + kOffVS, c.v_scales + scale_src(r, nrows) * kRowScales, nrows * 16, bar);
       }
       atomicMax(const_cast<int *>(issued), it + 1);
     };
@@ -302,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint16_t sc;
         q4v::quantize_vector_q8<BF16>(valid ? src : k_new, valid, lane, scratch + 64 * vg, bytes, sc);
         const int64_t row = q4_row(c, bs, kvh, p_new);
-        if (valid && row >= 0) {
+        if (valid && row >= 0 && in_bounds(row, row + 1, cache_rows(c), err)) {
           uint8_t *dst = (vg ? c.v_codes : c.k_codes) + row * kCodeRow + 32 * i;
           *reinterpret_cast<uint4 *>(dst) = bytes[0];
           *reinterpret_cast<uint4 *>(dst + 16) = bytes[1];
