@@ -60,7 +60,8 @@ TRAFFIC_SOURCES = {
     "q4_decode_combine": _DECODE,
     "q4_append_prefill": _COMMON + ["q4_vec.cuh", "q4_quant.cu"],
     "octave_decode": _COMMON + ["octave.cu", "octave_decode_mma.cu"],
-    "octave_quantize": _COMMON + ["octave.cu"],
+    "octave_quantize": _COMMON + ["octave_quant.cuh", "octave_quant.cu",
+                                  "octave_quant_bf16_v3.cu", "octave_quant_bf16_v4.cu"],
 }
 
 

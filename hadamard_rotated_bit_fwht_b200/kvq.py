@@ -126,12 +126,15 @@ def _check(fn, status):
 
 
 def _stream(stream=None):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return C.c_void_p(s.cuda_stream)
+    if stream is not None:
+        return stream.cuda_stream
+    # the raw handle of torch's current stream on the current device, without
+    # building a Stream object (this sits on the per-token decode path)
+    return torch._C._cuda_getCurrentRawStream(torch.cuda.current_device())
 
 
 def _ptr(t):
-    return None if t is None else C.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -187,6 +190,7 @@ class Q4Cache:
         append a single sequence of a paged batch)."""
         view = Q4Cache.__new__(Q4Cache)
         view.__dict__.update(self.__dict__)
+        view.__dict__.pop("_desc", None)
         view.block_table = block_table.to(device=self.k_codes.device,
                                           dtype=torch.int32).contiguous()
         return view
@@ -198,12 +202,18 @@ class Q4Cache:
         return self.block_table.shape[1] * self.page_size
 
     def desc(self) -> CacheDesc:
-        bt = self.block_table
-        return CacheDesc(self.k_codes.data_ptr(), self.k_scales.data_ptr(),
-                         self.v_codes.data_ptr(), self.v_scales.data_ptr(),
-                         self.num_kv_heads, 256, self.max_tokens, self.batch_capacity,
-                         None if bt is None else bt.data_ptr(), self.page_size,
-                         0 if bt is None else bt.shape[1], self.num_pages, self.bits)
+        """The C descriptor, built once (the planes and the block table of a
+        Q4Cache object never change; with_block_table makes a new object)."""
+        d = self.__dict__.get("_desc")
+        if d is None:
+            bt = self.block_table
+            d = CacheDesc(self.k_codes.data_ptr(), self.k_scales.data_ptr(),
+                          self.v_codes.data_ptr(), self.v_scales.data_ptr(),
+                          self.num_kv_heads, 256, self.max_tokens, self.batch_capacity,
+                          None if bt is None else bt.data_ptr(), self.page_size,
+                          0 if bt is None else bt.shape[1], self.num_pages, self.bits)
+            self._desc = d
+        return d
 
     def nbytes_per_row(self):
         return 2 * (32 * self.bits + 16)

@@ -20,14 +20,17 @@
  *     memory of the current CUDA device; "host" pointers to host memory.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
  *     call is asynchronous on that stream; the library never allocates, never
- *     frees and never synchronizes.
+ *     frees and never synchronizes (the one exception is the diagnostic
+ *     kvq_device_errors, which reads the device error word after the device
+ *     has finished its work).
  *   - Argument checks happen on the host before any launch and return
  *     KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED / KVQ_ERR_WORKSPACE without
  *     touching the GPU.  A failed launch returns KVQ_ERR_CUDA.  Values that live
  *     in device memory (positions, lengths, page tables) cannot be checked on
  *     the host; the kernels clamp them so that no access leaves the buffers the
  *     caller described, and document what an out-of-range value does.
- *   - Kernels never trap or assert.
+ *   - Kernels never trap or assert; what they cannot return as a status they
+ *     record in the device error word (kvq_device_errors).
  *   - Inputs must be finite; the bit-exact contract for the quantizers covers
  *     finite inputs whose 32-value blocks have max |value| either 0 or at least
  *     2^-120 (below that the reciprocal of the block scale overflows).
