@@ -26,9 +26,13 @@
 //     digits, 14 bits, left up to 2.3e-3 of error in the outputs of the
 //     16 x 16384-token workload, whose keys carry x16 outlier channels.)
 //   * PV on the fp16 path (m16n8k16, fp32 accumulation): A = V^T codes through
-//     the biased table (each byte u becomes the exact fp16 1024 + u by pairing
-//     it with 0x64; one half2 subtract of 1152 leaves LUT[c]), read by
-//     ldmatrix.trans from the swizzled tile; B = p * s_v / 64 split hi + lo.
+//     the biased table (each byte u becomes the exact fp16 1024 + u = LUT[c] +
+//     1152 by pairing it with 0x64), read by ldmatrix.trans from the swizzled
+//     tile; B = p * s_v / 64 split hi + lo.  One more MMA per 16 tokens, with
+//     an all-ones A, sums B over the tokens, and the merge subtracts 1152
+//     times that sum.  Up to 4 heads per CTA, the hi parts sit in B columns
+//     0-3 and the lo parts in columns 4-7 (one MMA per tile instead of two);
+//     the merge adds the two halves.
 //     The V region starts 8 bytes into a 16-byte chunk: the used halves of
 //     chunks 3 and 7 are joined by one lane shuffle, so the 64 V bytes make
 //     exactly 8 M-tiles.
@@ -118,13 +122,13 @@ __device__ __forceinline__ uint32_t lut4_bytes(uint32_t sel, const Lut4 &T) {
   const uint32_t m = prmt(sel << 4, sel, 0xD9C8u);
   return lop3_sel(plo, phi, m);
 }
-// biased bytes (a, b) of R -> half2 (LUT, LUT) exactly: (1024 + U) - 1152
+// biased bytes (a, b) of R -> half2 (1024 + U, 1024 + U) exactly, U = LUT + 128;
+// the 1152 this adds to every code leaves the PV products as 1152 * sum_t w
+// per head, which the merge takes off
 __device__ __forceinline__ uint32_t lut_half2(uint32_t R, uint32_t selector) {
-  const uint32_t h = prmt(R, 0x64646464u, selector);
-  const __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&h),
-                            __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
-  return *reinterpret_cast<const uint32_t *>(&v);
+  return prmt(R, 0x64646464u, selector);
 }
+constexpr float kVBias = 1152.f;
 
 __device__ __forceinline__ void split_hilo(float2 w, uint32_t &hi, uint32_t &lo) {
   __half2 h = __float22half2_rn(w);
@@ -305,6 +309,8 @@ __global__ void __launch_bounds__(kThreads, 4)
   float o[8][4];
 #pragma unroll
   for (int mt = 0; mt < 8; mt++) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  float wsum[4] = {0.f, 0.f, 0.f, 0.f};  // sum_t of the B columns, as the PV MMAs see them
+  const uint32_t ones[4] = {0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u};
   float m_run = -INFINITY, l_run = 0.f;
   float *fsc = reinterpret_cast<float *>(smem + kOffF);
 
@@ -427,8 +433,11 @@ __global__ void __launch_bounds__(kThreads, 4)
         const float alpha = exp2f(m_run - mn);
         m_run = mn;
         l_run *= alpha;
-        const float a0 = __shfl_sync(kFull, alpha, 8 * tg);
-        const float a1 = __shfl_sync(kFull, alpha, 8 * tg + 4);
+        // columns 2tg, 2tg + 1 belong to heads 2tg, 2tg + 1 (PACK: to heads
+        // (2tg) & 3, (2tg + 1) & 3, hi in columns 0-3 and lo in 4-7)
+        const int src = PACK ? 8 * (tg & 1) : 8 * tg;
+        const float a0 = __shfl_sync(kFull, alpha, src);
+        const float a1 = __shfl_sync(kFull, alpha, src + 4);
 #pragma unroll
         for (int mt = 0; mt < 8; mt++) {
           o[mt][0] *= a0;
@@ -436,6 +445,10 @@ __global__ void __launch_bounds__(kThreads, 4)
           o[mt][2] *= a0;
           o[mt][3] *= a1;
         }
+        wsum[0] *= a0;
+        wsum[1] *= a1;
+        wsum[2] *= a0;
+        wsum[3] *= a1;
       }
       float p[4];
 #pragma unroll
@@ -458,6 +471,18 @@ __global__ void __launch_bounds__(kThreads, 4)
       uint32_t bh0, bl0, bh1, bl1;
       split_hilo(w0, bh0, bl0);
       split_hilo(w1, bh1, bl1);
+      if (PACK) {  // columns 4-7: the lo parts of heads 0-3 (lanes 16 apart)
+        const uint32_t xl0 = __shfl_xor_sync(kFull, bl0, 16);
+        const uint32_t xl1 = __shfl_xor_sync(kFull, bl1, 16);
+        if (g >= 4) {
+          bh0 = xl0;
+          bh1 = xl1;
+        }
+        mma16816(wsum, ones, bh0, bh1);
+      } else {
+        mma16816(wsum, ones, bh0, bh1);
+        mma16816(wsum, ones, bl0, bl1);
+      }
       // x2.trans: matrices (T0, chunk), (T1, chunk); lanes 0..15 give the rows
       const int vrow = 16 * warp + (lane & 15);
       const uint32_t vaddr = base + vrow * 128;
@@ -486,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 4)
                                  lut_half2(R1, 0x4240u), lut_half2(R1, 0x4341u)};
           float(&acc)[4] = o[2 * vc + par];
           mma16816(acc, a, bh0, bh1);
-          mma16816(acc, a, bl0, bl1);
+          if (!PACK) mma16816(acc, a, bl0, bl1);
         }
       }
     }
@@ -511,7 +536,14 @@ __global__ void __launch_bounds__(kThreads, 4)
       // V byte of row g: joined chunk -> 2g (+48 for g >= 4); chunk 3 + vc -> 16 vc - 8 + 2g
       const int vb = (vc == 0 ? (g < 4 ? 2 * g : 48 + 2 * g) : 16 * vc - 8 + 2 * g) + par;
       const int d = 8 * (vb >> 2) + (vb & 3);  // low nibble; high nibble is d + 4
-      const float(&acc)[4] = o[2 * vc + par];
+      float acc[4];
+#pragma unroll
+      for (int e = 0; e < 4; e++) acc[e] = fmaf(-kVBias, wsum[e & 1], o[2 * vc + par][e]);
+      if (PACK) {  // hi (columns 0-3, tg < 2) + lo (columns 4-7, tg + 2)
+#pragma unroll
+        for (int e = 0; e < 4; e++) acc[e] += __shfl_xor_sync(kFull, acc[e], 2);
+        if (tg >= 2) continue;
+      }
       float *w = red_o + warp * 8 * kHead;
       w[(2 * tg) * kHead + d] = acc[0];
       w[(2 * tg + 1) * kHead + d] = acc[1];
