@@ -63,13 +63,13 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
       : "memory");
   return done != 0;
 }
-// true once the phase with this parity has completed; false after `polls`
-// polls (0: one non-blocking test) or once *abort is set (by any thread of
-// the CTA)
+// true once the phase with this parity has completed; false after one
+// non-blocking test and `polls` further polls (0: the test alone), or once
+// *abort is set (by any thread of the CTA).  The common case, a tile that has
+// already landed, is the one test and a branch.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           const volatile int *abort, int polls) {
-  if (polls <= 0) return mbar_test(bar, parity);
-  if (mbar_try(bar, parity)) return true;
+  if (mbar_test(bar, parity)) return true;
   for (int i = 0; i < polls; i++) {
     if (mbar_try(bar, parity)) return true;
     if (*abort) return false;

@@ -255,8 +255,13 @@ __device__ __forceinline__ void q4_quantize_l1(const float r[32], int lane, int 
     // element-in-block i + 8m: byte i = c0 | c2 << 4, byte i + 8 = c1 | c3 << 4
     const uint32_t x02 = min_u16x2(__byte_perm(__float_as_uint(f02.x), __float_as_uint(f02.y), 0x5410), fifteen);
     const uint32_t x13 = min_u16x2(__byte_perm(__float_as_uint(f13.x), __float_as_uint(f13.y), 0x5410), fifteen);
-    const uint32_t y02 = x02 | (x02 >> 12), y13 = x13 | (x13 >> 12);
-    o.items[B] = __byte_perm(y02, y13, 0x0040);  // (byte i, byte i + 8) in the low 16 bits
+    // y = x + (x >> 12) = x | (x >> 12) (no overlapping bits), as a high
+    // multiply-add; item = y02 + 256 y13 in the low 16 bits
+    uint32_t y02, y13, it;
+    asm("mad.hi.u32 %0, %1, 1048576, %1;" : "=r"(y02) : "r"(x02));
+    asm("mad.hi.u32 %0, %1, 1048576, %1;" : "=r"(y13) : "r"(x13));
+    asm("mad.lo.u32 %0, %1, 256, %2;" : "=r"(it) : "r"(y13), "r"(y02));
+    o.items[B] = it;  // (byte i, byte i + 8) in the low 16 bits
   }
 }
 
