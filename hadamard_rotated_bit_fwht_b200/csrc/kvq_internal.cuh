@@ -25,7 +25,11 @@ __device__ __forceinline__ uint4 ldg_stream_u4(const void *p) {
   return r;
 }
 
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16lo(uint32_t w) {
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, 65536, 0;" : "=r"(r) : "r"(w));
+  return __uint_as_float(r);
+}
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // ---------------------------------------------------------------- packed fp32

@@ -103,15 +103,29 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(s));
   return r;
 }
+// a * 2^k + b and (a >> (32 - k)) + b as integer multiply-adds, which issue
+// to the FMA pipe (this kernel's ALU pipe is its busiest)
+template <int K>
+__device__ __forceinline__ uint32_t shl_add(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "n"(1u << K), "r"(b));
+  return r;
+}
+template <int K>
+__device__ __forceinline__ uint32_t shr_add(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "n"(1u << (32 - K)), "r"(b));
+  return r;
+}
 __device__ __forceinline__ uint32_t lop3_sel(uint32_t lo, uint32_t hi, uint32_t m) {
   uint32_t r;  // m ? hi : lo, bitwise
   asm("lop3.b32 %0, %1, %2, %3, 0xD8;" : "=r"(r) : "r"(lo), "r"(hi), "r"(m));
   return r;
 }
 
-// Table bytes T[c] for four nibble-packed 4-bit codes (sel bits 0-15): two
-// 8-entry lookups on the low three bits, then a per-byte choice by the fourth
-// bit (sign-replicated into a mask by prmt).
+// Table bytes T[c] for four nibble-packed 4-bit codes (sel bits 0-15; the
+// higher bits are ignored): two 8-entry lookups on the low three bits, then a
+// per-byte choice by the fourth bit (sign-replicated into a mask by prmt).
 struct Lut4 {
   uint32_t lo0, lo1, hi0, hi1;
 };
@@ -119,7 +133,7 @@ __device__ __forceinline__ uint32_t lut4_bytes(uint32_t sel, const Lut4 &T) {
   const uint32_t s = sel & 0x7777u;
   const uint32_t plo = prmt(T.lo0, T.lo1, s);
   const uint32_t phi = prmt(T.hi0, T.hi1, s);
-  const uint32_t m = prmt(sel << 4, sel, 0xD9C8u);
+  const uint32_t m = prmt(shl_add<4>(sel, 0u), sel, 0xD9C8u);
   return lop3_sel(plo, phi, m);
 }
 // biased bytes (a, b) of R -> half2 (1024 + U, 1024 + U) exactly, U = LUT + 128;
@@ -141,11 +155,15 @@ __device__ __forceinline__ void split_hilo(float2 w, uint32_t &hi, uint32_t &lo)
 // Head dim of column k (0..31) of the query's virtual chunk vc: chunks 0, 1
 // follow the RoPE codes as lut4_bytes returns them (word of lane tg = dims
 // 32 vc + 8 tg + 0..7, bytes in the order 0 4 1 5 | 2 6 3 7); chunks 2, 3 the
-// NoPE codes (lane tg: dims 64 + 16 tg + 8 (vc - 2) + 0..7 in order).
+// NoPE codes as the NoPE lookup returns them: lane tg holds dims
+// 64 + 16 tg + 4 f + j (2-bit field f of plane byte j), chunk 2 fields 0 and
+// 2, chunk 3 fields 1 and 3, byte order (f, j) = (a, 0) (a + 2, 0) (a, 1)
+// (a + 2, 1) | the same for j = 2, 3.
 __device__ __forceinline__ int qcol_dim(int vc, int k) {
-  const int tg = (k & 15) >> 2, j = k & 3, hi = k >> 4;
-  return vc < 2 ? 32 * vc + 8 * tg + 2 * hi + (j >> 1) + 4 * (j & 1)
-                : 64 + 16 * tg + 8 * (vc - 2) + 4 * hi + j;
+  const int tg = (k & 15) >> 2, jp = k & 3, hi = k >> 4;
+  if (vc < 2) return 32 * vc + 8 * tg + 2 * hi + (jp >> 1) + 4 * (jp & 1);
+  const int f = (vc - 2) + 2 * (jp & 1), j = 2 * hi + (jp >> 1);
+  return 64 + 16 * tg + 4 * f + j;
 }
 
 // PACK: gc <= 4, the three query digits in one A tile
@@ -361,7 +379,8 @@ __global__ void __launch_bounds__(kThreads, 4)
         for (int m = 0; m < 4; m++) {
           const int T = m & 1, c = m >> 1;
           const uint32_t w = kr[m];
-          const uint32_t b0 = lut4_bytes(w & 0xFFFFu, T4), b1 = lut4_bytes(w >> 16, T4);
+          // lut4_bytes reads selector bits 0..15 only
+          const uint32_t b0 = lut4_bytes(w, T4), b1 = lut4_bytes(shr_add<16>(w, 0u), T4);
           imma16832(accr[T], qa[c], b0, b1);
           if (!PACK) imma16832(accrl[T], qb[c], b0, b1);
         }
@@ -373,22 +392,29 @@ __global__ void __launch_bounds__(kThreads, 4)
           ldsm_x4(chunk_addr(2 + mc), r4);  // (T0, c2), (T1, c2), (T0, c3), (T1, c3)
           lo[0] = r4[0];
           lo[1] = r4[1];
-          // the 1-bit plane word this lane needs (tg >> 1) sits in lane 4g + (tg >> 1)
-          hi[0] = __shfl_sync(kFull, r4[2], (lane & ~3) | (tg >> 1));
-          hi[1] = __shfl_sync(kFull, r4[3], (lane & ~3) | (tg >> 1));
+          // the 1-bit plane word this lane needs (tg >> 1) sits in lane 4g + (tg >> 1),
+          // its 4 bits per byte at 4 (tg & 1)
+          hi[0] = __shfl_sync(kFull, r4[2], (lane & ~3) | (tg >> 1)) >> (4 * (tg & 1));
+          hi[1] = __shfl_sync(kFull, r4[3], (lane & ~3) | (tg >> 1)) >> (4 * (tg & 1));
         }
 #pragma unroll
         for (int T = 0; T < 2; T++) {
+          // code of dim 16tg + 4f + j: 2-bit field f of lo byte j, bit f of hi
+          // byte j on top.  Fields f and f + 2 go to the low and high nibble of
+          // byte j (disjoint bits, so the multiply-adds only place them), and
+          // each 16-bit half is then a selector of four codes.
+          const uint32_t h = hi[T];
+          uint32_t x02 = lo[T] & 0x33333333u;                 // fields 0, 2
+          x02 = shl_add<2>(h & 0x01010101u, x02);             // bit 0 -> 2
+          x02 = shl_add<4>(h & 0x04040404u, x02);             // bit 2 -> 6
+          uint32_t x13 = shr_add<2>(lo[T] & 0xCCCCCCCCu, 0u);  // fields 1, 3
+          x13 = shl_add<1>(h & 0x02020202u, x13);             // bit 1 -> 2
+          x13 = shl_add<3>(h & 0x08080808u, x13);             // bit 3 -> 6
           uint32_t R[4];
-#pragma unroll
-          for (int i = 0; i < 4; i++) {
-            // code byte j: (lo >> 2i) & 3 | ((hi >> (4(tg & 1) + i)) & 1) << 2
-            const uint32_t lb = (lo[T] >> (2 * i)) & 0x03030303u;
-            const uint32_t hb = (hi[T] >> (4 * (tg & 1) + i)) & 0x01010101u;
-            uint32_t x = hb * 4u + lb;
-            x = x | (x >> 4);
-            R[i] = prmt(T3lo, T3hi, prmt(x, 0u, 0x0020u));  // dims 16tg + 4i + 0..3
-          }
+          R[0] = prmt(T3lo, T3hi, x02);
+          R[1] = prmt(T3lo, T3hi, shr_add<16>(x02, 0u));
+          R[2] = prmt(T3lo, T3hi, x13);
+          R[3] = prmt(T3lo, T3hi, shr_add<16>(x13, 0u));
           imma16832(accn[T], qa[2], R[0], R[1]);
           imma16832(accn[T], qa[3], R[2], R[3]);
           if (!PACK) {

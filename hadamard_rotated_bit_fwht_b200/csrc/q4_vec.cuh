@@ -178,6 +178,13 @@ __device__ __forceinline__ float key_value(uint32_t key) {
   return __uint_as_float((key >> 1) | ((~key & 1u) << 31));
 }
 
+// three-input maximum (one instruction on sm_100); exact, like fmaxf
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
@@ -201,9 +208,11 @@ __device__ __forceinline__ void q4_quantize_l1(const float r[32], int lane, int 
   for (int B = 0; B < 8; B++) {
     const int r0 = 4 * (B & 1) + 8 * (B >> 1);
     const float z0 = r[r0], z1 = r[r0 + 1], z2 = r[r0 + 2], z3 = r[r0 + 3];
-    const float am = fmaxf(fmaxf(fabsf(z0), fabsf(z1)), fmaxf(fabsf(z2), fabsf(z3)));
-    const float mz = fmaxf(fmaxf(z0, z1), fmaxf(z2, z3));
-    key[B] = (__float_as_uint(am) << 1) | (mz == am ? 1u : 0u);
+    const float am = fmaxf(max3f(fabsf(z0), fabsf(z1), fabsf(z2)), fabsf(z3));
+    const float mz = fmaxf(max3f(z0, z1, z2), z3);
+    uint32_t k;
+    asm("mad.lo.u32 %0, %1, 2, %2;" : "=r"(k) : "r"(__float_as_uint(am)), "r"(mz == am ? 1u : 0u));
+    key[B] = k;
   }
   // transposed max-reduction over the 8 lanes of the vector: each xor level
   // halves the blocks a lane keeps, so lane i ends with the key of block i
@@ -298,7 +307,7 @@ __device__ __forceinline__ void q8_quantize_l1(const float r[32], int lane, int 
 #pragma unroll
   for (int B = 0; B < 8; B++) {
     const int r0 = 4 * (B & 1) + 8 * (B >> 1);
-    const float am = fmaxf(fmaxf(fabsf(r[r0]), fabsf(r[r0 + 1])), fmaxf(fabsf(r[r0 + 2]), fabsf(r[r0 + 3])));
+    const float am = fmaxf(max3f(fabsf(r[r0]), fabsf(r[r0 + 1]), fabsf(r[r0 + 2])), fabsf(r[r0 + 3]));
     key[B] = __float_as_uint(am);
   }
 #pragma unroll
