@@ -31,6 +31,13 @@ __device__ __forceinline__ float bf16lo(uint32_t w) {
   return __uint_as_float(r);
 }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// maximum that returns NaN if either input is NaN (split-K combines: a record
+// left NaN by a split that gave up must reach the output)
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
 
 // ---------------------------------------------------------------- packed fp32
 // Packed fp32x2 arithmetic.  Used only where no multiply feeds an add

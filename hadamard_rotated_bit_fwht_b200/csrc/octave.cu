@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kHead)
   if (req < 0 || req >= num_reqs) klen = 0;
   const float *rec = ws + (int64_t)qh * splits * kORec;
   float M = -INFINITY;
-  for (int s = 0; s < splits && klen > 0; s++) M = fmaxf(M, rec[s * kORec]);
+  for (int s = 0; s < splits && klen > 0; s++) M = fmax_nan(M, rec[s * kORec]);
   float L = 0.f, O = 0.f;
   if (klen > 0 && M != -INFINITY) {
     for (int s = 0; s < splits; s++) {
@@ -220,7 +220,8 @@ __global__ void __launch_bounds__(kHead)
       O += rec[s * kORec + 4 + j] * f;
     }
   }
-  ob[j] = L > 0.f ? O / L : 0.f;
+  // L = 0: no token; L NaN: a split that gave up (its record is NaN)
+  ob[j] = L > 0.f ? O / L : (L == 0.f ? 0.f : __int_as_float(0x7fc00000));
   for (int h = 1; h < kHead; h <<= 1) {
     __syncthreads();
     if (j < 64) {

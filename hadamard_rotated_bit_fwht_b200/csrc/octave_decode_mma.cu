@@ -40,7 +40,9 @@
 // the 128-byte XOR swizzle through a 3-stage ring; each row is addressed
 // through the block table by one lookup, so any block size works, and a
 // token whose block entry names no block contributes nothing.
-#include "kvq_internal.cuh"
+#include <cstring>
+
+#include "decode_common.cuh"
 
 namespace kvq {
 namespace {
@@ -59,7 +61,13 @@ constexpr int kOffF = kStages * kStageBytes;  // fp32 scales [3][64] of the curr
 constexpr int kOffV = kOffF + 3 * kTile * 4;  // per stage, per token: 1 if its block is mapped
 constexpr int kQStride = 144;                 // int8 query row: 128 B + 16 B pad
 constexpr int kOffQ = kOffV + kStages * kTile;  // int8 query rows: 0-7 H, 8-15 M, 16-23 L, 24-31 zero
-constexpr int kSmemBytes = kOffQ + 32 * kQStride;
+constexpr int kOffBar = kOffQ + 32 * kQStride;  // TMA staging: full barriers [kStages]
+constexpr int kOffTok = kOffBar + 8 * kStages;  // TMA staging: 1 if the tile's block is mapped [kStages]
+constexpr int kOffAbort = kOffTok + 8;          // TMA staging: a wait gave up
+constexpr int kSmemUsed = kOffAbort + 8;
+constexpr int kSmemBytes = kSmemUsed + 1024;    // slack for the 1024-byte alignment
+static_assert(kStageBytes % 1024 == 0, "stages keep the 128-byte swizzle atoms aligned");
+static_assert(kOffBar % 8 == 0, "mbarrier alignment");
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -166,10 +174,14 @@ __device__ __forceinline__ int qcol_dim(int vc, int k) {
   return 64 + 16 * tg + 4 * f + j;
 }
 
-// PACK: gc <= 4, the three query digits in one A tile
-template <bool BF16, bool PACK>
+// PACK: gc <= 4, the three query digits in one A tile.  TMA: the tiles come
+// by one 64-row tensor copy each (block sizes that are multiples of 64: a
+// tile lies in one block), staged through mbarriers; otherwise by cp.async,
+// row by row through the block table.
+template <bool BF16, bool PACK, bool TMA>
 __global__ void __launch_bounds__(kThreads, 4)
-    octave_decode_mma_kernel(OctaveParams P, const void *__restrict__ query, int n_q_heads,
+    octave_decode_mma_kernel(const __grid_constant__ CUtensorMap slots, int wait_polls,
+                             OctaveParams P, const void *__restrict__ query, int n_q_heads,
                              int group, int gc, const uint8_t *__restrict__ cache, int n_kv_heads,
                              int block_size, int64_t num_blocks,
                              const int32_t *__restrict__ block_table, int num_reqs,
@@ -177,7 +189,8 @@ __global__ void __launch_bounds__(kThreads, 4)
                              const int32_t *__restrict__ q_to_klen, int max_klen,
                              float scale_log2, int split_tokens, int splits,
                              float *__restrict__ ws, uint32_t *__restrict__ err) {
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int s = blockIdx.x, hg = blockIdx.y, qi = blockIdx.z;
   const int h0 = hg * gc, kvh = h0 / group;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -302,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 4)
   const int lr = tid >> 1, lc0 = 4 * (tid & 1);
   // block index of a token: a shift for power-of-two block sizes
   const int bs_shift = (block_size & (block_size - 1)) == 0 ? __ffs(block_size) - 1 : -1;
-  auto issue = [&](int it) {
+  auto issue = [&](int it) {  // cp.async staging (all threads)
     uint8_t *st = smem + (it % kStages) * kStageBytes;
     const int t = t0 + it * kTile + lr;
     bool ok = t < t1;
@@ -324,6 +337,44 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
   };
 
+  // TMA staging: thread 0 issues each tile as one 64 x 128-byte box of the
+  // slot rows (the map's 128-byte swizzle is the XOR pattern used above) and
+  // records whether its block is mapped
+  const uint32_t full0 = smem_u32(smem + kOffBar);
+  volatile uint8_t *tok = smem + kOffTok;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffAbort);
+  int issued = 0;  // thread 0: tiles issued so far
+  auto issue_tma = [&](int it) {
+    const int st = it % kStages;
+    const int t = t0 + it * kTile;  // a multiple of 64, inside one block
+    const int bi = bs_shift >= 0 ? t >> bs_shift : t / block_size;
+    const int blk = __ldg(block_table + (int64_t)req * max_blocks + bi);
+    bool ok = blk >= 0 && blk < num_blocks;
+    const int64_t row = ((int64_t)blk * n_kv_heads + kvh) * block_size + (t - bi * block_size);
+    ok = ok && in_bounds(row, row + kTile, num_blocks * n_kv_heads * block_size, err);
+    tok[st] = ok ? 1 : 0;
+    const uint32_t bar = full0 + 8 * st;
+    if (ok) {
+      dec::mbar_arrive_tx(bar, kStageBytes);
+      dec::tma_load_2d(smem_u32(smem + st * kStageBytes), &slots, 0, (int)row, bar);
+    } else {
+      dec::mbar_arrive(bar);
+    }
+    issued = it + 1;
+  };
+  if (TMA) {
+    if (tid == 0) {
+      dec::prefetch_map(&slots);
+#pragma unroll
+      for (int i = 0; i < kStages; i++) dec::mbar_init(full0 + 8 * i, 1);
+      *abort_flag = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      // the query set-up above wrote stage 0 through the generic proxy
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncthreads();
+  }
+
   float o[8][4];
 #pragma unroll
   for (int mt = 0; mt < 8; mt++) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
@@ -332,14 +383,30 @@ __global__ void __launch_bounds__(kThreads, 4)
   float m_run = -INFINITY, l_run = 0.f;
   float *fsc = reinterpret_cast<float *>(smem + kOffF);
 
+  if (TMA) {
+    if (tid == 0)
+      for (int i = 0; i < kStages - 1 && i < ntiles; i++) issue_tma(i);
+  } else {
 #pragma unroll
-  for (int i = 0; i < kStages - 1; i++) {
-    if (i < ntiles) issue(i);
-    cp_async_commit();
+    for (int i = 0; i < kStages - 1; i++) {
+      if (i < ntiles) issue(i);
+      cp_async_commit();
+    }
   }
+  bool aborted = false;
   for (int it = 0; it < ntiles; it++) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
+    if (TMA) {
+      if (!dec::mbar_wait(full0 + 8 * (it % kStages), (it / kStages) & 1, abort_flag, wait_polls))
+        *abort_flag = 1;
+      __syncthreads();
+      if (*abort_flag) {  // read by every thread after the barrier: a uniform exit
+        aborted = true;
+        break;
+      }
+    } else {
+      cp_async_wait<kStages - 2>();
+      __syncthreads();
+    }
     uint8_t *st = smem + (it % kStages) * kStageBytes;
     if (tid < kTile) {  // scales at bytes 120..125 (chunk 7, offset 8): fp16 -> fp32 / 64
       const int r = tid;
@@ -351,15 +418,28 @@ __global__ void __launch_bounds__(kThreads, 4)
       fsc[kTile + r] = f01.y * 0.015625f;
       fsc[2 * kTile + r] = __half2float(__ushort_as_half((uint16_t)w2)) * 0.015625f;
     }
-    if (it + kStages - 1 < ntiles) issue(it + kStages - 1);
-    cp_async_commit();
+    if (TMA) {
+      // every thread is past the barrier above, so the stage of tile it - 1
+      // is free; its generic reads precede the async-proxy write
+      if (tid == 0 && it + kStages - 1 < ntiles) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue_tma(it + kStages - 1);
+      }
+    } else {
+      if (it + kStages - 1 < ntiles) issue(it + kStages - 1);
+      cp_async_commit();
+    }
     __syncthreads();
 
     // bit k: token k of this warp's 16 is in range and on a mapped block
     const unsigned okmask =
-        __ballot_sync(kFull, (lane < 16) &&
-                                 smem[kOffV + (it % kStages) * kTile + 16 * warp + (lane & 15)] != 0) &
-        0xFFFFu;
+        TMA ? __ballot_sync(kFull, (lane < 16) && tok[it % kStages] != 0 &&
+                                       t0 + it * kTile + 16 * warp + (lane & 15) < t1) &
+                  0xFFFFu
+            : __ballot_sync(kFull,
+                            (lane < 16) &&
+                                smem[kOffV + (it % kStages) * kTile + 16 * warp + (lane & 15)] != 0) &
+                  0xFFFFu;
     if (okmask != 0) {
       const bool partial = okmask != 0xFFFFu;
       const uint32_t base = smem_u32(st);
@@ -542,7 +622,30 @@ __global__ void __launch_bounds__(kThreads, 4)
       }
     }
   }
-  cp_async_wait<0>();
+  if (TMA) {
+    if (aborted) {
+      // a tile never arrived: let the copies still in flight land (bounded,
+      // ignoring the flag) before shared memory is reused, then write NaN
+      // records, which the combine turns into NaN outputs
+      if (tid == 0) {
+        dec::report(err, KVQ_DEVERR_WAIT_TIMEOUT);
+        for (int j = issued > kStages ? issued - kStages : 0; j < issued; j++)
+          for (int i = 0; i < dec::kWaitPolls && !dec::mbar_try(full0 + 8 * (j % kStages), (j / kStages) & 1); i++) {
+          }
+      }
+      __syncthreads();
+      const float nan = __int_as_float(0x7fc00000);
+      for (int p = tid; p < gc * kHead; p += kThreads) {
+        const int hh = p >> 7, j = p & 127;
+        float *rec = ws + (((int64_t)qi * n_q_heads + h0 + hh) * splits + s) * kORec;
+        rec[4 + j] = nan;
+        if (j == 0) rec[0] = rec[1] = nan;
+      }
+      return;
+    }
+  } else {
+    cp_async_wait<0>();
+  }
   __syncthreads();
 
   // ---- merge the warps and write the partial records
@@ -618,16 +721,31 @@ cudaError_t launch_octave_decode_mma(const OctaveParams &P, const void *query, i
   const int gc = group < 8 ? group : 8;
   dim3 grid(plan.splits, n_q_heads / gc, num_q);
   const float sl2 = scale * kLog2e;
-  if (bf16)
-    (gc <= 4 ? octave_decode_mma_kernel<true, true> : octave_decode_mma_kernel<true, false>)<<<grid, kThreads, kSmemBytes, s>>>(
-        P, query, n_q_heads, group, gc, cache, n_kv_heads, block_size, num_blocks, block_table,
-        num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2, plan.split_tokens,
-        plan.splits, ws, device_error_word());
-  else
-    (gc <= 4 ? octave_decode_mma_kernel<false, true> : octave_decode_mma_kernel<false, false>)<<<grid, kThreads, kSmemBytes, s>>>(
-        P, query, n_q_heads, group, gc, cache, n_kv_heads, block_size, num_blocks, block_table,
-        num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2, plan.split_tokens,
-        plan.splits, ws, device_error_word());
+  // one 64-row tensor copy per tile when every tile lies in one block (block
+  // sizes that are multiples of 64; the splits are whole 64-token tiles) and
+  // the slot rows fit the map's 32-bit coordinate
+  const int64_t rows = num_blocks * n_kv_heads * block_size;
+  CUtensorMap map;
+  std::memset(&map, 0, sizeof(map));
+  const bool tma = block_size % kTile == 0 && plan.split_tokens % kTile == 0 && rows > 0 &&
+                   rows < (int64_t{1} << 31) &&
+                   dec::make_map(&map, cache, (uint64_t)rows, 128, 128, kTile, true);
+  const int idx = (bf16 ? 4 : 0) + (gc <= 4 ? 2 : 0) + (tma ? 1 : 0);
+  auto fn = octave_decode_mma_kernel<false, false, false>;
+  switch (idx) {
+    case 1: fn = octave_decode_mma_kernel<false, false, true>; break;
+    case 2: fn = octave_decode_mma_kernel<false, true, false>; break;
+    case 3: fn = octave_decode_mma_kernel<false, true, true>; break;
+    case 4: fn = octave_decode_mma_kernel<true, false, false>; break;
+    case 5: fn = octave_decode_mma_kernel<true, false, true>; break;
+    case 6: fn = octave_decode_mma_kernel<true, true, false>; break;
+    case 7: fn = octave_decode_mma_kernel<true, true, true>; break;
+    default: break;
+  }
+  fn<<<grid, kThreads, kSmemBytes, s>>>(map, wait_poll_limit(), P, query, n_q_heads, group, gc,
+                                        cache, n_kv_heads, block_size, num_blocks, block_table,
+                                        num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2,
+                                        plan.split_tokens, plan.splits, ws, device_error_word());
   return cudaGetLastError();
 }
 

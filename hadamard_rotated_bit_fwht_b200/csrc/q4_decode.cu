@@ -96,9 +96,9 @@ __global__ void __launch_bounds__(256, kB <= 16 ? 4 : 1)
   }
   if (ns > 0) fetch(0);
   if (warp == 0 && ns <= 64) {
-    float M = fmaxf(r0.x, r1.x);
+    float M = fmax_nan(r0.x, r1.x);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    for (int off = 16; off > 0; off >>= 1) M = fmax_nan(M, __shfl_xor_sync(0xffffffffu, M, off));
     const float f0 = (M == -INFINITY || r0.x == -INFINITY) ? 0.f : exp2f(r0.x - M);
     const float f1 = (M == -INFINITY || r1.x == -INFINITY) ? 0.f : exp2f(r1.x - M);
     if (lane < ns) wgt[lane] = f0;
@@ -109,9 +109,9 @@ __global__ void __launch_bounds__(256, kB <= 16 ? 4 : 1)
     if (lane == 0) lsum = L;
   } else if (warp == 0) {
     float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldg(rec + s * rstride));
+    for (int s = lane; s < ns; s += 32) M = fmax_nan(M, __ldg(rec + s * rstride));
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    for (int off = 16; off > 0; off >>= 1) M = fmax_nan(M, __shfl_xor_sync(0xffffffffu, M, off));
     float L = 0.f;
     for (int s = lane; s < ns; s += 32) {
       const float ms = __ldg(rec + s * rstride);

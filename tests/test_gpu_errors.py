@@ -50,6 +50,43 @@ def test_wait_timeout_is_reported_and_recovers(bits):
     assert torch.equal(again, want)
 
 
+def test_octave_wait_timeout_is_reported_and_recovers():
+    """The Octave k3v4 decode with 256-token blocks stages its tiles by tensor
+    copies behind bounded mbarrier waits: the same timeout path."""
+    F = kvq.OctaveFormat(128, 64, 4)
+    B, Hkv, Hq, T, bs = 2, 2, 8, 8192, 256
+    nblk = B * T // bs
+    k = synth.to_bf16_bits(synth.gaussian(517, (B * T, Hkv, 128)))
+    v = synth.to_bf16_bits(synth.gaussian(518, (B * T, Hkv, 128)))
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    kd, vd = dev(k).view(torch.bfloat16), dev(v).view(torch.bfloat16)
+    cache = torch.zeros((nblk, Hkv, bs, 128), dtype=torch.uint8, device="cuda")
+    signs = kvq.sign_words(synth.sign_pattern(128))
+    kvq.octave_quantize(F, kd, vd, torch.arange(B * T, dtype=torch.int64, device="cuda"), cache,
+                        signs)
+    bt = torch.arange(nblk, dtype=torch.int32, device="cuda").view(B, T // bs)
+    q = dev(synth.queries(519, B, Hq, 128)).to(torch.bfloat16)
+    q2r = torch.arange(B, dtype=torch.int32, device="cuda")
+    q2l = torch.full((B,), T, dtype=torch.int32, device="cuda")
+
+    def run():
+        return kvq.octave_decode_attn(F, q, cache, bt, q2r, q2l, T, 128 ** -0.5, signs)
+
+    want = run()
+    assert kvq.device_errors() == 0
+    kvq.set_wait_limit(0)
+    try:
+        got = run()
+        flags = kvq.device_errors()
+    finally:
+        kvq.set_wait_limit(-1)
+    assert flags & kvq.KVQ_DEVERR_WAIT_TIMEOUT
+    assert torch.isnan(got).any(), "a CTA that gave up leaves NaN partial results"
+    again = run()
+    assert kvq.device_errors() == 0
+    assert torch.equal(again, want)
+
+
 def test_wait_limit_validation():
     with pytest.raises(kvq.KVQError):
         kvq.set_wait_limit(-2)

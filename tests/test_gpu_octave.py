@@ -126,20 +126,22 @@ def test_decode_block_sizes(v_bits, bs):
     assert np.abs(got - want).max() <= ATOL
 
 
-@pytest.mark.parametrize("v_bits", [4, 3])
-def test_decode_unmapped_blocks_contribute_nothing(v_bits):
+@pytest.mark.parametrize("v_bits,bs", [(4, 16), (3, 16), (4, 64)])
+def test_decode_unmapped_blocks_contribute_nothing(v_bits, bs):
     """A block-table entry that names no block (-1 or past the cache) drops its
     tokens: decode attention has no positional term, so the result equals the
-    oracle over the table with those entries removed."""
-    bs = 16
+    oracle over the table with those entries removed.  (64-token blocks take
+    the tensor-copy staging, whole tiles at a time.)"""
     F, fmt, cache, bt, q, signs = decode_case(v_bits, 8, bs, "bf16", seed=60)
     nblk = cache.shape[0]
     holes = bt.copy()
-    holes[0, 3] = -1
-    holes[0, 7] = nblk + 5
+    nb = bt.shape[1]
+    gone0 = (1, 2) if nb < 8 else (3, 7)
+    holes[0, gone0[0]] = -1
+    holes[0, gone0[1]] = nblk + 5
     holes[1, 0] = -1
-    keep0 = [j for j in range(bt.shape[1]) if j not in (3, 7)]
-    keep1 = [j for j in range(bt.shape[1]) if j != 0]
+    keep0 = [j for j in range(nb) if j not in gone0]
+    keep1 = [j for j in range(nb) if j != 0]
     q_to_req = np.array([0, 1], np.int32)
     q_to_klen = np.array([192, 192], np.int32)
     got = kvq.octave_decode_attn(F, to_dev(q[:2]), cache, to_dev(holes), to_dev(q_to_req),
