@@ -225,35 +225,40 @@ __device__ __forceinline__ void pack_3(const uint8_t *cbb, int t, int W, int ND,
   }
 }
 
-// this thread's 16 contiguous dims 16 q .. 16 q + 15 of a row, sign flips
-// applied (sg: their 16 sign bits)
+// this thread's 16 contiguous dims 16 q .. 16 q + 15 of a row: fetched raw
+// (so that the load of the next vector overlaps the work on this one), then
+// widened with the sign flips applied (sm: for bf16 the XOR masks of the 8
+// words, bits 15 and 31; for fp32 bit m of sm[0] is the sign of dim 16 q + m)
 template <bool BF16>
-__device__ __forceinline__ void load16(const void *row, int q, uint32_t sg, bool valid,
-                                       float (&x)[16]) {
-  if (!valid) {
+struct Raw16 {
+  uint4 w[BF16 ? 2 : 4];
+};
+template <bool BF16>
+__device__ __forceinline__ void fetch16(const void *row, int q, bool valid, Raw16<BF16> &r) {
+  const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const char *>(row) +
+                                                     16 * q * (BF16 ? 2 : 4));
 #pragma unroll
-    for (int m = 0; m < 16; m++) x[m] = 0.f;
-    return;
-  }
+  for (int j = 0; j < (BF16 ? 2 : 4); j++)
+    r.w[j] = valid ? __ldg(src + j) : make_uint4(0u, 0u, 0u, 0u);
+}
+template <bool BF16>
+__device__ __forceinline__ void unpack16(const Raw16<BF16> &r, const uint32_t (&sm)[8],
+                                         float (&x)[16]) {
   if constexpr (BF16) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(row) + 16 * q);
-    const uint4 a = __ldg(src), b = __ldg(src + 1);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int j = 0; j < 8; j++) {
-      x[2 * j] = __uint_as_float((w[j] << 16) ^ (((sg >> (2 * j)) & 1u) << 31));
-      x[2 * j + 1] = __uint_as_float((w[j] & 0xffff0000u) ^ (((sg >> (2 * j + 1)) & 1u) << 31));
+      const uint4 u = r.w[j / 4];
+      const uint32_t w = (j % 4 == 0 ? u.x : j % 4 == 1 ? u.y : j % 4 == 2 ? u.z : u.w) ^ sm[j];
+      x[2 * j] = __uint_as_float(w << 16);
+      x[2 * j + 1] = __uint_as_float(w & 0xffff0000u);
     }
   } else {
-    const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(row) + 16 * q);
 #pragma unroll
     for (int j = 0; j < 4; j++) {
-      const float4 a = __ldg(src + j);
-      const float f[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t f[4] = {r.w[j].x, r.w[j].y, r.w[j].z, r.w[j].w};
 #pragma unroll
       for (int i = 0; i < 4; i++)
-        x[4 * j + i] =
-            __uint_as_float(__float_as_uint(f[i]) ^ (((sg >> (4 * j + i)) & 1u) << 31));
+        x[4 * j + i] = __uint_as_float(f[i] ^ (((sm[0] >> (4 * j + i)) & 1u) << 31));
     }
   }
 }
@@ -292,33 +297,44 @@ __global__ void __launch_bounds__(kThreads)
   const int o = threadIdx.x >> 3;  // octet of the CTA
   float *xr = S.xb[o];
   uint8_t *cbb = reinterpret_cast<uint8_t *>(S.cb[o]);
-  // sign bits of dims 16 q .. 16 q + 15
+  // sign bits of dims 16 q .. 16 q + 15, as XOR masks
   const uint32_t sg = (P.sign_words[q >> 1] >> (16 * (q & 1))) & 0xffffu;
+  uint32_t sm[8];
+#pragma unroll
+  for (int j = 0; j < 8; j++)
+    sm[j] = BF16 ? (((sg >> (2 * j)) & 1u) << 15) | (((sg >> (2 * j + 1)) & 1u) << 31)
+                 : (j == 0 ? sg : 0u);
 
   // whole warps step through the items together (the shuffles), four octets each
   const int64_t wbase0 = ((int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31)) / 8;
   const int64_t wstride = (int64_t)gridDim.x * kOct;
+  auto row_of = [&](const void *base, int64_t item) {
+    return static_cast<const char *>(base) + item * kHead * (BF16 ? 2 : 4);
+  };
+  Raw16<BF16> kraw, vraw;
+  {
+    const int64_t it0 = wbase0 + (lane >> 3);
+    fetch16<BF16>(row_of(key, it0 < items ? it0 : 0), q, it0 < items, kraw);
+  }
   for (int64_t wb = wbase0; wb < items; wb += wstride) {
     const int64_t it = wb + (lane >> 3);
     const bool valid = it < items;
+    fetch16<BF16>(row_of(value, valid ? it : 0), q, valid, vraw);
     uint32_t *dst = nullptr;  // the slot, or null for a skipped token
     if (valid) {
       const int tok = (int)(it / n_kv_heads);
       const int h = (int)(it - (int64_t)tok * n_kv_heads);
-      const int64_t sm = __ldg(slot_mapping + tok);
-      if (sm >= 0) {
-        const int64_t blk = sm / block_size, off = sm - blk * block_size;
+      const int64_t sm_ = __ldg(slot_mapping + tok);
+      if (sm_ >= 0) {
+        const int64_t blk = sm_ / block_size, off = sm_ - blk * block_size;
         const int64_t si = (blk * n_kv_heads + h) * block_size + off;
         if (blk < num_blocks && in_bounds(si, si + 1, num_blocks * n_kv_heads * block_size, err))
           dst = reinterpret_cast<uint32_t *>(cache + si * (int64_t)kSlotBytes);
       }
     }
-    const int64_t itc = valid ? it : 0;
-    const void *krow = static_cast<const char *>(key) + itc * kHead * (BF16 ? 2 : 4);
-    const void *vrow = static_cast<const char *>(value) + itc * kHead * (BF16 ? 2 : 4);
     float x[16];
     float ks0, ks1 = 0.f;
-    load16<BF16>(krow, q, sg, valid, x);
+    unpack16<BF16>(kraw, sm, x);
     if constexpr (COMPACT) {
       ks0 = quantize_vec<8>(x, q, vscale, P.mult3, 0, S.T, xr, cbb);
       __syncwarp();
@@ -338,8 +354,12 @@ __global__ void __launch_bounds__(kThreads)
       ks1 = __shfl_sync(kFull, ks, (lane & ~7) | 4);
     }
     __syncwarp();  // the code row is free again
+    {  // the next item's K row, while this one's V is worked on
+      const int64_t itn = it + wstride;
+      fetch16<BF16>(row_of(key, itn < items ? itn : 0), q, itn < items, kraw);
+    }
     float vs;
-    load16<BF16>(vrow, q, sg, valid, x);
+    unpack16<BF16>(vraw, sm, x);
     vs = quantize_vec<8>(x, q, vscale, VBITS == 4 ? P.mult4 : P.mult3, VBITS == 4 ? 1 : 0, S.T,
                          xr, cbb);
     __syncwarp();
