@@ -83,12 +83,15 @@ static __device__ __noinline__ uint2 exact_code(float x, float rms, float mult, 
 // {code, fp32 bits of x * LUT[code]} of one element from the floor table of
 // code width tb + 3, given y2 ~ 2y (see the file comment); near is set when
 // |y2| lies within 2^-13 of an integer, where only the exact path decides.
+__device__ __forceinline__ bool near_int(float a, float f) {  // a = min(|y2|, 255.5)
+  const float frac = __fsub_rn(a, __fsub_rn(f, 8388608.f));
+  return fabsf(__fsub_rn(frac, 0.5f)) > 0.5f - kNearEps;
+}
 __device__ __forceinline__ uint2 code_fast(float x, float y2, const uint2 *tab, bool &near) {
   const uint32_t yb = __float_as_uint(y2);
   const float a = fminf(__uint_as_float(yb & 0x7fffffffu), 255.5f);
   const float f = __fadd_rz(a, 8388608.f);  // 2^23 + floor(a)
-  const float frac = __fsub_rn(a, __fsub_rn(f, 8388608.f));
-  near = fabsf(__fsub_rn(frac, 0.5f)) > 0.5f - kNearEps;
+  near = near_int(a, f);
   uint2 e = tab[(__float_as_uint(f) & 0xffu) | ((yb >> 23) & 0x100u)];
   e.y = __float_as_uint(__fmul_rn(x, __uint_as_float(e.y)));
   return e;
@@ -159,23 +162,30 @@ __device__ __forceinline__ float quantize_vec(float (&x)[16], int t, float scale
   rms = rms < 1e-12f ? 1e-12f : rms;
   const float c2 = __fdiv_rn(2.f * mult, rms);
   const uint2 *tab = Q.e[tb];
-  uint32_t near = 0;
+  bool any_near = false;
 #pragma unroll
   for (int k = 0; k < 16; k++) {
     bool nk;
     const uint2 e = code_fast(y[k], __fmul_rn(y[k], c2), tab, nk);
     cbb[t + T * k] = (uint8_t)e.x;
     v[k] = __uint_as_float(e.y);
-    near |= nk ? 1u << k : 0u;
+    any_near = any_near || nk;
   }
-  if (near) {
-    // the exact path for the flagged elements, as a rolled loop over this
-    // thread's segment of the (free) transpose row, so that y and v stay in
-    // registers: y in, x * LUT[code] back
+  if (any_near) {
+    // the exact path for the flagged elements (the flags recomputed here, off
+    // the common path), as a rolled loop over this thread's segment of the
+    // (free) transpose row, so that y and v stay in registers: y in, x *
+    // LUT[code] back
     float *seg = xr + 20 * t;
+    uint32_t near = 0;
 #pragma unroll
-    for (int k = 0; k < 16; k++)
-      if (near & (1u << k)) seg[k] = y[k];
+    for (int k = 0; k < 16; k++) {
+      const float a = fminf(fabsf(__fmul_rn(y[k], c2)), 255.5f);
+      if (near_int(a, __fadd_rz(a, 8388608.f))) {
+        near |= 1u << k;
+        seg[k] = y[k];
+      }
+    }
 #pragma unroll 1
     for (int k = 0; k < 16; k++)
       if (near & (1u << k)) {
