@@ -53,7 +53,9 @@ constexpr float kNearEps = 1.f / 8192.f;  // 2^-13, twice the bound on |y2 - 2y|
 constexpr unsigned kFull = 0xffffffffu;
 
 struct QTables {
-  uint2 e[2][512];   // [bits - 3][neg * 256 + floor|2y|] = {code, fp32 bits of LUT[code]}
+  // [bits - 3][neg * 256 + floor|2y|]: fp32 bits of LUT[code] with the code
+  // in the low byte (an int8 LUT value leaves the low 16 bits of its fp32 zero)
+  uint32_t e[2][512];
   float lut[2][16];  // exact path: LUT values
   float mid[2][16];  // exact path: midpoints
 };
@@ -61,7 +63,8 @@ struct QTables {
 struct Smem {
   QTables T;
   float xb[kOct][kXb];     // transpose rows: element 16 q + m of thread q at 20 q + m
-  uint32_t cb[kOct][32];   // code bytes in element order
+  uint32_t cb[kOct][34];   // code bytes in element order (rows 34 words apart: the
+                           // byte stores of the four octets of a warp meet no bank twice)
 };
 
 __device__ __forceinline__ uint32_t bit(const OctaveParams &P, int d) {
@@ -87,14 +90,13 @@ __device__ __forceinline__ bool near_int(float a, float f) {  // a = min(|y2|, 2
   const float frac = __fsub_rn(a, __fsub_rn(f, 8388608.f));
   return fabsf(__fsub_rn(frac, 0.5f)) > 0.5f - kNearEps;
 }
-__device__ __forceinline__ uint2 code_fast(float x, float y2, const uint2 *tab, bool &near) {
+__device__ __forceinline__ uint2 code_fast(float x, float y2, const uint32_t *tab, bool &near) {
   const uint32_t yb = __float_as_uint(y2);
   const float a = fminf(__uint_as_float(yb & 0x7fffffffu), 255.5f);
   const float f = __fadd_rz(a, 8388608.f);  // 2^23 + floor(a)
   near = near_int(a, f);
-  uint2 e = tab[(__float_as_uint(f) & 0xffu) | ((yb >> 23) & 0x100u)];
-  e.y = __float_as_uint(__fmul_rn(x, __uint_as_float(e.y)));
-  return e;
+  const uint32_t w = tab[(__float_as_uint(f) & 0xffu) | ((yb >> 23) & 0x100u)];
+  return make_uint2(w, __float_as_uint(__fmul_rn(x, __uint_as_float(w & 0xffffff00u))));
 }
 
 // One vector of n = 16 T values over T threads (t = this thread's index in
@@ -161,7 +163,7 @@ __device__ __forceinline__ float quantize_vec(float (&x)[16], int t, float scale
   float rms = __fsqrt_rn(__fmul_rn(ss, 1.f / (float)N));
   rms = rms < 1e-12f ? 1e-12f : rms;
   const float c2 = __fdiv_rn(2.f * mult, rms);
-  const uint2 *tab = Q.e[tb];
+  const uint32_t *tab = Q.e[tb];
   bool any_near = false;
 #pragma unroll
   for (int k = 0; k < 16; k++) {
@@ -288,7 +290,7 @@ __global__ void __launch_bounds__(kThreads)
     const float y2 = neg ? -(n + 0.5f) : (n + 0.5f);
     uint32_t c = 0;
     for (int i = 0; i < L - 1; i++) c += (float)(lut[i] + lut[i + 1]) < y2 ? 1u : 0u;
-    S.T.e[tb][t & 511] = make_uint2(c, __float_as_uint((float)lut[c]));
+    S.T.e[tb][t & 511] = __float_as_uint((float)lut[c]) | c;
   }
   for (int t = threadIdx.x; t < 32; t += blockDim.x) {
     const int tb = t >> 4, i = t & 15, L = tb ? 16 : 8;
