@@ -56,6 +56,28 @@ def test_quantize_bitexact(v_bits, dt):
     assert bad[0].size == 0, f"{bad[0].size} slots differ, first token {bad[0][:3]}"
 
 
+@pytest.mark.parametrize("T,Hkv", [(1, 1), (3, 1), (5, 3), (7, 5)])
+@pytest.mark.parametrize("fmt", [(128, 64, 4, 0), (128, 64, 3, 1)])
+def test_quantize_few_items_bitexact(T, Hkv, fmt):
+    """Item counts that leave octets of the last warp without an item (the
+    kernel runs eight threads per (token, kv head) and whole warps together)."""
+    F = kvq.OctaveFormat(fmt[0], fmt[1], fmt[2], compact=bool(fmt[3]))
+    slot_bytes = F.layout()["slot_bytes"]
+    bs = 4
+    k, v, slot, nblk = make_cache(fmt, T, Hkv, bs, 90 + T * Hkv, "bf16")
+    signs = synth.sign_pattern(128)
+    cache = torch.zeros((nblk, Hkv, bs, slot_bytes), dtype=torch.uint8, device="cuda")
+    kvq.octave_quantize(F, to_dev(k), to_dev(v), to_dev(slot), cache, kvq.sign_words(signs))
+    want = oracle.octave_quantize(k, v, fmt, signs)
+    c = cache.cpu().numpy()
+    got = c.transpose(0, 2, 1, 3).reshape(-1, Hkv, slot_bytes)[slot]
+    assert np.array_equal(got, want)
+    # slots no token maps to stay untouched
+    used = np.zeros(nblk * bs, bool)
+    used[slot] = True
+    assert not c.transpose(0, 2, 1, 3).reshape(-1, Hkv, slot_bytes)[~used].any()
+
+
 def test_quantize_skips_negative_and_out_of_range_slots():
     F = kvq.OctaveFormat(128, 64, 4)
     T, Hkv, bs = 8, 2, 16
