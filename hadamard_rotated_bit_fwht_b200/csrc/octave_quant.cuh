@@ -90,13 +90,25 @@ __device__ __forceinline__ bool near_int(float a, float f) {  // a = min(|y2|, 2
   const float frac = __fsub_rn(a, __fsub_rn(f, 8388608.f));
   return fabsf(__fsub_rn(frac, 0.5f)) > 0.5f - kNearEps;
 }
-__device__ __forceinline__ uint2 code_fast(float x, float y2, const uint32_t *tab, bool &near) {
-  const uint32_t yb = __float_as_uint(y2);
-  const float a = fminf(__uint_as_float(yb & 0x7fffffffu), 255.5f);
-  const float f = __fadd_rz(a, 8388608.f);  // 2^23 + floor(a)
-  near = near_int(a, f);
-  const uint32_t w = tab[(__float_as_uint(f) & 0xffu) | ((yb >> 23) & 0x100u)];
-  return make_uint2(w, __float_as_uint(__fmul_rn(x, __uint_as_float(w & 0xffffff00u))));
+// The same for two elements at once, the floating-point steps as packed
+// fp32x2 operations (each lane rounds as the scalar form): table words (the
+// code in the low byte) in w0, w1, the products x * LUT[code] in prod (a zero
+// product comes out +0, which no sum or scale below can tell from -0), and
+// near when either element is near an integer.
+__device__ __forceinline__ void code_fast2(float2 x, float2 y2, const uint32_t *tab, uint32_t &w0,
+                                          uint32_t &w1, float2 &prod, bool &near) {
+  const uint32_t b0 = __float_as_uint(y2.x), b1 = __float_as_uint(y2.y);
+  const float2 a = make_float2(fminf(__uint_as_float(b0 & 0x7fffffffu), 255.5f),
+                               fminf(__uint_as_float(b1 & 0x7fffffffu), 255.5f));
+  const float2 f = add2_rz(a, make_float2(8388608.f, 8388608.f));  // 2^23 + floor(a)
+  const float2 fl = add2_rn(f, make_float2(-8388608.f, -8388608.f));
+  const float2 frac = add2_rn(a, make_float2(-fl.x, -fl.y));
+  const float2 g = add2_rn(frac, make_float2(-0.5f, -0.5f));
+  near = fabsf(g.x) > 0.5f - kNearEps || fabsf(g.y) > 0.5f - kNearEps;
+  w0 = tab[(__float_as_uint(f.x) & 0xffu) | ((b0 >> 23) & 0x100u)];
+  w1 = tab[(__float_as_uint(f.y) & 0xffu) | ((b1 >> 23) & 0x100u)];
+  prod = mul2_rn_p0(x, make_float2(__uint_as_float(w0 & 0xffffff00u),
+                                   __uint_as_float(w1 & 0xffffff00u)));
 }
 
 // One vector of n = 16 T values over T threads (t = this thread's index in
@@ -166,11 +178,16 @@ __device__ __forceinline__ float quantize_vec(float (&x)[16], int t, float scale
   const uint32_t *tab = Q.e[tb];
   bool any_near = false;
 #pragma unroll
-  for (int k = 0; k < 16; k++) {
+  for (int k = 0; k < 8; k++) {  // elements k and k + 8
     bool nk;
-    const uint2 e = code_fast(y[k], __fmul_rn(y[k], c2), tab, nk);
-    cbb[t + T * k] = (uint8_t)e.x;
-    v[k] = __uint_as_float(e.y);
+    uint32_t w0, w1;
+    float2 pr;
+    const float2 yy = make_float2(y[k], y[k + 8]);
+    code_fast2(yy, mul2_rn_p0(yy, make_float2(c2, c2)), tab, w0, w1, pr, nk);
+    cbb[t + T * k] = (uint8_t)w0;
+    cbb[t + T * (k + 8)] = (uint8_t)w1;
+    v[k] = pr.x;
+    v[k + 8] = pr.y;
     any_near = any_near || nk;
   }
   if (any_near) {
