@@ -125,12 +125,18 @@ def _check(fn, status):
         raise KVQError(fn, status)
 
 
+# the raw handle of torch's current stream on the current device, without
+# building a Stream object (this sits on the per-token decode path); the
+# public route where this torch build lacks the internal accessor
+_RAW_STREAM = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream=None):
     if stream is not None:
         return stream.cuda_stream
-    # the raw handle of torch's current stream on the current device, without
-    # building a Stream object (this sits on the per-token decode path)
-    return torch._C._cuda_getCurrentRawStream(torch.cuda.current_device())
+    if _RAW_STREAM is not None:
+        return _RAW_STREAM(torch.cuda.current_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _ptr(t):
