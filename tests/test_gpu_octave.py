@@ -118,7 +118,7 @@ def decode_case(v_bits, G, bs, qdt, seed=21):
 
 
 @pytest.mark.parametrize("v_bits", [4, 3])  # 4: tensor-core kernel, 3: SIMT kernel
-@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
 @pytest.mark.parametrize("qdt", ["bf16", "f32"])
 def test_decode_vs_oracle(v_bits, G, qdt):
     F, fmt, cache, bt, q, signs = decode_case(v_bits, G, 16, qdt)
@@ -241,7 +241,7 @@ def test_compact_quantize_bitexact(v_bits, dt):
 
 
 @pytest.mark.parametrize("v_bits", [3, 4])
-@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_compact_decode_vs_oracle(v_bits, G):
     fmt = (128, 64, v_bits, 1)
     F = kvq.OctaveFormat(128, 64, v_bits, True)
