@@ -27,12 +27,15 @@
 //     16 x 16384-token workload, whose keys carry x16 outlier channels.)
 //   * PV on the fp16 path (m16n8k16, fp32 accumulation): A = V^T codes through
 //     the biased table (each byte u becomes the exact fp16 1024 + u = LUT[c] +
-//     1152 by pairing it with 0x64), read by ldmatrix.trans from the swizzled
-//     tile; B = p * s_v / 64 split hi + lo.  One more MMA per 16 tokens, with
-//     an all-ones A, sums B over the tokens, and the merge subtracts 1152
-//     times that sum.  Up to 4 heads per CTA, the hi parts sit in B columns
-//     0-3 and the lo parts in columns 4-7 (one MMA per tile instead of two);
-//     the merge adds the two halves.
+//     1152 by pairing it with 0x64, and one half2 subtract of 1152 leaves the
+//     exact LUT[c]), read by ldmatrix.trans from the swizzled tile; B = p *
+//     s_v / 64 split hi + lo.  The subtract stays ahead of the MMA: folding
+//     the 1152 out of the fp32 accumulators after the sum instead (an
+//     all-ones MMA for sum_t p) carried the accumulation error of 1152 * l,
+//     2e-3 in the outputs at 16k-256k tokens, against 5e-5 this way.  Up to
+//     4 heads per CTA, the hi parts sit in B columns 0-3 and the lo parts in
+//     columns 4-7 (one MMA per tile instead of two); the merge adds the two
+//     halves.
 //     The V region starts 8 bytes into a 16-byte chunk: the used halves of
 //     chunks 3 and 7 are joined by one lane shuffle, so the 64 V bytes make
 //     exactly 8 M-tiles.
@@ -144,13 +147,14 @@ __device__ __forceinline__ uint32_t lut4_bytes(uint32_t sel, const Lut4 &T) {
   const uint32_t m = prmt(shl_add<4>(sel, 0u), sel, 0xD9C8u);
   return lop3_sel(plo, phi, m);
 }
-// biased bytes (a, b) of R -> half2 (1024 + U, 1024 + U) exactly, U = LUT + 128;
-// the 1152 this adds to every code leaves the PV products as 1152 * sum_t w
-// per head, which the merge takes off
+// biased bytes (a, b) of R, U = LUT + 128 -> half2 (LUT_a, LUT_b) exactly: the
+// pairing with 0x64 makes the fp16 1024 + U, and 1024 + U - 1152 is exact
 __device__ __forceinline__ uint32_t lut_half2(uint32_t R, uint32_t selector) {
-  return prmt(R, 0x64646464u, selector);
+  const uint32_t biased = prmt(R, 0x64646464u, selector);
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(biased), "r"(0x64806480u));  // 1152, 1152
+  return r;
 }
-constexpr float kVBias = 1152.f;
 
 __device__ __forceinline__ void split_hilo(float2 w, uint32_t &hi, uint32_t &lo) {
   __half2 h = __float22half2_rn(w);
@@ -378,8 +382,6 @@ __global__ void __launch_bounds__(kThreads, 4)
   float o[8][4];
 #pragma unroll
   for (int mt = 0; mt < 8; mt++) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-  float wsum[4] = {0.f, 0.f, 0.f, 0.f};  // sum_t of the B columns, as the PV MMAs see them
-  const uint32_t ones[4] = {0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u};
   float m_run = -INFINITY, l_run = 0.f;
   float *fsc = reinterpret_cast<float *>(smem + kOffF);
 
@@ -551,10 +553,6 @@ __global__ void __launch_bounds__(kThreads, 4)
           o[mt][2] *= a0;
           o[mt][3] *= a1;
         }
-        wsum[0] *= a0;
-        wsum[1] *= a1;
-        wsum[2] *= a0;
-        wsum[3] *= a1;
       }
       float p[4];
 #pragma unroll
@@ -584,10 +582,6 @@ __global__ void __launch_bounds__(kThreads, 4)
           bh0 = xl0;
           bh1 = xl1;
         }
-        mma16816(wsum, ones, bh0, bh1);
-      } else {
-        mma16816(wsum, ones, bh0, bh1);
-        mma16816(wsum, ones, bl0, bl1);
       }
       // x2.trans: matrices (T0, chunk), (T1, chunk); lanes 0..15 give the rows
       const int vrow = 16 * warp + (lane & 15);
@@ -667,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 4)
       const int d = 8 * (vb >> 2) + (vb & 3);  // low nibble; high nibble is d + 4
       float acc[4];
 #pragma unroll
-      for (int e = 0; e < 4; e++) acc[e] = fmaf(-kVBias, wsum[e & 1], o[2 * vc + par][e]);
+      for (int e = 0; e < 4; e++) acc[e] = o[2 * vc + par][e];
       if (PACK) {  // hi (columns 0-3, tg < 2) + lo (columns 4-7, tg + 2)
 #pragma unroll
         for (int e = 0; e < 4; e++) acc[e] += __shfl_xor_sync(kFull, acc[e], 2);

@@ -220,6 +220,43 @@ def test_octave_workload_full_size():
     assert err.max() <= ATOL, f"requests over 2e-3: {np.nonzero(err > ATOL)[0]}"
 
 
+def test_octave_decode_longest_context():
+    """One request of 262144 tokens (1024 shuffled 256-token blocks, 8 kv
+    heads, GQA 4, the workload's outlier channels): the k3v4 decode sums 16x
+    more tokens per request than the benchmark workload, so an error that
+    grows with the summed tokens shows here.  Slots bit-exact, all 32 head
+    outputs within 2e-3 of the oracle over the oracle's own slots."""
+    W = synth.WORKLOADS["octave"]
+    fmt = (128, 64, 4, 0)
+    F = kvq.OctaveFormat(*fmt[:3])
+    Hkv, Hq, ctx, bs, seed = 8, 32, 262144, 256, 31
+    nblk = ctx // bs
+    bt, _ = synth.page_table(seed, 1, np.array([nblk]), nblk)
+    signs = synth.sign_pattern(128)
+    k, v = synth.kv_tokens(seed, 1, ctx, Hkv, 128, W["outlier_frac"], W["outlier_factor"])
+    kb, vb = synth.to_bf16_bits(k[0]), synth.to_bf16_bits(v[0])
+    del k, v
+    slot = (bt[0, np.arange(ctx) // bs] * bs + np.arange(ctx) % bs).astype(np.int64)
+    cache = torch.zeros((nblk, Hkv, bs, 128), dtype=torch.uint8, device="cuda")
+    kvq.octave_quantize(F, to_dev(kb), to_dev(vb), to_dev(slot), cache, kvq.sign_words(signs))
+    threads = oracle.host_threads()
+    want_by_slot = np.zeros((nblk * bs, Hkv, 128), np.uint8)
+    want_by_slot[slot] = oracle.octave_quantize(kb, vb, fmt, signs, threads=threads)
+    got_by_slot = cache.cpu().numpy().transpose(0, 2, 1, 3).reshape(-1, Hkv, 128)
+    assert np.array_equal(got_by_slot, want_by_slot)
+    want_cache = want_by_slot.reshape(nblk, bs, Hkv, 128).transpose(0, 2, 1, 3).copy()
+    q = synth.to_bf16_bits(synth.queries(seed, 1, Hq, 128))
+    q_to_req = np.zeros(1, np.int32)
+    q_to_klen = np.full(1, ctx, np.int32)
+    got = kvq.octave_decode_attn(F, to_dev(q), cache, to_dev(bt), to_dev(q_to_req),
+                                 to_dev(q_to_klen), ctx, 128 ** -0.5,
+                                 kvq.sign_words(signs)).cpu().numpy()
+    want = oracle.octave_attention(q, want_cache, bt, q_to_req, q_to_klen, fmt, 128 ** -0.5,
+                                   signs, threads=threads)
+    err = np.abs(got - want).max()
+    assert err <= ATOL, f"max abs error {err}"
+
+
 # ------------------------------------------------------------------ compact K
 @pytest.mark.parametrize("v_bits", [3, 4])
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
