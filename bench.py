@@ -746,8 +746,10 @@ def cpu_oracle_octave(threads: int):
 def cpu_baselines(threads: int):
     """The headline (long-context decode) oracle figure on all cores and on one,
     plus bounded multi-core samples of the other workloads."""
-    gbs1, dt1, sample1, _ = cpu_oracle_long_decode(steps=3, threads=1)
-    gbs, dt, sample, used = cpu_oracle_long_decode(steps=2, threads=threads)
+    # about 3 s of wall time each: 8 quarter steps on one core, 6 whole steps
+    # (about 12 s of CPU work on 4 threads)
+    gbs1, dt1, sample1, _ = cpu_oracle_long_decode(steps=8, threads=1)
+    gbs, dt, sample, used = cpu_oracle_long_decode(steps=6, threads=threads)
     per = {"long_decode": {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle",
                            "sample": sample, "seconds": dt},
            "long_decode_1_core": {"value": gbs1, "unit": "GB/s", "cores": 1, "kind": "oracle",
@@ -766,8 +768,9 @@ def run_reference(args):
         return
     import oracle
     threads = oracle.host_threads()
-    # bounded sample: at most 4 timed and 2 warm-up whole oracle steps
-    steps = max(1, min(args.steps, 4))
+    # bounded sample: at most 8 timed and 2 warm-up whole oracle steps (about
+    # 0.5 s of wall time and 2 s of CPU work each on 4 threads)
+    steps = max(1, min(args.steps, 8))
     warm = max(0, min(args.warmup, 2))
     gbs, dt, sample, used = cpu_oracle_long_decode(steps, warm, threads=threads)
     W = synth.WORKLOADS["long_decode"]
