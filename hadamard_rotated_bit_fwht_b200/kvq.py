@@ -9,6 +9,7 @@ is missing the import of the first call fails with a message saying so.
 from __future__ import annotations
 
 import ctypes as C
+import functools
 import os
 from dataclasses import dataclass
 
@@ -385,6 +386,21 @@ class OctaveFormat:
         return {n: getattr(out, n) for n, _ in OctaveLayoutDesc._fields_}
 
 
+@functools.lru_cache(maxsize=None)
+def _slot_bytes(fmt: OctaveFormat) -> int:
+    return fmt.layout()["slot_bytes"]
+
+
+def _octave_cache_shape(fmt: OctaveFormat, cache: torch.Tensor):
+    """(num_blocks, kv heads, block_size) of a cache [num_blocks, Hkv,
+    block_size, slot bytes of fmt]; the C ABI takes the slot width from the
+    format, so a cache of another width is refused here."""
+    if cache.dim() != 4 or cache.shape[3] != _slot_bytes(fmt):
+        raise ValueError(f"cache must be [num_blocks, kv heads, block_size, {_slot_bytes(fmt)}] "
+                         f"for this format, got {tuple(cache.shape)}")
+    return cache.shape[0], cache.shape[1], cache.shape[2]
+
+
 def octave_codebook(bits: int):
     lut = np.zeros(1 << bits, np.int8)
     mult = C.c_float(0)
@@ -410,7 +426,7 @@ def octave_quantize(fmt: OctaveFormat, key: torch.Tensor, value: torch.Tensor,
     if slot_mapping.dtype != torch.int64 or cache.dtype != torch.uint8:
         raise TypeError("slot_mapping must be int64 and cache uint8")
     T, hkv, _ = key.shape
-    num_blocks, _, block_size, _ = cache.shape
+    num_blocks, _, block_size = _octave_cache_shape(fmt, cache)
     f = fmt.desc()
     sb = np.ascontiguousarray(sign_bits, dtype=np.int32)
     _check("kvq_octave_quantize",
@@ -434,7 +450,7 @@ def octave_decode_attn(fmt: OctaveFormat, query: torch.Tensor, cache: torch.Tens
                  ("q_to_req", q_to_req), ("q_to_klen", q_to_klen)):
         _cuda_contig(n, t)
     nq, hq, d = query.shape
-    num_blocks, hkv, block_size, _ = cache.shape
+    num_blocks, hkv, block_size = _octave_cache_shape(fmt, cache)
     if out is None:
         out = torch.empty((nq, hq, d), dtype=torch.float32, device=query.device)
     if workspace is None:

@@ -352,3 +352,24 @@ def test_quantize_rejects_misaligned_inputs():
     with pytest.raises(kvq.KVQError) as e:
         kvq.octave_quantize(F, kk, kk, slot, cache, kvq.sign_words(synth.sign_pattern(128)))
     assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_bindings_refuse_a_cache_of_another_slot_width():
+    """The C ABI takes the slot width from the format, so the bindings check
+    the cache's last dimension against it: a k3v3 format (112-byte slots)
+    with a 128-byte-slot cache is refused before any launch."""
+    F = kvq.OctaveFormat(128, 64, 3)
+    assert F.layout()["slot_bytes"] == 112
+    cache = torch.zeros((1, 2, 16, 128), dtype=torch.uint8, device="cuda")
+    k = torch.zeros((1, 2, 128), dtype=torch.bfloat16, device="cuda")
+    signs = kvq.sign_words(synth.sign_pattern(128))
+    with pytest.raises(ValueError):
+        kvq.octave_quantize(F, k, k, torch.zeros(1, dtype=torch.int64, device="cuda"), cache,
+                            signs)
+    i32 = lambda *v: torch.tensor(v, dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError):
+        kvq.octave_decode_attn(F, torch.zeros((1, 4, 128), dtype=torch.bfloat16, device="cuda"),
+                               cache, torch.zeros((1, 1), dtype=torch.int32, device="cuda"),
+                               i32(0), i32(16), 16, 0.1, signs)
+    torch.cuda.synchronize()
+    assert not cache.any().item()
