@@ -202,6 +202,9 @@ __global__ void __launch_bounds__(kHead)
                           const int32_t *__restrict__ q_to_klen, int num_reqs, int n_q_heads,
                           int splits, int max_klen, int cap, float *__restrict__ out) {
   __shared__ float ob[kHead];
+  // after the tensor-core split kernel this grid is a programmatic dependent:
+  // the records are read only once that grid has finished (a no-op otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int qh = blockIdx.x, j = threadIdx.x;
   const int qi = qh / n_q_heads;
   const int req = __ldg(q_to_req + qi);
@@ -263,10 +266,20 @@ cudaError_t launch_octave_decode(const OctaveParams &P, const void *query, int b
                                              max_blocks, q_to_req, q_to_klen, max_klen, scale, ws,
                                              plan, s);
     if (e != cudaSuccess) return e;
-    octave_combine_kernel<<<num_q * n_q_heads, kHead, 0, s>>>(P, ws, q_to_req, q_to_klen,
-                                                             num_reqs, n_q_heads, plan.splits,
-                                                             max_klen, max_blocks * block_size,
-                                                             out);
+    // programmatic dependent launch: scheduled while the split kernel drains
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_q * n_q_heads);
+    cfg.blockDim = dim3(kHead);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, octave_combine_kernel, P, (const float *)ws, q_to_req, q_to_klen,
+                           num_reqs, n_q_heads, plan.splits, max_klen, max_blocks * block_size,
+                           out);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
 #define KVQ_LAUNCH(G)                                                                         \

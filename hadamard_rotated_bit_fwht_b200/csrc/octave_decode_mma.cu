@@ -42,7 +42,11 @@
 // Tiles of 64 slots (one 128-byte row per token) are staged by cp.async with
 // the 128-byte XOR swizzle through a 3-stage ring; each row is addressed
 // through the block table by one lookup, so any block size works, and a
-// token whose block entry names no block contributes nothing.
+// token whose block entry names no block contributes nothing.  (Block sizes
+// that are multiples of 64 take one 64-row TMA box per tile instead.)
+// The kernel and the combine after it are programmatic dependent launches:
+// each is scheduled while the grid before it drains and waits for that grid
+// (griddepcontrol.wait) before its first global read.
 #include <cstring>
 
 #include "decode_common.cuh"
@@ -199,6 +203,11 @@ __global__ void __launch_bounds__(kThreads, 4)
   const int h0 = hg * gc, kvh = h0 / group;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tg = lane & 3;
+  // launched as a programmatic dependent of the kernel before it (which may
+  // write the slots or the inputs): wait for that grid before the first global
+  // read, then let the combine grid be scheduled behind this one
+  dec::grid_dependency_wait();
+  dec::launch_dependents();
   const int req = __ldg(q_to_req + qi);
   int klen = min(max(__ldg(q_to_klen + qi), 0), min(max_klen, max_blocks * block_size));
   if (req < 0 || req >= num_reqs) klen = 0;
@@ -736,10 +745,21 @@ cudaError_t launch_octave_decode_mma(const OctaveParams &P, const void *query, i
     case 7: fn = octave_decode_mma_kernel<true, true, true>; break;
     default: break;
   }
-  fn<<<grid, kThreads, kSmemBytes, s>>>(map, wait_poll_limit(), P, query, n_q_heads, group, gc,
-                                        cache, n_kv_heads, block_size, num_blocks, block_table,
-                                        num_reqs, max_blocks, q_to_req, q_to_klen, max_klen, sl2,
-                                        plan.split_tokens, plan.splits, ws, device_error_word());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(
+      &cfg, fn, map, wait_poll_limit(), P, query, n_q_heads, group, gc, cache, n_kv_heads,
+      block_size, num_blocks, block_table, num_reqs, max_blocks, q_to_req, q_to_klen, max_klen,
+      sl2, plan.split_tokens, plan.splits, ws, device_error_word());
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
