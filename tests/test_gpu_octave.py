@@ -257,6 +257,57 @@ def test_octave_decode_longest_context():
     assert err <= ATOL, f"max abs error {err}"
 
 
+@pytest.mark.parametrize("v_bits,bs", [(4, 256), (4, 16), (3, 16)])
+def test_decode_right_after_quantize_sees_the_new_slots(v_bits, bs):
+    """Append and decode back to back on one stream with every input already
+    on the device, so no copy or synchronisation separates the two launches
+    (on the tensor-core path the decode and its combine are programmatic
+    dependent launches): four rounds, each appending 200 tokens to each of 2
+    requests and decoding over everything so far, must see every slot the
+    append before them wrote.  All outputs within 2e-3 of the oracle."""
+    fmt = (128, 64, v_bits, 0)
+    F = kvq.OctaveFormat(128, 64, v_bits)
+    sbytes = F.layout()["slot_bytes"]
+    Hkv, G, R, step, rounds = 2, 4, 2, 200, 4
+    T = step * rounds
+    per_req = -(-T // bs)
+    nblk = R * per_req + 3
+    blocks = np.random.default_rng(bs).permutation(nblk)[:R * per_req].reshape(R, per_req)
+    bt = blocks.astype(np.int32)
+    signs = synth.sign_pattern(128)
+    k, v = synth.kv_tokens(919, R, T, Hkv, 128, 0.01, 16.0)
+    kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+    t = np.arange(T)
+    slot = np.stack([bt[r, t // bs].astype(np.int64) * bs + t % bs for r in range(R)])
+    q = synth.to_bf16_bits(synth.queries(920, rounds * R, Hkv * G, 128))
+    # every round's inputs staged on the device before the first launch
+    chunks = [(to_dev(kb[:, i * step:(i + 1) * step].reshape(-1, Hkv, 128)),
+               to_dev(vb[:, i * step:(i + 1) * step].reshape(-1, Hkv, 128)),
+               to_dev(slot[:, i * step:(i + 1) * step].reshape(-1)),
+               to_dev(q[i * R:(i + 1) * R]),
+               to_dev(np.full(R, (i + 1) * step, np.int32))) for i in range(rounds)]
+    bt_d, q2r_d = to_dev(bt), to_dev(np.arange(R, dtype=np.int32))
+    sw = kvq.sign_words(signs)
+    cache = torch.zeros((nblk, Hkv, bs, sbytes), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    outs = []
+    for kc, vc, sc, qc, lc in chunks:
+        kvq.octave_quantize(F, kc, vc, sc, cache, sw)
+        outs.append(kvq.octave_decode_attn(F, qc, cache, bt_d, q2r_d, lc, T, 128 ** -0.5, sw))
+    got = [o.cpu().numpy() for o in outs]
+    want_slots = oracle.octave_quantize(kb.reshape(-1, Hkv, 128), vb.reshape(-1, Hkv, 128), fmt,
+                                        signs)
+    oc = np.zeros((nblk * bs, Hkv, sbytes), np.uint8)
+    oc[slot.reshape(-1)] = want_slots
+    oc = oc.reshape(nblk, bs, Hkv, sbytes).transpose(0, 2, 1, 3).copy()
+    for i in range(rounds):
+        want = oracle.octave_attention(q[i * R:(i + 1) * R], oc, bt, np.arange(R, dtype=np.int32),
+                                       np.full(R, (i + 1) * step, np.int32), fmt, 128 ** -0.5,
+                                       signs)
+        err = np.abs(got[i] - want).max()
+        assert err <= ATOL, f"round {i}: max abs error {err}"
+
+
 # ------------------------------------------------------------------ compact K
 @pytest.mark.parametrize("v_bits", [3, 4])
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
