@@ -315,6 +315,28 @@ def test_long_decode_full_size_sampled():
     assert np.abs(got - want).max() <= ATOL
 
 
+def test_long_decode_longest_context():
+    """One sequence of 524288 tokens (4x the long-context workload; 32 q / 4
+    kv heads, bf16, the workload's outlier channels): the decode sums 4x more
+    tokens per split, so an error that grows with the summed tokens shows
+    here.  Sampled cache rows bit-exact, all 32 head outputs within 2e-3."""
+    W = synth.WORKLOADS["long_decode"]
+    B, H, Hq, T = 1, W["n_kv_heads"], W["n_q_heads"], 524288
+    k, v = synth.kv_tokens(W["seed"] + T, B, T, H, 256, W["outlier_frac"], W["outlier_factor"])
+    k, v = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+    q = synth.to_bf16_bits(synth.queries(W["seed"] + T, B, Hq, 256))
+    gc = kvq.Q4Cache.contiguous(B, H, T)
+    kvq.quantize_append(gc, to_dev(k), to_dev(v), to_dev(np.zeros(B, np.int32)))
+    got = kvq.decode_attn(gc, to_dev(q), to_dev(np.full(B, T, np.int32)), T, 1 / 16).cpu().numpy()
+    threads = oracle.host_threads()
+    oc = oracle.Q4Cache(B * H * T, H, max_tokens=T)
+    oc.append(k, v, np.zeros(B, np.int32), threads=threads)
+    rng = np.random.default_rng(1)
+    compare_cache(gc, oc, rows=rng.choice(B * H * T, 4096, replace=False))
+    want = oc.decode_attn(q, [T], 1 / 16, threads=threads)
+    assert np.abs(got - want).max() <= ATOL
+
+
 def test_quantize_workload_full_size():
     """Quantize-on-append workload at full size (8 sequences x 8 kv heads,
     bf16): a 4096-token prefill, then 256 single-token appends, as the
