@@ -420,13 +420,13 @@ def octave_quantize(fmt: OctaveFormat, key: torch.Tensor, value: torch.Tensor,
                     slot_mapping: torch.Tensor, cache: torch.Tensor, sign_bits: np.ndarray,
                     stream=None) -> None:
     """key/value [T, Hkv, D] -> slots of cache [num_blocks, Hkv, block_size, slot]."""
+    num_blocks, _, block_size = _octave_cache_shape(fmt, cache)
     for n, t in (("key", key), ("value", value), ("slot_mapping", slot_mapping),
                  ("cache", cache)):
         _cuda_contig(n, t)
     if slot_mapping.dtype != torch.int64 or cache.dtype != torch.uint8:
         raise TypeError("slot_mapping must be int64 and cache uint8")
     T, hkv, _ = key.shape
-    num_blocks, _, block_size = _octave_cache_shape(fmt, cache)
     f = fmt.desc()
     sb = np.ascontiguousarray(sign_bits, dtype=np.int32)
     _check("kvq_octave_quantize",
@@ -446,11 +446,11 @@ def octave_decode_attn(fmt: OctaveFormat, query: torch.Tensor, cache: torch.Tens
                        q_to_klen: torch.Tensor, max_klen: int, scale: float,
                        sign_bits: np.ndarray, out: torch.Tensor | None = None,
                        workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    num_blocks, hkv, block_size = _octave_cache_shape(fmt, cache)
     for n, t in (("query", query), ("cache", cache), ("block_table", block_table),
                  ("q_to_req", q_to_req), ("q_to_klen", q_to_klen)):
         _cuda_contig(n, t)
     nq, hq, d = query.shape
-    num_blocks, hkv, block_size = _octave_cache_shape(fmt, cache)
     if out is None:
         out = torch.empty((nq, hq, d), dtype=torch.float32, device=query.device)
     if workspace is None:

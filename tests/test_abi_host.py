@@ -140,3 +140,21 @@ def test_device_error_calls_validate_on_host(L):
     assert L.kvq_device_errors(None) == kvq.KVQ_ERR_INVALID_ARG
     assert L.kvq_set_wait_limit(-2) == kvq.KVQ_ERR_INVALID_ARG
     assert L.kvq_set_wait_limit(-1) == kvq.KVQ_OK
+
+
+def test_octave_bindings_check_the_slot_width_first(L):
+    """The C ABI takes the slot width from the format; the bindings refuse a
+    cache of another width before any device check or library call."""
+    import torch
+    F = kvq.OctaveFormat(128, 64, 3)  # 112-byte slots
+    cache = torch.zeros((1, 2, 16, 128), dtype=torch.uint8)
+    k = torch.zeros((1, 2, 128), dtype=torch.bfloat16)
+    i32 = torch.zeros(1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="cache must be"):
+        kvq.octave_quantize(F, k, k, torch.zeros(1, dtype=torch.int64), cache, np.zeros(4))
+    with pytest.raises(ValueError, match="cache must be"):
+        kvq.octave_decode_attn(F, torch.zeros((1, 4, 128)), cache, i32.view(1, 1), i32, i32, 16,
+                               0.1, np.zeros(4))
+    with pytest.raises(ValueError, match="cache must be"):  # not 4-D
+        kvq.octave_quantize(F, k, k, torch.zeros(1, dtype=torch.int64), cache.view(-1),
+                            np.zeros(4))
