@@ -371,7 +371,11 @@ KVQ_API size_t kvq_octave_decode_attn_workspace(const kvq_octave_fmt *fmt, int32
  *   max_klen: host upper bound of q_to_klen (sizes the grid).
  *   sign_bits: host, as for kvq_octave_quantize.
  *   out: device, [num_q][num_q_heads][head_size] fp32.
- * Same implemented formats as kvq_octave_quantize; group size 1, 2, 4 or 8. */
+ * Same implemented formats as kvq_octave_quantize; group size 1, 2, 4 or 8.
+ * On the k3v4 tensor-core path the split kernel and the combine are launched
+ * as programmatic dependents of the work before them on `stream`; each
+ * waits for that work to finish before it reads any input, so stream order
+ * holds as for plain launches. */
 KVQ_API kvq_status kvq_octave_decode_attn(const kvq_octave_fmt *fmt, const void *query,
                                   kvq_dtype dtype, int32_t num_q, int32_t num_q_heads,
                                   const uint8_t *cache, int32_t num_kv_heads,
